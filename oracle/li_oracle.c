@@ -1,0 +1,335 @@
+/*
+ * Lightning Indexer forward pass: plain CPU oracle.
+ *
+ * TEST INFRASTRUCTURE. This file is the slow, obviously correct reference that the CUDA library
+ * is checked against. Only the tests, the package's smoke check and the benchmark's CPU-baseline
+ * leg may load it. It shares no code, header, table or helper with the CUDA library, and the
+ * library never calls it.
+ *
+ * What it computes, step by step, in the order the pages give it:
+ *
+ *   1. Per batch b, the query length L1_b and key length L2_b (lightning_indexer, "Constraints":
+ *      cu_seqlens are cumulative token counts, seqused_* are valid-token counts per batch;
+ *      aclnnLightningIndexerV2, constraints: TND padding of query rows past seqused_q, and
+ *      seqused_k being required for the paged key layout).
+ *   2. The key window of query row i (custom_pypto.npu_lightning_indexer_pto, sparse_mode:
+ *      0 = no mask, 3 = right-down causal, i.e. the lower triangle anchored at the bottom-right
+ *      corner): mode 0 keeps 0 <= j < L2_b, mode 3 additionally keeps j <= i + L2_b - L1_b.
+ *   3. The index score (custom_pypto.npu_lightning_indexer_pto, formula in the function
+ *      description; lightning_indexer, "Function" steps 1-3 and "Formula"):
+ *         I[i,j] = sum_h w[i,h] * ReLU( q[i,h,:] . k[j,:] )
+ *      with no 1/sqrt(d) scale (the scale belongs only to the main attention softmax in
+ *      torch_npu.npu_sparse_lightning_indexer_grad_kl_loss, formula 2).
+ *   4. Top-k selection per row, output sorted (npu_sparse_lightning_indexer_grad_kl_loss,
+ *      parameter sparse_indices: "sorted" token indices), padded with index -1 and value -inf
+ *      (aclnnLightningIndexerV2 and lightning_indexer, constraints), indices shifted by
+ *      output_idx_offset (aclnnLightningIndexerV2 constraints: the shifted index must not exceed
+ *      INT32_MAX).
+ *
+ * Precision. q, k and w arrive as bf16 bit patterns; every product and sum is taken in fp64, so
+ * the score is the exact real value up to fp64 rounding. The selection decision is then taken on
+ * the score rounded once to fp32, the precision the CUDA kernels decide in, and -0 is treated as
+ * +0. Order: score descending, then key index ascending (the pages only say "deterministic").
+ *
+ * Readings of points the pages leave open are listed in the design notes; each is marked
+ * [reading] below where it is applied.
+ *
+ * Planted mistakes. Building with -DORC_MUTANT=n plants mistake n (see the ORC_MUTANT blocks).
+ * A test builds each mutant and checks that the pins catch it. A normal build has none.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORC_MUTANT
+#define ORC_MUTANT 0
+#endif
+
+enum { ORC_BSND = 0, ORC_TND = 1, ORC_PA_BSND = 2 };
+enum { ORC_OK = 0, ORC_EARG = 1, ORC_EDATA = 2, ORC_ENOMEM = 3 };
+
+/* One problem. All arrays are host memory in the layouts the pages give:
+ *   q: BSND (B, S1, N1, D) or TND (T1, N1, D)
+ *   k: BSND (B, S2, 1, D), TND (T2, 1, D) or PA_BSND (num_blocks, block_size, 1, D)
+ *   w: (B, S1, N1) or (T1, N1)
+ * Optional arrays are NULL when absent. */
+typedef struct {
+    const uint16_t *q, *k, *w;
+    const int32_t *cu_seqlens_q, *cu_seqlens_k;
+    const int32_t *seqused_q, *seqused_k;
+    const int32_t *block_table;
+    const int32_t *output_idx_offset;
+    int64_t block_table_stride;
+    int32_t batch;
+    int32_t q_len;      /* BSND: S1; TND: T1 */
+    int32_t k_len;      /* BSND: S2; TND: T2; PA_BSND: unused */
+    int32_t num_blocks, block_size;
+    int32_t n_heads, head_dim, topk;
+    int32_t layout_q, layout_k, mask_mode;
+} orc_problem;
+
+static double bf16_value(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int64_t orc_num_rows(const orc_problem *p)
+{
+    return p->layout_q == ORC_TND ? (int64_t)p->q_len : (int64_t)p->batch * p->q_len;
+}
+
+/* Step 1: which batch a query row belongs to, its position there, and the lengths. */
+typedef struct {
+    int32_t b, i;          /* batch and row position within the batch                      */
+    int64_t L1, L2;        /* query rows allocated / keys valid for the batch              */
+    int64_t L1_used;       /* query rows in use (seqused_q), used for validity + alignment */
+} orc_row;
+
+static int orc_locate(const orc_problem *p, int64_t r, orc_row *o)
+{
+    if (p->layout_q == ORC_TND) {
+        int b = -1;
+        for (int bb = 0; bb < p->batch; ++bb)
+            if (p->cu_seqlens_q[bb] <= r && r < p->cu_seqlens_q[bb + 1]) { b = bb; break; }
+        if (b < 0) {            /* row not covered by any batch: no valid keys */
+            o->b = -1; o->i = 0; o->L1 = 0; o->L2 = 0; o->L1_used = 0;
+            return ORC_OK;
+        }
+        o->b = b;
+        o->i = (int32_t)(r - p->cu_seqlens_q[b]);
+        o->L1 = p->cu_seqlens_q[b + 1] - p->cu_seqlens_q[b];
+    } else {
+        o->b = (int32_t)(r / p->q_len);
+        o->i = (int32_t)(r % p->q_len);
+        o->L1 = p->q_len;
+    }
+    if (p->layout_k == ORC_TND)
+        o->L2 = p->cu_seqlens_k[o->b + 1] - p->cu_seqlens_k[o->b];
+    else if (p->layout_k == ORC_PA_BSND)
+        o->L2 = p->seqused_k[o->b];
+    else
+        o->L2 = p->k_len;
+    /* [reading] seqused_k, when given for a non-paged layout, is the valid key count. */
+    if (p->seqused_k && p->layout_k != ORC_PA_BSND && p->seqused_k[o->b] < o->L2)
+        o->L2 = p->seqused_k[o->b];
+    o->L1_used = o->L1;
+    if (p->seqused_q && p->seqused_q[o->b] < o->L1_used)
+        o->L1_used = p->seqused_q[o->b];
+    return ORC_OK;
+}
+
+/* Step 2: the window is always a prefix [0, hi) of the batch's keys. */
+static int64_t orc_window(const orc_problem *p, const orc_row *o)
+{
+    if (o->b < 0 || o->i >= o->L1_used || o->L2 <= 0) return 0;
+    int64_t hi = o->L2;
+    if (p->mask_mode == 3) {
+        /* [reading] right-down causal aligns the last used query row with the last key. */
+#if ORC_MUTANT == 3
+        int64_t lim = o->i + 1;                       /* mistake: top-left alignment */
+#else
+        int64_t lim = (int64_t)o->i + o->L2 - o->L1_used + 1;
+#endif
+        if (lim < hi) hi = lim;
+    }
+    return hi < 0 ? 0 : hi;
+}
+
+/* Key j of batch b (logical position within the batch's key sequence). */
+static const uint16_t *orc_key(const orc_problem *p, int32_t b, int64_t j)
+{
+    const int64_t D = p->head_dim;
+    if (p->layout_k == ORC_TND) {
+#if ORC_MUTANT == 8
+        return p->k + ((int64_t)p->cu_seqlens_q[b] + j) * D;   /* mistake: query offsets */
+#else
+        return p->k + ((int64_t)p->cu_seqlens_k[b] + j) * D;
+#endif
+    }
+    if (p->layout_k == ORC_PA_BSND) {
+#if ORC_MUTANT == 7
+        (void)b;
+        return p->k + j * D;                      /* mistake: block table ignored */
+#else
+        int64_t blk = p->block_table[(int64_t)b * p->block_table_stride + j / p->block_size];
+        return p->k + (blk * p->block_size + j % p->block_size) * D;
+#endif
+    }
+    return p->k + ((int64_t)b * p->k_len + j) * D;
+}
+
+static const uint16_t *orc_query(const orc_problem *p, int64_t r, int32_t h)
+{
+#if ORC_MUTANT == 6
+    /* mistake: head and row strides exchanged */
+    return p->q + ((int64_t)h * orc_num_rows(p) + r) * p->head_dim;
+#else
+    return p->q + (r * p->n_heads + h) * p->head_dim;
+#endif
+}
+
+/* Step 3: the exact score of row r against key j, in fp64. */
+static double orc_score(const orc_problem *p, int64_t r, const orc_row *o, int64_t j)
+{
+    const uint16_t *kj = orc_key(p, o->b, j);
+    double I = 0.0;
+#if ORC_MUTANT == 1
+    double sum_ws = 0.0;
+#endif
+    for (int32_t h = 0; h < p->n_heads; ++h) {
+        const uint16_t *qh = orc_query(p, r, h);
+        double s = 0.0;
+        for (int32_t d = 0; d < p->head_dim; ++d)
+            s += bf16_value(qh[d]) * bf16_value(kj[d]);
+        double wh = bf16_value(p->w[r * p->n_heads + h]);
+#if ORC_MUTANT == 1
+        sum_ws += wh * s;                              /* mistake: ReLU after the head sum */
+#elif ORC_MUTANT == 2
+        (void)wh;
+        I += (s > 0.0 ? s : 0.0);                      /* mistake: weights dropped */
+#elif ORC_MUTANT == 9
+        I += wh * s;                                   /* mistake: ReLU dropped */
+#elif ORC_MUTANT == 5
+        if (h == 0) I = wh * (s > 0.0 ? s : 0.0);     /* mistake: sum seeded with a -0 term */
+        else I += wh * (s > 0.0 ? s : 0.0);
+#else
+        I += wh * (s > 0.0 ? s : 0.0);
+#endif
+    }
+#if ORC_MUTANT == 1
+    I = sum_ws > 0.0 ? sum_ws : 0.0;
+#endif
+    return I;
+}
+
+typedef struct { float v; int64_t j; } orc_entry;
+
+/* Step 4 order: score descending, then key index ascending. */
+static int orc_cmp(const void *a, const void *b)
+{
+    const orc_entry *x = (const orc_entry *)a, *y = (const orc_entry *)b;
+    if (x->v > y->v) return -1;
+    if (x->v < y->v) return 1;
+#if ORC_MUTANT == 4
+    return (x->j < y->j) ? 1 : (x->j > y->j) ? -1 : 0;  /* mistake: higher index first */
+#else
+    return (x->j < y->j) ? -1 : (x->j > y->j) ? 1 : 0;
+#endif
+}
+
+static float orc_to_f32(double I)
+{
+    float v = (float)I;
+#if ORC_MUTANT != 5
+    if (v == 0.0f) v = 0.0f;   /* -0 counts as +0 */
+#endif
+    return v;
+}
+
+static int orc_check(const orc_problem *p)
+{
+    if (!p || !p->q || !p->k || !p->w) return ORC_EARG;
+    if (p->n_heads < 1 || p->head_dim < 1 || p->topk < 1 || p->batch < 0) return ORC_EARG;
+    if (p->mask_mode != 0 && p->mask_mode != 3) return ORC_EARG;
+    if (p->layout_q != ORC_BSND && p->layout_q != ORC_TND) return ORC_EARG;
+    if (p->layout_k < ORC_BSND || p->layout_k > ORC_PA_BSND) return ORC_EARG;
+    if (p->layout_q == ORC_TND && !p->cu_seqlens_q) return ORC_EARG;
+    if (p->layout_k == ORC_TND && !p->cu_seqlens_k) return ORC_EARG;
+    if (p->layout_k == ORC_PA_BSND && (!p->seqused_k || !p->block_table || p->block_size < 1))
+        return ORC_EARG;
+    return ORC_OK;
+}
+
+/* Number of query rows of the problem (B*S1 for BSND, T1 for TND). */
+int64_t orc_rows(const orc_problem *p) { return orc_num_rows(p); }
+
+/* The exact scores of one row over its window: scores[j] for 0 <= j < *hi (fp64).
+ * scores must hold at least the batch's key count. */
+int orc_scores(const orc_problem *p, int64_t r, double *scores, int64_t *hi)
+{
+    int rc = orc_check(p);
+    if (rc) return rc;
+    if (r < 0 || r >= orc_num_rows(p)) return ORC_EARG;
+    orc_row o;
+    orc_locate(p, r, &o);
+    *hi = orc_window(p, &o);
+    for (int64_t j = 0; j < *hi; ++j) scores[j] = orc_score(p, r, &o, j);
+    return ORC_OK;
+}
+
+/* The window length, batch and in-batch position of a row. */
+int orc_row_info(const orc_problem *p, int64_t r, int64_t *hi, int32_t *b, int32_t *i)
+{
+    int rc = orc_check(p);
+    if (rc) return rc;
+    if (r < 0 || r >= orc_num_rows(p)) return ORC_EARG;
+    orc_row o;
+    orc_locate(p, r, &o);
+    *hi = orc_window(p, &o);
+    *b = o.b;
+    *i = o.i;
+    return ORC_OK;
+}
+
+/* Top-k of the listed rows (all rows when rows == NULL). Row n of the output is the n-th listed
+ * row: out_idx[n*topk + m], out_val[n*topk + m]. Returns ORC_EDATA when an offset index would
+ * pass INT32_MAX. */
+int orc_topk(const orc_problem *p, const int64_t *rows, int64_t n_rows,
+             int32_t *out_idx, float *out_val)
+{
+    int rc = orc_check(p);
+    if (rc) return rc;
+    const int64_t R = rows ? n_rows : orc_num_rows(p);
+    int64_t cap = 0;
+    for (int64_t n = 0; n < R; ++n) {
+        int64_t r = rows ? rows[n] : n;
+        if (r < 0 || r >= orc_num_rows(p)) return ORC_EARG;
+        orc_row o;
+        orc_locate(p, r, &o);
+        int64_t hi = orc_window(p, &o);
+        if (hi > cap) cap = hi;
+    }
+    orc_entry *e = (orc_entry *)malloc((size_t)(cap > 0 ? cap : 1) * sizeof(orc_entry));
+    if (!e) return ORC_ENOMEM;
+    rc = ORC_OK;
+    for (int64_t n = 0; n < R; ++n) {
+        int64_t r = rows ? rows[n] : n;
+        orc_row o;
+        orc_locate(p, r, &o);
+        int64_t hi = orc_window(p, &o);
+        for (int64_t j = 0; j < hi; ++j) {
+            e[j].v = orc_to_f32(orc_score(p, r, &o, j));
+            e[j].j = j;
+        }
+        qsort(e, (size_t)hi, sizeof(orc_entry), orc_cmp);
+        int64_t m = hi < p->topk ? hi : p->topk;
+        int64_t off = 0;
+#if ORC_MUTANT != 10
+        if (p->output_idx_offset && o.b >= 0) off = p->output_idx_offset[o.b];
+#endif
+        for (int64_t s = 0; s < p->topk; ++s) {
+            int32_t *ix = out_idx + n * p->topk + s;
+            float *vx = out_val + n * p->topk + s;
+            if (s < m) {
+                int64_t idx = e[s].j + off;
+                if (idx > INT32_MAX) { rc = ORC_EDATA; idx = -1; }
+                *ix = (int32_t)idx;
+                *vx = e[s].v;
+            } else {
+#if ORC_MUTANT == 11
+                *ix = 0;                                /* mistake: wrong padding */
+                *vx = 0.0f;
+#else
+                *ix = -1;
+                *vx = -INFINITY;
+#endif
+            }
+        }
+    }
+    free(e);
+    return rc;
+}

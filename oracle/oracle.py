@@ -1,0 +1,190 @@
+"""ctypes wrapper around the C oracle (``li_oracle.c``).
+
+TEST INFRASTRUCTURE: only the tests, the package's smoke check and the benchmark's CPU-baseline
+leg use this module. It marshals arguments and nothing else; every step of the computation is
+in the C file. It accepts any problem object that carries the attributes listed in
+``_FIELDS`` (q, k, w as bf16 CPU tensors or uint16 numpy arrays, int32 side arrays or None,
+layouts as strings) and never imports the CUDA package.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+HERE = Path(__file__).resolve().parent
+SOURCE = HERE / "li_oracle.c"
+BUILD_DIR = HERE / "_build"
+
+LAYOUTS = {"BSND": 0, "TND": 1, "PA_BSND": 2}
+ORC_OK, ORC_EARG, ORC_EDATA, ORC_ENOMEM = 0, 1, 2, 3
+
+
+def build(mutant: int = 0, out_dir: Path | None = None, openmp: bool = False) -> Path:
+    """Compile the oracle with gcc. ``mutant`` > 0 plants the numbered mistake (for tests)."""
+    out_dir = Path(out_dir) if out_dir is not None else BUILD_DIR
+    out_dir.mkdir(parents=True, exist_ok=True)
+    name = "liorc" + (f"_m{mutant}" if mutant else "") + ".so"
+    out = out_dir / name
+    if out.exists() and out.stat().st_mtime >= SOURCE.stat().st_mtime:
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-Wall", "-fPIC", "-shared", f"-DORC_MUTANT={mutant}",
+           "-o", str(out), str(SOURCE), "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("w", ctypes.c_void_p),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("output_idx_offset", ctypes.c_void_p),
+        ("block_table_stride", ctypes.c_int64),
+        ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("k_len", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32),
+        ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
+    ]
+
+
+def _bits16(x) -> np.ndarray:
+    """bf16 tensor or uint16 array -> contiguous uint16 numpy array of the bit patterns."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch  # local: the oracle does not need torch unless handed tensors
+    assert x.dtype == torch.bfloat16, x.dtype
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _i32(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+class Oracle:
+    """One loaded build of the oracle (the normal one, or a planted mutant)."""
+
+    def __init__(self, lib_path: Path | str | None = None):
+        self.path = Path(lib_path) if lib_path is not None else build()
+        lib = ctypes.CDLL(str(self.path))
+        P = ctypes.POINTER(_Problem)
+        lib.orc_rows.argtypes = [P]
+        lib.orc_rows.restype = ctypes.c_int64
+        lib.orc_scores.argtypes = [P, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+        lib.orc_scores.restype = ctypes.c_int
+        lib.orc_row_info.argtypes = [P, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p]
+        lib.orc_row_info.restype = ctypes.c_int
+        lib.orc_topk.argtypes = [P, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                 ctypes.c_void_p]
+        lib.orc_topk.restype = ctypes.c_int
+        self.lib = lib
+
+    # -- marshalling -----------------------------------------------------------------------
+    def _marshal(self, pb):
+        keep = {}
+
+        def ptr(name, arr):
+            if arr is None:
+                return None
+            keep[name] = arr
+            return arr.ctypes.data
+
+        s = _Problem()
+        s.q = ptr("q", _bits16(pb.q))
+        s.k = ptr("k", _bits16(pb.k))
+        s.w = ptr("w", _bits16(pb.w))
+        for f in ("cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k", "block_table",
+                  "output_idx_offset"):
+            setattr(s, f, ptr(f, _i32(getattr(pb, f, None))))
+        bt = keep.get("block_table")
+        s.block_table_stride = int(bt.shape[-1]) if bt is not None and bt.ndim == 2 else 0
+        s.batch = int(pb.batch)
+        s.q_len = int(pb.q_len)
+        s.k_len = int(getattr(pb, "k_len", 0) or 0)
+        s.num_blocks = int(getattr(pb, "num_blocks", 0) or 0)
+        s.block_size = int(getattr(pb, "block_size", 0) or 0)
+        s.n_heads = int(pb.n_heads)
+        s.head_dim = int(pb.head_dim)
+        s.topk = int(pb.topk)
+        s.layout_q = LAYOUTS[pb.layout_q]
+        s.layout_k = LAYOUTS[pb.layout_k]
+        s.mask_mode = int(pb.mask_mode)
+        return s, keep
+
+    # -- entry points ----------------------------------------------------------------------
+    def rows(self, pb) -> int:
+        s, _keep = self._marshal(pb)
+        return int(self.lib.orc_rows(ctypes.byref(s)))
+
+    def topk(self, pb, rows=None, check: bool = True):
+        """Top-k of the given query rows (all when None). Returns (idx, val, status)."""
+        s, keep = self._marshal(pb)
+        if rows is None:
+            n = int(self.lib.orc_rows(ctypes.byref(s)))
+            rows_arr = None
+        else:
+            rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            n = rows_arr.size
+        idx = np.empty((n, s.topk), dtype=np.int32)
+        val = np.empty((n, s.topk), dtype=np.float32)
+        rc = self.lib.orc_topk(ctypes.byref(s),
+                               None if rows_arr is None else rows_arr.ctypes.data, n,
+                               idx.ctypes.data, val.ctypes.data)
+        del keep
+        if check and rc not in (ORC_OK,):
+            raise RuntimeError(f"oracle orc_topk returned {rc}")
+        return idx, val, rc
+
+    def scores(self, pb, row: int) -> np.ndarray:
+        """Exact (fp64) scores I[row, j] over the row's key window."""
+        s, keep = self._marshal(pb)
+        hi = ctypes.c_int64(0)
+        b = ctypes.c_int32(0)
+        i = ctypes.c_int32(0)
+        rc = self.lib.orc_row_info(ctypes.byref(s), row, ctypes.byref(hi), ctypes.byref(b),
+                                   ctypes.byref(i))
+        if rc:
+            raise RuntimeError(f"oracle orc_row_info returned {rc}")
+        out = np.empty(max(hi.value, 1), dtype=np.float64)
+        rc = self.lib.orc_scores(ctypes.byref(s), row, out.ctypes.data, ctypes.byref(hi))
+        del keep
+        if rc:
+            raise RuntimeError(f"oracle orc_scores returned {rc}")
+        return out[: hi.value]
+
+    def row_info(self, pb, row: int):
+        """(window length, batch, position in batch) of a query row."""
+        s, keep = self._marshal(pb)
+        hi = ctypes.c_int64(0)
+        b = ctypes.c_int32(0)
+        i = ctypes.c_int32(0)
+        rc = self.lib.orc_row_info(ctypes.byref(s), row, ctypes.byref(hi), ctypes.byref(b),
+                                   ctypes.byref(i))
+        del keep
+        if rc:
+            raise RuntimeError(f"oracle orc_row_info returned {rc}")
+        return hi.value, b.value, i.value
+
+
+_DEFAULT: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The normal (unmutated) oracle build, compiled on first use."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT
+
+
+def host_cores() -> int:
+    return os.cpu_count() or 1

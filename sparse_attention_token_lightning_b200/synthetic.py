@@ -1,0 +1,244 @@
+"""Seeded synthetic inputs for the Lightning Indexer forward pass.
+
+This module only draws and lays out inputs; it holds none of the indexer's arithmetic, so the
+CUDA path and the CPU oracle can both be fed from it. Every workload is synthetic (the pages
+name no dataset): q and k are N(0, 1) and w is N(0, 1/N1), drawn in fp32 from a seeded CPU
+``torch.Generator`` and rounded to bf16 (round-to-nearest-even). Shapes follow the pages:
+
+* q: BSND (B, S1, N1, D) or TND (T1, N1, D)
+* k: BSND (B, S2, 1, D), TND (T2, 1, D) or PA_BSND (num_blocks, block_size, 1, D)
+* w: (B, S1, N1) or (T1, N1)
+
+Draw order (fixed, so a seed names one input): structure first (lengths, cut points), then q,
+k, w, then the paged block permutation.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+D_DEFAULT = 128
+
+
+@dataclass
+class Problem:
+    """One indexer invocation: inputs plus the scalar arguments of the call."""
+
+    name: str
+    q: torch.Tensor
+    k: torch.Tensor
+    w: torch.Tensor
+    topk: int
+    batch: int
+    q_len: int                      # BSND: S1; TND: T1
+    k_len: int                      # BSND: S2; TND: T2; PA_BSND: 0
+    n_heads: int
+    head_dim: int = D_DEFAULT
+    layout_q: str = "BSND"
+    layout_k: str = "BSND"
+    mask_mode: int = 3
+    max_seqlen_q: int = 0
+    max_seqlen_k: int = 0
+    cu_seqlens_q: Optional[torch.Tensor] = None
+    cu_seqlens_k: Optional[torch.Tensor] = None
+    seqused_q: Optional[torch.Tensor] = None
+    seqused_k: Optional[torch.Tensor] = None
+    block_table: Optional[torch.Tensor] = None
+    output_idx_offset: Optional[torch.Tensor] = None
+    num_blocks: int = 0
+    block_size: int = 0
+    meta: dict = field(default_factory=dict)
+
+    TENSORS = ("q", "k", "w", "cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k",
+               "block_table", "output_idx_offset")
+
+    @property
+    def rows(self) -> int:
+        """Number of query rows (B*S1 for BSND, T1 for TND)."""
+        return self.q_len if self.layout_q == "TND" else self.batch * self.q_len
+
+    def to(self, device) -> "Problem":
+        kw = {}
+        for f in self.TENSORS:
+            t = getattr(self, f)
+            kw[f] = None if t is None else t.to(device)
+        return dataclasses.replace(self, **kw)
+
+    def replace(self, **kw) -> "Problem":
+        return dataclasses.replace(self, **kw)
+
+    def nbytes(self) -> int:
+        return sum(getattr(self, f).numel() * getattr(self, f).element_size()
+                   for f in self.TENSORS if getattr(self, f) is not None)
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def _normal(g, shape, std=1.0) -> torch.Tensor:
+    x = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
+    return x.to(torch.bfloat16)
+
+
+def _integer_valued(g, shape, kind) -> torch.Tensor:
+    """Values whose products and sums are exact in fp32: q,k in {-2..2}; w in {+-1/2,+-1,+-2}."""
+    if kind == "qk":
+        x = torch.randint(-2, 3, shape, generator=g).to(torch.float32)
+    else:
+        mag = torch.tensor([0.5, 1.0, 2.0])[torch.randint(0, 3, shape, generator=g)]
+        sgn = torch.randint(0, 2, shape, generator=g).to(torch.float32) * 2 - 1
+        x = mag * sgn
+    return x.to(torch.bfloat16)
+
+
+def _qkw(g, q_shape, k_shape, w_shape, n_heads, integer):
+    if integer:
+        return (_integer_valued(g, q_shape, "qk"), _integer_valued(g, k_shape, "qk"),
+                _integer_valued(g, w_shape, "w"))
+    return (_normal(g, q_shape), _normal(g, k_shape),
+            _normal(g, w_shape, std=1.0 / math.sqrt(n_heads)))
+
+
+def _i32(x) -> torch.Tensor:
+    return torch.as_tensor(x, dtype=torch.int32)
+
+
+def bsnd(B, S1, S2, N1, topk, mask_mode=3, seed=0, D=D_DEFAULT, integer=False, name="bsnd",
+         seqused_q=None, seqused_k=None, output_idx_offset=None) -> Problem:
+    """Dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)."""
+    g = _gen(seed)
+    q, k, w = _qkw(g, (B, S1, N1, D), (B, S2, 1, D), (B, S1, N1), N1, integer)
+    return Problem(name=name, q=q, k=k, w=w, topk=topk, batch=B, q_len=S1, k_len=S2,
+                   n_heads=N1, head_dim=D, layout_q="BSND", layout_k="BSND",
+                   mask_mode=mask_mode, max_seqlen_q=S1, max_seqlen_k=S2,
+                   seqused_q=None if seqused_q is None else _i32(seqused_q),
+                   seqused_k=None if seqused_k is None else _i32(seqused_k),
+                   output_idx_offset=None if output_idx_offset is None else _i32(output_idx_offset))
+
+
+def tnd(lens_q, lens_k, N1, topk, mask_mode=3, seed=0, D=D_DEFAULT, integer=False, name="tnd",
+        seqused_q=None, output_idx_offset=None, layout_k="TND") -> Problem:
+    """Packed varlen: q (T1,N1,D), k (T2,1,D), w (T1,N1) with cumulative cu_seqlens."""
+    g = _gen(seed)
+    lens_q = [int(x) for x in lens_q]
+    lens_k = [int(x) for x in lens_k]
+    B = len(lens_q)
+    cu_q = [0]
+    for x in lens_q:
+        cu_q.append(cu_q[-1] + x)
+    cu_k = [0]
+    for x in lens_k:
+        cu_k.append(cu_k[-1] + x)
+    T1, T2 = cu_q[-1], cu_k[-1]
+    if layout_k == "BSND":
+        S2 = max(lens_k) if lens_k else 0
+        q, k, w = _qkw(g, (T1, N1, D), (B, S2, 1, D), (T1, N1), N1, integer)
+        return Problem(name=name, q=q, k=k, w=w, topk=topk, batch=B, q_len=T1, k_len=S2,
+                       n_heads=N1, head_dim=D, layout_q="TND", layout_k="BSND",
+                       mask_mode=mask_mode, max_seqlen_q=max(lens_q) if lens_q else 0,
+                       max_seqlen_k=S2, cu_seqlens_q=_i32(cu_q),
+                       seqused_k=_i32(lens_k),
+                       seqused_q=None if seqused_q is None else _i32(seqused_q),
+                       output_idx_offset=None if output_idx_offset is None
+                       else _i32(output_idx_offset))
+    q, k, w = _qkw(g, (T1, N1, D), (T2, 1, D), (T1, N1), N1, integer)
+    return Problem(name=name, q=q, k=k, w=w, topk=topk, batch=B, q_len=T1, k_len=T2,
+                   n_heads=N1, head_dim=D, layout_q="TND", layout_k="TND", mask_mode=mask_mode,
+                   max_seqlen_q=max(lens_q) if lens_q else 0,
+                   max_seqlen_k=max(lens_k) if lens_k else 0,
+                   cu_seqlens_q=_i32(cu_q), cu_seqlens_k=_i32(cu_k),
+                   seqused_q=None if seqused_q is None else _i32(seqused_q),
+                   output_idx_offset=None if output_idx_offset is None
+                   else _i32(output_idx_offset))
+
+
+def paged(seqused_k, S1, N1, topk, block_size=64, table_width=None, mask_mode=3, seed=0,
+          D=D_DEFAULT, integer=False, name="paged", layout_q="BSND", lens_q=None,
+          output_idx_offset=None, spare_blocks=0) -> Problem:
+    """Paged key cache PA_BSND (num_blocks, block_size, 1, D) addressed through block_table.
+
+    Batch b owns ceil(seqused_k[b] / block_size) physical blocks, taken from a seeded random
+    permutation of all blocks; unused table entries are -1. ``spare_blocks`` adds physical
+    blocks no batch uses (the cache need not be dense)."""
+    g = _gen(seed)
+    seqused_k = [int(x) for x in seqused_k]
+    B = len(seqused_k)
+    nb = [max(0, -(-L // block_size)) for L in seqused_k]
+    NB = sum(nb) + int(spare_blocks)
+    width = table_width if table_width is not None else max(1, max(nb) if nb else 1)
+    if layout_q == "TND":
+        lens_q = [int(x) for x in lens_q]
+        cu_q = [0]
+        for x in lens_q:
+            cu_q.append(cu_q[-1] + x)
+        T1 = cu_q[-1]
+        q_shape, w_shape = (T1, N1, D), (T1, N1)
+    else:
+        q_shape, w_shape = (B, S1, N1, D), (B, S1, N1)
+    q, k, w = _qkw(g, q_shape, (max(NB, 1), block_size, 1, D), w_shape, N1, integer)
+    perm = torch.randperm(max(NB, 1), generator=g)[:NB]
+    table = torch.full((B, width), -1, dtype=torch.int32)
+    pos = 0
+    for b in range(B):
+        table[b, : nb[b]] = perm[pos: pos + nb[b]].to(torch.int32)
+        pos += nb[b]
+    pb = Problem(name=name, q=q, k=k, w=w, topk=topk, batch=B,
+                 q_len=T1 if layout_q == "TND" else S1, k_len=0, n_heads=N1, head_dim=D,
+                 layout_q=layout_q, layout_k="PA_BSND", mask_mode=mask_mode,
+                 max_seqlen_q=(max(lens_q) if layout_q == "TND" else S1),
+                 max_seqlen_k=max(seqused_k) if seqused_k else 0,
+                 seqused_k=_i32(seqused_k), block_table=table, num_blocks=max(NB, 1),
+                 block_size=block_size,
+                 output_idx_offset=None if output_idx_offset is None else _i32(output_idx_offset))
+    if layout_q == "TND":
+        pb.cu_seqlens_q = _i32(cu_q)
+    return pb
+
+
+# ---------------------------------------------------------------------------------------------
+# The named workloads. Sizes and distributions follow the indexer's target configurations:
+# q, k ~ N(0,1), w ~ N(0, 1/N1), D = 128, one key head.
+# ---------------------------------------------------------------------------------------------
+
+def varlen_lengths(total=32768, n_seq=8, seed=0):
+    """n_seq lengths >= 1 summing to total: n_seq-1 distinct cut points uniform in [1,total-1]."""
+    g = _gen(seed)
+    cuts = (torch.randperm(total - 1, generator=g)[: n_seq - 1] + 1).sort().values.tolist()
+    pts = [0] + cuts + [total]
+    return [pts[i + 1] - pts[i] for i in range(n_seq)], g
+
+
+def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
+    if name == "tiny":
+        return bsnd(1, 256, 256, 4, 32, 3, seed, integer=integer, name=name)
+    if name == "causal_prefill":
+        return bsnd(1, 4096, 4096, 64, 2048, 3, seed, integer=integer, name=name)
+    if name == "paged_decode":
+        g = _gen(seed)
+        lens = torch.randint(4096, 32769, (64,), generator=g).tolist()
+        return paged(lens, 1, 64, 2048, block_size=64, table_width=512, mask_mode=3,
+                     seed=seed + 1, integer=integer, name=name)
+    if name == "varlen":
+        lens, _ = varlen_lengths(32768, 8, seed)
+        return tnd(lens, lens, 64, 2048, 3, seed + 1, integer=integer, name=name)
+    if name == "long_2048":
+        return bsnd(1, 65536, 65536, 64, 2048, 3, seed, integer=integer, name=name)
+    if name == "long_8192":
+        return bsnd(1, 65536, 65536, 64, 8192, 3, seed, integer=integer, name=name)
+    if name == "pages_example":
+        # The shape of the pages' worked example (B=2, S1=64, N1=16, topk=32) with the key
+        # length it compresses to (130 // 4 = 32), taken uncompressed.
+        return bsnd(2, 64, 32, 16, 32, 3, seed, integer=integer, name=name)
+    raise KeyError(name)
+
+
+CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192")

@@ -1,0 +1,280 @@
+"""Pins for the CPU oracle: checks against facts fixed by the pages and by mathematics, not by
+the oracle itself.
+
+Each ``pin_*`` takes an ``Oracle`` and raises AssertionError when it disagrees. They are run on
+the real oracle by test_oracle_pins.py and on every planted-mistake build by
+test_oracle_mutants.py, which requires each planted mistake to fail at least one of them.
+"""
+import numpy as np
+import torch
+
+import golden_cases
+from sparse_attention_token_lightning_b200 import synthetic
+
+INT32_MAX = 2**31 - 1
+
+
+def _bits(v):
+    return np.asarray(v, dtype=np.float32).view(np.uint32)
+
+
+def _assert_same(a, b, what=""):
+    ia, va = a[0], a[1]
+    ib, vb = b[0], b[1]
+    assert np.array_equal(ia, ib), f"{what}: indices differ"
+    assert np.array_equal(_bits(va), _bits(vb)), f"{what}: values differ"
+
+
+def pin_golden(orc):
+    """Hand-worked fixtures under tests/golden (each cites the passages it follows)."""
+    for pb, ei, ev in golden_cases.all_cases():
+        i, v, rc = orc.topk(pb, check=False)
+        assert rc == 0, pb.name
+        assert np.array_equal(i, ei), f"{pb.name}: indices {i.tolist()} != {ei.tolist()}"
+        assert np.array_equal(_bits(v), _bits(ev)), f"{pb.name}: values {v.tolist()} != {ev.tolist()}"
+
+
+def _torch_desc(scores64, topk):
+    """Reference top-k of a float64 score row by a library sort: values rounded to fp32 once,
+    stable descending sort (equal values keep ascending index order)."""
+    s32 = torch.as_tensor(scores64).to(torch.float32)
+    s32 = torch.where(s32 == 0, torch.zeros_like(s32), s32)
+    vals, idx = torch.sort(s32, descending=True, stable=True)
+    m = min(topk, s32.numel())
+    out_i = np.full(topk, -1, dtype=np.int32)
+    out_v = np.full(topk, -np.inf, dtype=np.float32)
+    out_i[:m] = idx[:m].numpy()
+    out_v[:m] = vals[:m].numpy()
+    return out_i, out_v
+
+
+def pin_single_head_reduces_to_relu_matmul(orc):
+    """N1 = 1 and w = 1: the score is ReLU(q . k), a float64 matmul plus ReLU (library calls),
+    and the selection is a stable descending sort. topk covers zero scores, so the tie order of
+    the ReLU zeros is pinned too. No mask."""
+    pb = synthetic.bsnd(1, 6, 200, 1, 150, mask_mode=0, seed=11, name="n1")
+    pb.w = torch.ones_like(pb.w)
+    idx, val, _ = orc.topk(pb)
+    q64 = pb.q.to(torch.float64).reshape(6, 128)
+    k64 = pb.k.to(torch.float64).reshape(200, 128)
+    ref = torch.relu(q64 @ k64.T)
+    for r in range(6):
+        ei, ev = _torch_desc(ref[r], 150)
+        assert np.array_equal(idx[r], ei), f"row {r}: indices"
+        assert np.array_equal(_bits(val[r]), _bits(ev)), f"row {r}: values"
+
+
+def pin_one_hot_weights_pick_a_head(orc):
+    """w[t] = e_h selects head h alone: I[t,j] = ReLU(q[t,h] . k_j) (float64 matmul + ReLU)."""
+    pb = synthetic.bsnd(1, 8, 96, 4, 96, mask_mode=0, seed=12, name="onehot")
+    heads = [t % 4 for t in range(8)]
+    w = torch.zeros(1, 8, 4)
+    for t, h in enumerate(heads):
+        w[0, t, h] = 1.0
+    pb.w = w.to(torch.bfloat16)
+    idx, val, _ = orc.topk(pb)
+    q64 = pb.q.to(torch.float64).reshape(8, 4, 128)
+    k64 = pb.k.to(torch.float64).reshape(96, 128)
+    for t, h in enumerate(heads):
+        ei, ev = _torch_desc(torch.relu(q64[t, h] @ k64.T), 96)
+        assert np.array_equal(idx[t], ei), f"row {t}: indices"
+        assert np.array_equal(_bits(val[t]), _bits(ev)), f"row {t}: values"
+
+
+def pin_linear_in_weights(orc):
+    """I is linear in w: I(w1 + w2) = I(w1) + I(w2). Integer-valued inputs keep every sum exact,
+    so the identity holds bit for bit in fp64."""
+    base = synthetic.bsnd(1, 5, 40, 4, 8, mask_mode=0, seed=13, integer=True, name="lin")
+    g = torch.Generator().manual_seed(5)
+    w1 = torch.randint(-2, 3, base.w.shape, generator=g).to(torch.bfloat16)
+    w2 = torch.randint(-2, 3, base.w.shape, generator=g).to(torch.bfloat16)
+    for r in range(5):
+        s1 = orc.scores(base.replace(w=w1), r)
+        s2 = orc.scores(base.replace(w=w2), r)
+        s12 = orc.scores(base.replace(w=(w1.float() + w2.float()).to(torch.bfloat16)), r)
+        assert np.array_equal(s1 + s2, s12), f"row {r}: not linear in w"
+        s_neg = orc.scores(base.replace(w=(-w1.float()).to(torch.bfloat16)), r)
+        assert np.array_equal(s_neg, -s1), f"row {r}: not odd in w"
+
+
+def pin_head_permutation_invariance(orc):
+    """Permuting the heads of q and w together leaves every output unchanged (the head sum is a
+    sum, and integer-valued inputs make it exact)."""
+    pb = synthetic.bsnd(2, 16, 24, 6, 10, mask_mode=3, seed=14, integer=True, name="perm")
+    perm = torch.tensor([3, 0, 5, 1, 4, 2])
+    pp = pb.replace(q=pb.q[:, :, perm].contiguous(), w=pb.w[:, :, perm].contiguous())
+    _assert_same(orc.topk(pb), orc.topk(pp), "head permutation")
+
+
+def pin_key_permutation_equivariance(orc):
+    """Without a mask, permuting the keys permutes the scores: the score multiset of every row
+    is unchanged and score(j) follows its key."""
+    pb = synthetic.bsnd(1, 4, 50, 4, 50, mask_mode=0, seed=15, name="kperm")
+    perm = torch.randperm(50, generator=torch.Generator().manual_seed(3))
+    pp = pb.replace(k=pb.k[:, perm].contiguous())
+    for r in range(4):
+        a = orc.scores(pb, r)
+        b = orc.scores(pp, r)
+        assert np.array_equal(b, a[perm.numpy()]), f"row {r}"
+
+
+def _logical_varlen(seed=16):
+    """Three batches with L1 != L2 and one empty query batch, as TND/TND."""
+    lens_q, lens_k = [5, 1, 0, 7], [9, 4, 3, 12]
+    return synthetic.tnd(lens_q, lens_k, 3, 6, mask_mode=3, seed=seed, name="lv"), lens_q, lens_k
+
+
+def pin_layouts_agree(orc):
+    """The same logical data laid out as TND keys, as a paged cache with a shuffled block table,
+    and as one dense BSND batch per sequence gives the same outputs bit for bit."""
+    pt, lens_q, lens_k = _logical_varlen()
+    out_t = orc.topk(pt)
+    cu_q = np.cumsum([0] + lens_q)
+    cu_k = np.cumsum([0] + lens_k)
+    # paged: block size 4, blocks in a shuffled order, two spare blocks
+    bs = 4
+    nb = [(L + bs - 1) // bs for L in lens_k]
+    NB = sum(nb) + 2
+    perm = torch.randperm(NB, generator=torch.Generator().manual_seed(9)).tolist()
+    cache = torch.zeros(NB, bs, 1, 128, dtype=torch.bfloat16)
+    table = torch.full((len(lens_k), max(nb)), -1, dtype=torch.int32)
+    pos = 0
+    for b, L in enumerate(lens_k):
+        for blk in range(nb[b]):
+            phys = perm[pos]
+            pos += 1
+            table[b, blk] = phys
+            for s in range(bs):
+                j = blk * bs + s
+                if j < L:
+                    cache[phys, s, 0] = pt.k[cu_k[b] + j, 0]
+    pp = pt.replace(layout_k="PA_BSND", k=cache, block_table=table,
+                    seqused_k=torch.tensor(lens_k, dtype=torch.int32), cu_seqlens_k=None,
+                    num_blocks=NB, block_size=bs, k_len=0)
+    _assert_same(out_t, orc.topk(pp), "TND vs PA_BSND")
+    # dense, one batch at a time
+    for b in range(len(lens_q)):
+        if lens_q[b] == 0:
+            continue
+        qb = pt.q[cu_q[b]:cu_q[b + 1]].unsqueeze(0).contiguous()
+        wb = pt.w[cu_q[b]:cu_q[b + 1]].unsqueeze(0).contiguous()
+        kb = pt.k[cu_k[b]:cu_k[b + 1]].unsqueeze(0).contiguous()
+        pd = synthetic.Problem(name="dense", q=qb, k=kb, w=wb, topk=pt.topk, batch=1,
+                               q_len=lens_q[b], k_len=lens_k[b], n_heads=pt.n_heads,
+                               layout_q="BSND", layout_k="BSND", mask_mode=3)
+        i_d, v_d, _ = orc.topk(pd)
+        assert np.array_equal(out_t[0][cu_q[b]:cu_q[b + 1]], i_d), f"batch {b}: TND vs BSND idx"
+        assert np.array_equal(_bits(out_t[1][cu_q[b]:cu_q[b + 1]]), _bits(v_d)), f"batch {b}"
+
+
+def pin_single_query_row_sees_all_keys(orc):
+    """Right-down causal with one query row (decode) keeps every key: equals the unmasked result.
+    With S1 = S2 the last row also sees every key and the first row sees only key 0."""
+    pb = synthetic.bsnd(2, 1, 37, 4, 40, mask_mode=3, seed=17, name="dec")
+    _assert_same(orc.topk(pb), orc.topk(pb.replace(mask_mode=0)), "decode mask 3 vs 0")
+    sq = synthetic.bsnd(1, 20, 20, 4, 25, mask_mode=3, seed=18, name="sq")
+    i3, v3, _ = orc.topk(sq)
+    i0, v0, _ = orc.topk(sq.replace(mask_mode=0))
+    assert np.array_equal(i3[-1], i0[-1]) and np.array_equal(_bits(v3[-1]), _bits(v0[-1]))
+    assert i3[0, 0] == 0 and (i3[0, 1:] == -1).all()
+
+
+def pin_zero_query_ties_by_index(orc):
+    """q = 0 makes every score exactly 0: each row returns keys 0, 1, ... in order, values +0."""
+    pb = synthetic.bsnd(1, 8, 30, 4, 12, mask_mode=3, seed=19, name="zero")
+    pb.q = torch.zeros_like(pb.q)
+    idx, val, _ = orc.topk(pb)
+    off = 30 - 8
+    for t in range(8):
+        m = min(12, t + off + 1)
+        assert np.array_equal(idx[t, :m], np.arange(m)), f"row {t}"
+        assert (_bits(val[t, :m]) == 0).all(), f"row {t}: zero scores must be +0"
+        assert (idx[t, m:] == -1).all()
+
+
+def pin_negative_weights_zero_is_positive(orc):
+    """All weights negative: every score is <= 0, keys whose head scores are all <= 0 score zero,
+    and that zero is +0; zeros rank first, by index."""
+    pb = synthetic.bsnd(1, 6, 64, 2, 64, mask_mode=0, seed=20, integer=True, name="negw")
+    pb.w = -pb.w.abs()
+    idx, val, _ = orc.topk(pb)
+    for t in range(6):
+        v = val[t]
+        assert (v <= 0).all()
+        zeros = v == 0
+        assert (_bits(v[zeros]) == 0).all(), f"row {t}: -0 in the output"
+        nz = int(zeros.sum())
+        assert nz > 0
+        assert np.array_equal(idx[t, :nz], np.sort(idx[t, :nz]))
+
+
+def pin_offset_overflow_is_an_error(orc):
+    """An output_idx_offset that pushes an index past INT32_MAX is reported (the pages forbid it)."""
+    pb = synthetic.bsnd(1, 2, 3, 1, 3, mask_mode=0, seed=21, name="ovf",
+                        output_idx_offset=[INT32_MAX - 1])
+    _i, _v, rc = orc.topk(pb, check=False)
+    assert rc == 2
+    ok = pb.replace(output_idx_offset=torch.tensor([INT32_MAX - 2], dtype=torch.int32))
+    i2, _v2, rc2 = orc.topk(ok, check=False)
+    assert rc2 == 0 and i2.max() == INT32_MAX
+
+
+def check_row_invariants(orc, pb, idx, val, rows=None):
+    """Invariants of any correct output: m = min(topk, |window|) valid entries then padding;
+    indices unique and inside the window; values non-increasing and equal to the fp32 score at
+    their index; every selected key beats every unselected one (score, then lower index)."""
+    rows = range(pb.rows) if rows is None else rows
+    for n, r in enumerate(rows):
+        s = orc.scores(pb, r)
+        hi = s.size
+        m = min(pb.topk, hi)
+        ii, vv = idx[n], val[n]
+        assert (ii[m:] == -1).all() and np.isneginf(vv[m:]).all(), f"row {r}: padding"
+        off = 0
+        if pb.output_idx_offset is not None:
+            _hi, b, _i = orc.row_info(pb, r)
+            off = int(pb.output_idx_offset[b])
+        sel = ii[:m].astype(np.int64) - off
+        assert (sel >= 0).all() and (sel < hi).all(), f"row {r}: index outside window"
+        assert np.unique(sel).size == m, f"row {r}: duplicate index"
+        s32 = s.astype(np.float32)
+        s32[s32 == 0] = 0.0
+        assert np.array_equal(_bits(vv[:m]), _bits(s32[sel])), f"row {r}: value != score"
+        assert (np.diff(vv[:m]) <= 0).all(), f"row {r}: not sorted"
+        if m < hi:
+            mask = np.ones(hi, dtype=bool)
+            mask[sel] = False
+            un = np.nonzero(mask)[0]
+            kth_v, kth_i = vv[m - 1], sel[m - 1]
+            worse = (s32[un] < kth_v) | ((s32[un] == kth_v) & (un > kth_i))
+            assert worse.all(), f"row {r}: an unselected key beats the k-th"
+
+
+def pin_invariants_on_random_problems(orc):
+    """The invariants on small random problems of every layout and both masks."""
+    cases = [
+        synthetic.bsnd(2, 33, 70, 4, 16, mask_mode=3, seed=22, name="b3"),
+        synthetic.bsnd(1, 20, 20, 3, 7, mask_mode=0, seed=23, name="b0"),
+        synthetic.tnd([3, 9, 1], [12, 9, 30], 5, 8, mask_mode=3, seed=24, name="t3"),
+        synthetic.paged([17, 5, 40], 2, 4, 12, block_size=8, mask_mode=3, seed=25, name="p3",
+                        spare_blocks=3),
+        synthetic.bsnd(1, 12, 40, 4, 9, mask_mode=3, seed=26, integer=True, name="int"),
+    ]
+    for pb in cases:
+        idx, val, _ = orc.topk(pb)
+        check_row_invariants(orc, pb, idx, val)
+
+
+def pin_pages_example_shape(orc):
+    """The pages' worked example shape (B=2, S1=64, N1=16, topk=32) with 32 keys and mask 3:
+    rows i < 32 see no key (i + S2 - S1 < 0) and row i >= 32 sees i - 31 keys."""
+    pb = synthetic.config("pages_example")
+    idx, val, _ = orc.topk(pb)
+    assert idx.shape == (128, 32)
+    for r in range(128):
+        i = r % 64
+        valid = int((idx[r] >= 0).sum())
+        assert valid == max(0, min(32, i - 31)), f"row {r}: {valid} valid entries"
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
