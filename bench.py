@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of the Lightning Indexer forward pass on B200.
+
+One step = one li_indexer call on one batch of synthetic input: schedule build, score kernel
+(ReLU, weights, head sum, mask fused), top-k selection and padding, i.e. the whole hot path.
+Default workload: causal prefill, B=1, S1=S2=4096, N1=64, D=128, topk=2048, right-down causal
+mask, BSND, bf16 inputs (fp32 accumulation). The metric is query tokens per second; the
+roofline object reports the score kernel's tensor throughput against the measured bf16 peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+Multi-GPU (torchrun): each rank runs its own independent problem (seed = rank); no data-path
+collective exists because query rows are independent (weak scaling). The reported time is the
+max over ranks of the device time of the K steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from sparse_attention_token_lightning_b200 import li, synthetic  # noqa: E402
+
+METRIC = "indexer query-tokens/s; TFLOP/s as % bf16 tensor peak (N1=64,D=128,topk=2048)"
+UNIT = "query-tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+WORKLOAD_TEXT = {
+    "causal_prefill": "causal prefill: B=1, S1=S2=4096, N1=64, N2=1, D=128, topk=2048, "
+                      "mask_mode=3, BSND, q,k ~N(0,1), w ~N(0,1/64), bf16",
+    "tiny": "tiny prefill: B=1, S1=S2=256, N1=4, D=128, topk=32, mask_mode=3, BSND",
+    "paged_decode": "paged decode: B=64, S1=1, N1=64, D=128, topk=2048, mask_mode=3, PA_BSND "
+                    "block_size=64, seqused_k~U[4096,32768], permuted block_table",
+    "varlen": "varlen TND: 8 sequences summing to T1=T2=32768, N1=64, D=128, topk=2048, "
+              "mask_mode=3",
+    "long_2048": "long-context prefill: B=1, S1=S2=65536, N1=64, D=128, topk=2048, mask_mode=3",
+    "long_8192": "long-context prefill: B=1, S1=S2=65536, N1=64, D=128, topk=8192, mask_mode=3",
+}
+
+
+def valid_pairs(pb) -> int:
+    """(query row, key) pairs inside the mask windows, from the integer lengths alone."""
+    if pb.layout_q == "TND":
+        cu = pb.cu_seqlens_q.tolist()
+        L1s = [cu[i + 1] - cu[i] for i in range(pb.batch)]
+    else:
+        L1s = [pb.q_len] * pb.batch
+    if pb.layout_k == "TND":
+        cu = pb.cu_seqlens_k.tolist()
+        L2s = [cu[i + 1] - cu[i] for i in range(pb.batch)]
+    elif pb.layout_k == "PA_BSND":
+        L2s = pb.seqused_k.tolist()
+    else:
+        L2s = [pb.k_len] * pb.batch
+    if pb.seqused_k is not None and pb.layout_k != "PA_BSND":
+        L2s = [min(a, b) for a, b in zip(L2s, pb.seqused_k.tolist())]
+    total = 0
+    for b in range(pb.batch):
+        L1, L2 = L1s[b], L2s[b]
+        used = L1 if pb.seqused_q is None else min(L1, int(pb.seqused_q[b]))
+        if pb.mask_mode == 0:
+            total += used * max(L2, 0)
+            continue
+        # row i sees min(L2, max(0, i + L2 - used + 1)) keys
+        lo = L2 - used + 1
+        for i in range(used):
+            total += min(L2, max(0, i + lo))
+    return total
+
+
+def key_bytes(pb) -> int:
+    """Bytes of keys the path must read once: 256 B per valid key per batch."""
+    if pb.layout_k == "PA_BSND":
+        return int(pb.seqused_k.sum()) * pb.head_dim * 2
+    return pb.k.numel() * 2
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(pb, seconds: float, seed: int = 0):
+    """Time the CPU oracle (as it stands, one thread) on seeded random rows of the workload for
+    about `seconds`; returns (query rows per second, rows timed)."""
+    import numpy as np
+    from oracle import oracle as orc
+
+    bound = orc.default().bind(pb)
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(pb.rows)
+    done, t_total, chunk = 0, 0.0, 4
+    while done < pb.rows and t_total < seconds:
+        rows = order[done: done + chunk]
+        t0 = time.perf_counter()
+        bound.topk(rows)
+        t_total += time.perf_counter() - t0
+        done += len(rows)
+        chunk = min(chunk * 2, 256)
+    return done / t_total, done, t_total
+
+
+def run_reference(a):
+    """The CPU oracle as the reference arm: each step times a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    pb = synthetic.config(a.config)
+    step_seconds = a.ref_step_seconds
+    for s in range(a.warmup):
+        cpu_oracle_rate(pb, step_seconds / 4, seed=1000 + s)
+    rates, rows = [], 0
+    for s in range(a.steps):
+        r, n, _t = cpu_oracle_rate(pb, step_seconds, seed=s)
+        rates.append(r)
+        rows += n
+    value = statistics.mean(rates)
+    ms = pb.rows / value * 1e3
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT.get(a.config, a.config), "name": a.config,
+                       "rows_per_step": pb.rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} seeded-random query rows over {a.steps} steps "
+                                       f"(~{step_seconds:.0f} s each), single-threaded C oracle; "
+                                       "per-row cost is unbiased so rows/s scales to the workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="causal_prefill", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU-oracle sample budget for cpu_baseline (0 = skip)")
+    ap.add_argument("--ref-step-seconds", type=float, default=3.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.impl == "reference":
+        return run_reference(a)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    def barrier():
+        if dist:
+            torch.distributed.barrier()
+
+    li.lib()
+    pb_cpu = synthetic.config(a.config, seed=rank)
+    pb = pb_cpu.to(dev)
+    args = li.make_args(pb)
+    ws = li.empty_workspace(args, dev)
+    idx = torch.empty(li.out_shape(pb), dtype=torch.int32, device=dev)
+    val = torch.empty(li.out_shape(pb), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        li.li_indexer(args, None, ws, idx, val, stream)
+
+    for _ in range(a.warmup):
+        step()
+    st, bits = li.li_check_status(ws)
+    if st != li.LI_OK:
+        raise SystemExit(f"device status {st} bits {bits:#x}")
+
+    K = a.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    for e in ev:
+        for x in e:
+            x.record(stream)            # materialise the CUDA events before handing them out
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for s in range(K):
+        flush.zero_()                   # evict the inputs from L2 (outside the step's events)
+        e = ev[s]
+        li.li_set_stage_events(e[2:8])
+        e[0].record(stream)
+        step()
+        e[1].record(stream)
+    li.li_set_stage_events(None)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+
+    step_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    meta_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(K)]
+    score_ms = [ev[s][4].elapsed_time(ev[s][5]) for s in range(K)]
+    sel_ms = [ev[s][6].elapsed_time(ev[s][7]) for s in range(K)]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    rows = pb.rows
+    value = rows * world / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers ---------------------------------
+    e2e = None
+    if not a.no_e2e:
+        host = {f: getattr(pb_cpu, f).pin_memory() for f in synthetic.Problem.TENSORS
+                if getattr(pb_cpu, f) is not None}
+        h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+        h_val = torch.empty(val.shape, dtype=val.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = h_idx.numel() * 4 + h_val.numel() * 4
+
+        def e2e_step():
+            for f, t in host.items():
+                getattr(pb, f).copy_(t, non_blocking=True)
+            li.li_indexer(args, None, ws, idx, val, stream)
+            h_idx.copy_(idx, non_blocking=True)
+            h_val.copy_(val, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / K
+        if dist:
+            t = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        barrier()
+        e2e = {"value": rows * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    peaks = load_peaks()
+    flops = 2.0 * valid_pairs(pb_cpu) * pb.n_heads * pb.head_dim
+    sc = statistics.mean(score_ms)
+    achieved = flops / (sc / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "score kernel (q.k contraction + ReLU/weight/head-sum epilogue)",
+                "peak_source": f"{peaks['source']} bf16 burst"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
+                       "rows_per_step_per_gpu": rows, "valid_pairs": valid_pairs(pb_cpu),
+                       "l2": "flushed before every step by a 256 MB write outside the step's "
+                             "CUDA events",
+                       "parallelism": f"{world} independent replicas (one problem per GPU)"},
+            "roofline": roofline,
+            "stages_ms": {"schedule": statistics.mean(meta_ms), "score": sc,
+                          "select": statistics.mean(sel_ms)},
+            "tflops_whole_step": flops / (ms_per_step / 1e3) / 1e12,
+            "clocks": clk, "gpu_launches": 3 * K}
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and a.cpu_seconds > 0:
+        rate, n, t = cpu_oracle_rate(pb_cpu, a.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{n} seeded-random query rows of the same workload, "
+                                          f"{t:.1f} s, single-threaded C oracle (fp64)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+/*
+ * li.h -- C ABI of the Lightning Indexer forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (custom_pypto.npu_lightning_indexer_pto, function description formula;
+ * lightning_indexer, "Function" steps 1-3 and "Formula"; aclnnLightningIndexerV2, formula and
+ * main computation steps): for every query row t of batch b and every key j in the row's window,
+ *
+ *     I[t,j] = sum_{h < N1} w[t,h] * ReLU( q[t,h,:] . k[j,:] ),      D = 128, one key head,
+ *
+ * then the topk keys with the largest I, sorted by I descending (lower key index first on equal
+ * scores), returned as int32 sparse_indices (-1 padded) and fp32 sparse_values (-inf padded)
+ * (lightning_indexer and aclnnLightningIndexerV2, constraints on the invalid part).
+ *
+ * Windows (custom_pypto.npu_lightning_indexer_pto, parameter sparse_mode):
+ *     mask_mode 0 (defaultMask):       0 <= j < L2_b
+ *     mask_mode 3 (rightDownCausal):   0 <= j < L2_b  and  j <= i + L2_b - L1_b
+ * where i is the row's position inside batch b, L1_b the batch's query rows in use (seqused_q[b]
+ * when given, else all of them) and L2_b its key count. Indices are positions inside batch b's key
+ * sequence, plus output_idx_offset[b] when given.
+ *
+ * Conventions shared by every entry point
+ *   - All data pointers are DEVICE pointers of the current CUDA device; NULL means "absent".
+ *   - The caller owns every buffer; the library never allocates device or pinned memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every launch
+ *     is stream-ordered; no entry point except li_check_status synchronizes or reads device
+ *     memory on the host, so li_metadata and li_indexer can be captured in a CUDA graph.
+ *   - Argument errors are detected on the host before anything is launched and are returned as a
+ *     status; the message is available from li_last_error_string(). Errors that depend on device
+ *     data (non-monotone cu_seqlens, out-of-range block table entries, offsets overflowing int32,
+ *     lengths above the declared maxima) are recorded in a device status word inside the
+ *     workspace and reported by li_check_status(); the affected rows hold unspecified values but
+ *     no access leaves the caller's buffers.
+ */
+#ifndef LI_H_
+#define LI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LI_ABI_VERSION 1
+
+typedef enum li_layout {
+    LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
+    LI_LAYOUT_TND = 1,      /* packed varlen: q (T1,N1,D), k (T2,1,D), w (T1,N1) + cu_seqlens   */
+    LI_LAYOUT_PA_BSND = 2   /* paged keys only: k (num_blocks, block_size, 1, D) + block_table  */
+} li_layout;
+
+typedef enum li_status {
+    LI_OK = 0,
+    LI_ERR_INVALID_ARG = 1,     /* an argument violates the documented contract             */
+    LI_ERR_UNSUPPORTED = 2,     /* a valid request this build does not implement            */
+    LI_ERR_WORKSPACE = 3,       /* workspace / metadata buffer too small or misaligned      */
+    LI_ERR_CUDA = 4,            /* a CUDA runtime call failed (message has the CUDA error)  */
+    LI_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait gave up (li_check_status)     */
+    LI_ERR_DEVICE_DATA = 6      /* device-resident lengths/tables/offsets were invalid      */
+} li_status;
+
+typedef enum li_dtype {
+    LI_DTYPE_BF16 = 0
+} li_dtype;
+
+/* Device status word bits, as reported through li_check_status(). */
+#define LI_DEVERR_TIMEOUT   0x1u   /* a bounded wait (mbarrier / scheduler) ran out            */
+#define LI_DEVERR_LENGTHS   0x2u   /* cu_seqlens not monotone, or a length above its maximum  */
+#define LI_DEVERR_TABLE     0x4u   /* a block_table entry in use is outside [0, num_blocks)    */
+#define LI_DEVERR_OFFSET    0x8u   /* output_idx_offset < 0, or index + offset > INT32_MAX     */
+
+/*
+ * Arguments of one indexer call. Mirrors the pages' prototypes (lightning_indexer, "Prototype":
+ * q, k, w, topk, cu_seqlens_q/k, seqused_q/k, block_table, output_idx_offset, max_seqlen_q/k,
+ * layout_q/k, mask_mode, return_value) with the tensor shapes made explicit.
+ */
+typedef struct li_args {
+    const void *q;                      /* bf16, BSND (B,S1,N1,128) or TND (T1,N1,128), dense  */
+    const void *k;                      /* bf16, BSND (B,S2,1,128), TND (T2,1,128) or
+                                           PA_BSND (num_blocks, block_size, 1, 128), dense     */
+    const void *w;                      /* bf16, (B,S1,N1) or (T1,N1), dense                    */
+    const int32_t *cu_seqlens_q;        /* [B+1], non-decreasing; required iff layout_q == TND  */
+    const int32_t *cu_seqlens_k;        /* [B+1], non-decreasing; required iff layout_k == TND  */
+    const int32_t *seqused_q;           /* [B] or NULL: query rows in use per batch; rows past
+                                           it are all padding and the causal window aligns to it */
+    const int32_t *seqused_k;           /* [B]: keys per batch. Required for PA_BSND; for the
+                                           other layouts, when given, caps the batch's keys      */
+    const int32_t *block_table;         /* [B, block_table_stride]; required for PA_BSND        */
+    int64_t block_table_stride;         /* entries per batch row of block_table                 */
+    const int32_t *output_idx_offset;   /* [B] or NULL: added to every valid output index      */
+    int32_t batch;                      /* B (number of sequences)                              */
+    int32_t q_len;                      /* BSND: S1 ; TND: T1 (rows of q)                       */
+    int32_t k_len;                      /* BSND: S2 ; TND: T2 (rows of k) ; PA_BSND: ignored    */
+    int32_t max_seqlen_q;               /* upper bound of every batch's query rows (BSND: S1)   */
+    int32_t max_seqlen_k;               /* upper bound of every batch's key count (BSND: S2)    */
+    int32_t num_blocks;                 /* PA_BSND: blocks in the cache                         */
+    int32_t block_size;                 /* PA_BSND: keys per block, 1..1024                     */
+    int32_t num_heads_q;                /* N1, 1..64                                            */
+    int32_t num_heads_k;                /* N2, must be 1                                        */
+    int32_t head_dim;                   /* D, must be 128                                       */
+    int32_t topk;                       /* 1..8192                                              */
+    int32_t layout_q;                   /* li_layout: BSND or TND                               */
+    int32_t layout_k;                   /* li_layout: BSND, TND or PA_BSND                      */
+    int32_t mask_mode;                  /* 0 (no mask) or 3 (right-down causal)                 */
+    int32_t dtype_qk;                   /* li_dtype of q and k: LI_DTYPE_BF16                   */
+    int32_t dtype_w;                    /* li_dtype of w: LI_DTYPE_BF16                         */
+    int32_t return_value;               /* 1: write sparse_values too; 0: indices only          */
+} li_args;
+
+/*
+ * li_metadata_workspace_size -- bytes of the metadata buffer li_metadata() fills.
+ * Host only. Validates `args` (same checks as li_indexer_workspace_size, device pointers are not
+ * dereferenced). Counterpart of the pages' lightning_indexer_metadata sizing (lightning_indexer,
+ * "Function": the metadata op produces the per-core task list) and of the first phase of the
+ * two-phase call (aclnnLightningIndexerV2: GetWorkspaceSize validates and sizes, then execute).
+ * Returns LI_OK and writes *bytes, or an argument error.
+ */
+li_status li_metadata_workspace_size(const li_args *args, size_t *bytes);
+
+/*
+ * li_metadata -- build the schedule (work list) for li_indexer on `stream`.
+ * Replaces the pages' per-AI-core task list (lightning_indexer, "Function" and "Prototype":
+ * lightning_indexer_metadata must run before lightning_indexer) by a list of query blocks and key
+ * ranges ordered longest first, read by the persistent sm_100a kernels. It reads the
+ * device-resident lengths (cu_seqlens, seqused) on the device; nothing is read back to the host.
+ * `metadata` is a device buffer of at least li_metadata_workspace_size() bytes, 256-byte aligned,
+ * owned by the caller and valid until the li_indexer calls that use it have completed. Invalid
+ * device data sets bits in the metadata's status word, which li_indexer copies to its own.
+ */
+li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *stream);
+
+/*
+ * li_indexer_workspace_size -- bytes of scratch li_indexer() needs for `args`.
+ * Host only; validates like li_metadata_workspace_size. The size covers the device status word,
+ * the scheduler counters, room for an inline schedule, and the fp32 score rows the selection step
+ * reads (rows x max_seqlen_k x 4 bytes).
+ */
+li_status li_indexer_workspace_size(const li_args *args, size_t *bytes);
+
+/*
+ * li_indexer -- the forward pass (lightning_indexer, "Prototype" and "Function"): scores,
+ * ReLU, weights, head sum, mask, top-k, padding, for every query row.
+ *   metadata        schedule from li_metadata() for the same args, or NULL to build it inline
+ *                   into the workspace (one extra small kernel launch).
+ *   workspace       device scratch of >= li_indexer_workspace_size() bytes, 256-byte aligned.
+ *                   Contents on entry are ignored; after the call it holds the status word.
+ *   sparse_indices  int32 output, (B,S1,1,topk) for BSND q or (T1,1,topk) for TND q.
+ *   sparse_values   fp32 output of the same shape, or NULL when args->return_value == 0.
+ * Every output row is written (valid entries first, then -1 / -inf). Deterministic: the same
+ * inputs give bit-identical outputs (aclnnLightningIndexerV2 and lightning_indexer, deterministic
+ * computation). Returns after queueing the kernels; use li_check_status to learn about device
+ * data errors.
+ */
+li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
+                     size_t workspace_bytes, int32_t *sparse_indices, float *sparse_values,
+                     void *stream);
+
+/*
+ * li_check_status -- synchronize `stream`, read the device status word of `workspace` (the one
+ * passed to the last li_indexer on that stream) into *device_bits (LI_DEVERR_* bits, may be NULL)
+ * and map it to a status: LI_OK, LI_ERR_DEVICE_TIMEOUT or LI_ERR_DEVICE_DATA. A CUDA error
+ * raised by the stream is returned as LI_ERR_CUDA.
+ */
+li_status li_check_status(const void *workspace, void *stream, uint32_t *device_bits);
+
+/*
+ * li_set_stage_events -- benchmarking hook. With n_events == 6, every later li_indexer call
+ * records events[0]/[1] around the inline schedule build (only when metadata == NULL),
+ * events[2]/[3] around the score kernel and events[4]/[5] around the selection kernel, on the
+ * call's stream, so a caller can time each kernel with cudaEventElapsedTime. The events are
+ * cudaEvent_t handles passed as void*, created by the caller (timing enabled) and owned by it.
+ * n_events == 0 turns the hook off. The setting is process-wide; do not change it while another
+ * host thread is inside li_indexer. Returns LI_ERR_INVALID_ARG for any other count.
+ */
+li_status li_set_stage_events(void *const *events, int32_t n_events);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *li_last_error_string(void);
+
+/* LI_ABI_VERSION of the loaded library. */
+int32_t li_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LI_H_ */

@@ -275,11 +275,25 @@ int orc_row_info(const orc_problem *p, int64_t r, int64_t *hi, int32_t *b, int32
     return ORC_OK;
 }
 
+/* The exact score of one (row, key) pair; ORC_EARG when j is outside the row's window. */
+int orc_score_at(const orc_problem *p, int64_t r, int64_t j, double *out)
+{
+    int rc = orc_check(p);
+    if (rc) return rc;
+    if (r < 0 || r >= orc_num_rows(p)) return ORC_EARG;
+    orc_row o;
+    orc_locate(p, r, &o);
+    if (j < 0 || j >= orc_window(p, &o)) return ORC_EARG;
+    *out = orc_score(p, r, &o, j);
+    return ORC_OK;
+}
+
 /* Top-k of the listed rows (all rows when rows == NULL). Row n of the output is the n-th listed
- * row: out_idx[n*topk + m], out_val[n*topk + m]. Returns ORC_EDATA when an offset index would
- * pass INT32_MAX. */
+ * row: out_idx[n*topk + m], out_val[n*topk + m]. When row_maxabs is not NULL it receives, per
+ * listed row, the largest |I| over the row's window (0 for an empty window). Returns ORC_EDATA
+ * when an offset index would pass INT32_MAX. */
 int orc_topk(const orc_problem *p, const int64_t *rows, int64_t n_rows,
-             int32_t *out_idx, float *out_val)
+             int32_t *out_idx, float *out_val, double *row_maxabs)
 {
     int rc = orc_check(p);
     if (rc) return rc;
@@ -301,10 +315,14 @@ int orc_topk(const orc_problem *p, const int64_t *rows, int64_t n_rows,
         orc_row o;
         orc_locate(p, r, &o);
         int64_t hi = orc_window(p, &o);
+        double maxabs = 0.0;
         for (int64_t j = 0; j < hi; ++j) {
-            e[j].v = orc_to_f32(orc_score(p, r, &o, j));
+            double I = orc_score(p, r, &o, j);
+            if (fabs(I) > maxabs) maxabs = fabs(I);
+            e[j].v = orc_to_f32(I);
             e[j].j = j;
         }
+        if (row_maxabs) row_maxabs[n] = maxabs;
         qsort(e, (size_t)hi, sizeof(orc_entry), orc_cmp);
         int64_t m = hi < p->topk ? hi : p->topk;
         int64_t off = 0;

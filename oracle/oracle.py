@@ -84,7 +84,9 @@ class Oracle:
                                      ctypes.c_void_p]
         lib.orc_row_info.restype = ctypes.c_int
         lib.orc_topk.argtypes = [P, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
-                                 ctypes.c_void_p]
+                                 ctypes.c_void_p, ctypes.c_void_p]
+        lib.orc_score_at.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+        lib.orc_score_at.restype = ctypes.c_int
         lib.orc_topk.restype = ctypes.c_int
         self.lib = lib
 
@@ -121,58 +123,87 @@ class Oracle:
         return s, keep
 
     # -- entry points ----------------------------------------------------------------------
-    def rows(self, pb) -> int:
-        s, _keep = self._marshal(pb)
-        return int(self.lib.orc_rows(ctypes.byref(s)))
+    def bind(self, pb) -> "Bound":
+        """Marshal a problem once; the returned object answers repeated queries on it."""
+        return Bound(self, pb)
 
-    def topk(self, pb, rows=None, check: bool = True):
-        """Top-k of the given query rows (all when None). Returns (idx, val, status)."""
-        s, keep = self._marshal(pb)
+    def rows(self, pb) -> int:
+        return self.bind(pb).rows()
+
+    def topk(self, pb, rows=None, check: bool = True, with_maxabs: bool = False):
+        """Top-k of the given query rows (all when None). Returns (idx, val, status), plus the
+        per-row max |I| over the window when with_maxabs."""
+        return self.bind(pb).topk(rows, check, with_maxabs)
+
+    def score_at(self, pb, row: int, j: int) -> float:
+        return self.bind(pb).score_at(row, j)
+
+    def scores(self, pb, row: int) -> np.ndarray:
+        return self.bind(pb).scores(row)
+
+    def row_info(self, pb, row: int):
+        return self.bind(pb).row_info(row)
+
+
+class Bound:
+    """A problem marshalled for one oracle build."""
+
+    def __init__(self, orc: Oracle, pb):
+        self.lib = orc.lib
+        self.s, self._keep = orc._marshal(pb)
+        self.topk_k = int(self.s.topk)
+
+    def rows(self) -> int:
+        return int(self.lib.orc_rows(ctypes.byref(self.s)))
+
+    def topk(self, rows=None, check: bool = True, with_maxabs: bool = False):
         if rows is None:
-            n = int(self.lib.orc_rows(ctypes.byref(s)))
+            n = self.rows()
             rows_arr = None
         else:
             rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
             n = rows_arr.size
-        idx = np.empty((n, s.topk), dtype=np.int32)
-        val = np.empty((n, s.topk), dtype=np.float32)
-        rc = self.lib.orc_topk(ctypes.byref(s),
+        idx = np.empty((n, self.topk_k), dtype=np.int32)
+        val = np.empty((n, self.topk_k), dtype=np.float32)
+        mx = np.zeros(max(n, 1), dtype=np.float64)
+        rc = self.lib.orc_topk(ctypes.byref(self.s),
                                None if rows_arr is None else rows_arr.ctypes.data, n,
-                               idx.ctypes.data, val.ctypes.data)
-        del keep
+                               idx.ctypes.data, val.ctypes.data, mx.ctypes.data)
         if check and rc not in (ORC_OK,):
             raise RuntimeError(f"oracle orc_topk returned {rc}")
+        if with_maxabs:
+            return idx, val, rc, mx[:n]
         return idx, val, rc
 
-    def scores(self, pb, row: int) -> np.ndarray:
-        """Exact (fp64) scores I[row, j] over the row's key window."""
-        s, keep = self._marshal(pb)
-        hi = ctypes.c_int64(0)
-        b = ctypes.c_int32(0)
-        i = ctypes.c_int32(0)
-        rc = self.lib.orc_row_info(ctypes.byref(s), row, ctypes.byref(hi), ctypes.byref(b),
-                                   ctypes.byref(i))
+    def score_at(self, row: int, j: int) -> float:
+        """Exact (fp64) score of one (row, key) pair inside the row's window."""
+        out = ctypes.c_double(0.0)
+        rc = self.lib.orc_score_at(ctypes.byref(self.s), int(row), int(j), ctypes.byref(out))
         if rc:
-            raise RuntimeError(f"oracle orc_row_info returned {rc}")
-        out = np.empty(max(hi.value, 1), dtype=np.float64)
-        rc = self.lib.orc_scores(ctypes.byref(s), row, out.ctypes.data, ctypes.byref(hi))
-        del keep
-        if rc:
-            raise RuntimeError(f"oracle orc_scores returned {rc}")
-        return out[: hi.value]
+            raise RuntimeError(f"oracle orc_score_at({row}, {j}) returned {rc}")
+        return out.value
 
-    def row_info(self, pb, row: int):
+    def row_info(self, row: int):
         """(window length, batch, position in batch) of a query row."""
-        s, keep = self._marshal(pb)
         hi = ctypes.c_int64(0)
         b = ctypes.c_int32(0)
         i = ctypes.c_int32(0)
-        rc = self.lib.orc_row_info(ctypes.byref(s), row, ctypes.byref(hi), ctypes.byref(b),
-                                   ctypes.byref(i))
-        del keep
+        rc = self.lib.orc_row_info(ctypes.byref(self.s), int(row), ctypes.byref(hi),
+                                   ctypes.byref(b), ctypes.byref(i))
         if rc:
             raise RuntimeError(f"oracle orc_row_info returned {rc}")
         return hi.value, b.value, i.value
+
+    def scores(self, row: int) -> np.ndarray:
+        """Exact (fp64) scores I[row, j] over the row's key window."""
+        hi0, _b, _i = self.row_info(row)
+        out = np.empty(max(hi0, 1), dtype=np.float64)
+        hi = ctypes.c_int64(0)
+        rc = self.lib.orc_scores(ctypes.byref(self.s), int(row), out.ctypes.data,
+                                 ctypes.byref(hi))
+        if rc:
+            raise RuntimeError(f"oracle orc_scores returned {rc}")
+        return out[: hi.value]
 
 
 _DEFAULT: Oracle | None = None

@@ -1,0 +1,321 @@
+// Host side of the C ABI declared in include/li.h: argument validation, schedule choice,
+// workspace sizing and the launch sequence. Mirrors the pages' two-phase convention
+// (aclnnLightningIndexerV2: a first call validates the arguments and sizes the workspace, a
+// second call runs on a stream) and their metadata-then-indexer order (lightning_indexer,
+// "Prototype").
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "li_internal.cuh"
+
+namespace li {
+cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
+                            float *scores, int64_t ld, cudaStream_t st, bool *launched);
+}
+
+namespace {
+
+thread_local std::string g_err;
+
+li_status fail(li_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+li_status ok() {
+    g_err.clear();
+    return LI_OK;
+}
+
+int sm_count() {
+    static int cached = 0;
+    if (cached) return cached;
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) {
+        cached = n;
+        return n;
+    }
+    (void)cudaGetLastError();
+    return 148;
+}
+
+cudaEvent_t g_stage_events[6] = {};
+bool g_stage_events_on = false;
+
+void stage_mark(int i, cudaStream_t st) {
+    if (g_stage_events_on && g_stage_events[i]) cudaEventRecord(g_stage_events[i], st);
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Which score kernel runs: the tensor-core kernel unless LI_SCORE_KERNEL=simple selects the
+// CUDA-core one (a debugging switch; both write the same score rows).
+bool use_simple_kernel() {
+    const char *e = std::getenv("LI_SCORE_KERNEL");
+    return e && std::strcmp(e, "simple") == 0;
+}
+
+li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
+    if (!a) return fail(LI_ERR_INVALID_ARG, "args is NULL");
+    if (a->num_heads_q < 1 || a->num_heads_q > li::kMaxHeads)
+        return fail(LI_ERR_INVALID_ARG, "num_heads_q=%d outside [1, 64]", a->num_heads_q);
+    if (a->num_heads_k != 1)
+        return fail(LI_ERR_INVALID_ARG, "num_heads_k=%d, only 1 key head is supported",
+                    a->num_heads_k);
+    if (a->head_dim != li::kHeadDim)
+        return fail(LI_ERR_INVALID_ARG, "head_dim=%d, only 128 is supported", a->head_dim);
+    if (a->topk < 1 || a->topk > li::kMaxTopk)
+        return fail(LI_ERR_INVALID_ARG, "topk=%d outside [1, 8192]", a->topk);
+    if (a->mask_mode != 0 && a->mask_mode != 3)
+        return fail(LI_ERR_INVALID_ARG, "mask_mode=%d, must be 0 or 3", a->mask_mode);
+    if (a->layout_q != LI_LAYOUT_BSND && a->layout_q != LI_LAYOUT_TND)
+        return fail(LI_ERR_INVALID_ARG, "layout_q=%d, must be BSND or TND", a->layout_q);
+    if (a->layout_k != LI_LAYOUT_BSND && a->layout_k != LI_LAYOUT_TND &&
+        a->layout_k != LI_LAYOUT_PA_BSND)
+        return fail(LI_ERR_INVALID_ARG, "layout_k=%d, must be BSND, TND or PA_BSND", a->layout_k);
+    if (a->dtype_qk != LI_DTYPE_BF16 || a->dtype_w != LI_DTYPE_BF16)
+        return fail(LI_ERR_UNSUPPORTED, "only bf16 q, k and w are supported");
+    if (a->return_value != 0 && a->return_value != 1)
+        return fail(LI_ERR_INVALID_ARG, "return_value=%d, must be 0 or 1", a->return_value);
+    if (a->batch < 0) return fail(LI_ERR_INVALID_ARG, "batch=%d < 0", a->batch);
+    if (a->q_len < 0) return fail(LI_ERR_INVALID_ARG, "q_len=%d < 0", a->q_len);
+    if (a->layout_k != LI_LAYOUT_PA_BSND && a->k_len < 0)
+        return fail(LI_ERR_INVALID_ARG, "k_len=%d < 0", a->k_len);
+    if (a->max_seqlen_k < 0) return fail(LI_ERR_INVALID_ARG, "max_seqlen_k=%d < 0", a->max_seqlen_k);
+    if (a->max_seqlen_q < 0) return fail(LI_ERR_INVALID_ARG, "max_seqlen_q=%d < 0", a->max_seqlen_q);
+    if (!a->q || !a->k || !a->w) return fail(LI_ERR_INVALID_ARG, "q, k and w are required");
+    if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->w, 2))
+        return fail(LI_ERR_INVALID_ARG, "q and k must be 16-byte aligned, w 2-byte aligned");
+    if (a->layout_q == LI_LAYOUT_TND && !a->cu_seqlens_q)
+        return fail(LI_ERR_INVALID_ARG, "layout_q TND requires cu_seqlens_q");
+    if (a->layout_k == LI_LAYOUT_TND && !a->cu_seqlens_k)
+        return fail(LI_ERR_INVALID_ARG, "layout_k TND requires cu_seqlens_k");
+    if (a->layout_q == LI_LAYOUT_BSND && a->cu_seqlens_q)
+        return fail(LI_ERR_INVALID_ARG, "cu_seqlens_q is only for layout_q TND");
+    if (a->layout_k != LI_LAYOUT_TND && a->cu_seqlens_k)
+        return fail(LI_ERR_INVALID_ARG, "cu_seqlens_k is only for layout_k TND");
+    if (a->layout_k == LI_LAYOUT_PA_BSND) {
+        if (!a->seqused_k) return fail(LI_ERR_INVALID_ARG, "layout_k PA_BSND requires seqused_k");
+        if (!a->block_table) return fail(LI_ERR_INVALID_ARG, "layout_k PA_BSND requires block_table");
+        if (a->block_size < 1 || a->block_size > 1024)
+            return fail(LI_ERR_INVALID_ARG, "block_size=%d outside [1, 1024]", a->block_size);
+        if (a->num_blocks < 1) return fail(LI_ERR_INVALID_ARG, "num_blocks=%d < 1", a->num_blocks);
+        if (a->block_table_stride < 1)
+            return fail(LI_ERR_INVALID_ARG, "block_table_stride=%lld < 1",
+                        (long long)a->block_table_stride);
+        // 32-byte block alignment (lightning_indexer, Constraints) holds for any block size:
+        // one key is 128 bf16 = 256 bytes.
+    } else if (a->block_table) {
+        return fail(LI_ERR_INVALID_ARG, "block_table is only for layout_k PA_BSND");
+    }
+    if (a->layout_q == LI_LAYOUT_BSND && a->max_seqlen_q != 0 && a->max_seqlen_q != a->q_len)
+        return fail(LI_ERR_INVALID_ARG, "BSND: max_seqlen_q=%d must equal S1=%d (or be 0)",
+                    a->max_seqlen_q, a->q_len);
+    const int64_t rows = a->layout_q == LI_LAYOUT_TND ? (int64_t)a->q_len
+                                                     : (int64_t)a->batch * a->q_len;
+    if (rows > INT32_MAX) return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 query rows");
+
+    li::Problem &P = *p;
+    std::memset(&P, 0, sizeof P);
+    P.q = static_cast<const uint16_t *>(a->q);
+    P.k = static_cast<const uint16_t *>(a->k);
+    P.w = static_cast<const uint16_t *>(a->w);
+    P.cu_seqlens_q = a->cu_seqlens_q;
+    P.cu_seqlens_k = a->cu_seqlens_k;
+    P.seqused_q = a->seqused_q;
+    P.seqused_k = a->seqused_k;
+    P.block_table = a->block_table;
+    P.output_idx_offset = a->output_idx_offset;
+    P.bt_stride = a->block_table_stride;
+    P.batch = a->batch;
+    P.q_len = a->q_len;
+    P.k_len = a->layout_k == LI_LAYOUT_PA_BSND ? 0 : a->k_len;
+    P.max_seqlen_q = a->layout_q == LI_LAYOUT_BSND ? a->q_len : a->max_seqlen_q;
+    int32_t mk = a->max_seqlen_k;
+    if (a->layout_k == LI_LAYOUT_BSND) {
+        if (mk == 0) mk = a->k_len;
+        if (mk > a->k_len)
+            return fail(LI_ERR_INVALID_ARG, "BSND: max_seqlen_k=%d > S2=%d", mk, a->k_len);
+    }
+    P.max_seqlen_k = mk;
+    P.num_blocks = a->num_blocks;
+    P.block_size = a->layout_k == LI_LAYOUT_PA_BSND ? a->block_size : 0;
+    P.n_heads = a->num_heads_q;
+    P.topk = a->topk;
+    P.layout_q = a->layout_q;
+    P.layout_k = a->layout_k;
+    P.mask_mode = a->mask_mode;
+    P.return_value = a->return_value;
+    P.rows = (int32_t)rows;
+
+    // Schedule: query blocks of tq rows (all N1 heads of tq rows fill one 256-column MMA tile),
+    // split along the keys when there are too few blocks to fill the GPU.
+    li::Schedule &S = *s;
+    S.tq = li::kMaxHeads * 4 / P.n_heads;           // 256 / N1
+    if (S.tq > 128) S.tq = 128;
+    if (S.tq < 1) S.tq = 1;
+    int64_t qblocks = (int64_t)P.batch * ((P.q_len + S.tq - 1) / S.tq);
+    if (P.layout_q == LI_LAYOUT_TND) {
+        qblocks = (rows + S.tq - 1) / S.tq + P.batch;
+        if (qblocks > rows) qblocks = rows;
+    }
+    S.kc = 0;
+    const int64_t target = 4LL * sm_count();
+    if (qblocks < 2LL * sm_count() && P.max_seqlen_k >= 2048) {
+        int64_t kc = ((int64_t)P.max_seqlen_k * (qblocks > 0 ? qblocks : 1) + target - 1) / target;
+        kc = (kc + li::kKeyTile - 1) / li::kKeyTile * li::kKeyTile;
+        if (kc < 1024) kc = 1024;
+        if (kc < P.max_seqlen_k) S.kc = (int)kc;
+    }
+    const int64_t splits = S.kc > 0 ? ((int64_t)P.max_seqlen_k + S.kc - 1) / S.kc : 1;
+    const int64_t max_items = qblocks * splits;
+    if (max_items > INT32_MAX / 2) return fail(LI_ERR_UNSUPPORTED, "schedule too large");
+    S.max_items = (int)(max_items > 0 ? max_items : 0);
+    return LI_OK;
+}
+
+size_t scores_ld(const li::Problem &p) {
+    const size_t mk = p.max_seqlen_k > 0 ? (size_t)p.max_seqlen_k : 1;
+    return li::align_up(mk, 4);
+}
+
+size_t indexer_ws_bytes(const li::Problem &p, const li::Schedule &s) {
+    return sizeof(li::WsHeader) + li::meta_bytes(p.batch, s.max_items) +
+           (size_t)p.rows * scores_ld(p) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+li_status li_metadata_workspace_size(const li_args *args, size_t *bytes) {
+    li::Problem p;
+    li::Schedule s;
+    li_status st = validate(args, &p, &s);
+    if (st != LI_OK) return st;
+    if (!bytes) return fail(LI_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = li::meta_bytes(p.batch, s.max_items);
+    return ok();
+}
+
+li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *stream) {
+    li::Problem p;
+    li::Schedule s;
+    li_status st = validate(args, &p, &s);
+    if (st != LI_OK) return st;
+    if (!metadata || !aligned(metadata, 256))
+        return fail(LI_ERR_WORKSPACE, "metadata must be a 256-byte aligned device buffer");
+    const size_t need = li::meta_bytes(p.batch, s.max_items);
+    if (bytes < need)
+        return fail(LI_ERR_WORKSPACE, "metadata buffer of %zu bytes, %zu needed", bytes, need);
+    cudaError_t e = li::launch_metadata(p, s, metadata, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "metadata launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+li_status li_indexer_workspace_size(const li_args *args, size_t *bytes) {
+    li::Problem p;
+    li::Schedule s;
+    li_status st = validate(args, &p, &s);
+    if (st != LI_OK) return st;
+    if (!bytes) return fail(LI_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = indexer_ws_bytes(p, s);
+    return ok();
+}
+
+li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
+                     size_t workspace_bytes, int32_t *sparse_indices, float *sparse_values,
+                     void *stream) {
+    li::Problem p;
+    li::Schedule s;
+    li_status st = validate(args, &p, &s);
+    if (st != LI_OK) return st;
+    if (!sparse_indices || !aligned(sparse_indices, 4))
+        return fail(LI_ERR_INVALID_ARG, "sparse_indices must be a 4-byte aligned device buffer");
+    if (p.return_value && (!sparse_values || !aligned(sparse_values, 4)))
+        return fail(LI_ERR_INVALID_ARG, "return_value=1 requires sparse_values");
+    if (metadata && !aligned(metadata, 256))
+        return fail(LI_ERR_WORKSPACE, "metadata must be 256-byte aligned");
+    if (!workspace || !aligned(workspace, 256))
+        return fail(LI_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+    const size_t need = indexer_ws_bytes(p, s);
+    if (workspace_bytes < need)
+        return fail(LI_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    auto *ws = static_cast<li::WsHeader *>(workspace);
+    char *base = static_cast<char *>(workspace);
+    void *inline_meta = base + sizeof(li::WsHeader);
+    float *scores = reinterpret_cast<float *>(base + sizeof(li::WsHeader) +
+                                              li::meta_bytes(p.batch, s.max_items));
+    const int64_t ld = (int64_t)scores_ld(p);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(li::WsHeader), cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "workspace clear: %s", cudaGetErrorString(e));
+    if (p.rows == 0) return ok();
+    const void *meta = metadata;
+    if (!meta) {
+        stage_mark(0, cs);
+        e = li::launch_metadata(p, s, inline_meta, cs);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "metadata launch: %s", cudaGetErrorString(e));
+        stage_mark(1, cs);
+        meta = inline_meta;
+    }
+    bool launched = false;
+    stage_mark(2, cs);
+    if (!use_simple_kernel()) {
+        e = li::launch_score_tc(p, s, meta, ws, scores, ld, cs, &launched);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
+    }
+    if (!launched) {
+        e = li::launch_score_simple(p, s, meta, ws, scores, ld, cs);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
+    }
+    stage_mark(3, cs);
+    stage_mark(4, cs);
+    e = li::launch_select(p, s, meta, ws, scores, ld, sparse_indices,
+                          p.return_value ? sparse_values : nullptr, cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+    stage_mark(5, cs);
+    return ok();
+}
+
+li_status li_check_status(const void *workspace, void *stream, uint32_t *device_bits) {
+    if (!workspace) return fail(LI_ERR_INVALID_ARG, "workspace is NULL");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    uint32_t bits = 0;
+    e = cudaMemcpy(&bits, workspace, sizeof bits, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (device_bits) *device_bits = bits;
+    if (bits & LI_DEVERR_TIMEOUT) return fail(LI_ERR_DEVICE_TIMEOUT, "device wait timed out (bits 0x%x)", bits);
+    if (bits) return fail(LI_ERR_DEVICE_DATA, "invalid device data (bits 0x%x)", bits);
+    return ok();
+}
+
+li_status li_set_stage_events(void *const *events, int32_t n_events) {
+    if (n_events == 0) {
+        g_stage_events_on = false;
+        for (auto &ev : g_stage_events) ev = nullptr;
+        return ok();
+    }
+    if (n_events != 6 || !events) return fail(LI_ERR_INVALID_ARG, "li_set_stage_events wants 0 or 6 events");
+    for (int i = 0; i < 6; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_stage_events_on = true;
+    return ok();
+}
+
+const char *li_last_error_string(void) { return g_err.c_str(); }
+
+int32_t li_abi_version(void) { return LI_ABI_VERSION; }
+
+}  // extern "C"

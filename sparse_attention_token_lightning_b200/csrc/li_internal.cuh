@@ -1,0 +1,171 @@
+// Internal definitions shared by the library's kernels and host code (not part of the ABI).
+//
+// Device memory layout of the two caller-owned buffers:
+//
+//   metadata (li_metadata):   MetaHeader | BatchInfo[B] | WorkItem[max_items]
+//   workspace (li_indexer):   WsHeader (256 B) | inline metadata | fp32 scores [rows][ld]
+//
+// The fp32 score rows hold I[t, j] for every key j of row t's window; the selection kernel reads
+// them back. Rows are indexed by the global query row (B*S1 rows for BSND, T1 rows for TND).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "li.h"
+
+namespace li {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxHeads = 64;
+constexpr int kMaxTopk = 8192;
+constexpr int kKeyTile = 128;          // keys per tile of the score kernels
+constexpr uint32_t kMetaMagic = 0x4c494d31u;   // "LIM1"
+
+// Device status bit used when metadata does not match the call it is used with.
+constexpr uint32_t kDevErrMetadata = 0x10u;
+
+struct MetaHeader {
+    uint32_t magic;
+    uint32_t status;       // LI_DEVERR_* bits found while building the schedule
+    int32_t n_items;       // items written
+    int32_t max_items;     // capacity
+    int32_t batch;
+    int32_t tq;            // query rows per work item
+    int32_t kc;            // keys per work item (key-range split), 0 = whole window
+    uint32_t signature;    // hash of the scalar arguments the schedule was built for
+    int32_t pad[8];
+};
+static_assert(sizeof(MetaHeader) == 64, "MetaHeader size");
+
+struct BatchInfo {
+    int32_t L1;            // query rows allocated to the batch
+    int32_t L1u;           // query rows in use (seqused_q), <= L1
+    int32_t L2;            // keys of the batch
+    int32_t q_row0;        // global query row of the batch's row 0
+    int32_t k_row0;        // BSND: b*S2, TND: cu_seqlens_k[b], PA: 0
+    int32_t pad[3];
+};
+static_assert(sizeof(BatchInfo) == 32, "BatchInfo size");
+
+struct WorkItem {
+    int32_t b;             // batch
+    int32_t q0;            // first query row (position inside the batch)
+    int32_t nq;            // query rows (<= tq)
+    int32_t j0;            // first key of the item's range
+    int32_t j1;            // one past the last key any of its rows needs
+    int32_t cost;          // key tiles, for ordering
+    int32_t pad[2];
+};
+static_assert(sizeof(WorkItem) == 32, "WorkItem size");
+
+struct WsHeader {
+    uint32_t status;       // LI_DEVERR_* bits of the last li_indexer on this workspace
+    int32_t sched_next;    // dynamic scheduler ticket counter
+    int32_t pad[62];
+};
+static_assert(sizeof(WsHeader) == 256, "WsHeader size");
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline size_t meta_bytes(int batch, int max_items) {
+    return align_up(sizeof(MetaHeader) + sizeof(BatchInfo) * (size_t)batch +
+                    sizeof(WorkItem) * (size_t)max_items, 256);
+}
+
+__host__ __device__ inline const BatchInfo *meta_batches(const void *meta) {
+    return reinterpret_cast<const BatchInfo *>(static_cast<const char *>(meta) + sizeof(MetaHeader));
+}
+__host__ __device__ inline const WorkItem *meta_items(const void *meta, int batch) {
+    return reinterpret_cast<const WorkItem *>(static_cast<const char *>(meta) + sizeof(MetaHeader) +
+                                              sizeof(BatchInfo) * (size_t)batch);
+}
+
+// Window of row i of a batch: keys [0, hi). mask 0: hi = L2. mask 3 (right-down causal):
+// hi = min(L2, i + L2 - L1u + 1), clipped at 0. Rows past L1u have no window.
+__host__ __device__ inline int32_t window_hi(int mask_mode, int32_t i, int32_t L1u, int32_t L2) {
+    if (i >= L1u || L2 <= 0) return 0;
+    if (mask_mode != 3) return L2;
+    int64_t lim = (int64_t)i + L2 - L1u + 1;
+    if (lim > L2) lim = L2;
+    return lim < 0 ? 0 : (int32_t)lim;
+}
+
+// Scalars every kernel needs, copied by value into kernel parameters.
+struct Problem {
+    const uint16_t *q, *k, *w;            // bf16 bit patterns
+    const int32_t *cu_seqlens_q, *cu_seqlens_k, *seqused_q, *seqused_k;
+    const int32_t *block_table;
+    const int32_t *output_idx_offset;
+    int64_t bt_stride;
+    int32_t batch, q_len, k_len, max_seqlen_q, max_seqlen_k;
+    int32_t num_blocks, block_size;
+    int32_t n_heads, topk;
+    int32_t layout_q, layout_k, mask_mode;
+    int32_t return_value;
+    int32_t rows;                          // B*S1 or T1
+};
+
+// Signature of the scalar arguments a schedule depends on.
+__host__ __device__ inline uint32_t problem_signature(const Problem &p, int tq, int kc) {
+    uint32_t h = 2166136261u;
+    auto mix = [&](uint32_t v) { h = (h ^ v) * 16777619u; };
+    mix((uint32_t)p.batch); mix((uint32_t)p.q_len); mix((uint32_t)p.k_len);
+    mix((uint32_t)p.max_seqlen_q); mix((uint32_t)p.max_seqlen_k); mix((uint32_t)p.n_heads);
+    mix((uint32_t)p.layout_q); mix((uint32_t)p.layout_k); mix((uint32_t)p.mask_mode);
+    mix((uint32_t)p.block_size); mix((uint32_t)tq); mix((uint32_t)kc);
+    return h;
+}
+
+// Schedule parameters chosen on the host for a problem (shared by li_metadata and li_indexer).
+struct Schedule {
+    int tq;          // query rows per item
+    int kc;          // key-range split (0 = none)
+    int max_items;   // capacity of the item list
+};
+
+// Device-side: batch of a global query row (TND: binary search in cu_seqlens_q).
+__device__ inline int32_t row_batch(const Problem &p, int32_t r, int32_t *pos) {
+    if (p.layout_q != LI_LAYOUT_TND) {
+        int32_t b = r / p.q_len;
+        *pos = r - b * p.q_len;
+        return b;
+    }
+    // largest b with cu[b] <= r and r < cu[b+1]; rows past cu[B] have no batch
+    int32_t lo = 0, hi = p.batch;   // search in cu[0..B]
+    if (p.batch <= 0 || r < p.cu_seqlens_q[0] || r >= p.cu_seqlens_q[p.batch]) { *pos = 0; return -1; }
+    while (hi - lo > 1) {
+        int32_t mid = (lo + hi) >> 1;
+        if (p.cu_seqlens_q[mid] <= r) lo = mid; else hi = mid;
+    }
+    *pos = r - p.cu_seqlens_q[lo];
+    return lo;
+}
+
+// Pointer to logical key j of batch b (paged: through the block table). Returns nullptr when
+// the block table entry is out of range.
+__device__ inline const uint16_t *key_ptr(const Problem &p, const BatchInfo &bi, int32_t b, int32_t j) {
+    if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        int32_t blk = p.block_table[(int64_t)b * p.bt_stride + j / p.block_size];
+        if (blk < 0 || blk >= p.num_blocks) return nullptr;
+        return p.k + ((int64_t)blk * p.block_size + j % p.block_size) * kHeadDim;
+    }
+    return p.k + ((int64_t)bi.k_row0 + j) * kHeadDim;
+}
+
+__device__ inline float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ inline float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ inline void set_status(uint32_t *status, uint32_t bits) {
+    if (bits) atomicOr(status, bits);
+}
+
+// ---- launchers implemented in the .cu files --------------------------------------------------
+cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st);
+cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
+                                WsHeader *ws, float *scores, int64_t ld, cudaStream_t st);
+cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
+                          const float *scores, int64_t ld, int32_t *out_idx, float *out_val,
+                          cudaStream_t st);
+
+}  // namespace li

@@ -1,0 +1,196 @@
+// Schedule builder (li_metadata). Replaces the pages' per-AI-core task list (lightning_indexer,
+// "Function": lightning_indexer_metadata produces per-core tasks of batch, head and Q/K block
+// ranges) with a list of work items for persistent CTAs:
+//
+//   item = (batch b, query rows [q0, q0+nq), key range [j0, j1))
+//
+// ordered by cost (key tiles) descending, so CTAs that pull items in order finish together.
+// One CTA builds it: per-batch lengths first (validating the device-resident cu_seqlens, seqused
+// and offsets), then a counting sort of the items by cost: a histogram pass, a descending scan of
+// the histogram, and a placement pass. The order of equal-cost items may vary between runs; every
+// item writes its own rows, so results do not depend on it.
+#include "li_internal.cuh"
+
+namespace li {
+namespace {
+
+constexpr int kMetaThreads = 1024;
+constexpr int kCostBins = 1024;
+
+struct MetaParams {
+    Problem p;
+    Schedule s;
+    void *meta;
+};
+
+__device__ inline int item_cost(int32_t j0, int32_t j1) {
+    int c = (j1 - j0 + kKeyTile - 1) / kKeyTile;
+    return c < kCostBins ? c : kCostBins - 1;
+}
+
+// Enumerate the items of batch b for the lanes of one warp; f(item) is called once per item.
+template <class F>
+__device__ inline void for_items_of_batch(const Problem &p, const Schedule &s, int32_t b,
+                                          const BatchInfo &bi, int lane, F &&f) {
+    const int32_t nqb = (bi.L1u + s.tq - 1) / s.tq;
+    for (int32_t qb = lane; qb < nqb; qb += 32) {
+        WorkItem it;
+        it.b = b;
+        it.q0 = qb * s.tq;
+        it.nq = min(s.tq, bi.L1u - it.q0);
+        // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
+        const int32_t jend = window_hi(p.mask_mode, it.q0 + it.nq - 1, bi.L1u, bi.L2);
+        if (jend <= 0) continue;
+        const int32_t kc = s.kc > 0 ? s.kc : jend;
+        for (int32_t j0 = 0; j0 < jend; j0 += kc) {
+            it.j0 = j0;
+            it.j1 = min(jend, j0 + kc);
+            it.cost = item_cost(it.j0, it.j1);
+            it.pad[0] = it.pad[1] = 0;
+            f(it);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
+    const Problem &p = mp.p;
+    const Schedule &s = mp.s;
+    MetaHeader *hdr = reinterpret_cast<MetaHeader *>(mp.meta);
+    BatchInfo *binfo = reinterpret_cast<BatchInfo *>(static_cast<char *>(mp.meta) + sizeof(MetaHeader));
+    WorkItem *items = reinterpret_cast<WorkItem *>(binfo + p.batch);
+
+    __shared__ int32_t hist[kCostBins];
+    __shared__ uint32_t s_status;
+    __shared__ int32_t s_total;
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kCostBins; i += kMetaThreads) hist[i] = 0;
+    if (tid == 0) { s_status = 0; s_total = 0; }
+    __syncthreads();
+
+    // ---- pass 0: per-batch lengths ------------------------------------------------------------
+    for (int32_t b = tid; b < p.batch; b += kMetaThreads) {
+        uint32_t err = 0;
+        BatchInfo bi;
+        int64_t L1, q0, L2, k0;
+        if (p.layout_q == LI_LAYOUT_TND) {
+            const int64_t c0 = p.cu_seqlens_q[b], c1 = p.cu_seqlens_q[b + 1];
+            if (c0 < 0 || c1 < c0 || c1 > p.q_len) { err |= LI_DEVERR_LENGTHS; }
+            L1 = (c1 >= c0 && c0 >= 0 && c1 <= p.q_len) ? c1 - c0 : 0;
+            q0 = c0 < 0 ? 0 : c0;
+        } else {
+            L1 = p.q_len;
+            q0 = (int64_t)b * p.q_len;
+        }
+        int64_t L1u = L1;
+        if (p.seqused_q) {
+            const int64_t u = p.seqused_q[b];
+            if (u < 0 || u > L1) err |= LI_DEVERR_LENGTHS;
+            L1u = u < 0 ? 0 : (u > L1 ? L1 : u);
+        }
+        if (p.layout_k == LI_LAYOUT_TND) {
+            const int64_t c0 = p.cu_seqlens_k[b], c1 = p.cu_seqlens_k[b + 1];
+            if (c0 < 0 || c1 < c0 || c1 > p.k_len) { err |= LI_DEVERR_LENGTHS; }
+            L2 = (c1 >= c0 && c0 >= 0 && c1 <= p.k_len) ? c1 - c0 : 0;
+            k0 = c0 < 0 ? 0 : c0;
+        } else if (p.layout_k == LI_LAYOUT_PA_BSND) {
+            const int64_t u = p.seqused_k[b];
+            const int64_t cap = p.bt_stride * (int64_t)p.block_size;
+            if (u < 0 || u > cap) err |= LI_DEVERR_LENGTHS;
+            L2 = u < 0 ? 0 : (u > cap ? cap : u);
+            k0 = 0;
+        } else {
+            L2 = p.k_len;
+            k0 = (int64_t)b * p.k_len;
+        }
+        if (p.seqused_k && p.layout_k != LI_LAYOUT_PA_BSND) {
+            const int64_t u = p.seqused_k[b];
+            if (u < 0 || u > L2) err |= LI_DEVERR_LENGTHS;
+            L2 = u < 0 ? 0 : (u < L2 ? u : L2);
+        }
+        if (L2 > p.max_seqlen_k) { err |= LI_DEVERR_LENGTHS; L2 = p.max_seqlen_k; }
+        if (p.output_idx_offset) {
+            const int64_t off = p.output_idx_offset[b];
+            if (off < 0 || off + (L2 > 0 ? L2 - 1 : 0) > (int64_t)INT32_MAX) err |= LI_DEVERR_OFFSET;
+        }
+        bi.L1 = (int32_t)L1;
+        bi.L1u = (int32_t)L1u;
+        bi.L2 = (int32_t)L2;
+        bi.q_row0 = (int32_t)q0;
+        bi.k_row0 = (int32_t)k0;
+        bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
+        binfo[b] = bi;
+        if (err) atomicOr(&s_status, err);
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    constexpr int kWarps = kMetaThreads / 32;
+
+    // ---- pass 1: cost histogram ---------------------------------------------------------------
+    for (int32_t b = warp; b < p.batch; b += kWarps) {
+        const BatchInfo bi = binfo[b];
+        for_items_of_batch(p, s, b, bi, lane, [&](const WorkItem &it) {
+            atomicAdd(&hist[it.cost], 1);
+            atomicAdd(&s_total, 1);
+        });
+    }
+    __syncthreads();
+
+    // ---- descending exclusive scan of the histogram: cursor[c] = items with cost > c ----------
+    if (warp == 0) {
+        // each lane owns kCostBins/32 consecutive bins; highest bins first
+        constexpr int per = kCostBins / 32;
+        int32_t local = 0;
+        for (int i = 0; i < per; ++i) local += hist[lane * per + i];
+        // suffix sum over lanes above this one
+        int32_t incl = local;
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += v;
+        }
+        int32_t above = incl - local;
+        for (int i = per - 1; i >= 0; --i) {
+            const int bin = lane * per + i;
+            const int32_t c = hist[bin];
+            hist[bin] = above;
+            above += c;
+        }
+    }
+    __syncthreads();
+
+    // ---- pass 2: placement --------------------------------------------------------------------
+    const int32_t cap = s.max_items;
+    for (int32_t b = warp; b < p.batch; b += kWarps) {
+        const BatchInfo bi = binfo[b];
+        for_items_of_batch(p, s, b, bi, lane, [&](const WorkItem &it) {
+            const int32_t slot = atomicAdd(&hist[it.cost], 1);
+            if (slot < cap) items[slot] = it;
+        });
+    }
+    __syncthreads();
+
+    if (tid == 0) {
+        uint32_t st = s_status;
+        int32_t n = s_total;
+        if (n > cap) { st |= LI_DEVERR_LENGTHS; n = cap; }
+        hdr->magic = kMetaMagic;
+        hdr->status = st;
+        hdr->n_items = n;
+        hdr->max_items = cap;
+        hdr->batch = p.batch;
+        hdr->tq = s.tq;
+        hdr->kc = s.kc;
+        hdr->signature = problem_signature(p, s.tq, s.kc);
+        for (int i = 0; i < 8; ++i) hdr->pad[i] = 0;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st) {
+    MetaParams mp{p, s, meta};
+    metadata_kernel<<<1, kMetaThreads, 0, st>>>(mp);
+    return cudaGetLastError();
+}
+
+}  // namespace li

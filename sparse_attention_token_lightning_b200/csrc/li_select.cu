@@ -1,0 +1,356 @@
+// Per-row top-k selection from the fp32 score rows (second pass of the two-pass design).
+//
+// For query row t with window [0, n): keep the m = min(topk, n) keys with the largest I[t, j],
+// ordered by I descending and, on equal scores, by lower key index first; write their indices
+// (+ output_idx_offset[b]) and scores, then pad with -1 / -inf up to topk (lightning_indexer and
+// aclnnLightningIndexerV2, constraints on the invalid part; torch_npu.npu_sparse_lightning_
+// indexer_grad_kl_loss, sparse_indices are sorted). Rows past seqused_q, rows of no batch and
+// rows with an empty causal window are all padding.
+//
+// Method, one CTA per row:
+//   1. Scores become order-preserving 32-bit keys (-0 maps to +0, so both zeros tie).
+//   2. Radix select, most significant byte first: four histogram passes narrow a prefix until
+//      the m-th largest key is known, or until every key sharing the prefix is taken.
+//   3. Gather in index order with block-wide ballot scans: keys above the threshold first, then
+//      the lowest-index keys equal to it. This fixes the tie rule.
+//   4. Stable LSD radix sort (8-bit digits, warp match for in-round ranks) of the m selected keys
+//      descending; stability keeps equal scores in index order. Passes whose digit is constant
+//      are skipped.
+// Rows of up to `row_cap` keys are staged in shared memory once; longer rows are re-read from
+// global memory (L2) in each pass.
+#include "li_internal.cuh"
+
+namespace li {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kDigits = 256;
+
+struct Params {
+    Problem p;
+    const void *meta;
+    WsHeader *ws;
+    const float *scores;
+    int64_t ld;
+    int32_t *out_idx;
+    float *out_val;
+    int32_t row_cap;
+    uint32_t signature;
+};
+
+__device__ __forceinline__ uint32_t score_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+struct Smem {
+    int32_t hist[kDigits];
+    int32_t wsum[2][kWarps];
+    int32_t s_digit, s_rem, s_cnt;
+    int32_t s_skip[4];      // one flag per sort pass, so no pass resets a flag still being read
+};
+
+// Block-wide exclusive scan of cnt[0..kWarps*kDigits) in place (512 threads x 8 entries).
+__device__ void block_exclusive_scan_4096(int32_t *cnt, Smem &sm) {
+    constexpr int per = kWarps * kDigits / kThreads;   // 8
+    const int tid = threadIdx.x;
+    int32_t v[per];
+    int32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) { v[i] = cnt[tid * per + i]; local += v[i]; }
+    // warp inclusive scan of local
+    const int lane = tid & 31, warp = tid >> 5;
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) sm.wsum[0][warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t x = lane < kWarps ? sm.wsum[0][lane] : 0;
+        int32_t xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t t = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += t;
+        }
+        if (lane < kWarps) sm.wsum[1][lane] = xi - x;
+    }
+    __syncthreads();
+    int32_t run = sm.wsum[1][warp] + incl - local;
+#pragma unroll
+    for (int i = 0; i < per; ++i) { cnt[tid * per + i] = run; run += v[i]; }
+    __syncthreads();
+}
+
+template <bool kCached>
+__device__ __forceinline__ uint32_t get_key(const uint32_t *rowc, const float *src, int32_t e) {
+    if (kCached) return rowc[e];
+    return score_key(__ldg(src + e));
+}
+
+// Radix select: the m-th largest key of n. Leaves (prefix, mask, need) such that the selected
+// set is {keys with (u & mask) > prefix} plus the first `need` keys (by index) with
+// (u & mask) == prefix.
+template <bool kCached>
+__device__ void radix_select(const uint32_t *rowc, const float *src, int32_t n, int32_t m,
+                             Smem &sm, uint32_t &prefix, uint32_t &mask, int32_t &need) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    prefix = 0u;
+    mask = 0u;
+    int32_t rem = m;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < kDigits; i += kThreads) sm.hist[i] = 0;
+        __syncthreads();
+        for (int32_t e0 = 0; e0 < n; e0 += kThreads) {
+            const int32_t e = e0 + tid;
+            uint32_t d = kDigits;   // no digit
+            if (e < n) {
+                const uint32_t u = get_key<kCached>(rowc, src, e);
+                if ((u & mask) == prefix) d = (u >> shift) & 0xffu;
+            }
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            if (d < kDigits && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], __popc(peers));
+        }
+        __syncthreads();
+        if (tid < 32) {
+            constexpr int per = kDigits / 32;
+            int32_t local = 0;
+#pragma unroll
+            for (int i = 0; i < per; ++i) local += sm.hist[lane * per + i];
+            int32_t incl = local;   // suffix sum over lanes >= this one
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t t = __shfl_down_sync(0xffffffffu, incl, o);
+                if (lane + o < 32) incl += t;
+            }
+            int32_t above = incl - local;
+            for (int i = per - 1; i >= 0; --i) {
+                const int d = lane * per + i;
+                const int32_t c = sm.hist[d];
+                if (above < rem && rem <= above + c) {
+                    sm.s_digit = d;
+                    sm.s_rem = rem - above;
+                    sm.s_cnt = c;
+                }
+                above += c;
+            }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sm.s_digit << shift;
+        mask |= 0xffu << shift;
+        rem = sm.s_rem;
+        const int32_t cnt = sm.s_cnt;
+        __syncthreads();
+        if (cnt == rem) break;   // every key with this prefix is taken
+    }
+    need = rem;
+}
+
+// Gather the selected keys in index order into keyA/idxA[0..m).
+template <bool kCached>
+__device__ void gather(const uint32_t *rowc, const float *src, int32_t n, int32_t m,
+                       uint32_t prefix, uint32_t mask, int32_t need, uint32_t *keyA,
+                       int32_t *idxA, Smem &sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t gt = m - need;
+    int32_t run_gt = 0, run_eq = 0;
+    for (int32_t e0 = 0; e0 < n; e0 += kThreads) {
+        const int32_t e = e0 + tid;
+        uint32_t u = 0;
+        bool is_gt = false, is_eq = false;
+        if (e < n) {
+            u = get_key<kCached>(rowc, src, e);
+            const uint32_t mu = u & mask;
+            is_gt = mu > prefix;
+            is_eq = mu == prefix;
+        }
+        const uint32_t bg = __ballot_sync(0xffffffffu, is_gt);
+        const uint32_t be = __ballot_sync(0xffffffffu, is_eq);
+        if (lane == 0) { sm.wsum[0][warp] = __popc(bg); sm.wsum[1][warp] = __popc(be); }
+        __syncthreads();
+        int32_t pre_g = 0, pre_e = 0, tot_g = 0, tot_e = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int32_t a = sm.wsum[0][w], b = sm.wsum[1][w];
+            if (w < warp) { pre_g += a; pre_e += b; }
+            tot_g += a;
+            tot_e += b;
+        }
+        const uint32_t lt = lanemask_lt();
+        if (is_gt) {
+            const int32_t pos = run_gt + pre_g + __popc(bg & lt);
+            keyA[pos] = u;
+            idxA[pos] = e;
+        } else if (is_eq) {
+            const int32_t r = run_eq + pre_e + __popc(be & lt);
+            if (r < need) {
+                keyA[gt + r] = u;
+                idxA[gt + r] = e;
+            }
+        }
+        run_gt += tot_g;
+        run_eq += tot_e;
+        __syncthreads();
+    }
+}
+
+// Stable LSD radix sort of keyA/idxA[0..m) by key descending. Returns true when the result
+// ended in the B buffers.
+__device__ bool sort_desc(int32_t m, uint32_t *keyA, int32_t *idxA, uint32_t *keyB, int32_t *idxB,
+                          int32_t *cnt, Smem &sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t seg = (m + kWarps - 1) / kWarps;
+    const int32_t s0 = warp * seg, s1 = min(m, s0 + seg);
+    bool inB = false;
+    if (tid < 4) sm.s_skip[tid] = 0;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 8 * pass;
+        uint32_t *ks = inB ? keyB : keyA;
+        int32_t *is = inB ? idxB : idxA;
+        uint32_t *kd = inB ? keyA : keyB;
+        int32_t *id = inB ? idxA : idxB;
+        for (int i = tid; i < kWarps * kDigits; i += kThreads) cnt[i] = 0;
+        __syncthreads();
+        // counts, digit-major: cnt[d * kWarps + w]
+        for (int32_t e0 = s0; e0 < s1; e0 += 32) {
+            const int32_t e = e0 + lane;
+            const uint32_t d = e < s1 ? ((~ks[e]) >> shift) & 0xffu : kDigits;
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            if (d < kDigits && lane == __ffs(peers) - 1) cnt[d * kWarps + warp] += __popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (tid < kDigits) {
+            int32_t tot = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) tot += cnt[tid * kWarps + w];
+            if (tot == m) sm.s_skip[pass] = 1;
+        }
+        __syncthreads();
+        if (sm.s_skip[pass]) continue;   // one digit value for all keys: order unchanged
+        block_exclusive_scan_4096(cnt, sm);
+        for (int32_t e0 = s0; e0 < s1; e0 += 32) {
+            const int32_t e = e0 + lane;
+            const bool valid = e < s1;
+            const uint32_t key = valid ? ks[e] : 0u;
+            const uint32_t d = valid ? ((~key) >> shift) & 0xffu : kDigits;
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            if (valid) {
+                const int32_t base = cnt[d * kWarps + warp];
+                const int32_t dst = base + __popc(peers & lanemask_lt());
+                kd[dst] = key;
+                id[dst] = is[e];
+            }
+            __syncwarp();
+            if (valid && lane == __ffs(peers) - 1) cnt[d * kWarps + warp] += __popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();
+        inB = !inB;
+    }
+    return inB;
+}
+
+__global__ void __launch_bounds__(kThreads) select_kernel(Params sp) {
+    const Problem &p = sp.p;
+    const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(sp.meta);
+    const int tid = threadIdx.x;
+    const bool meta_ok = hdr->magic == kMetaMagic && hdr->signature == sp.signature;
+    if (blockIdx.x == 0 && tid == 0) {
+        set_status(&sp.ws->status, meta_ok ? hdr->status : kDevErrMetadata);
+    }
+
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ Smem sm;
+    const int32_t topk = p.topk;
+    uint32_t *keyA = reinterpret_cast<uint32_t *>(dsm);
+    uint32_t *keyB = keyA + topk;
+    int32_t *idxA = reinterpret_cast<int32_t *>(keyB + topk);
+    int32_t *idxB = idxA + topk;
+    int32_t *cnt = idxB + topk;                                   // kWarps * kDigits
+    uint32_t *rowc = reinterpret_cast<uint32_t *>(cnt + kWarps * kDigits);
+
+    const int32_t r = blockIdx.x;
+    int32_t pos = 0;
+    int32_t b = meta_ok ? row_batch(p, r, &pos) : -1;
+    int32_t n = 0, off = 0;
+    if (b >= 0) {
+        const BatchInfo bi = meta_batches(sp.meta)[b];
+        n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2);
+        if (p.output_idx_offset) off = p.output_idx_offset[b];
+    }
+    const int32_t m = min(n, topk);
+    int32_t *oi = sp.out_idx + (int64_t)r * topk;
+    float *ov = sp.out_val ? sp.out_val + (int64_t)r * topk : nullptr;
+
+    bool inB = false;
+    if (m > 0) {
+        const float *src = sp.scores + (int64_t)r * sp.ld;
+        const bool cached = n <= sp.row_cap;
+        if (cached) {
+            for (int32_t e = tid; e < n; e += kThreads) rowc[e] = score_key(__ldg(src + e));
+            __syncthreads();
+        }
+        uint32_t prefix = 0u, mask = 0u;
+        int32_t need = m;
+        if (m < n) {
+            if (cached) radix_select<true>(rowc, src, n, m, sm, prefix, mask, need);
+            else radix_select<false>(rowc, src, n, m, sm, prefix, mask, need);
+        }
+        if (cached) gather<true>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
+        else gather<false>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
+        __syncthreads();
+        inB = sort_desc(m, keyA, idxA, keyB, idxB, cnt, sm);
+    }
+    const uint32_t *kf = inB ? keyB : keyA;
+    const int32_t *jf = inB ? idxB : idxA;
+    for (int32_t s = tid; s < topk; s += kThreads) {
+        if (s < m) {
+            oi[s] = jf[s] + off;
+            if (ov) ov[s] = key_score(kf[s]);
+        } else {
+            oi[s] = -1;
+            if (ov) ov[s] = -__int_as_float(0x7f800000);
+        }
+    }
+}
+
+}  // namespace
+
+static size_t select_smem_bytes(int topk, int row_cap) {
+    return (size_t)4 * topk * 4 + (size_t)kWarps * kDigits * 4 + (size_t)row_cap * 4;
+}
+
+cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
+                          const float *scores, int64_t ld, int32_t *out_idx, float *out_val,
+                          cudaStream_t st) {
+    if (p.rows <= 0) return cudaSuccess;
+    constexpr int64_t kSmemLimit = 227 * 1024 - (int64_t)sizeof(Smem) - 1024;
+    const int64_t cap = (kSmemLimit - (int64_t)select_smem_bytes(p.topk, 0)) / 4 / 32 * 32;
+    const int64_t want = ((int64_t)(p.max_seqlen_k > 0 ? p.max_seqlen_k : 1) + 31) / 32 * 32;
+    const int32_t row_cap = (int32_t)(want < cap ? want : (cap > 0 ? cap : 0));
+    const size_t smem = select_smem_bytes(p.topk, row_cap);
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    Params sp{p, meta, ws, scores, ld, out_idx, out_val, row_cap,
+              problem_signature(p, s.tq, s.kc)};
+    select_kernel<<<p.rows, kThreads, smem, st>>>(sp);
+    return cudaGetLastError();
+}
+
+}  // namespace li

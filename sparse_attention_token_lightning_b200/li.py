@@ -1,0 +1,221 @@
+"""Thin ctypes binding over ``libli.so`` (C ABI in include/li.h).
+
+Argument marshalling only: every step of the indexer runs in the library's CUDA kernels. The
+functions keep the C names (``li_metadata``, ``li_indexer``, ...). ``indexer()`` is a convenience
+that allocates the outputs and the workspace with torch and calls ``li_indexer`` on the current
+stream. There is no fallback: if the library is missing, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libli.so"
+LAYOUTS = {"BSND": 0, "TND": 1, "PA_BSND": 2}
+STATUS = {0: "LI_OK", 1: "LI_ERR_INVALID_ARG", 2: "LI_ERR_UNSUPPORTED", 3: "LI_ERR_WORKSPACE",
+          4: "LI_ERR_CUDA", 5: "LI_ERR_DEVICE_TIMEOUT", 6: "LI_ERR_DEVICE_DATA"}
+LI_OK = 0
+DEVERR_TIMEOUT, DEVERR_LENGTHS, DEVERR_TABLE, DEVERR_OFFSET, DEVERR_METADATA = 1, 2, 4, 8, 16
+
+
+class LiError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class LiArgs(ctypes.Structure):
+    """Mirror of ``li_args`` (include/li.h)."""
+
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("w", ctypes.c_void_p),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("seqused_q", ctypes.c_void_p), ("seqused_k", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("block_table_stride", ctypes.c_int64),
+        ("output_idx_offset", ctypes.c_void_p),
+        ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("k_len", ctypes.c_int32),
+        ("max_seqlen_q", ctypes.c_int32), ("max_seqlen_k", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("num_heads_q", ctypes.c_int32), ("num_heads_k", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32),
+        ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
+        ("dtype_qk", ctypes.c_int32), ("dtype_w", ctypes.c_int32),
+        ("return_value", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
+           "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
+           "li_abi_version")
+
+
+def lib_path() -> Path:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libli.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not _LIB_PATH.exists():
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m sparse_attention_token_lightning_b200.build`")
+    L = ctypes.CDLL(str(_LIB_PATH))
+    P = ctypes.POINTER(LiArgs)
+    sz = ctypes.POINTER(ctypes.c_size_t)
+    vp = ctypes.c_void_p
+    L.li_metadata_workspace_size.argtypes = [P, sz]
+    L.li_metadata.argtypes = [P, vp, ctypes.c_size_t, vp]
+    L.li_indexer_workspace_size.argtypes = [P, sz]
+    L.li_indexer.argtypes = [P, vp, vp, ctypes.c_size_t, vp, vp, vp]
+    L.li_check_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    for f in ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
+              "li_indexer", "li_check_status"):
+        getattr(L, f).restype = ctypes.c_int
+    L.li_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+    L.li_set_stage_events.restype = ctypes.c_int
+    L.li_last_error_string.argtypes = []
+    L.li_last_error_string.restype = ctypes.c_char_p
+    L.li_abi_version.argtypes = []
+    L.li_abi_version.restype = ctypes.c_int32
+    _lib = L
+    return L
+
+
+def li_last_error_string() -> str:
+    return lib().li_last_error_string().decode()
+
+
+def li_abi_version() -> int:
+    return int(lib().li_abi_version())
+
+
+def _check(st: int):
+    if st != LI_OK:
+        raise LiError(st, li_last_error_string())
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream or None
+
+
+def make_args(pb, return_value: int = 1) -> LiArgs:
+    """li_args for a problem whose tensors are already on the device (see synthetic.Problem)."""
+    a = LiArgs()
+    for name in ("q", "k", "w"):
+        t = getattr(pb, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    a.q, a.k, a.w = _ptr(pb.q), _ptr(pb.k), _ptr(pb.w)
+    a.cu_seqlens_q = _ptr(pb.cu_seqlens_q)
+    a.cu_seqlens_k = _ptr(pb.cu_seqlens_k)
+    a.seqused_q = _ptr(pb.seqused_q)
+    a.seqused_k = _ptr(pb.seqused_k)
+    a.block_table = _ptr(pb.block_table)
+    a.block_table_stride = int(pb.block_table.shape[-1]) if pb.block_table is not None else 0
+    a.output_idx_offset = _ptr(pb.output_idx_offset)
+    a.batch = pb.batch
+    a.q_len = pb.q_len
+    a.k_len = pb.k_len
+    a.max_seqlen_q = pb.max_seqlen_q
+    a.max_seqlen_k = pb.max_seqlen_k
+    a.num_blocks = pb.num_blocks
+    a.block_size = pb.block_size
+    a.num_heads_q = pb.n_heads
+    a.num_heads_k = 1
+    a.head_dim = pb.head_dim
+    a.topk = pb.topk
+    a.layout_q = LAYOUTS[pb.layout_q]
+    a.layout_k = LAYOUTS[pb.layout_k]
+    a.mask_mode = pb.mask_mode
+    a.dtype_qk = 0
+    a.dtype_w = 0
+    a.return_value = int(return_value)
+    return a
+
+
+def li_metadata_workspace_size(args: LiArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().li_metadata_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def li_indexer_workspace_size(args: LiArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().li_indexer_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def li_metadata(args: LiArgs, metadata: torch.Tensor, stream=None):
+    _check(lib().li_metadata(ctypes.byref(args), metadata.data_ptr(),
+                             metadata.numel() * metadata.element_size(), _stream_handle(stream)))
+
+
+def li_indexer(args: LiArgs, metadata, workspace: torch.Tensor, sparse_indices: torch.Tensor,
+               sparse_values, stream=None):
+    _check(lib().li_indexer(ctypes.byref(args), _ptr(metadata), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(),
+                            sparse_indices.data_ptr(), _ptr(sparse_values),
+                            _stream_handle(stream)))
+
+
+def li_check_status(workspace: torch.Tensor, stream=None):
+    """Synchronize and read the device status word: returns (status, LI_DEVERR_* bits)."""
+    bits = ctypes.c_uint32(0)
+    st = lib().li_check_status(workspace.data_ptr(), _stream_handle(stream), ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def li_set_stage_events(events):
+    """Time li_indexer's kernels: six recorded torch.cuda.Event objects, or None to stop."""
+    if not events:
+        _check(lib().li_set_stage_events(None, 0))
+        return
+    assert len(events) == 6
+    arr = (ctypes.c_void_p * 6)(*[int(e.cuda_event) for e in events])
+    _check(lib().li_set_stage_events(arr, 6))
+
+
+def out_shape(pb):
+    return (pb.batch, pb.q_len, 1, pb.topk) if pb.layout_q == "BSND" else (pb.q_len, 1, pb.topk)
+
+
+def empty_workspace(args: LiArgs, device) -> torch.Tensor:
+    n = li_indexer_workspace_size(args)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def indexer(pb, return_value: bool = True, metadata: bool | torch.Tensor = False,
+            workspace: torch.Tensor | None = None, stream=None, check: bool = True):
+    """Run the indexer on a device-resident problem. Returns (sparse_indices, sparse_values).
+
+    metadata: False = built inline by li_indexer; True = built by a separate li_metadata call;
+    a tensor = a schedule the caller built before."""
+    args = make_args(pb, int(return_value))
+    dev = pb.q.device
+    idx = torch.empty(out_shape(pb), dtype=torch.int32, device=dev)
+    val = torch.empty(out_shape(pb), dtype=torch.float32, device=dev) if return_value else None
+    ws = workspace if workspace is not None else empty_workspace(args, dev)
+    meta = None
+    if isinstance(metadata, torch.Tensor):
+        meta = metadata
+    elif metadata:
+        meta = torch.empty(li_metadata_workspace_size(args), dtype=torch.uint8, device=dev)
+        li_metadata(args, meta, stream)
+    li_indexer(args, meta, ws, idx, val, stream)
+    if check:
+        st, bits = li_check_status(ws, stream)
+        if st != LI_OK:
+            raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
+    return idx, val

@@ -1,0 +1,78 @@
+"""Comparison of the CUDA path's outputs with the CPU oracle.
+
+Tolerance (the indexer's accuracy target): per entry
+    |value_gpu - value_oracle| <= 2e-3 * max_j |I[t, j]| + 1e-4
+position-wise on the sorted lists, where max_j runs over the row's window. The index sets must be
+equal except for keys whose exact oracle score lies within that tolerance of the row's k-th
+score (near-ties may legitimately swap). The count of valid entries and the padding are exact.
+With integer-valued inputs every score is exact in fp32 and the outputs must match bit for bit.
+"""
+import numpy as np
+
+TOL_REL = 2e-3
+TOL_ABS = 1e-4
+
+
+def _bits(a):
+    return np.asarray(a, dtype=np.float32).view(np.uint32)
+
+
+def as_rows(t, topk):
+    return t.detach().cpu().numpy().reshape(-1, topk)
+
+
+def check(orc, pb_cpu, gpu_idx, gpu_val, rows=None, exact=False, label=""):
+    """Compare GPU outputs (all rows, as [rows, topk] numpy arrays) with the oracle on `rows`
+    (all rows when None). Returns the number of rows checked."""
+    bound = orc.bind(pb_cpu)
+    rows = np.arange(pb_cpu.rows) if rows is None else np.asarray(rows, dtype=np.int64)
+    o_idx, o_val, rc, maxabs = bound.topk(rows, with_maxabs=True)
+    assert rc == 0
+    topk = pb_cpu.topk
+    for n, r in enumerate(rows):
+        gi, gv = gpu_idx[r], gpu_val[r] if gpu_val is not None else None
+        oi, ov = o_idx[n], o_val[n]
+        where = f"{label} row {int(r)}"
+        m = int((oi >= 0).sum())
+        mg = int((gi >= 0).sum())
+        assert mg == m, f"{where}: {mg} valid entries, oracle {m}"
+        assert (gi[m:] == -1).all(), f"{where}: index padding"
+        if gv is not None:
+            assert np.isneginf(gv[m:]).all(), f"{where}: value padding"
+        if exact:
+            assert np.array_equal(gi, oi), f"{where}: indices differ (exact inputs)"
+            if gv is not None:
+                assert np.array_equal(_bits(gv), _bits(ov)), f"{where}: values differ (exact)"
+            continue
+        if m == 0:
+            continue
+        tol = TOL_REL * maxabs[n] + TOL_ABS
+        if gv is not None:
+            err = np.abs(gv[:m].astype(np.float64) - ov[:m].astype(np.float64))
+            bad = np.nonzero(err > tol)[0]
+            assert bad.size == 0, (f"{where}: value err {err.max():.3g} > tol {tol:.3g} at "
+                                   f"positions {bad[:5].tolist()}")
+            assert (np.diff(gv[:m]) <= 0).all(), f"{where}: values not sorted"
+        assert np.unique(gi[:m]).size == m, f"{where}: duplicate indices"
+        sg, so = set(gi[:m].tolist()), set(oi[:m].tolist())
+        diff = sg ^ so
+        if diff:
+            kth = float(ov[m - 1])
+            hi, b, _pos = bound.row_info(int(r))
+            off = int(pb_cpu.output_idx_offset[b]) if pb_cpu.output_idx_offset is not None else 0
+            for jj in diff:
+                j = jj - off
+                assert 0 <= j < hi, f"{where}: index {jj} outside the window"
+                s = bound.score_at(int(r), j)
+                assert abs(s - kth) <= tol, (f"{where}: key {jj} (score {s:.6g}) differs from the "
+                                             f"oracle's set, k-th score {kth:.6g}, tol {tol:.3g}")
+    return len(rows)
+
+
+def sample_rows(pb, n, seed=0, must=()):
+    """n seeded-random query rows plus the listed ones (deduplicated, sorted)."""
+    rng = np.random.default_rng(seed)
+    pick = set(int(x) for x in must if 0 <= x < pb.rows)
+    if pb.rows > 0:
+        pick.update(rng.choice(pb.rows, size=min(n, pb.rows), replace=False).tolist())
+    return np.array(sorted(pick), dtype=np.int64)

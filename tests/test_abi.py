@@ -1,0 +1,135 @@
+"""The C ABI without a GPU: the library loads, exports every function include/li.h declares, the
+ctypes mirror of li_args matches the C layout, and host-side validation rejects bad arguments
+before any launch."""
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+
+from sparse_attention_token_lightning_b200 import li
+from sparse_attention_token_lightning_b200 import build as libbuild
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "li.h"
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return li.lib()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"^[a-z0-9_ ]+[ *](li_[a-z_]+)\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in li.EXPORTS:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", str(li.lib_path())], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (li_[a-z_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(L, n)
+
+
+def test_abi_version(L):
+    assert li.li_abi_version() == 1
+
+
+def test_ctypes_struct_matches_c_layout(tmp_path):
+    fields = [f for f, _ in li.LiArgs._fields_]
+    prog = tmp_path / "probe.c"
+    body = "\n".join(f'  printf("%zu\\n", offsetof(li_args, {f}));' for f in fields)
+    prog.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "li.h"\nint main(void){\n'
+                    f'  printf("%zu\\n", sizeof(li_args));\n{body}\n  return 0;\n}}\n')
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c11", "-I", str(ROOT / "include"), str(prog), "-o", str(exe)],
+                   check=True)
+    vals = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                           check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(li.LiArgs)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(li.LiArgs, f).offset == off, f
+
+
+def _args(**kw):
+    """A valid BSND argument set with fake (never dereferenced) aligned device pointers."""
+    a = li.LiArgs()
+    a.q, a.k, a.w = 0x10000, 0x20000, 0x30000
+    a.batch, a.q_len, a.k_len = 1, 64, 64
+    a.max_seqlen_q, a.max_seqlen_k = 64, 64
+    a.num_heads_q, a.num_heads_k, a.head_dim, a.topk = 8, 1, 128, 16
+    a.layout_q = a.layout_k = 0
+    a.mask_mode = 3
+    a.return_value = 1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _ws_status(a):
+    n = ctypes.c_size_t(0)
+    return li.lib().li_indexer_workspace_size(ctypes.byref(a), ctypes.byref(n)), n.value
+
+
+def test_valid_args_size_the_workspace(L):
+    st, n = _ws_status(_args())
+    assert st == 0
+    # header + schedule + fp32 score rows (64 rows x 64 keys)
+    assert n >= 256 + 64 * 64 * 4
+    st, m = 0, ctypes.c_size_t(0)
+    st = L.li_metadata_workspace_size(ctypes.byref(_args()), ctypes.byref(m))
+    assert st == 0 and m.value > 0 and m.value % 256 == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_heads_q=0), 1), (dict(num_heads_q=65), 1), (dict(num_heads_k=2), 1),
+    (dict(head_dim=64), 1), (dict(topk=0), 1), (dict(topk=8193), 1), (dict(mask_mode=1), 1),
+    (dict(layout_q=2), 1), (dict(layout_k=5), 1), (dict(dtype_qk=1), 2), (dict(q=None), 1),
+    (dict(q=0x10008), 1), (dict(layout_q=1), 1), (dict(layout_k=1), 1), (dict(layout_k=2), 1),
+    (dict(layout_k=2, seqused_k=0x40000, block_table=0x50000, block_table_stride=4,
+          num_blocks=4, block_size=0), 1),
+    (dict(layout_k=2, seqused_k=0x40000, block_table=0x50000, block_table_stride=4,
+          num_blocks=4, block_size=1025), 1),
+    (dict(cu_seqlens_q=0x40000), 1), (dict(block_table=0x40000), 1), (dict(batch=-1), 1),
+    (dict(max_seqlen_k=65), 1), (dict(return_value=2), 1),
+])
+def test_invalid_args_rejected_on_host(L, kw, status):
+    st, _ = _ws_status(_args(**kw))
+    assert st == status, li.li_last_error_string()
+    assert li.li_last_error_string()
+
+
+def test_topk_accepts_every_value_up_to_8192(L):
+    # the pages' Atlas set is [1, 2048] plus multiples of 1024 up to 8192; every value in
+    # [1, 8192] is accepted here
+    for k in (1, 2047, 2048, 2049, 3000, 3072, 8191, 8192):
+        st, _ = _ws_status(_args(topk=k))
+        assert st == 0, k
+
+
+def test_paged_args_accepted(L):
+    st, n = _ws_status(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
+                             block_table_stride=8, num_blocks=16, block_size=64,
+                             max_seqlen_k=512))
+    assert st == 0 and n > 0
+
+
+def test_indexer_rejects_small_workspace(L):
+    a = _args()
+    st = L.li_indexer(ctypes.byref(a), None, 0x100000, 16, 0x200000, 0x300000, None)
+    assert st == 3
+    st = L.li_indexer(ctypes.byref(a), None, 0x100010, 1 << 30, 0x200000, 0x300000, None)
+    assert st == 3   # misaligned workspace
+    st = L.li_indexer(ctypes.byref(a), None, 0x100000, 1 << 30, None, 0x300000, None)
+    assert st == 1   # no output

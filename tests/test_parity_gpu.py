@@ -1,0 +1,180 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
+
+Small problems span several 128-key tiles with ragged tails and are compared on every row; the
+full-size workloads (causal prefill, paged decode, varlen, long context) run in the benchmark's
+configuration and are compared on seeded samples of rows. Integer-valued inputs make every score
+exact in fp32, so there the outputs must match the oracle bit for bit, ties included.
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from sparse_attention_token_lightning_b200 import li, synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    li.lib()
+
+
+def run(pb, **kw):
+    g = pb.to("cuda")
+    idx, val = li.indexer(g, **kw)
+    torch.cuda.synchronize()
+    return (parity.as_rows(idx, pb.topk), None if val is None else parity.as_rows(val, pb.topk))
+
+
+# ---- small problems, every row ------------------------------------------------------------------
+
+SMALL = {
+    "tiny": lambda: synthetic.config("tiny"),
+    "pages_example": lambda: synthetic.config("pages_example"),
+    "bsnd_causal_ragged": lambda: synthetic.bsnd(2, 300, 459, 64, 200, 3, seed=3),
+    "bsnd_nomask_n1": lambda: synthetic.bsnd(1, 40, 333, 1, 64, 0, seed=4),
+    "bsnd_n3_topk_gt_keys": lambda: synthetic.bsnd(1, 50, 130, 3, 256, 3, seed=5),
+    "bsnd_n16_q_longer": lambda: synthetic.bsnd(2, 200, 150, 16, 32, 3, seed=6),
+    "tnd_varlen": lambda: synthetic.tnd([1, 130, 77, 0, 256], [300, 130, 500, 9, 256], 64, 100,
+                                        3, seed=7),
+    "tnd_nomask": lambda: synthetic.tnd([17, 5], [40, 290], 8, 50, 0, seed=8),
+    "paged_bs64": lambda: synthetic.paged([700, 129, 1, 64], 3, 64, 128, block_size=64,
+                                          seed=9, spare_blocks=5),
+    "paged_bs16_tnd_q": lambda: synthetic.paged([300, 45], 0, 32, 64, block_size=16, seed=10,
+                                                layout_q="TND", lens_q=[4, 2]),
+    "paged_bs48": lambda: synthetic.paged([333, 200], 2, 16, 40, block_size=48, seed=11),
+    "paged_bs1": lambda: synthetic.paged([37, 3], 1, 4, 8, block_size=1, seed=12),
+    "topk1": lambda: synthetic.bsnd(1, 64, 200, 8, 1, 3, seed=13),
+    "topk8192": lambda: synthetic.bsnd(1, 8, 9000, 2, 8192, 0, seed=14),
+    "offset_seqused": lambda: synthetic.tnd([10, 30], [60, 90], 4, 40, 3, seed=15,
+                                            seqused_q=[7, 30], output_idx_offset=[1000, 5]),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_parity(orc, name):
+    pb = SMALL[name]()
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, label=name)
+
+
+EXACT = {
+    "bsnd_causal": lambda: synthetic.bsnd(2, 333, 333, 64, 100, 3, seed=20, integer=True),
+    "bsnd_n4_nomask": lambda: synthetic.bsnd(1, 100, 260, 4, 300, 0, seed=21, integer=True),
+    "tnd": lambda: synthetic.tnd([5, 200, 1], [129, 200, 700], 16, 64, 3, seed=22, integer=True),
+    "paged": lambda: synthetic.paged([500, 64, 65], 2, 64, 96, block_size=64, seed=23,
+                                     integer=True, spare_blocks=2),
+}
+
+
+@pytest.mark.parametrize("name", list(EXACT))
+def test_integer_inputs_bit_exact(orc, name):
+    pb = EXACT[name]()
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, exact=True, label=name)
+
+
+def test_indices_only(orc):
+    pb = synthetic.bsnd(1, 64, 300, 8, 50, 3, seed=30)
+    gi, gv = run(pb, return_value=False)
+    assert gv is None
+    gi2, gv2 = run(pb)
+    assert np.array_equal(gi, gi2)
+
+
+def test_separate_metadata_matches_inline():
+    pb = synthetic.tnd([100, 3, 250], [100, 400, 260], 64, 64, 3, seed=31)
+    a = run(pb, metadata=False)
+    b = run(pb, metadata=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+
+
+def test_deterministic_reruns():
+    pb = synthetic.bsnd(1, 1024, 1024, 64, 256, 3, seed=32).to("cuda")
+    i1, v1 = li.indexer(pb)
+    i2, v2 = li.indexer(pb)
+    assert torch.equal(i1, i2) and torch.equal(v1.view(torch.int32), v2.view(torch.int32))
+
+
+def test_batch_without_rows():
+    pb = synthetic.bsnd(0, 16, 16, 4, 8, 3, seed=33)
+    gi, gv = run(pb)
+    assert gi.size == 0
+
+
+# ---- device-data errors are reported, not faulted ------------------------------------------------
+
+def _status_of(pb):
+    g = pb.to("cuda")
+    args = li.make_args(g)
+    ws = li.empty_workspace(args, "cuda")
+    idx = torch.empty(li.out_shape(g), dtype=torch.int32, device="cuda")
+    val = torch.empty(li.out_shape(g), dtype=torch.float32, device="cuda")
+    li.li_indexer(args, None, ws, idx, val)
+    return li.li_check_status(ws)
+
+
+def test_bad_cu_seqlens_reported():
+    pb = synthetic.tnd([10, 10], [20, 20], 4, 8, 3, seed=34)
+    pb.cu_seqlens_k = torch.tensor([0, 25, 20], dtype=torch.int32)   # not monotone
+    st, bits = _status_of(pb)
+    assert st == 6 and bits & li.DEVERR_LENGTHS
+
+
+def test_bad_block_table_reported():
+    pb = synthetic.paged([100, 50], 1, 4, 8, block_size=16, seed=35)
+    pb.block_table[0, 2] = pb.num_blocks + 7                            # outside the cache
+    st, bits = _status_of(pb)
+    assert st == 6 and bits & li.DEVERR_TABLE
+
+
+def test_offset_overflow_reported():
+    pb = synthetic.bsnd(1, 4, 40, 4, 8, 3, seed=36, output_idx_offset=[2**31 - 10])
+    st, bits = _status_of(pb)
+    assert st == 6 and bits & li.DEVERR_OFFSET
+
+
+def test_mismatched_metadata_reported():
+    pb = synthetic.bsnd(1, 64, 64, 4, 8, 3, seed=37).to("cuda")
+    other = synthetic.bsnd(1, 64, 64, 4, 8, 0, seed=37).to("cuda")    # other mask mode
+    meta = torch.empty(li.li_metadata_workspace_size(li.make_args(other)), dtype=torch.uint8,
+                       device="cuda")
+    li.li_metadata(li.make_args(other), meta)
+    args = li.make_args(pb)
+    ws = li.empty_workspace(args, "cuda")
+    idx = torch.empty(li.out_shape(pb), dtype=torch.int32, device="cuda")
+    val = torch.empty(li.out_shape(pb), dtype=torch.float32, device="cuda")
+    li.li_indexer(args, meta, ws, idx, val)
+    st, bits = li.li_check_status(ws)
+    assert st == 6 and bits & li.DEVERR_METADATA
+
+
+def test_seqused_k_above_max_reported():
+    pb = synthetic.paged([100, 50], 1, 4, 8, block_size=16, seed=38)
+    pb.max_seqlen_k = 60                                               # batch 0 has 100 keys
+    st, bits = _status_of(pb)
+    assert st == 6 and bits & li.DEVERR_LENGTHS
+
+
+# ---- full-size workloads, sampled rows -----------------------------------------------------------
+
+FULL = {
+    # name: (rows to sample, rows that must be checked)
+    "causal_prefill": (24, (0, 1, 127, 128, 2046, 2047, 2048, 2049, 4095)),
+    "paged_decode": (8, (0, 63)),
+    "varlen": (16, (0, 32767)),
+    "long_2048": (6, (0, 2047, 2048, 65535)),
+    "long_8192": (4, (8191, 8192, 65535)),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_sampled(orc, name):
+    pb = synthetic.config(name)
+    n, must = FULL[name]
+    rows = parity.sample_rows(pb, n, seed=1, must=must)
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, rows=rows, label=name)
