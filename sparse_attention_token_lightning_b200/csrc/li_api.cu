@@ -92,7 +92,13 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
         return fail(LI_ERR_INVALID_ARG, "k_len=%d < 0", a->k_len);
     if (a->max_seqlen_k < 0) return fail(LI_ERR_INVALID_ARG, "max_seqlen_k=%d < 0", a->max_seqlen_k);
     if (a->max_seqlen_q < 0) return fail(LI_ERR_INVALID_ARG, "max_seqlen_q=%d < 0", a->max_seqlen_q);
-    if (!a->q || !a->k || !a->w) return fail(LI_ERR_INVALID_ARG, "q, k and w are required");
+    const int64_t rows0 = a->layout_q == LI_LAYOUT_TND ? (int64_t)a->q_len
+                                                      : (int64_t)a->batch * a->q_len;
+    const bool may_have_keys = a->layout_k == LI_LAYOUT_PA_BSND || a->k_len > 0;
+    // Empty tensors may come with NULL data pointers: q and w are needed only when there are
+    // query rows, k only when there can be keys.
+    if (rows0 > 0 && (!a->q || !a->w)) return fail(LI_ERR_INVALID_ARG, "q and w are required");
+    if (rows0 > 0 && may_have_keys && !a->k) return fail(LI_ERR_INVALID_ARG, "k is required");
     if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->w, 2))
         return fail(LI_ERR_INVALID_ARG, "q and k must be 16-byte aligned, w 2-byte aligned");
     if (a->layout_q == LI_LAYOUT_TND && !a->cu_seqlens_q)
@@ -239,9 +245,10 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
     li::Schedule s;
     li_status st = validate(args, &p, &s);
     if (st != LI_OK) return st;
-    if (!sparse_indices || !aligned(sparse_indices, 4))
+    // Outputs are needed only when there are rows (empty tensors may have NULL data).
+    if (p.rows > 0 && (!sparse_indices || !aligned(sparse_indices, 4)))
         return fail(LI_ERR_INVALID_ARG, "sparse_indices must be a 4-byte aligned device buffer");
-    if (p.return_value && (!sparse_values || !aligned(sparse_values, 4)))
+    if (p.rows > 0 && p.return_value && (!sparse_values || !aligned(sparse_values, 4)))
         return fail(LI_ERR_INVALID_ARG, "return_value=1 requires sparse_values");
     if (metadata && !aligned(metadata, 256))
         return fail(LI_ERR_WORKSPACE, "metadata must be 256-byte aligned");
