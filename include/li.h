@@ -174,6 +174,36 @@ li_status li_check_status(const void *workspace, void *stream, uint32_t *device_
  */
 li_status li_set_stage_events(void *const *events, int32_t n_events);
 
+/*
+ * li_indexer_noalloc -- li_indexer for callers that may not allocate device memory.
+ * The pages have no counterpart; this entry point exists for integrations where the caller
+ * cannot obtain a workspace: plugin or custom-op interfaces whose enqueue step offers no
+ * allocator, runtimes that reserve all device memory up front and forbid allocation afterwards,
+ * and real-time loops where cudaMalloc's implicit synchronization and latency are not allowed.
+ *
+ * It runs exactly the li_indexer path with metadata built inline, using as workspace a scratch
+ * array compiled into the library (a static device array of LI_NOALLOC_SCRATCH_BYTES). The
+ * caller passes the inputs in `args` and the outputs as with li_indexer, plus `device_status`:
+ * a device uint32 (or NULL) that receives the call's device status word, stream-ordered, so
+ * li_check_status(device_status, stream, &bits) reports data errors of this call.
+ *
+ *   - Problems whose workspace (li_indexer_workspace_size) exceeds LI_NOALLOC_SCRATCH_BYTES are
+ *     rejected on the host with LI_ERR_WORKSPACE and a message giving both sizes.
+ *   - No cudaMalloc, cudaFree or other allocating call is made. The array occupies
+ *     LI_NOALLOC_SCRATCH_BYTES on every device where the library's module is loaded (from the
+ *     first call on that device, or from library load under eager module loading) until the
+ *     process exits.
+ *   - The first call on a device looks up the array's device address (once per device, with that
+ *     device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, and its contents persist between calls (the
+ *     call clears what must start at zero). Calls whose kernels overlap on the GPU -- concurrent
+ *     streams, or several host threads -- race on the array and give undefined results:
+ *     serialize them.
+ */
+#define LI_NOALLOC_SCRATCH_BYTES (32u << 20)
+li_status li_indexer_noalloc(const li_args *args, int32_t *sparse_indices, float *sparse_values,
+                             uint32_t *device_status, void *stream);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char *li_last_error_string(void);
 

@@ -201,6 +201,10 @@ size_t indexer_ws_bytes(const li::Problem &p, const li::Schedule &s) {
 
 }  // namespace
 
+namespace li {
+void set_last_error(const char *msg) { g_err = msg; }
+}  // namespace li
+
 extern "C" {
 
 li_status li_metadata_workspace_size(const li_args *args, size_t *bytes) {

@@ -160,6 +160,9 @@ __device__ inline void set_status(uint32_t *status, uint32_t bits) {
     if (bits) atomicOr(status, bits);
 }
 
+// Sets the message li_last_error_string() returns on this host thread.
+void set_last_error(const char *msg);
+
 // ---- launchers implemented in the .cu files --------------------------------------------------
 cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st);
 cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,

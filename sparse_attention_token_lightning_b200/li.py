@@ -50,7 +50,7 @@ _lib = None
 
 EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
            "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
-           "li_abi_version")
+           "li_abi_version", "li_indexer_noalloc")
 
 
 def lib_path() -> Path:
@@ -77,6 +77,8 @@ def lib():
     for f in ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
               "li_indexer", "li_check_status"):
         getattr(L, f).restype = ctypes.c_int
+    L.li_indexer_noalloc.argtypes = [P, vp, vp, vp, vp]
+    L.li_indexer_noalloc.restype = ctypes.c_int
     L.li_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
     L.li_set_stage_events.restype = ctypes.c_int
     L.li_last_error_string.argtypes = []
@@ -168,6 +170,16 @@ def li_indexer(args: LiArgs, metadata, workspace: torch.Tensor, sparse_indices: 
                             workspace.numel() * workspace.element_size(),
                             sparse_indices.data_ptr(), _ptr(sparse_values),
                             _stream_handle(stream)))
+
+
+def li_indexer_noalloc(args: LiArgs, sparse_indices: torch.Tensor, sparse_values,
+                       device_status=None, stream=None):
+    """li_indexer without a caller workspace (the library's static scratch is used); for
+    callers that may not allocate device memory. device_status: a 4-byte device tensor that
+    receives the call's status word, or None."""
+    _check(lib().li_indexer_noalloc(ctypes.byref(args), sparse_indices.data_ptr(),
+                                    _ptr(sparse_values), _ptr(device_status),
+                                    _stream_handle(stream)))
 
 
 def li_check_status(workspace: torch.Tensor, stream=None):

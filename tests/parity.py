@@ -76,3 +76,33 @@ def sample_rows(pb, n, seed=0, must=()):
     if pb.rows > 0:
         pick.update(rng.choice(pb.rows, size=min(n, pb.rows), replace=False).tolist())
     return np.array(sorted(pick), dtype=np.int64)
+
+
+def check_pair(orc, pb_cpu, a_idx, a_val, b_idx, b_val, label=""):
+    """Two GPU outputs of the same problem agree under the same tolerance rule (values within
+    2e-3 * max|I| + 1e-4 position-wise; index sets equal outside the near-tie band), with the
+    oracle supplying each row's max |I| and exact scores for any differing keys."""
+    bound = orc.bind(pb_cpu)
+    rows = np.arange(pb_cpu.rows)
+    _oi, o_val, rc, maxabs = bound.topk(rows, with_maxabs=True)
+    assert rc == 0
+    for r in rows:
+        where = f"{label} row {int(r)}"
+        ai, bi = a_idx[r], b_idx[r]
+        m = int((ai >= 0).sum())
+        assert int((bi >= 0).sum()) == m, f"{where}: valid counts differ"
+        assert (ai[m:] == -1).all() and (bi[m:] == -1).all(), f"{where}: index padding"
+        assert np.isneginf(a_val[r][m:]).all() and np.isneginf(b_val[r][m:]).all(), where
+        if m == 0:
+            continue
+        tol = TOL_REL * maxabs[r] + TOL_ABS
+        err = np.abs(a_val[r][:m].astype(np.float64) - b_val[r][:m].astype(np.float64))
+        assert (err <= tol).all(), f"{where}: values differ by {err.max():.3g} > {tol:.3g}"
+        diff = set(ai[:m].tolist()) ^ set(bi[:m].tolist())
+        if diff:
+            kth = float(o_val[r][m - 1])
+            _hi, b, _p = bound.row_info(int(r))
+            off = int(pb_cpu.output_idx_offset[b]) if pb_cpu.output_idx_offset is not None else 0
+            for jj in diff:
+                s = bound.score_at(int(r), jj - off)
+                assert abs(s - kth) <= tol, f"{where}: key {jj} is not a near-tie"
