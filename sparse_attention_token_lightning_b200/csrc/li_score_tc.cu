@@ -1,12 +1,599 @@
-// Tensor-core score kernel (tcgen05 + TMA + TMEM) -- placeholder until the kernel lands.
+// Score kernel on the 5th-generation tensor cores (tcgen05 + TMA + TMEM), sm_100a.
+//
+// Computes, for every work item (batch b, query rows [q0, q0+nq), keys [j0, j1)), the index score
+//     I[t, j] = sum_h w[t,h] * ReLU(q[t,h,:] . k[j,:])
+// (custom_pypto.npu_lightning_indexer_pto, function description formula; lightning_indexer,
+// "Function" steps 1-3) and writes it to the fp32 score rows of the workspace for the keys of
+// each row's window (right-down causal or none, custom_pypto.npu_lightning_indexer_pto,
+// sparse_mode). The head-by-key score tensor never leaves the SM.
+//
+// Orientation: keys on the MMA M axis (128 TMEM lanes), query rows x heads on N:
+//     D[key, t*N1 + h] = k_key . q[t, h]          M = 128, N = tq*N1 (<= 256), K = 128
+// so every epilogue thread owns one key (one TMEM lane) and reduces the heads of a row in
+// registers; no cross-lane reduction is needed and w is a per-row broadcast.
+//
+// Warp roles (one CTA per SM, persistent, work items pulled from a global ticket counter):
+//   warp 0      scheduler + TMA producer: takes a ticket, stages the item's header and w in a
+//               shared-memory slot, loads the item's Q tile (double buffered) and streams its
+//               K tiles through a 3-stage ring. Paged keys come block by block through the
+//               block table.
+//   warp 1      allocates TMEM (512 columns = two 256-column accumulators); one thread issues
+//               the tcgen05.mma chain (8 x K16 per tile) and commits to the barriers.
+//   warps 2-9   epilogue: two warps per TMEM lane quarter, each taking every other query row of
+//               the item; tcgen05.ld of a row's N1 columns, ReLU, weight, head sum, causal mask,
+//               coalesced fp32 stores.
+// Every wait on an mbarrier is bounded in time; on expiry the kernel records LI_DEVERR_TIMEOUT,
+// the roles leave their loops, TMEM is freed and the kernel returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "li_internal.cuh"
 
 namespace li {
+namespace {
 
-cudaError_t launch_score_tc(const Problem &, const Schedule &, const void *, WsHeader *, float *,
-                            int64_t, cudaStream_t, bool *launched) {
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kStages = 3;
+constexpr int kSlots = 2;
+constexpr int kNmax = 256;
+constexpr uint32_t kQHalfBytes = kNmax * 128;            // 256 rows x 64 bf16
+constexpr uint32_t kQBufBytes = 2 * kQHalfBytes;         // both K halves
+constexpr uint32_t kKHalfBytes = kKeyTile * 128;         // 128 keys x 64 bf16
+constexpr uint32_t kKStageBytes = 2 * kKHalfBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256;
+constexpr uint32_t kDevErrInternal = 0x20u;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+
+struct Slot {
+    int32_t valid, b, q0, nq, j0, j1, row0, L1u, L2;
+    int32_t pad[7];
+    float w[kNmax];
+};
+static_assert(sizeof(Slot) == 64 + 4 * kNmax, "Slot size");
+
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kKOff = kQOff + 2 * kQBufBytes;
+constexpr uint32_t kSlotOff = kKOff + kStages * kKStageBytes;
+constexpr uint32_t kBarOff = kSlotOff + kSlots * sizeof(Slot);
+constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 * 2 + 2 * kSlots;
+constexpr uint32_t kFlagOff = kBarOff + 8 * kNumBars;
+constexpr uint32_t kSmemBytes = kFlagOff + 16;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct TcParams {
+    Problem p;
+    const void *meta;
+    WsHeader *ws;
+    float *scores;
+    int64_t ld;
+    uint32_t signature;
+    int32_t N;            // MMA N
+    int32_t tq;           // query rows per item
+    uint32_t idesc;       // tcgen05 instruction descriptor
+    int32_t piece_rows;   // paged: keys per TMA load (min(block_size, 128)); 0 for dense keys
+};
+
+// ---- PTX wrappers --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of the given parity. Returns false when the time limit passes or
+// another role has already given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle layout TMA writes
+// (8-row x 128-byte atoms, 1024 bytes apart), start address in 16-byte units.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane, waited for before returning.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+          "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+          "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+          "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+          "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive fp32 columns, waited for before returning.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct Bars {
+    uint32_t base;
+    __device__ uint32_t k_full(int s) const { return base + 8 * s; }
+    __device__ uint32_t k_empty(int s) const { return base + 8 * (kStages + s); }
+    __device__ uint32_t q_full(int i) const { return base + 8 * (2 * kStages + i); }
+    __device__ uint32_t q_empty(int i) const { return base + 8 * (2 * kStages + 2 + i); }
+    __device__ uint32_t acc_full(int i) const { return base + 8 * (2 * kStages + 4 + i); }
+    __device__ uint32_t acc_empty(int i) const { return base + 8 * (2 * kStages + 6 + i); }
+    __device__ uint32_t sl_full(int i) const { return base + 8 * (2 * kStages + 8 + i); }
+    __device__ uint32_t sl_empty(int i) const { return base + 8 * (2 * kStages + 8 + kSlots + i); }
+};
+
+__device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
+    return (j1 - j0 + kKeyTile - 1) / kKeyTile;
+}
+
+// ---- roles ---------------------------------------------------------------------------------
+__device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
+                         uint8_t *smem, const Bars &bars, volatile int *abort_flag,
+                         const BatchInfo *binfo, const WorkItem *items, int n_items) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
+    const int N1 = P.p.n_heads;
+    uint32_t err = 0;
+    int kcount = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+        const int sl = it % kSlots;
+        if (!mbar_wait(bars.sl_empty(sl), ((it / kSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(&P.ws->sched_next, 1);
+        ticket = __shfl_sync(0xffffffffu, ticket, 0);
+        const bool valid = ticket < n_items;
+        Slot &S = slots[sl];
+        WorkItem wi{};
+        BatchInfo bi{};
+        if (valid) {
+            wi = items[ticket];
+            bi = binfo[wi.b];
+            const int64_t wbase = ((int64_t)bi.q_row0 + wi.q0) * N1;
+            const int nw = wi.nq * N1;
+            for (int e = lane; e < kNmax; e += 32)
+                S.w[e] = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+            if (lane == 0) {
+                S.b = wi.b; S.q0 = wi.q0; S.nq = wi.nq; S.j0 = wi.j0; S.j1 = wi.j1;
+                S.row0 = bi.q_row0 + wi.q0; S.L1u = bi.L1u; S.L2 = bi.L2;
+            }
+        }
+        if (lane == 0) S.valid = valid ? 1 : 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.sl_full(sl));
+        if (!valid) break;
+
+        // Q tile of the item (all heads of tq rows): two TMA loads, one per 64-wide K half.
+        const int qb = it & 1;
+        if (!mbar_wait(bars.q_empty(qb), ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) {
+            const uint32_t qdst = sbase + kQOff + qb * kQBufBytes;
+            const int32_t y = (bi.q_row0 + wi.q0) * N1;
+            mbar_arrive_expect_tx(bars.q_full(qb), 2u * P.N * 128u);
+            tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
+            tma_load_2d(qdst + kQHalfBytes, tmq, bars.q_full(qb), 64, y);
+        }
+        // K tiles of the item's key range.
+        const int32_t nt = n_tiles_of(wi.j0, wi.j1);
+        for (int32_t tile = 0; tile < nt; ++tile, ++kcount) {
+            const int st = kcount % kStages;
+            if (!mbar_wait(bars.k_empty(st), ((kcount / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
+                const int32_t jt = wi.j0 + tile * kKeyTile;
+                const uint32_t kdst = sbase + kKOff + st * kKStageBytes;
+                if (P.piece_rows == 0) {
+                    mbar_arrive_expect_tx(bars.k_full(st), kKStageBytes);
+                    tma_load_2d(kdst, tmk, bars.k_full(st), 0, bi.k_row0 + jt);
+                    tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, bi.k_row0 + jt);
+                } else {
+                    // Paged keys: one load per (part of a) block, at most 128 / piece_rows.
+                    const int pr = P.piece_rows;
+                    const int pieces = kKeyTile / pr;
+                    int32_t rows[kKeyTile / 8];
+                    int loads = 0;
+                    for (int pc = 0; pc < pieces; ++pc) {
+                        const int32_t jp = jt + pc * pr;
+                        rows[pc] = -1;
+                        if (jp >= wi.j1) continue;
+                        const int32_t blk = P.p.block_table[(int64_t)wi.b * P.p.bt_stride + jp / P.p.block_size];
+                        if (blk < 0 || blk >= P.p.num_blocks) { err |= LI_DEVERR_TABLE; continue; }
+                        rows[pc] = blk * P.p.block_size + jp % P.p.block_size;
+                        ++loads;
+                    }
+                    mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)loads * pr * 256u);
+                    for (int pc = 0; pc < pieces; ++pc) {
+                        if (rows[pc] < 0) continue;
+                        const uint32_t off = (uint32_t)pc * pr * 128u;
+                        tma_load_2d(kdst + off, tmk, bars.k_full(st), 0, rows[pc]);
+                        tma_load_2d(kdst + kKHalfBytes + off, tmk, bars.k_full(st), 64, rows[pc]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    if (!ok) *abort_flag = 1;
+    if (lane == 0 && err) set_status(&P.ws->status, err);
+}
+
+__device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
+                           volatile int *abort_flag, uint32_t tmem_base) {
+    const uint32_t sbase = smem_u32(smem);
+    Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
+    int kcount = 0, acount = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+        const int sl = it % kSlots;
+        if (!mbar_wait(bars.sl_full(sl), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
+        const Slot &S = slots[sl];
+        const int valid = S.valid;
+        const int32_t j0 = S.j0, j1 = S.j1;
+        mbar_arrive(bars.sl_empty(sl));
+        if (!valid) break;
+        const int qb = it & 1;
+        if (!mbar_wait(bars.q_full(qb), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        const uint32_t qsm = sbase + kQOff + qb * kQBufBytes;
+        const int32_t nt = n_tiles_of(j0, j1);
+        for (int32_t tile = 0; tile < nt; ++tile, ++kcount, ++acount) {
+            const int st = kcount % kStages;
+            const int ab = acount & 1;
+            if (!mbar_wait(bars.k_full(st), (kcount / kStages) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bars.acc_empty(ab), ((acount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ksm = sbase + kKOff + st * kKStageBytes;
+            const uint32_t d = tmem_base + ab * kAccCols;
+#pragma unroll
+            for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+                const uint32_t half = (uint32_t)(kk >> 2), sub = (uint32_t)(kk & 3) * 32u;
+                const uint64_t adesc = sw128_desc(ksm + half * kKHalfBytes + sub);
+                const uint64_t bdesc = sw128_desc(qsm + half * kQHalfBytes + sub);
+                umma_bf16(d, adesc, bdesc, P.idesc, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bars.k_empty(st));
+            umma_commit(bars.acc_full(ab));
+        }
+        if (!ok) break;
+        umma_commit(bars.q_empty(qb));
+    }
+    if (!ok) *abort_flag = 1;
+}
+
+__device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
+                         volatile int *abort_flag, uint32_t tmem_base) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;          // TMEM lanes this warp may access
+    const int group = (warp - 2) >> 2;     // 0 or 1: which rows of the item
+    Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
+    const int N1 = P.p.n_heads;
+    const int mask_mode = P.p.mask_mode;
+    const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+    int acount = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+        const int sl = it % kSlots;
+        if (!mbar_wait(bars.sl_full(sl), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
+        const Slot &S = slots[sl];
+        const int valid = S.valid;
+        if (!valid) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.sl_empty(sl));
+            break;
+        }
+        const int32_t q0 = S.q0, nq = S.nq, j0 = S.j0, j1 = S.j1, row0 = S.row0, L1u = S.L1u,
+                      L2 = S.L2;
+        const int32_t nt = n_tiles_of(j0, j1);
+        for (int32_t tile = 0; tile < nt; ++tile, ++acount) {
+            const int ab = acount & 1;
+            if (!mbar_wait(bars.acc_full(ab), (acount >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const int32_t jt = j0 + tile * kKeyTile;
+            const int32_t j = jt + 32 * quarter + lane;
+            const uint32_t acc = tmem_base + lane_addr + ab * kAccCols;
+            for (int t = group; t < nq; t += 2) {
+                const int32_t hi = min(window_hi(mask_mode, q0 + t, L1u, L2), j1);
+                if (jt >= hi) continue;                       // tile past this row's window
+                float I;
+                if (N1 == 64) {
+                    float v[64];
+                    tmem_ld64(acc + t * 64, v);
+                    const float4 *w4 = reinterpret_cast<const float4 *>(S.w + t * 64);
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                    for (int h4 = 0; h4 < 16; ++h4) {
+                        const float4 ww = w4[h4];
+                        a0 = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), a0);
+                        a1 = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), a1);
+                        a2 = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), a2);
+                        a3 = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), a3);
+                    }
+                    I = (a0 + a1) + (a2 + a3);
+                } else {
+                    const int c_lo = t * N1, c_hi = c_lo + N1;
+                    float a = 0.f;
+                    for (int ch = c_lo & ~15; ch < c_hi; ch += 16) {
+                        float v[16];
+                        tmem_ld16(acc + ch, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = ch + i;
+                            if (c >= c_lo && c < c_hi) a = fmaf(S.w[c], fmaxf(v[i], 0.f), a);
+                        }
+                    }
+                    I = a;
+                }
+                if (j < hi) P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.acc_empty(ab));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.sl_empty(sl));
+    }
+    if (!ok) *abort_flag = 1;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                const TcParams P) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {                              // the swizzled tiles need 1 KB alignment
+        if (threadIdx.x == 0) set_status(&P.ws->status, kDevErrInternal);
+        return;
+    }
+    const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(P.meta);
+    if (hdr->magic != kMetaMagic || hdr->signature != P.signature) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) set_status(&P.ws->status, kDevErrMetadata);
+        return;
+    }
+    const int n_items = hdr->n_items;
+    const BatchInfo *binfo = meta_batches(P.meta);
+    const WorkItem *items = meta_items(P.meta, hdr->batch);
+
+    Bars bars{sbase + kBarOff};
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff + 4);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bars.k_full(s), 1);
+            mbar_init(bars.k_empty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bars.q_full(i), 1);
+            mbar_init(bars.q_empty(i), 1);
+            mbar_init(bars.acc_full(i), 1);
+            mbar_init(bars.acc_empty(i), kEpiWarps);
+        }
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(bars.sl_full(i), 1);
+            mbar_init(bars.sl_empty(i), 1 + kEpiWarps);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag, binfo, items, n_items);
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);
+        __syncwarp();
+    } else {
+        epilogue(P, smem, bars, abort_flag, tmem_base);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) set_status(&P.ws->status, LI_DEVERR_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---- host ----------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn || rows == 0) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count_cached() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
+}
+
+}  // namespace
+
+// Launches the tensor-core kernel when the problem fits it; *launched = false leaves the call
+// to the CUDA-core kernel (paged caches whose block size is not a multiple of 8 dividing 128 or
+// a multiple of 128, and empty tensors).
+cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
+                            float *scores, int64_t ld, cudaStream_t st, bool *launched) {
     *launched = false;
-    return cudaSuccess;
+    if (s.max_items <= 0 || p.rows <= 0) return cudaSuccess;
+    TcParams P{};
+    P.p = p;
+    P.meta = meta;
+    P.ws = ws;
+    P.scores = scores;
+    P.ld = ld;
+    P.signature = problem_signature(p, s.tq, s.kc);
+    P.tq = s.tq;
+    P.N = (s.tq * p.n_heads + 15) / 16 * 16;
+    if (P.N > kNmax || P.N < 16) return cudaSuccess;
+    P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(P.N >> 3) << 17) |
+              ((uint32_t)(128 >> 4) << 24);
+    uint64_t k_rows = 0;
+    if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        const int bs = p.block_size;
+        if (bs <= kKeyTile) {
+            if (bs % 8 != 0 || kKeyTile % bs != 0) return cudaSuccess;
+            P.piece_rows = bs;
+        } else {
+            if (bs % kKeyTile != 0) return cudaSuccess;
+            P.piece_rows = kKeyTile;
+        }
+        k_rows = (uint64_t)p.num_blocks * bs;
+    } else {
+        P.piece_rows = 0;
+        k_rows = p.layout_k == LI_LAYOUT_TND ? (uint64_t)p.k_len : (uint64_t)p.batch * p.k_len;
+    }
+    const uint64_t q_rows = (uint64_t)(p.layout_q == LI_LAYOUT_TND ? p.q_len : p.batch * p.q_len) *
+                            p.n_heads;
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N)) return cudaSuccess;
+    if (!make_map(&mk, p.k, k_rows, P.piece_rows ? (uint32_t)P.piece_rows : (uint32_t)kKeyTile))
+        return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int grid = sm_count_cached();
+    if (s.max_items < grid) grid = s.max_items;
+    score_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, P);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) *launched = true;
+    return e;
 }
 
 }  // namespace li

@@ -5,17 +5,20 @@
 // (+ output_idx_offset[b]) and scores, then pad with -1 / -inf up to topk (lightning_indexer and
 // aclnnLightningIndexerV2, constraints on the invalid part; torch_npu.npu_sparse_lightning_
 // indexer_grad_kl_loss, sparse_indices are sorted). Rows past seqused_q, rows of no batch and
-// rows with an empty causal window are all padding.
+// rows with an empty causal window are all padding. -0 and +0 are the same score.
 //
-// Method, one CTA per row:
-//   1. Scores become order-preserving 32-bit keys (-0 maps to +0, so both zeros tie).
-//   2. Radix select, most significant byte first: four histogram passes narrow a prefix until
-//      the m-th largest key is known, or until every key sharing the prefix is taken.
-//   3. Gather in index order with block-wide ballot scans: keys above the threshold first, then
-//      the lowest-index keys equal to it. This fixes the tie rule.
-//   4. Stable LSD radix sort (8-bit digits, warp match for in-round ranks) of the m selected keys
-//      descending; stability keeps equal scores in index order. Passes whose digit is constant
-//      are skipped.
+// One CTA per row. Main path (value buckets):
+//   1. min and max score of the row; if they are equal every key ties and the answer is keys
+//      0..m-1 in order.
+//   2. A monotone linear map of the score to ~n buckets (bucket 0 = highest scores), an
+//      atomic histogram, and a warp-striped exclusive scan give each bucket its output range;
+//      the bucket holding output position m-1 is the last one needed.
+//   3. The keys of the needed buckets are scattered to their ranges as 64-bit composites
+//      (score key << 32 | ~index), in any order, then each bucket (about one key on average) is
+//      insertion-sorted descending, which fixes the exact order including ties.
+// Exact fallback, for rows whose needed buckets hold more than kBinCap keys (heavy exact ties)
+// or whose score range overflows: radix select of the m-th key (most significant byte first),
+// gather in index order, stable LSD radix sort.
 // Rows of up to `row_cap` keys are staged in shared memory once; longer rows are re-read from
 // global memory (L2) in each pass.
 #include "li_internal.cuh"
@@ -37,6 +40,7 @@ struct Params {
     float *out_val;
     int32_t row_cap;
     uint32_t signature;
+    size_t work_bytes;      // dynamic shared memory before the row cache
 };
 
 __device__ __forceinline__ uint32_t score_key(float v) {
@@ -53,11 +57,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
+constexpr int kBinCap = 128;          // largest bucket the per-bucket insertion sort takes
+constexpr int kBucketsMax = 4096;
+
 struct Smem {
     int32_t hist[kDigits];
     int32_t wsum[2][kWarps];
     int32_t s_digit, s_rem, s_cnt;
     int32_t s_skip[4];      // one flag per sort pass, so no pass resets a flag still being read
+    float red_min[kWarps], red_max[kWarps];
+    float s_vmin, s_vmax;
+    int32_t s_cut, s_maxbin;
 };
 
 // Block-wide exclusive scan of cnt[0..kWarps*kDigits) in place (512 threads x 8 entries).
@@ -265,10 +275,101 @@ __device__ bool sort_desc(int32_t m, uint32_t *keyA, int32_t *idxA, uint32_t *ke
     return inB;
 }
 
+template <bool kCached>
+__device__ __forceinline__ float get_val(const uint32_t *rowc, const float *src, int32_t e) {
+    if (kCached) return key_score(rowc[e]);
+    const float v = __ldg(src + e);
+    return v == 0.0f ? 0.0f : v;
+}
+
+__device__ __forceinline__ int32_t bucket_of(float v, float vmin, float scale, int32_t nb) {
+    int32_t b = (int32_t)((v - vmin) * scale);     // monotone in v
+    b = b < 0 ? 0 : (b >= nb ? nb - 1 : b);
+    return nb - 1 - b;                             // bucket 0 holds the highest scores
+}
+
+// Bucket path: writes buf[0..m) sorted descending. Returns false (uniformly) when a needed
+// bucket holds more than kBinCap keys; the caller then takes the exact radix path.
+template <bool kCached>
+__device__ bool bucket_topk(const uint32_t *rowc, const float *src, int32_t n, int32_t m,
+                            float vmin, float vmax, int32_t *hist, uint64_t *buf, Smem &sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int32_t nb = 256;
+    while (nb < n && nb < kBucketsMax) nb <<= 1;
+    const float scale = (float)nb / (vmax - vmin);
+    for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
+    if (tid == 0) { sm.s_cut = nb - 1; sm.s_maxbin = 0; }
+    __syncthreads();
+    for (int32_t e = tid; e < n; e += kThreads)
+        atomicAdd(&hist[bucket_of(get_val<kCached>(rowc, src, e), vmin, scale, nb)], 1);
+    __syncthreads();
+    // exclusive scan over buckets: each warp owns a contiguous chunk, lanes stride it
+    const int32_t chunk = nb / kWarps;
+    const int32_t base = warp * chunk;
+    int32_t part = 0;
+    for (int32_t i = lane; i < chunk; i += 32) part += hist[base + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) sm.wsum[0][warp] = part;
+    __syncthreads();
+    int32_t carry = 0;
+    for (int w = 0; w < warp; ++w) carry += sm.wsum[0][w];
+    int32_t lmax = 0;
+    for (int32_t r0 = 0; r0 < chunk; r0 += 32) {
+        const int32_t i = r0 + lane;
+        const int32_t x = i < chunk ? hist[base + i] : 0;
+        int32_t incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const int32_t start = carry + incl - x;
+        if (i < chunk) {
+            hist[base + i] = start;
+            if (start <= m - 1 && m - 1 < start + x) sm.s_cut = base + i;
+            if (start < m && x > lmax) lmax = x;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if (lane == 0 && lmax > 0) atomicMax(&sm.s_maxbin, lmax);
+    __syncthreads();
+    if (sm.s_maxbin > kBinCap) return false;
+    const int32_t cut = sm.s_cut;
+    // scatter the keys of buckets 0..cut to their ranges
+    for (int32_t e = tid; e < n; e += kThreads) {
+        const float v = get_val<kCached>(rowc, src, e);
+        const int32_t rb = bucket_of(v, vmin, scale, nb);
+        if (rb <= cut) {
+            const int32_t dst = atomicAdd(&hist[rb], 1);
+            buf[dst] = ((uint64_t)score_key(v) << 32) | (uint32_t)~(uint32_t)e;
+        }
+    }
+    __syncthreads();
+    // order each needed bucket: [end of previous bucket, end of this bucket)
+    for (int32_t rb = tid; rb <= cut; rb += kThreads) {
+        const int32_t beg = rb == 0 ? 0 : hist[rb - 1];
+        const int32_t end = hist[rb];
+        for (int32_t a = beg + 1; a < end; ++a) {
+            const uint64_t x = buf[a];
+            int32_t c = a - 1;
+            while (c >= beg && buf[c] < x) {
+                buf[c + 1] = buf[c];
+                --c;
+            }
+            buf[c + 1] = x;
+        }
+    }
+    __syncthreads();
+    return true;
+}
+
 __global__ void __launch_bounds__(kThreads) select_kernel(Params sp) {
     const Problem &p = sp.p;
     const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(sp.meta);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool meta_ok = hdr->magic == kMetaMagic && hdr->signature == sp.signature;
     if (blockIdx.x == 0 && tid == 0) {
         set_status(&sp.ws->status, meta_ok ? hdr->status : kDevErrMetadata);
@@ -277,12 +378,15 @@ __global__ void __launch_bounds__(kThreads) select_kernel(Params sp) {
     extern __shared__ __align__(16) unsigned char dsm[];
     __shared__ Smem sm;
     const int32_t topk = p.topk;
-    uint32_t *keyA = reinterpret_cast<uint32_t *>(dsm);
+    // work area shared by the two paths, then the row cache
+    uint64_t *buf = reinterpret_cast<uint64_t *>(dsm);                       // bucket path
+    int32_t *hist = reinterpret_cast<int32_t *>(buf + topk + kBinCap);
+    uint32_t *keyA = reinterpret_cast<uint32_t *>(dsm);                      // exact path
     uint32_t *keyB = keyA + topk;
     int32_t *idxA = reinterpret_cast<int32_t *>(keyB + topk);
     int32_t *idxB = idxA + topk;
-    int32_t *cnt = idxB + topk;                                   // kWarps * kDigits
-    uint32_t *rowc = reinterpret_cast<uint32_t *>(cnt + kWarps * kDigits);
+    int32_t *cnt = idxB + topk;                                             // kWarps * kDigits
+    uint32_t *rowc = reinterpret_cast<uint32_t *>(dsm + sp.work_bytes);
 
     const int32_t r = blockIdx.x;
     int32_t pos = 0;
@@ -296,43 +400,91 @@ __global__ void __launch_bounds__(kThreads) select_kernel(Params sp) {
     const int32_t m = min(n, topk);
     int32_t *oi = sp.out_idx + (int64_t)r * topk;
     float *ov = sp.out_val ? sp.out_val + (int64_t)r * topk : nullptr;
+    const float kNegInf = -__int_as_float(0x7f800000);
 
+    // 0: all padding, 1: bucket path (buf), 2: exact path (A or B buffers), 3: all keys tie
+    int mode = 0;
     bool inB = false;
+    float vtie = 0.0f;
     if (m > 0) {
         const float *src = sp.scores + (int64_t)r * sp.ld;
         const bool cached = n <= sp.row_cap;
-        if (cached) {
-            for (int32_t e = tid; e < n; e += kThreads) rowc[e] = score_key(__ldg(src + e));
-            __syncthreads();
+        float lo = __int_as_float(0x7f800000), hi = kNegInf;
+        for (int32_t e = tid; e < n; e += kThreads) {
+            const float v = __ldg(src + e);
+            if (cached) rowc[e] = score_key(v);
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
         }
-        uint32_t prefix = 0u, mask = 0u;
-        int32_t need = m;
-        if (m < n) {
-            if (cached) radix_select<true>(rowc, src, n, m, sm, prefix, mask, need);
-            else radix_select<false>(rowc, src, n, m, sm, prefix, mask, need);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
         }
-        if (cached) gather<true>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
-        else gather<false>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
+        if (lane == 0) { sm.red_min[warp] = lo; sm.red_max[warp] = hi; }
         __syncthreads();
-        inB = sort_desc(m, keyA, idxA, keyB, idxB, cnt, sm);
+        float vmin = sm.red_min[0], vmax = sm.red_max[0];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            vmin = fminf(vmin, sm.red_min[w]);
+            vmax = fmaxf(vmax, sm.red_max[w]);
+        }
+        if (vmin == vmax) {
+            mode = 3;
+            vtie = vmin == 0.0f ? 0.0f : vmin;
+        } else {
+            bool done = false;
+            if (vmax - vmin < __int_as_float(0x7f800000)) {
+                done = cached ? bucket_topk<true>(rowc, src, n, m, vmin, vmax, hist, buf, sm)
+                              : bucket_topk<false>(rowc, src, n, m, vmin, vmax, hist, buf, sm);
+            }
+            if (done) {
+                mode = 1;
+            } else {
+                mode = 2;
+                uint32_t prefix = 0u, mask = 0u;
+                int32_t need = m;
+                if (m < n) {
+                    if (cached) radix_select<true>(rowc, src, n, m, sm, prefix, mask, need);
+                    else radix_select<false>(rowc, src, n, m, sm, prefix, mask, need);
+                }
+                if (cached) gather<true>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
+                else gather<false>(rowc, src, n, m, prefix, mask, need, keyA, idxA, sm);
+                __syncthreads();
+                inB = sort_desc(m, keyA, idxA, keyB, idxB, cnt, sm);
+            }
+        }
     }
     const uint32_t *kf = inB ? keyB : keyA;
     const int32_t *jf = inB ? idxB : idxA;
     for (int32_t s = tid; s < topk; s += kThreads) {
+        int32_t id = -1;
+        float v = kNegInf;
         if (s < m) {
-            oi[s] = jf[s] + off;
-            if (ov) ov[s] = key_score(kf[s]);
-        } else {
-            oi[s] = -1;
-            if (ov) ov[s] = -__int_as_float(0x7f800000);
+            if (mode == 1) {
+                const uint64_t x = buf[s];
+                id = (int32_t)~(uint32_t)x + off;
+                v = key_score((uint32_t)(x >> 32));
+            } else if (mode == 2) {
+                id = jf[s] + off;
+                v = key_score(kf[s]);
+            } else {
+                id = s + off;
+                v = vtie;
+            }
         }
+        oi[s] = id;
+        if (ov) ov[s] = v;
     }
 }
 
 }  // namespace
 
-static size_t select_smem_bytes(int topk, int row_cap) {
-    return (size_t)4 * topk * 4 + (size_t)kWarps * kDigits * 4 + (size_t)row_cap * 4;
+// Bytes of the work area shared by the bucket path and the exact path.
+static size_t select_work_bytes(int topk) {
+    const size_t bucket = (size_t)(topk + kBinCap) * 8 + (size_t)kBucketsMax * 4;
+    const size_t exact = (size_t)4 * topk * 4 + (size_t)kWarps * kDigits * 4;
+    return align_up(bucket > exact ? bucket : exact, 16);
 }
 
 cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
@@ -340,15 +492,16 @@ cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta,
                           cudaStream_t st) {
     if (p.rows <= 0) return cudaSuccess;
     constexpr int64_t kSmemLimit = 227 * 1024 - (int64_t)sizeof(Smem) - 1024;
-    const int64_t cap = (kSmemLimit - (int64_t)select_smem_bytes(p.topk, 0)) / 4 / 32 * 32;
+    const size_t work = select_work_bytes(p.topk);
+    const int64_t cap = (kSmemLimit - (int64_t)work) / 4 / 32 * 32;
     const int64_t want = ((int64_t)(p.max_seqlen_k > 0 ? p.max_seqlen_k : 1) + 31) / 32 * 32;
     const int32_t row_cap = (int32_t)(want < cap ? want : (cap > 0 ? cap : 0));
-    const size_t smem = select_smem_bytes(p.topk, row_cap);
+    const size_t smem = work + (size_t)row_cap * 4;
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     Params sp{p, meta, ws, scores, ld, out_idx, out_val, row_cap,
-              problem_signature(p, s.tq, s.kc)};
+              problem_signature(p, s.tq, s.kc), work};
     select_kernel<<<p.rows, kThreads, smem, st>>>(sp);
     return cudaGetLastError();
 }

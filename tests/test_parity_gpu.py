@@ -178,3 +178,16 @@ def test_full_size_sampled(orc, name):
     rows = parity.sample_rows(pb, n, seed=1, must=must)
     gi, gv = run(pb)
     parity.check(orc, pb, gi, gv, rows=rows, label=name)
+
+
+# ---- the two score kernels agree ------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "paged_bs64", "tnd_varlen"])
+def test_cuda_core_score_kernel_matches_tensor_core(orc, name, monkeypatch):
+    """LI_SCORE_KERNEL=simple selects the CUDA-core score kernel (a debugging path); both
+    kernels must produce outputs that agree under the parity tolerance."""
+    pb = SMALL[name]()
+    a = run(pb)
+    monkeypatch.setenv("LI_SCORE_KERNEL", "simple")
+    b = run(pb)
+    parity.check_pair(orc, pb, a[0], a[1], b[0], b[1], label=name)
