@@ -169,19 +169,27 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     S.tq = li::kMaxHeads * 4 / P.n_heads;           // 256 / N1
     if (S.tq > 128) S.tq = 128;
     if (S.tq < 1) S.tq = 1;
+    // a query block never spans batches, so it needs no more rows than the longest batch has
+    // (decode: one row, MMA N = N1 instead of 256)
+    if (P.max_seqlen_q > 0 && S.tq > P.max_seqlen_q) S.tq = P.max_seqlen_q;
     int64_t qblocks = (int64_t)P.batch * ((P.q_len + S.tq - 1) / S.tq);
     if (P.layout_q == LI_LAYOUT_TND) {
         qblocks = (rows + S.tq - 1) / S.tq + P.batch;
         if (qblocks > rows) qblocks = rows;
     }
     S.kc = 0;
-    const int64_t target = 4LL * sm_count();
+    // too few query blocks to fill the GPU (decode): split the key ranges so that there are
+    // about eight items per SM for the dynamic scheduler to balance
+    const int64_t target = 8LL * sm_count();
     if (qblocks < 2LL * sm_count() && P.max_seqlen_k >= 2048) {
         int64_t kc = ((int64_t)P.max_seqlen_k * (qblocks > 0 ? qblocks : 1) + target - 1) / target;
         kc = (kc + li::kKeyTile - 1) / li::kKeyTile * li::kKeyTile;
-        if (kc < 1024) kc = 1024;
+        if (kc < 512) kc = 512;
         if (kc < P.max_seqlen_k) S.kc = (int)kc;
     }
+    // dense BSND with no seqused and no key split: the work list has a closed form
+    S.dense = (P.layout_q == LI_LAYOUT_BSND && P.layout_k == LI_LAYOUT_BSND && !P.seqused_q &&
+               !P.seqused_k && S.kc == 0 && P.max_seqlen_k == P.k_len) ? 1 : 0;
     const int64_t splits = S.kc > 0 ? ((int64_t)P.max_seqlen_k + S.kc - 1) / S.kc : 1;
     const int64_t max_items = qblocks * splits;
     if (max_items > INT32_MAX / 2) return fail(LI_ERR_UNSUPPORTED, "schedule too large");
@@ -190,8 +198,7 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
 }
 
 size_t scores_ld(const li::Problem &p) {
-    const size_t mk = p.max_seqlen_k > 0 ? (size_t)p.max_seqlen_k : 1;
-    return li::align_up(mk, 4);
+    return (size_t)li::scores_row_floats(p.max_seqlen_k, p.topk);
 }
 
 size_t indexer_ws_bytes(const li::Problem &p, const li::Schedule &s) {
@@ -273,7 +280,11 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "workspace clear: %s", cudaGetErrorString(e));
     if (p.rows == 0) return ok();
     const void *meta = metadata;
-    if (!meta) {
+    if (!meta && s.dense) {
+        stage_mark(0, cs);          // no schedule kernel: the stage is empty
+        stage_mark(1, cs);
+    }
+    if (!meta && !s.dense) {
         stage_mark(0, cs);
         e = li::launch_metadata(p, s, inline_meta, cs);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "metadata launch: %s", cudaGetErrorString(e));

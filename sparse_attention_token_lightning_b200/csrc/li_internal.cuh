@@ -62,7 +62,8 @@ static_assert(sizeof(WorkItem) == 32, "WorkItem size");
 struct WsHeader {
     uint32_t status;       // LI_DEVERR_* bits of the last li_indexer on this workspace
     int32_t sched_next;    // dynamic scheduler ticket counter
-    int32_t pad[62];
+    int32_t exact_rows;    // rows the selection finished on its exact (tie-heavy) fallback path
+    int32_t pad[61];
 };
 static_assert(sizeof(WsHeader) == 256, "WsHeader size");
 
@@ -106,6 +107,13 @@ struct Problem {
     int32_t rows;                          // B*S1 or T1
 };
 
+// fp32 elements per score row of the workspace (16-byte aligned rows).
+__host__ __device__ inline int64_t scores_row_floats(int32_t max_seqlen_k, int32_t topk) {
+    (void)topk;
+    const int64_t ld = max_seqlen_k > 0 ? max_seqlen_k : 1;
+    return (ld + 3) / 4 * 4;
+}
+
 // Signature of the scalar arguments a schedule depends on.
 __host__ __device__ inline uint32_t problem_signature(const Problem &p, int tq, int kc) {
     uint32_t h = 2166136261u;
@@ -122,7 +130,56 @@ struct Schedule {
     int tq;          // query rows per item
     int kc;          // key-range split (0 = none)
     int max_items;   // capacity of the item list
+    int dense;       // 1: dense BSND without seqused and without key split; the work list is a
+                     //    closed-form function of the item number and needs no schedule kernel
 };
+
+// Work list and per-batch lengths as the kernels see them: either the schedule built by
+// li_metadata (a MetaHeader in device memory) or, for dense BSND problems, closed forms.
+struct SchedView {
+    const void *meta;      // nullptr: dense closed forms
+    int32_t tq;
+    int32_t n_items;
+    int32_t nqb;           // dense: query blocks per batch
+
+    __device__ BatchInfo batch(const Problem &p, int32_t b) const {
+        if (meta) return meta_batches(meta)[b];
+        BatchInfo bi;
+        bi.L1 = bi.L1u = p.q_len;
+        bi.L2 = p.k_len;
+        bi.q_row0 = b * p.q_len;
+        bi.k_row0 = b * p.k_len;
+        bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
+        return bi;
+    }
+    // Item t of the list (0 <= t < n_items). Dense: query blocks last-to-first (for the causal
+    // mask that is longest first), batches interleaved; an item whose window is empty has
+    // j1 <= j0 and is skipped by the caller.
+    __device__ WorkItem item(const Problem &p, int32_t t) const {
+        const int32_t hb = meta ? reinterpret_cast<const MetaHeader *>(meta)->batch : 0;
+        if (meta) return meta_items(meta, hb)[t];
+        WorkItem it;
+        const int32_t qb = nqb - 1 - t / p.batch;
+        it.b = t % p.batch;
+        it.q0 = qb * tq;
+        it.nq = min(tq, p.q_len - it.q0);
+        it.j0 = 0;
+        it.j1 = window_hi(p.mask_mode, it.q0 + it.nq - 1, p.q_len, p.k_len);
+        it.cost = 0;
+        it.pad[0] = it.pad[1] = 0;
+        return it;
+    }
+};
+
+// Builds the view for a kernel launch. meta == nullptr selects the dense closed forms.
+inline SchedView make_view(const Problem &p, const Schedule &s, const void *meta) {
+    SchedView v;
+    v.meta = meta;
+    v.tq = s.tq;
+    v.nqb = p.q_len > 0 ? (p.q_len + s.tq - 1) / s.tq : 0;
+    v.n_items = meta ? 0 : p.batch * v.nqb;   // with metadata the count is read on the device
+    return v;
+}
 
 // Device-side: batch of a global query row (TND: binary search in cu_seqlens_q).
 __device__ inline int32_t row_batch(const Problem &p, int32_t r, int32_t *pos) {
@@ -167,6 +224,7 @@ void set_last_error(const char *msg);
 cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st);
 cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
                                 WsHeader *ws, float *scores, int64_t ld, cudaStream_t st);
+// (meta == nullptr in the score and select launchers selects the dense closed-form schedule)
 cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
                           const float *scores, int64_t ld, int32_t *out_idx, float *out_val,
                           cudaStream_t st);

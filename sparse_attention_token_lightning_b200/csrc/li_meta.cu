@@ -28,28 +28,51 @@ __device__ inline int item_cost(int32_t j0, int32_t j1) {
     return c < kCostBins ? c : kCostBins - 1;
 }
 
-// Enumerate the items of batch b for the lanes of one warp; f(item) is called once per item.
+// Enumerate the items of query block qb of batch b; f(item) is called once per item.
 template <class F>
-__device__ inline void for_items_of_batch(const Problem &p, const Schedule &s, int32_t b,
-                                          const BatchInfo &bi, int lane, F &&f) {
-    const int32_t nqb = (bi.L1u + s.tq - 1) / s.tq;
-    for (int32_t qb = lane; qb < nqb; qb += 32) {
-        WorkItem it;
-        it.b = b;
-        it.q0 = qb * s.tq;
-        it.nq = min(s.tq, bi.L1u - it.q0);
-        // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
-        const int32_t jend = window_hi(p.mask_mode, it.q0 + it.nq - 1, bi.L1u, bi.L2);
-        if (jend <= 0) continue;
-        const int32_t kc = s.kc > 0 ? s.kc : jend;
-        for (int32_t j0 = 0; j0 < jend; j0 += kc) {
-            it.j0 = j0;
-            it.j1 = min(jend, j0 + kc);
-            it.cost = item_cost(it.j0, it.j1);
-            it.pad[0] = it.pad[1] = 0;
-            f(it);
-        }
+__device__ inline void for_items_of_block(const Problem &p, const Schedule &s, int32_t b,
+                                          const BatchInfo &bi, int32_t qb, F &&f) {
+    WorkItem it;
+    it.b = b;
+    it.q0 = qb * s.tq;
+    it.nq = min(s.tq, bi.L1u - it.q0);
+    // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
+    const int32_t jend = window_hi(p.mask_mode, it.q0 + it.nq - 1, bi.L1u, bi.L2);
+    if (jend <= 0) return;
+    const int32_t kc = s.kc > 0 ? s.kc : jend;
+    for (int32_t j0 = 0; j0 < jend; j0 += kc) {
+        it.j0 = j0;
+        it.j1 = min(jend, j0 + kc);
+        it.cost = item_cost(it.j0, it.j1);
+        it.pad[0] = it.pad[1] = 0;
+        f(it);
     }
+}
+
+// Block-wide inclusive scan of one value per thread (kMetaThreads threads).
+__device__ inline int32_t block_inclusive_scan(int32_t x, int32_t *warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t incl = x;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sums[w];
+    __syncthreads();
+    return before + incl;
+}
+
+// Batch of global query block g: the last batch whose first block is <= g.
+__device__ inline int32_t batch_of_block(const BatchInfo *binfo, int32_t batch, int32_t g) {
+    int32_t lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi + 1) >> 1;
+        if (binfo[mid].pad[1] <= g) lo = mid; else hi = mid - 1;
+    }
+    return lo;
 }
 
 __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
@@ -123,21 +146,42 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     }
     __syncthreads();
 
-    const int warp = tid >> 5, lane = tid & 31;
-    constexpr int kWarps = kMetaThreads / 32;
+    // ---- query blocks per batch and their global numbering ------------------------------------
+    __shared__ int32_t warp_sums[kMetaThreads / 32];
+    int32_t carry = 0;
+    for (int32_t b0 = 0; b0 < p.batch; b0 += kMetaThreads) {
+        const int32_t b = b0 + tid;
+        const int32_t nqb = b < p.batch ? (binfo[b].L1u + s.tq - 1) / s.tq : 0;
+        const int32_t incl = block_inclusive_scan(nqb, warp_sums);
+        if (b < p.batch) {
+            binfo[b].pad[0] = nqb;
+            binfo[b].pad[1] = carry + incl - nqb;
+        }
+        __syncthreads();
+        if (tid == kMetaThreads - 1) warp_sums[0] = incl;       // block total
+        __syncthreads();
+        carry += warp_sums[0];
+        __syncthreads();
+    }
+    const int32_t n_blocks = carry;
+    __syncthreads();
 
     // ---- pass 1: cost histogram ---------------------------------------------------------------
-    for (int32_t b = warp; b < p.batch; b += kWarps) {
+    int32_t mine = 0;
+    for (int32_t g = tid; g < n_blocks; g += kMetaThreads) {
+        const int32_t b = batch_of_block(binfo, p.batch, g);
         const BatchInfo bi = binfo[b];
-        for_items_of_batch(p, s, b, bi, lane, [&](const WorkItem &it) {
+        for_items_of_block(p, s, b, bi, g - bi.pad[1], [&](const WorkItem &it) {
             atomicAdd(&hist[it.cost], 1);
-            atomicAdd(&s_total, 1);
+            ++mine;
         });
     }
+    atomicAdd(&s_total, mine);
     __syncthreads();
 
     // ---- descending exclusive scan of the histogram: cursor[c] = items with cost > c ----------
-    if (warp == 0) {
+    if (tid < 32) {
+        const int lane = tid;
         // each lane owns kCostBins/32 consecutive bins; highest bins first
         constexpr int per = kCostBins / 32;
         int32_t local = 0;
@@ -160,9 +204,10 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
 
     // ---- pass 2: placement --------------------------------------------------------------------
     const int32_t cap = s.max_items;
-    for (int32_t b = warp; b < p.batch; b += kWarps) {
+    for (int32_t g = tid; g < n_blocks; g += kMetaThreads) {
+        const int32_t b = batch_of_block(binfo, p.batch, g);
         const BatchInfo bi = binfo[b];
-        for_items_of_batch(p, s, b, bi, lane, [&](const WorkItem &it) {
+        for_items_of_block(p, s, b, bi, g - bi.pad[1], [&](const WorkItem &it) {
             const int32_t slot = atomicAdd(&hist[it.cost], 1);
             if (slot < cap) items[slot] = it;
         });

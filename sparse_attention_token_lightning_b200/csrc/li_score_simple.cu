@@ -16,7 +16,7 @@ constexpr int kThreads = 256;
 
 struct Params {
     Problem p;
-    const void *meta;
+    SchedView view;
     WsHeader *ws;
     float *scores;
     int64_t ld;
@@ -25,14 +25,16 @@ struct Params {
 
 __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
     const Problem &p = sp.p;
-    const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(sp.meta);
-    if (hdr->magic != kMetaMagic || hdr->signature != sp.signature) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) set_status(&sp.ws->status, kDevErrMetadata);
-        return;
+    const SchedView &view = sp.view;
+    int n_items = view.n_items;
+    if (view.meta) {
+        const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(view.meta);
+        if (hdr->magic != kMetaMagic || hdr->signature != sp.signature) {
+            if (threadIdx.x == 0 && blockIdx.x == 0) set_status(&sp.ws->status, kDevErrMetadata);
+            return;
+        }
+        n_items = hdr->n_items;
     }
-    const BatchInfo *binfo = meta_batches(sp.meta);
-    const WorkItem *items = meta_items(sp.meta, hdr->batch);
-    const int n_items = hdr->n_items;
     const int H = p.n_heads;
 
     __shared__ float qs[kMaxHeads][kHeadDim];
@@ -40,8 +42,9 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
     uint32_t err = 0;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const WorkItem it = items[item];
-        const BatchInfo bi = binfo[it.b];
+        const WorkItem it = view.item(p, item);
+        if (it.j1 <= it.j0) continue;
+        const BatchInfo bi = view.batch(p, it.b);
         for (int r = 0; r < it.nq; ++r) {
             const int32_t i = it.q0 + r;
             const int64_t row = (int64_t)bi.q_row0 + i;
@@ -89,7 +92,7 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
 
 cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
                                 WsHeader *ws, float *scores, int64_t ld, cudaStream_t st) {
-    Params sp{p, meta, ws, scores, ld, problem_signature(p, s.tq, s.kc)};
+    Params sp{p, make_view(p, s, meta), ws, scores, ld, problem_signature(p, s.tq, s.kc)};
     int grid = s.max_items < 148 * 8 ? s.max_items : 148 * 8;
     if (grid < 1) grid = 1;
     score_simple_kernel<<<grid, kThreads, 0, st>>>(sp);

@@ -64,7 +64,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct TcParams {
     Problem p;
-    const void *meta;
+    SchedView view;
     WsHeader *ws;
     float *scores;
     int64_t ld;
@@ -226,8 +226,7 @@ __device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
 
 // ---- roles ---------------------------------------------------------------------------------
 __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
-                         uint8_t *smem, const Bars &bars, volatile int *abort_flag,
-                         const BatchInfo *binfo, const WorkItem *items, int n_items) {
+                         uint8_t *smem, const Bars &bars, volatile int *abort_flag, int n_items) {
     const int lane = threadIdx.x & 31;
     const uint32_t sbase = smem_u32(smem);
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
@@ -238,16 +237,21 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
     for (int it = 0; ok; ++it) {
         const int sl = it % kSlots;
         if (!mbar_wait(bars.sl_empty(sl), ((it / kSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        // next non-empty item (the dense closed forms can yield items with an empty window)
         int ticket = 0;
-        if (lane == 0) ticket = atomicAdd(&P.ws->sched_next, 1);
-        ticket = __shfl_sync(0xffffffffu, ticket, 0);
-        const bool valid = ticket < n_items;
-        Slot &S = slots[sl];
         WorkItem wi{};
+        bool valid = false;
+        for (;;) {
+            if (lane == 0) ticket = atomicAdd(&P.ws->sched_next, 1);
+            ticket = __shfl_sync(0xffffffffu, ticket, 0);
+            if (ticket >= n_items) break;
+            wi = P.view.item(P.p, ticket);
+            if (wi.j1 > wi.j0) { valid = true; break; }
+        }
+        Slot &S = slots[sl];
         BatchInfo bi{};
         if (valid) {
-            wi = items[ticket];
-            bi = binfo[wi.b];
+            bi = P.view.batch(P.p, wi.b);
             const int64_t wbase = ((int64_t)bi.q_row0 + wi.q0) * N1;
             const int nw = wi.nq * N1;
             for (int e = lane; e < kNmax; e += 32)
@@ -442,14 +446,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (threadIdx.x == 0) set_status(&P.ws->status, kDevErrInternal);
         return;
     }
-    const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(P.meta);
-    if (hdr->magic != kMetaMagic || hdr->signature != P.signature) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) set_status(&P.ws->status, kDevErrMetadata);
-        return;
+    int n_items = P.view.n_items;
+    if (P.view.meta) {
+        const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(P.view.meta);
+        if (hdr->magic != kMetaMagic || hdr->signature != P.signature) {
+            if (threadIdx.x == 0 && blockIdx.x == 0) set_status(&P.ws->status, kDevErrMetadata);
+            return;
+        }
+        n_items = hdr->n_items;
     }
-    const int n_items = hdr->n_items;
-    const BatchInfo *binfo = meta_batches(P.meta);
-    const WorkItem *items = meta_items(P.meta, hdr->batch);
 
     Bars bars{sbase + kBarOff};
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff);
@@ -486,7 +491,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag, binfo, items, n_items);
+        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag, n_items);
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);
         __syncwarp();
@@ -554,7 +559,7 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     if (s.max_items <= 0 || p.rows <= 0) return cudaSuccess;
     TcParams P{};
     P.p = p;
-    P.meta = meta;
+    P.view = make_view(p, s, meta);
     P.ws = ws;
     P.scores = scores;
     P.ld = ld;

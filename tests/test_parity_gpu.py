@@ -29,6 +29,17 @@ def run(pb, **kw):
     return (parity.as_rows(idx, pb.topk), None if val is None else parity.as_rows(val, pb.topk))
 
 
+def run_counting_fallbacks(pb):
+    """Like run(), also returning how many rows the selection finished on its exact fallback
+    path (read from the workspace header, third int32)."""
+    g = pb.to("cuda")
+    ws = li.empty_workspace(li.make_args(g), "cuda")
+    idx, val = li.indexer(g, workspace=ws)
+    torch.cuda.synchronize()
+    exact_rows = int(ws[8:12].view(torch.int32).item())
+    return parity.as_rows(idx, pb.topk), parity.as_rows(val, pb.topk), exact_rows
+
+
 # ---- small problems, every row ------------------------------------------------------------------
 
 SMALL = {
@@ -49,6 +60,7 @@ SMALL = {
     "paged_bs1": lambda: synthetic.paged([37, 3], 1, 4, 8, block_size=1, seed=12),
     "topk1": lambda: synthetic.bsnd(1, 64, 200, 8, 1, 3, seed=13),
     "topk8192": lambda: synthetic.bsnd(1, 8, 9000, 2, 8192, 0, seed=14),
+    "topk8192_n16": lambda: synthetic.bsnd(1, 4, 9000, 16, 8192, 0, seed=45),
     "offset_seqused": lambda: synthetic.tnd([10, 30], [60, 90], 4, 40, 3, seed=15,
                                             seqused_q=[7, 30], output_idx_offset=[1000, 5]),
 }
@@ -87,6 +99,17 @@ def test_indices_only(orc):
 
 def test_separate_metadata_matches_inline():
     pb = synthetic.tnd([100, 3, 250], [100, 400, 260], 64, 64, 3, seed=31)
+    a = run(pb, metadata=False)
+    b = run(pb, metadata=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", [(2, 300, 459, 64, 200, 3), (1, 200, 150, 16, 32, 3),
+                                   (3, 64, 64, 8, 16, 0)])
+def test_dense_closed_form_schedule_matches_metadata(shape):
+    """Dense BSND problems run without a schedule kernel (closed-form work list); a schedule
+    built by li_metadata for the same call must give bit-identical outputs."""
+    pb = synthetic.bsnd(*shape, seed=46)
     a = run(pb, metadata=False)
     b = run(pb, metadata=True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
@@ -176,8 +199,39 @@ def test_full_size_sampled(orc, name):
     pb = synthetic.config(name)
     n, must = FULL[name]
     rows = parity.sample_rows(pb, n, seed=1, must=must)
-    gi, gv = run(pb)
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
     parity.check(orc, pb, gi, gv, rows=rows, label=name)
+    assert exact_rows == 0, f"{exact_rows} rows left the bucket selection paths"
+
+
+@pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "tnd_varlen", "paged_bs64",
+                                  "topk8192_n16", "paged_bs16_tnd_q", "offset_seqused"])
+def test_tie_free_rows_use_the_bucket_paths(orc, name):
+    """Random-normal scores have (almost) no exact ties, so every row must finish on the bucket
+    paths (registers for short rows, digit histogram + candidates for long rows); the exact
+    radix path is only for tie-heavy rows. Guards against a fast path silently falling back."""
+    pb = SMALL[name]()
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
+    parity.check(orc, pb, gi, gv, label=name)
+    assert exact_rows == 0
+
+
+def test_long_rows_with_small_topk(orc):
+    """Rows well past the register path (up to 12000 keys) selecting few keys: exercises the
+    long-row digit histogram, the candidate gather and the bucket sort on the candidates."""
+    pb = synthetic.tnd([3, 1, 2], [12000, 4097, 9000], 64, 100, 3, seed=44)
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
+    parity.check(orc, pb, gi, gv, label="long rows")
+    assert exact_rows == 0
+
+
+def test_tie_heavy_rows_fall_back_correctly(orc):
+    """One head and no weight: about half the keys score exactly 0, one bucket overflows, and
+    the exact radix path must produce the same answer as the oracle."""
+    pb = SMALL["bsnd_nomask_n1"]()
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
+    parity.check(orc, pb, gi, gv, label="ties")
+    assert exact_rows > 0
 
 
 # ---- the two score kernels agree ------------------------------------------------------------------
