@@ -179,8 +179,8 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     }
     S.kc = 0;
     // too few query blocks to fill the GPU (decode): split the key ranges so that there are
-    // about eight items per SM for the dynamic scheduler to balance
-    const int64_t target = 8LL * sm_count();
+    // about 32 items per SM, small enough for the dynamic scheduler to end all SMs together
+    const int64_t target = 32LL * sm_count();
     if (qblocks < 2LL * sm_count() && P.max_seqlen_k >= 2048) {
         int64_t kc = ((int64_t)P.max_seqlen_k * (qblocks > 0 ? qblocks : 1) + target - 1) / target;
         kc = (kc + li::kKeyTile - 1) / li::kKeyTile * li::kKeyTile;

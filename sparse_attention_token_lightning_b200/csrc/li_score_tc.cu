@@ -33,34 +33,38 @@ namespace li {
 namespace {
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kStages = 3;
+constexpr int kSchedWarp = 2 + kEpiWarps;               // warp 10
+constexpr int kThreads = 32 * (3 + kEpiWarps);
+constexpr int kMaxStages = 8;
 constexpr int kSlots = 2;
 constexpr int kNmax = 256;
-constexpr uint32_t kQHalfBytes = kNmax * 128;            // 256 rows x 64 bf16
-constexpr uint32_t kQBufBytes = 2 * kQHalfBytes;         // both K halves
 constexpr uint32_t kKHalfBytes = kKeyTile * 128;         // 128 keys x 64 bf16
 constexpr uint32_t kKStageBytes = 2 * kKHalfBytes;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = 256;
+constexpr int kMaxAcc = 8;                               // TMEM accumulators (512 / stride)
 constexpr uint32_t kDevErrInternal = 0x20u;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 struct Slot {
-    int32_t valid, b, q0, nq, j0, j1, row0, L1u, L2;
-    int32_t pad[7];
+    int32_t valid, b, q0, nq, j0, j1, row0, L1u, L2, k_row0;
+    int32_t pad[6];
+    int32_t tbl[32];      // paged: block-table entries of the item's first 32 blocks
     float w[kNmax];
 };
-static_assert(sizeof(Slot) == 64 + 4 * kNmax, "Slot size");
+static_assert(sizeof(Slot) == 64 + 128 + 4 * kNmax, "Slot size");
 
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kKOff = kQOff + 2 * kQBufBytes;
-constexpr uint32_t kSlotOff = kKOff + kStages * kKStageBytes;
+// Shared memory: [Q buffers x2 | K stages][tail: slots, barriers, flags]. The Q buffers take
+// 2 x (2 halves x N x 128 B); the K ring gets as many 32 KB stages as fit before the tail, so
+// small N (decode) gets a deeper key pipeline.
+constexpr uint32_t kSmemBytes = 232448;
+constexpr int kNumBars = 2 * kMaxStages + 2 * 2 + 2 * kMaxAcc + 2 * kSlots;
+constexpr uint32_t kTailBytes = 2816;
+constexpr uint32_t kTailOff = kSmemBytes - kTailBytes;
+constexpr uint32_t kSlotOff = kTailOff;
 constexpr uint32_t kBarOff = kSlotOff + kSlots * sizeof(Slot);
-constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 * 2 + 2 * kSlots;
 constexpr uint32_t kFlagOff = kBarOff + 8 * kNumBars;
-constexpr uint32_t kSmemBytes = kFlagOff + 16;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kFlagOff + 16 <= kSmemBytes, "shared memory tail");
+static_assert(kTailOff % 16 == 0, "tail alignment");
 
 struct TcParams {
     Problem p;
@@ -73,6 +77,11 @@ struct TcParams {
     int32_t tq;           // query rows per item
     uint32_t idesc;       // tcgen05 instruction descriptor
     int32_t piece_rows;   // paged: keys per TMA load (min(block_size, 128)); 0 for dense keys
+    int32_t stages;       // K ring depth
+    int32_t n_acc;        // TMEM accumulators in use
+    uint32_t acc_stride;  // TMEM columns per accumulator (power of two >= N)
+    uint32_t q_half;      // bytes of one 64-wide half of a Q buffer (N x 128)
+    uint32_t k_off;       // start of the K ring (after the two Q buffers)
 };
 
 // ---- PTX wrappers --------------------------------------------------------------------------
@@ -144,14 +153,23 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
+// MMA with a compile-time accumulate flag (no predicate set-up on the issue path).
+template <bool kAccumulate>
+__device__ __forceinline__ void umma_bf16_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc) {
+    if constexpr (kAccumulate) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 1;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc)
+            : "memory");
+    }
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -211,13 +229,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 struct Bars {
     uint32_t base;
     __device__ uint32_t k_full(int s) const { return base + 8 * s; }
-    __device__ uint32_t k_empty(int s) const { return base + 8 * (kStages + s); }
-    __device__ uint32_t q_full(int i) const { return base + 8 * (2 * kStages + i); }
-    __device__ uint32_t q_empty(int i) const { return base + 8 * (2 * kStages + 2 + i); }
-    __device__ uint32_t acc_full(int i) const { return base + 8 * (2 * kStages + 4 + i); }
-    __device__ uint32_t acc_empty(int i) const { return base + 8 * (2 * kStages + 6 + i); }
-    __device__ uint32_t sl_full(int i) const { return base + 8 * (2 * kStages + 8 + i); }
-    __device__ uint32_t sl_empty(int i) const { return base + 8 * (2 * kStages + 8 + kSlots + i); }
+    __device__ uint32_t k_empty(int s) const { return base + 8 * (kMaxStages + s); }
+    __device__ uint32_t q_full(int i) const { return base + 8 * (2 * kMaxStages + i); }
+    __device__ uint32_t q_empty(int i) const { return base + 8 * (2 * kMaxStages + 2 + i); }
+    __device__ uint32_t acc_full(int i) const { return base + 8 * (2 * kMaxStages + 4 + i); }
+    __device__ uint32_t acc_empty(int i) const { return base + 8 * (2 * kMaxStages + 4 + kMaxAcc + i); }
+    __device__ uint32_t sl_full(int i) const { return base + 8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + i); }
+    __device__ uint32_t sl_empty(int i) const {
+        return base + 8 * (2 * kMaxStages + 4 + 2 * kMaxAcc + kSlots + i);
+    }
+};
+
+// Position in a ring of n buffers: index and phase parity, advanced without division.
+struct RingPos {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++idx == n) { idx = 0; phase ^= 1u; }
+    }
 };
 
 __device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
@@ -225,14 +254,14 @@ __device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
 }
 
 // ---- roles ---------------------------------------------------------------------------------
-__device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
-                         uint8_t *smem, const Bars &bars, volatile int *abort_flag, int n_items) {
+// Scheduler warp: takes tickets and stages each non-empty item (header, w, first block-table
+// entries) in the slot ring ahead of the producer, so item set-up latency stays off the
+// key-streaming path.
+__device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
+                          volatile int *abort_flag, int n_items) {
     const int lane = threadIdx.x & 31;
-    const uint32_t sbase = smem_u32(smem);
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
     const int N1 = P.p.n_heads;
-    uint32_t err = 0;
-    int kcount = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it % kSlots;
@@ -249,60 +278,107 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             if (wi.j1 > wi.j0) { valid = true; break; }
         }
         Slot &S = slots[sl];
-        BatchInfo bi{};
         if (valid) {
-            bi = P.view.batch(P.p, wi.b);
+            const BatchInfo bi = P.view.batch(P.p, wi.b);
             const int64_t wbase = ((int64_t)bi.q_row0 + wi.q0) * N1;
             const int nw = wi.nq * N1;
             for (int e = lane; e < kNmax; e += 32)
                 S.w[e] = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+            if (P.piece_rows) {
+                const int32_t bidx = wi.j0 / P.p.block_size + lane;
+                S.tbl[lane] = (int64_t)bidx * P.p.block_size < wi.j1
+                                  ? P.p.block_table[(int64_t)wi.b * P.p.bt_stride + bidx] : -1;
+            }
             if (lane == 0) {
                 S.b = wi.b; S.q0 = wi.q0; S.nq = wi.nq; S.j0 = wi.j0; S.j1 = wi.j1;
-                S.row0 = bi.q_row0 + wi.q0; S.L1u = bi.L1u; S.L2 = bi.L2;
+                S.row0 = bi.q_row0 + wi.q0; S.L1u = bi.L1u; S.L2 = bi.L2; S.k_row0 = bi.k_row0;
             }
         }
         if (lane == 0) S.valid = valid ? 1 : 0;
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.sl_full(sl));
         if (!valid) break;
+    }
+    if (!ok) *abort_flag = 1;
+}
 
+// TMA producer warp: per staged item, the Q tile (double buffered) and the K tiles of its key
+// range through the ring; paged keys block by block through the block table.
+__device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
+                         uint8_t *smem, const Bars &bars, volatile int *abort_flag) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(smem);
+    Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
+    const int N1 = P.p.n_heads;
+    uint32_t err = 0;
+    RingPos kr;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+        const int sl = it % kSlots;
+        if (!mbar_wait(bars.sl_full(sl), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
+        const Slot &S = slots[sl];
+        const int valid = S.valid;
+        const int32_t b = S.b, q0 = S.q0, j0 = S.j0, j1 = S.j1, row0 = S.row0, k_row0 = S.k_row0;
+        int32_t tbl_val = S.tbl[lane];
+        __syncwarp();
+        if (!valid) {
+            if (lane == 0) mbar_arrive(bars.sl_empty(sl));
+            break;
+        }
+        (void)q0;
         // Q tile of the item (all heads of tq rows): two TMA loads, one per 64-wide K half.
         const int qb = it & 1;
         if (!mbar_wait(bars.q_empty(qb), ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         if (lane == 0) {
-            const uint32_t qdst = sbase + kQOff + qb * kQBufBytes;
-            const int32_t y = (bi.q_row0 + wi.q0) * N1;
-            mbar_arrive_expect_tx(bars.q_full(qb), 2u * P.N * 128u);
+            const uint32_t qdst = sbase + qb * 2u * P.q_half;
+            const int32_t y = row0 * N1;
+            mbar_arrive_expect_tx(bars.q_full(qb), 2u * P.q_half);
             tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
-            tma_load_2d(qdst + kQHalfBytes, tmq, bars.q_full(qb), 64, y);
+            tma_load_2d(qdst + P.q_half, tmq, bars.q_full(qb), 64, y);
         }
-        // K tiles of the item's key range.
-        const int32_t nt = n_tiles_of(wi.j0, wi.j1);
-        for (int32_t tile = 0; tile < nt; ++tile, ++kcount) {
-            const int st = kcount % kStages;
-            if (!mbar_wait(bars.k_empty(st), ((kcount / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-            if (lane == 0) {
-                const int32_t jt = wi.j0 + tile * kKeyTile;
-                const uint32_t kdst = sbase + kKOff + st * kKStageBytes;
-                if (P.piece_rows == 0) {
+        // K tiles of the item's key range. Paged keys: the warp keeps 32 block-table entries
+        // in registers (lane l holds entry tbl_base + l), the first 32 staged by the scheduler,
+        // later ones refilled 32 at a time.
+        const int32_t nt = n_tiles_of(j0, j1);
+        const int32_t bs = P.p.block_size;
+        int32_t tbl_base = P.piece_rows ? j0 / bs : 0;
+        for (int32_t tile = 0; tile < nt; ++tile, kr.next(P.stages)) {
+            const int st = kr.idx;
+            if (!mbar_wait(bars.k_empty(st), kr.phase ^ 1u, abort_flag)) { ok = false; break; }
+            const int32_t jt = j0 + tile * kKeyTile;
+            const uint32_t kdst = sbase + P.k_off + st * kKStageBytes;
+            if (P.piece_rows == 0) {
+                if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), kKStageBytes);
-                    tma_load_2d(kdst, tmk, bars.k_full(st), 0, bi.k_row0 + jt);
-                    tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, bi.k_row0 + jt);
-                } else {
-                    // Paged keys: one load per (part of a) block, at most 128 / piece_rows.
-                    const int pr = P.piece_rows;
-                    const int pieces = kKeyTile / pr;
-                    int32_t rows[kKeyTile / 8];
-                    int loads = 0;
-                    for (int pc = 0; pc < pieces; ++pc) {
-                        const int32_t jp = jt + pc * pr;
-                        rows[pc] = -1;
-                        if (jp >= wi.j1) continue;
-                        const int32_t blk = P.p.block_table[(int64_t)wi.b * P.p.bt_stride + jp / P.p.block_size];
-                        if (blk < 0 || blk >= P.p.num_blocks) { err |= LI_DEVERR_TABLE; continue; }
-                        rows[pc] = blk * P.p.block_size + jp % P.p.block_size;
-                        ++loads;
-                    }
+                    tma_load_2d(kdst, tmk, bars.k_full(st), 0, k_row0 + jt);
+                    tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, k_row0 + jt);
+                }
+            } else {
+                // one load per block piece: 128 / piece_rows pieces, consecutive blocks when
+                // blocks are at most 128 keys, else one piece inside block jt / bs
+                const int pr = P.piece_rows;
+                const int pieces = kKeyTile / pr;
+                const int32_t blk0 = jt / bs;
+                const int32_t nblk = bs <= kKeyTile ? pieces : 1;
+                if (blk0 < tbl_base || blk0 + nblk > tbl_base + 32) {
+                    tbl_base = blk0;
+                    const int32_t bidx = blk0 + lane;
+                    tbl_val = (int64_t)bidx * bs < j1
+                                  ? P.p.block_table[(int64_t)b * P.p.bt_stride + bidx] : -1;
+                }
+                int32_t rows[kKeyTile / 8];
+                int loads = 0;
+                for (int pc = 0; pc < pieces; ++pc) {
+                    const int32_t jp = jt + pc * pr;
+                    const int32_t blk = __shfl_sync(0xffffffffu, tbl_val,
+                                                    (bs <= kKeyTile ? blk0 + pc : blk0) - tbl_base);
+                    rows[pc] = -1;
+                    if (jp >= j1) continue;
+                    if (blk < 0 || blk >= P.p.num_blocks) { err |= LI_DEVERR_TABLE; continue; }
+                    rows[pc] = blk * bs + jp % bs;
+                    ++loads;
+                }
+                if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)loads * pr * 256u);
                     for (int pc = 0; pc < pieces; ++pc) {
                         if (rows[pc] < 0) continue;
@@ -314,6 +390,8 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             }
             __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) mbar_arrive(bars.sl_empty(sl));
     }
     if (!ok) *abort_flag = 1;
     if (lane == 0 && err) set_status(&P.ws->status, err);
@@ -323,7 +401,7 @@ __device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
                            volatile int *abort_flag, uint32_t tmem_base) {
     const uint32_t sbase = smem_u32(smem);
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
-    int kcount = 0, acount = 0;
+    RingPos kr, ar;
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it % kSlots;
@@ -335,22 +413,26 @@ __device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
         if (!valid) break;
         const int qb = it & 1;
         if (!mbar_wait(bars.q_full(qb), (it >> 1) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t qsm = sbase + kQOff + qb * kQBufBytes;
+        const uint32_t qsm = sbase + qb * 2u * P.q_half;
+        const uint64_t b0 = sw128_desc(qsm);
+        const uint64_t b_half16 = P.q_half >> 4;
         const int32_t nt = n_tiles_of(j0, j1);
-        for (int32_t tile = 0; tile < nt; ++tile, ++kcount, ++acount) {
-            const int st = kcount % kStages;
-            const int ab = acount & 1;
-            if (!mbar_wait(bars.k_full(st), (kcount / kStages) & 1, abort_flag)) { ok = false; break; }
-            if (!mbar_wait(bars.acc_empty(ab), ((acount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        for (int32_t tile = 0; tile < nt; ++tile, kr.next(P.stages), ar.next(P.n_acc)) {
+            const int st = kr.idx;
+            const int ab = ar.idx;
+            if (!mbar_wait(bars.k_full(st), kr.phase, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bars.acc_empty(ab), ar.phase ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ksm = sbase + kKOff + st * kKStageBytes;
-            const uint32_t d = tmem_base + ab * kAccCols;
+            // descriptors advance by the byte offset / 16 in their address field (no carry:
+            // shared addresses stay below 2^18 bytes)
+            const uint64_t a0 = sw128_desc(sbase + P.k_off + st * kKStageBytes);
+            const uint32_t d = tmem_base + ab * P.acc_stride;
+            umma_bf16_c<false>(d, a0, b0, P.idesc);
 #pragma unroll
-            for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-                const uint32_t half = (uint32_t)(kk >> 2), sub = (uint32_t)(kk & 3) * 32u;
-                const uint64_t adesc = sw128_desc(ksm + half * kKHalfBytes + sub);
-                const uint64_t bdesc = sw128_desc(qsm + half * kQHalfBytes + sub);
-                umma_bf16(d, adesc, bdesc, P.idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 1; kk < kHeadDim / 16; ++kk) {
+                const uint64_t a_off = ((kk >> 2) * kKHalfBytes + (kk & 3) * 32u) >> 4;
+                const uint64_t b_off = ((uint64_t)(kk >> 2) * b_half16) + (uint64_t)((kk & 3) * 2);
+                umma_bf16_c<true>(d, a0 + a_off, b0 + b_off, P.idesc);
             }
             umma_commit(bars.k_empty(st));
             umma_commit(bars.acc_full(ab));
@@ -370,7 +452,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
     const int N1 = P.p.n_heads;
     const int mask_mode = P.p.mask_mode;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
-    int acount = 0;
+    RingPos ar;
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it % kSlots;
@@ -385,13 +467,13 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
         const int32_t q0 = S.q0, nq = S.nq, j0 = S.j0, j1 = S.j1, row0 = S.row0, L1u = S.L1u,
                       L2 = S.L2;
         const int32_t nt = n_tiles_of(j0, j1);
-        for (int32_t tile = 0; tile < nt; ++tile, ++acount) {
-            const int ab = acount & 1;
-            if (!mbar_wait(bars.acc_full(ab), (acount >> 1) & 1, abort_flag)) { ok = false; break; }
+        for (int32_t tile = 0; tile < nt; ++tile, ar.next(P.n_acc)) {
+            const int ab = ar.idx;
+            if (!mbar_wait(bars.acc_full(ab), ar.phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const int32_t jt = j0 + tile * kKeyTile;
             const int32_t j = jt + 32 * quarter + lane;
-            const uint32_t acc = tmem_base + lane_addr + ab * kAccCols;
+            const uint32_t acc = tmem_base + lane_addr + ab * P.acc_stride;
             for (int t = group; t < nq; t += 2) {
                 const int32_t hi = min(window_hi(mask_mode, q0 + t, L1u, L2), j1);
                 if (jt >= hi) continue;                       // tile past this row's window
@@ -460,19 +542,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff + 4);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(bars.k_full(s), 1);
             mbar_init(bars.k_empty(s), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.q_full(i), 1);
             mbar_init(bars.q_empty(i), 1);
+        }
+        for (int i = 0; i < kMaxAcc; ++i) {
             mbar_init(bars.acc_full(i), 1);
             mbar_init(bars.acc_empty(i), kEpiWarps);
         }
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(bars.sl_full(i), 1);
-            mbar_init(bars.sl_empty(i), 1 + kEpiWarps);
+            mbar_init(bars.sl_empty(i), 2 + kEpiWarps);   // producer, MMA, epilogue warps
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -491,7 +575,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag, n_items);
+        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
+    } else if (warp == kSchedWarp) {
+        scheduler(P, smem, bars, abort_flag, n_items);
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);
         __syncwarp();
@@ -569,6 +655,15 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     if (P.N > kNmax || P.N < 16) return cudaSuccess;
     P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(P.N >> 3) << 17) |
               ((uint32_t)(128 >> 4) << 24);
+    P.q_half = (uint32_t)P.N * 128u;               // N is a multiple of 16: 1 KB aligned halves
+    P.k_off = 4u * P.q_half;
+    P.acc_stride = 32;
+    while (P.acc_stride < (uint32_t)P.N) P.acc_stride <<= 1;
+    P.n_acc = (int)(kTmemCols / P.acc_stride);
+    if (P.n_acc > kMaxAcc) P.n_acc = kMaxAcc;
+    P.stages = (int)((kTailOff - P.k_off) / kKStageBytes);
+    if (P.stages > kMaxStages) P.stages = kMaxStages;
+    if (P.stages < 2) return cudaSuccess;
     uint64_t k_rows = 0;
     if (p.layout_k == LI_LAYOUT_PA_BSND) {
         const int bs = p.block_size;
