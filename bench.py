@@ -252,6 +252,7 @@ def main():
     pb_cpu = synthetic.config(a.config, seed=rank)
     pb = pb_cpu.to(dev)
     args = li.make_args(pb)
+    plan = li.li_plan(args)
     ws = li.empty_workspace(args, dev)
     idx = torch.empty(li.out_shape(pb), dtype=torch.int32, device=dev)
     val = torch.empty(li.out_shape(pb), dtype=torch.float32, device=dev)
@@ -368,12 +369,13 @@ def main():
                        "rows_per_step_per_gpu": rows, "valid_pairs": valid_pairs(pb_cpu),
                        "l2": "flushed before every step by a 256 MB write outside the step's "
                              "CUDA events",
-                       "parallelism": f"{world} independent replicas (one problem per GPU)"},
+                       "parallelism": f"{world} independent replicas (one problem per GPU)",
+                       "schedule": {k: plan[k] for k in ("tq", "kc", "dense", "score_tc")}},
             "roofline": roofline,
             "stages_ms": {"schedule": statistics.mean(meta_ms), "score": sc,
                           "select": statistics.mean(sel_ms)},
             "tflops_whole_step": flops / (ms_per_step / 1e3) / 1e12,
-            "clocks": clk, "gpu_launches": 3 * K}
+            "clocks": clk, "gpu_launches": plan["kernels"] * K}
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and a.cpu_seconds > 0:

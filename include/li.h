@@ -130,6 +130,32 @@ li_status li_metadata_workspace_size(const li_args *args, size_t *bytes);
 li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *stream);
 
 /*
+ * li_plan -- the schedule li_indexer() will use for `args`, and how many kernels it launches.
+ * Host only; validates like li_metadata_workspace_size and dereferences no device pointer. The
+ * pages split the work per AI core inside lightning_indexer_metadata (lightning_indexer,
+ * "Function"); this reports the sm_100a counterpart's choices so callers can size graphs and
+ * count launches:
+ *   tq            query rows per work item (tq x num_heads_q <= 256 MMA columns)
+ *   kc            keys per work item, 0 when each item covers its rows' whole window
+ *   max_items     capacity of the work list
+ *   dense         1 when the work list is a closed form of the shapes and no schedule kernel runs
+ *   kernels       kernels one li_indexer call launches with metadata == NULL (0 when there are no
+ *                 query rows); one fewer schedule kernel when a metadata buffer is passed
+ *   score_tc      1 when the score step runs on the tcgen05 kernel, 0 on the CUDA-core kernel
+ *                 (paged caches whose block_size the TMA pieces cannot tile)
+ * Returns LI_OK and fills *info, or an argument error.
+ */
+typedef struct li_plan_info {
+    int32_t tq;
+    int32_t kc;
+    int32_t max_items;
+    int32_t dense;
+    int32_t kernels;
+    int32_t score_tc;
+} li_plan_info;
+li_status li_plan(const li_args *args, li_plan_info *info);
+
+/*
  * li_indexer_workspace_size -- bytes of scratch li_indexer() needs for `args`.
  * Host only; validates like li_metadata_workspace_size. The size covers the device status word,
  * the scheduler counters, room for an inline schedule, and the fp32 score rows the selection step

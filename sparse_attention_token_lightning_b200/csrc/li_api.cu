@@ -11,11 +11,6 @@
 
 #include "li_internal.cuh"
 
-namespace li {
-cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
-                            float *scores, int64_t ld, cudaStream_t st, bool *launched);
-}
-
 namespace {
 
 thread_local std::string g_err;
@@ -236,6 +231,21 @@ li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *s
         return fail(LI_ERR_WORKSPACE, "metadata buffer of %zu bytes, %zu needed", bytes, need);
     cudaError_t e = li::launch_metadata(p, s, metadata, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "metadata launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+li_status li_plan(const li_args *args, li_plan_info *info) {
+    li::Problem p;
+    li::Schedule s;
+    li_status st = validate(args, &p, &s);
+    if (st != LI_OK) return st;
+    if (!info) return fail(LI_ERR_INVALID_ARG, "info is NULL");
+    info->tq = s.tq;
+    info->kc = s.kc;
+    info->max_items = s.max_items;
+    info->dense = s.dense ? 1 : 0;
+    info->kernels = p.rows > 0 ? (s.dense ? 2 : 3) : 0;
+    info->score_tc = !use_simple_kernel() && li::score_tc_eligible(p, s) ? 1 : 0;
     return ok();
 }
 

@@ -224,6 +224,11 @@ void set_last_error(const char *msg);
 cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st);
 cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
                                 WsHeader *ws, float *scores, int64_t ld, cudaStream_t st);
+// Tensor-core score kernel: whether the problem fits it, and its launcher (*launched = false
+// when it does not, leaving the step to launch_score_simple).
+bool score_tc_eligible(const Problem &p, const Schedule &s);
+cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
+                            float *scores, int64_t ld, cudaStream_t st, bool *launched);
 // (meta == nullptr in the score and select launchers selects the dense closed-form schedule)
 cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
                           const float *scores, int64_t ld, int32_t *out_idx, float *out_val,

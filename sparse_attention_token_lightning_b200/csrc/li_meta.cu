@@ -28,25 +28,23 @@ __device__ inline int item_cost(int32_t j0, int32_t j1) {
     return c < kCostBins ? c : kCostBins - 1;
 }
 
-// Enumerate the items of query block qb of batch b; f(item) is called once per item.
-template <class F>
-__device__ inline void for_items_of_block(const Problem &p, const Schedule &s, int32_t b,
-                                          const BatchInfo &bi, int32_t qb, F &&f) {
-    WorkItem it;
-    it.b = b;
-    it.q0 = qb * s.tq;
-    it.nq = min(s.tq, bi.L1u - it.q0);
+// Item `split` of query block qb of batch b (key range [split*kc, (split+1)*kc) of the block's
+// window); returns false when the block has no such item.
+__device__ inline bool item_of_block(const Problem &p, const Schedule &s, int32_t b,
+                                     const BatchInfo &bi, int32_t qb, int32_t split, WorkItem *it) {
+    it->b = b;
+    it->q0 = qb * s.tq;
+    it->nq = min(s.tq, bi.L1u - it->q0);
     // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
-    const int32_t jend = window_hi(p.mask_mode, it.q0 + it.nq - 1, bi.L1u, bi.L2);
-    if (jend <= 0) return;
+    const int32_t jend = window_hi(p.mask_mode, it->q0 + it->nq - 1, bi.L1u, bi.L2);
     const int32_t kc = s.kc > 0 ? s.kc : jend;
-    for (int32_t j0 = 0; j0 < jend; j0 += kc) {
-        it.j0 = j0;
-        it.j1 = min(jend, j0 + kc);
-        it.cost = item_cost(it.j0, it.j1);
-        it.pad[0] = it.pad[1] = 0;
-        f(it);
-    }
+    const int64_t j0 = (int64_t)split * kc;
+    if (jend <= 0 || j0 >= jend) return false;
+    it->j0 = (int32_t)j0;
+    it->j1 = min(jend, it->j0 + kc);
+    it->cost = item_cost(it->j0, it->j1);
+    it->pad[0] = it->pad[1] = 0;
+    return true;
 }
 
 // Block-wide inclusive scan of one value per thread (kMetaThreads threads).
@@ -65,12 +63,15 @@ __device__ inline int32_t block_inclusive_scan(int32_t x, int32_t *warp_sums) {
     return before + incl;
 }
 
-// Batch of global query block g: the last batch whose first block is <= g.
-__device__ inline int32_t batch_of_block(const BatchInfo *binfo, int32_t batch, int32_t g) {
+constexpr int kSmemBatches = 2048;     // batches whose lengths and block prefix stay in smem
+
+// Batch of global query block g: the last batch whose first block is <= g (qb0 holds each
+// batch's first block, in shared memory when the batch count allows, else in global memory).
+__device__ inline int32_t batch_of_block(const int32_t *qb0, int32_t batch, int32_t g) {
     int32_t lo = 0, hi = batch - 1;
     while (lo < hi) {
         const int32_t mid = (lo + hi + 1) >> 1;
-        if (binfo[mid].pad[1] <= g) lo = mid; else hi = mid - 1;
+        if (qb0[mid] <= g) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -85,6 +86,9 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     __shared__ int32_t hist[kCostBins];
     __shared__ uint32_t s_status;
     __shared__ int32_t s_total;
+    // per-batch query rows in use, keys and first query block (B <= kSmemBatches)
+    __shared__ int32_t s_L1u[kSmemBatches], s_L2[kSmemBatches], s_qb0[kSmemBatches];
+    const bool in_smem = p.batch <= kSmemBatches;
     const int tid = threadIdx.x;
     for (int i = tid; i < kCostBins; i += kMetaThreads) hist[i] = 0;
     if (tid == 0) { s_status = 0; s_total = 0; }
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         bi.k_row0 = (int32_t)k0;
         bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
         binfo[b] = bi;
+        if (in_smem) { s_L1u[b] = bi.L1u; s_L2[b] = bi.L2; }
         if (err) atomicOr(&s_status, err);
     }
     __syncthreads();
@@ -151,11 +156,13 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     int32_t carry = 0;
     for (int32_t b0 = 0; b0 < p.batch; b0 += kMetaThreads) {
         const int32_t b = b0 + tid;
-        const int32_t nqb = b < p.batch ? (binfo[b].L1u + s.tq - 1) / s.tq : 0;
+        const int32_t l1u = b < p.batch ? (in_smem ? s_L1u[b] : binfo[b].L1u) : 0;
+        const int32_t nqb = (l1u + s.tq - 1) / s.tq;
         const int32_t incl = block_inclusive_scan(nqb, warp_sums);
         if (b < p.batch) {
             binfo[b].pad[0] = nqb;
             binfo[b].pad[1] = carry + incl - nqb;
+            if (in_smem) s_qb0[b] = carry + incl - nqb;
         }
         __syncthreads();
         if (tid == kMetaThreads - 1) warp_sums[0] = incl;       // block total
@@ -165,23 +172,57 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     }
     const int32_t n_blocks = carry;
     __syncthreads();
+    // batch lookups: shared memory when it holds every batch, else the global records
+    const int32_t *qb0_arr = in_smem ? s_qb0 : nullptr;
+    auto batch_info = [&](int32_t b) {
+        BatchInfo bi;
+        if (in_smem) {
+            bi.L1u = s_L1u[b];
+            bi.L2 = s_L2[b];
+            bi.pad[1] = s_qb0[b];
+        } else {
+            bi = binfo[b];
+        }
+        return bi;
+    };
+    auto block_batch = [&](int32_t gb) {
+        if (qb0_arr) return batch_of_block(qb0_arr, p.batch, gb);
+        int32_t lo = 0, hi = p.batch - 1;
+        while (lo < hi) {
+            const int32_t mid = (lo + hi + 1) >> 1;
+            if (binfo[mid].pad[1] <= gb) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
 
-    // ---- pass 1: cost histogram ---------------------------------------------------------------
+    // ---- pass 1: cost histogram over (query block, key split) pairs -------------------------
+    // Most items share a handful of costs (every decode item has the same one), so lanes of a
+    // warp with equal cost add to the histogram once, through their leader.
+    const int32_t splits = s.kc > 0 ? (p.max_seqlen_k + s.kc - 1) / s.kc : 1;
+    const int64_t n_pairs = (int64_t)n_blocks * splits;
+    const int lane = tid & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    auto pair_item = [&](int64_t g, WorkItem *it) {
+        if (g >= n_pairs) return false;
+        const int32_t gb = (int32_t)(g / splits), sp = (int32_t)(g - (int64_t)gb * splits);
+        const int32_t b = block_batch(gb);
+        const BatchInfo bi = batch_info(b);
+        return item_of_block(p, s, b, bi, gb - bi.pad[1], sp, it);
+    };
     int32_t mine = 0;
-    for (int32_t g = tid; g < n_blocks; g += kMetaThreads) {
-        const int32_t b = batch_of_block(binfo, p.batch, g);
-        const BatchInfo bi = binfo[b];
-        for_items_of_block(p, s, b, bi, g - bi.pad[1], [&](const WorkItem &it) {
-            atomicAdd(&hist[it.cost], 1);
-            ++mine;
-        });
+    for (int64_t g0 = 0; g0 < n_pairs; g0 += kMetaThreads) {
+        WorkItem it;
+        const bool ok = pair_item(g0 + tid, &it);
+        const int key = ok ? it.cost : -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        if (ok && (peers & lt_mask) == 0) atomicAdd(&hist[key], __popc(peers));
+        mine += ok;
     }
     atomicAdd(&s_total, mine);
     __syncthreads();
 
     // ---- descending exclusive scan of the histogram: cursor[c] = items with cost > c ----------
     if (tid < 32) {
-        const int lane = tid;
         // each lane owns kCostBins/32 consecutive bins; highest bins first
         constexpr int per = kCostBins / 32;
         int32_t local = 0;
@@ -202,15 +243,19 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     }
     __syncthreads();
 
-    // ---- pass 2: placement --------------------------------------------------------------------
+    // ---- pass 2: placement (one atomic per equal-cost lane group; lanes take ranks in it) ------
     const int32_t cap = s.max_items;
-    for (int32_t g = tid; g < n_blocks; g += kMetaThreads) {
-        const int32_t b = batch_of_block(binfo, p.batch, g);
-        const BatchInfo bi = binfo[b];
-        for_items_of_block(p, s, b, bi, g - bi.pad[1], [&](const WorkItem &it) {
-            const int32_t slot = atomicAdd(&hist[it.cost], 1);
-            if (slot < cap) items[slot] = it;
-        });
+    for (int64_t g0 = 0; g0 < n_pairs; g0 += kMetaThreads) {
+        WorkItem it;
+        const bool ok = pair_item(g0 + tid, &it);
+        const int key = ok ? it.cost : -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        const int leader = __ffs(peers) - 1;
+        int32_t base = 0;
+        if (ok && lane == leader) base = atomicAdd(&hist[key], __popc(peers));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        const int32_t slot = base + __popc(peers & lt_mask);
+        if (ok && slot < cap) items[slot] = it;
     }
     __syncthreads();
 

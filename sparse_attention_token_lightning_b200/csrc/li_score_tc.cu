@@ -32,8 +32,12 @@
 namespace li {
 namespace {
 
-constexpr int kEpiWarps = 8;
-constexpr int kSchedWarp = 2 + kEpiWarps;               // warp 10
+#ifndef LI_EPI_WARPS
+#define LI_EPI_WARPS 16
+#endif
+constexpr int kEpiWarps = LI_EPI_WARPS;                 // multiple of 4 (one per TMEM lane quarter)
+constexpr int kEpiGroups = kEpiWarps / 4;               // warps sharing a lane quarter split the rows
+constexpr int kSchedWarp = 2 + kEpiWarps;
 constexpr int kThreads = 32 * (3 + kEpiWarps);
 constexpr int kMaxStages = 8;
 constexpr int kSlots = 2;
@@ -447,7 +451,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                          volatile int *abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3;          // TMEM lanes this warp may access
-    const int group = (warp - 2) >> 2;     // 0 or 1: which rows of the item
+    const int group = (warp - 2) >> 2;     // which rows of the item: t = group (mod kEpiGroups)
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
     const int N1 = P.p.n_heads;
     const int mask_mode = P.p.mask_mode;
@@ -474,7 +478,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
             const int32_t jt = j0 + tile * kKeyTile;
             const int32_t j = jt + 32 * quarter + lane;
             const uint32_t acc = tmem_base + lane_addr + ab * P.acc_stride;
-            for (int t = group; t < nq; t += 2) {
+            for (int t = group; t < nq; t += kEpiGroups) {
                 const int32_t hi = min(window_hi(mask_mode, q0 + t, L1u, L2), j1);
                 if (jt >= hi) continue;                       // tile past this row's window
                 float I;
@@ -636,13 +640,27 @@ int sm_count_cached() {
 
 }  // namespace
 
+// Shape checks of the tensor-core kernel: MMA width 16..256, at least two key stages in shared
+// memory, paged blocks the TMA pieces tile (a multiple of 8 dividing 128, or a multiple of 128),
+// and 16-byte aligned q and k for the tensor maps.
+bool score_tc_eligible(const Problem &p, const Schedule &s) {
+    if (s.max_items <= 0 || p.rows <= 0) return false;
+    const int N = (s.tq * p.n_heads + 15) / 16 * 16;
+    if (N > kNmax || N < 16) return false;
+    if ((kTailOff - 4u * (uint32_t)N * 128u) / kKStageBytes < 2) return false;
+    if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        const int bs = p.block_size;
+        if (bs <= kKeyTile ? (bs % 8 != 0 || kKeyTile % bs != 0) : bs % kKeyTile != 0) return false;
+    }
+    return (reinterpret_cast<uintptr_t>(p.q) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.k) & 15) == 0;
+}
+
 // Launches the tensor-core kernel when the problem fits it; *launched = false leaves the call
-// to the CUDA-core kernel (paged caches whose block size is not a multiple of 8 dividing 128 or
-// a multiple of 128, and empty tensors).
+// to the CUDA-core kernel (see score_tc_eligible, and a tensor map the driver refuses).
 cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
                             float *scores, int64_t ld, cudaStream_t st, bool *launched) {
     *launched = false;
-    if (s.max_items <= 0 || p.rows <= 0) return cudaSuccess;
+    if (!score_tc_eligible(p, s)) return cudaSuccess;
     TcParams P{};
     P.p = p;
     P.view = make_view(p, s, meta);

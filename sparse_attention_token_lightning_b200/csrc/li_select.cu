@@ -53,6 +53,13 @@ constexpr int kWarps = kThreads / 32;
 #include "li_select_impl.cuh"
 }  // namespace sel512
 
+// Few long rows (fewer than two per SM, e.g. decode): 1024 threads per row shorten each row.
+namespace sel1024 {
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+#include "li_select_impl.cuh"
+}  // namespace sel1024
+
 }  // namespace
 
 // Launch on a problem's rows: the 256-thread kernel when no row can exceed 4096 keys, else the
@@ -79,6 +86,18 @@ cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta,
         const size_t smem = sel256::select_work_bytes(p.topk, false, &cand_cap);
         return launch_one<256, false, sel256::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val,
                                                     smem, cand_cap, sel256::select_kernel<false>, st);
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        sms = 148;
+    }
+    if (p.rows < 2 * sms) {
+        const size_t smem = sel1024::select_work_bytes(p.topk, true, &cand_cap);
+        return launch_one<1024, true, sel1024::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val,
+                                                     smem, cand_cap, sel1024::select_kernel<true>,
+                                                     st);
     }
     const size_t smem = sel512::select_work_bytes(p.topk, true, &cand_cap);
     return launch_one<512, true, sel512::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val, smem,

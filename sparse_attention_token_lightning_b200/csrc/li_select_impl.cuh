@@ -624,7 +624,7 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
 // kLong: the problem may have rows longer than kRegKeys * kThreads keys (long-row path compiled
 // in; two CTAs per SM). Otherwise only the register path and the exact fallback exist.
 template <bool kLong>
-__global__ void __launch_bounds__(kThreads, kLong ? 2 : 4) select_kernel(Params sp) {
+__global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) : 4) select_kernel(Params sp) {
     const Problem &p = sp.p;
     const int tid = threadIdx.x;
     bool meta_ok = true;

@@ -46,11 +46,19 @@ class LiArgs(ctypes.Structure):
     ]
 
 
+class LiPlanInfo(ctypes.Structure):
+    """Mirror of ``li_plan_info`` (include/li.h)."""
+
+    _fields_ = [("tq", ctypes.c_int32), ("kc", ctypes.c_int32), ("max_items", ctypes.c_int32),
+                ("dense", ctypes.c_int32), ("kernels", ctypes.c_int32),
+                ("score_tc", ctypes.c_int32)]
+
+
 _lib = None
 
 EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
            "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
-           "li_abi_version", "li_indexer_noalloc")
+           "li_abi_version", "li_indexer_noalloc", "li_plan")
 
 
 def lib_path() -> Path:
@@ -72,6 +80,8 @@ def lib():
     L.li_metadata_workspace_size.argtypes = [P, sz]
     L.li_metadata.argtypes = [P, vp, ctypes.c_size_t, vp]
     L.li_indexer_workspace_size.argtypes = [P, sz]
+    L.li_plan.argtypes = [P, ctypes.POINTER(LiPlanInfo)]
+    L.li_plan.restype = ctypes.c_int
     L.li_indexer.argtypes = [P, vp, vp, ctypes.c_size_t, vp, vp, vp]
     L.li_check_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     for f in ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
@@ -157,6 +167,12 @@ def li_indexer_workspace_size(args: LiArgs) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().li_indexer_workspace_size(ctypes.byref(args), ctypes.byref(n)))
     return int(n.value)
+
+
+def li_plan(args: LiArgs) -> dict:
+    info = LiPlanInfo()
+    _check(lib().li_plan(ctypes.byref(args), ctypes.byref(info)))
+    return {f: int(getattr(info, f)) for f, _ in LiPlanInfo._fields_}
 
 
 def li_metadata(args: LiArgs, metadata: torch.Tensor, stream=None):

@@ -46,20 +46,21 @@ def test_abi_version(L):
     assert li.li_abi_version() == 1
 
 
-def test_ctypes_struct_matches_c_layout(tmp_path):
-    fields = [f for f, _ in li.LiArgs._fields_]
+@pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
+def test_ctypes_struct_matches_c_layout(tmp_path, cls, cname):
+    fields = [f for f, _ in cls._fields_]
     prog = tmp_path / "probe.c"
-    body = "\n".join(f'  printf("%zu\\n", offsetof(li_args, {f}));' for f in fields)
+    body = "\n".join(f'  printf("%zu\\n", offsetof({cname}, {f}));' for f in fields)
     prog.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "li.h"\nint main(void){\n'
-                    f'  printf("%zu\\n", sizeof(li_args));\n{body}\n  return 0;\n}}\n')
+                    f'  printf("%zu\\n", sizeof({cname}));\n{body}\n  return 0;\n}}\n')
     exe = tmp_path / "probe"
     subprocess.run(["gcc", "-std=c11", "-I", str(ROOT / "include"), str(prog), "-o", str(exe)],
                    check=True)
     vals = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
                                            check=True).stdout.split()]
-    assert vals[0] == ctypes.sizeof(li.LiArgs)
+    assert vals[0] == ctypes.sizeof(cls)
     for f, off in zip(fields, vals[1:]):
-        assert getattr(li.LiArgs, f).offset == off, f
+        assert getattr(cls, f).offset == off, f
 
 
 def _args(**kw):
@@ -133,3 +134,28 @@ def test_indexer_rejects_small_workspace(L):
     assert st == 3   # misaligned workspace
     st = L.li_indexer(ctypes.byref(a), None, 0x100000, 1 << 30, None, 0x300000, None)
     assert st == 1   # no output
+
+
+def test_plan_reports_schedule_and_kernel_count(L):
+    # dense causal BSND: closed-form work list, score + select kernels only
+    pl = li.li_plan(_args(q_len=4096, k_len=4096, max_seqlen_q=4096, max_seqlen_k=4096,
+                          num_heads_q=64, topk=2048))
+    assert pl == dict(tq=4, kc=0, max_items=1024, dense=1, kernels=2, score_tc=1)
+    # one query row per batch (decode): tq capped by max_seqlen_q, schedule kernel needed
+    pl = li.li_plan(_args(layout_k=2, k_len=0, q_len=1, max_seqlen_q=1, batch=64,
+                          num_heads_q=64, seqused_k=0x40000, block_table=0x50000,
+                          block_table_stride=512, num_blocks=64 * 512, block_size=64,
+                          max_seqlen_k=32768, topk=2048))
+    assert pl["tq"] == 1 and pl["dense"] == 0 and pl["kernels"] == 3 and pl["score_tc"] == 1
+    assert pl["kc"] > 0 and pl["max_items"] >= 64 * (32768 // pl["kc"])
+    # block sizes the TMA pieces cannot tile go to the CUDA-core score kernel
+    pl = li.li_plan(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
+                          block_table_stride=64, num_blocks=64, block_size=12,
+                          max_seqlen_k=512))
+    assert pl["score_tc"] == 0 and pl["kernels"] == 3
+    # no query rows: nothing launches
+    assert li.li_plan(_args(batch=0))["kernels"] == 0
+    # argument errors come back as status codes
+    a = _args(num_heads_q=0)
+    assert L.li_plan(ctypes.byref(a), ctypes.byref(li.LiPlanInfo())) == 1
+    assert L.li_plan(ctypes.byref(_args()), None) == 1
