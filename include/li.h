@@ -52,7 +52,9 @@ typedef enum li_layout {
 typedef enum li_status {
     LI_OK = 0,
     LI_ERR_INVALID_ARG = 1,     /* an argument violates the documented contract             */
-    LI_ERR_UNSUPPORTED = 2,     /* a valid request this build does not implement            */
+    LI_ERR_UNSUPPORTED = 2,     /* a valid request this build does not implement, e.g. more
+                                   than 2^31-1 query-head rows (query rows x num_heads_q) or
+                                   key rows (B*S2, T2 or num_blocks*block_size)                 */
     LI_ERR_WORKSPACE = 3,       /* workspace / metadata buffer too small or misaligned      */
     LI_ERR_CUDA = 4,            /* a CUDA runtime call failed (message has the CUDA error)  */
     LI_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait gave up (li_check_status)     */

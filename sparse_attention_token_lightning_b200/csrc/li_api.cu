@@ -124,6 +124,13 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     const int64_t rows = a->layout_q == LI_LAYOUT_TND ? (int64_t)a->q_len
                                                      : (int64_t)a->batch * a->q_len;
     if (rows > INT32_MAX) return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 query rows");
+    // the kernels address query-head rows and key-cache rows with 32-bit coordinates
+    if (rows * a->num_heads_q > INT32_MAX)
+        return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 query-head rows");
+    const int64_t key_rows = a->layout_k == LI_LAYOUT_PA_BSND ? (int64_t)a->num_blocks * a->block_size
+                             : a->layout_k == LI_LAYOUT_TND  ? (int64_t)a->k_len
+                                                             : (int64_t)a->batch * a->k_len;
+    if (key_rows > INT32_MAX) return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 key rows");
 
     li::Problem &P = *p;
     std::memset(&P, 0, sizeof P);

@@ -48,16 +48,22 @@ struct BatchInfo {
 };
 static_assert(sizeof(BatchInfo) == 32, "BatchInfo size");
 
-struct WorkItem {
+// One unit of score work. It carries its batch's lengths and row bases too, so the kernels that
+// take items need no second dependent load of the batch record.
+struct alignas(16) WorkItem {
     int32_t b;             // batch
     int32_t q0;            // first query row (position inside the batch)
     int32_t nq;            // query rows (<= tq)
     int32_t j0;            // first key of the item's range
     int32_t j1;            // one past the last key any of its rows needs
     int32_t cost;          // key tiles, for ordering
-    int32_t pad[2];
+    int32_t row0;          // global query row of q0 (the batch's q_row0 + q0)
+    int32_t L1u;           // the batch's query rows in use
+    int32_t L2;            // the batch's keys
+    int32_t k_row0;        // the batch's first key row
+    int32_t pad[6];
 };
-static_assert(sizeof(WorkItem) == 32, "WorkItem size");
+static_assert(sizeof(WorkItem) == 64, "WorkItem size");
 
 struct WsHeader {
     uint32_t status;       // LI_DEVERR_* bits of the last li_indexer on this workspace
@@ -166,7 +172,11 @@ struct SchedView {
         it.j0 = 0;
         it.j1 = window_hi(p.mask_mode, it.q0 + it.nq - 1, p.q_len, p.k_len);
         it.cost = 0;
-        it.pad[0] = it.pad[1] = 0;
+        it.row0 = it.b * p.q_len + it.q0;
+        it.L1u = p.q_len;
+        it.L2 = p.k_len;
+        it.k_row0 = it.b * p.k_len;
+        for (int i = 0; i < 6; ++i) it.pad[i] = 0;
         return it;
     }
 };

@@ -28,39 +28,40 @@ __device__ inline int item_cost(int32_t j0, int32_t j1) {
     return c < kCostBins ? c : kCostBins - 1;
 }
 
-// Item `split` of query block qb of batch b (key range [split*kc, (split+1)*kc) of the block's
-// window); returns false when the block has no such item.
-__device__ inline bool item_of_block(const Problem &p, const Schedule &s, int32_t b,
-                                     const BatchInfo &bi, int32_t qb, int32_t split, WorkItem *it) {
-    it->b = b;
-    it->q0 = qb * s.tq;
-    it->nq = min(s.tq, bi.L1u - it->q0);
-    // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
-    const int32_t jend = window_hi(p.mask_mode, it->q0 + it->nq - 1, bi.L1u, bi.L2);
-    const int32_t kc = s.kc > 0 ? s.kc : jend;
-    const int64_t j0 = (int64_t)split * kc;
-    if (jend <= 0 || j0 >= jend) return false;
-    it->j0 = (int32_t)j0;
-    it->j1 = min(jend, it->j0 + kc);
-    it->cost = item_cost(it->j0, it->j1);
-    it->pad[0] = it->pad[1] = 0;
-    return true;
-}
-
-// Block-wide inclusive scan of one value per thread (kMetaThreads threads).
+// Block-wide inclusive scan of one value per thread (kMetaThreads threads): warp scans, then
+// one warp scans the 32 warp totals.
 __device__ inline int32_t block_inclusive_scan(int32_t x, int32_t *warp_sums) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int32_t incl = x;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
     }
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
-    int32_t before = 0;
-    for (int w = 0; w < warp; ++w) before += warp_sums[w];
+    if (warp == 0) {
+        int32_t ws = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t t = __shfl_up_sync(0xffffffffu, ws, o);
+            if (lane >= o) ws += t;
+        }
+        warp_sums[lane] = ws;                       // inclusive prefix of the warp totals
+    }
+    __syncthreads();
+    const int32_t before = warp > 0 ? warp_sums[warp - 1] : 0;
     __syncthreads();
     return before + incl;
+}
+
+// Writes one item as four 16-byte stores (items land at scattered slots; a warp's scalar
+// stores to scattered slots cost one memory transaction per lane each).
+__device__ inline void store_item(WorkItem *dst, const WorkItem &it) {
+    const int4 *src = reinterpret_cast<const int4 *>(&it);
+    int4 *d = reinterpret_cast<int4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(WorkItem) / sizeof(int4)); ++i) d[i] = src[i];
 }
 
 constexpr int kSmemBatches = 2048;     // batches whose lengths and block prefix stay in smem
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     __shared__ int32_t s_total;
     // per-batch query rows in use, keys and first query block (B <= kSmemBatches)
     __shared__ int32_t s_L1u[kSmemBatches], s_L2[kSmemBatches], s_qb0[kSmemBatches];
+    __shared__ int32_t s_qr0[kSmemBatches], s_kr0[kSmemBatches];   // first query / key rows
     const bool in_smem = p.batch <= kSmemBatches;
     const int tid = threadIdx.x;
     for (int i = tid; i < kCostBins; i += kMetaThreads) hist[i] = 0;
@@ -146,7 +148,12 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         bi.k_row0 = (int32_t)k0;
         bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
         binfo[b] = bi;
-        if (in_smem) { s_L1u[b] = bi.L1u; s_L2[b] = bi.L2; }
+        if (in_smem) {
+            s_L1u[b] = bi.L1u;
+            s_L2[b] = bi.L2;
+            s_qr0[b] = bi.q_row0;
+            s_kr0[b] = bi.k_row0;
+        }
         if (err) atomicOr(&s_status, err);
     }
     __syncthreads();
@@ -179,6 +186,8 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         if (in_smem) {
             bi.L1u = s_L1u[b];
             bi.L2 = s_L2[b];
+            bi.q_row0 = s_qr0[b];
+            bi.k_row0 = s_kr0[b];
             bi.pad[1] = s_qb0[b];
         } else {
             bi = binfo[b];
@@ -195,67 +204,113 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         return lo;
     };
 
-    // ---- pass 1: cost histogram over (query block, key split) pairs -------------------------
-    // Most items share a handful of costs (every decode item has the same one), so lanes of a
-    // warp with equal cost add to the histogram once, through their leader.
-    const int32_t splits = s.kc > 0 ? (p.max_seqlen_k + s.kc - 1) / s.kc : 1;
-    const int64_t n_pairs = (int64_t)n_blocks * splits;
-    const int lane = tid & 31;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    auto pair_item = [&](int64_t g, WorkItem *it) {
-        if (g >= n_pairs) return false;
-        const int32_t gb = (int32_t)(g / splits), sp = (int32_t)(g - (int64_t)gb * splits);
-        const int32_t b = block_batch(gb);
-        const BatchInfo bi = batch_info(b);
-        return item_of_block(p, s, b, bi, gb - bi.pad[1], sp, it);
+    // Items of query block gb: its window [0, jend) cut into n_s pieces of kc keys; every piece
+    // but the last costs full_cost tiles, the last costs last_cost.
+    struct BlockItems {
+        int32_t b, q0, nq, jend, kc, n_s, full_cost, last_cost, row0, L1u, L2, k_row0;
     };
-    int32_t mine = 0;
-    for (int64_t g0 = 0; g0 < n_pairs; g0 += kMetaThreads) {
+    auto block_items = [&](int32_t gb) {
+        BlockItems r;
+        r.b = block_batch(gb);
+        const BatchInfo bi = batch_info(r.b);
+        r.q0 = (gb - bi.pad[1]) * s.tq;
+        r.nq = min(s.tq, bi.L1u - r.q0);
+        // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
+        r.jend = window_hi(p.mask_mode, r.q0 + r.nq - 1, bi.L1u, bi.L2);
+        r.kc = s.kc > 0 ? s.kc : r.jend;
+        r.n_s = r.jend > 0 ? (r.jend + r.kc - 1) / r.kc : 0;
+        r.full_cost = item_cost(0, r.kc);
+        r.last_cost = r.n_s > 0 ? item_cost((r.n_s - 1) * r.kc, r.jend) : 0;
+        r.row0 = bi.q_row0 + r.q0;
+        r.L1u = bi.L1u;
+        r.L2 = bi.L2;
+        r.k_row0 = bi.k_row0;
+        return r;
+    };
+    auto make_item = [&](const BlockItems &r, int32_t sp) {
         WorkItem it;
-        const bool ok = pair_item(g0 + tid, &it);
-        const int key = ok ? it.cost : -1;
+        it.b = r.b;
+        it.q0 = r.q0;
+        it.nq = r.nq;
+        it.j0 = sp * r.kc;
+        it.j1 = min(r.jend, it.j0 + r.kc);
+        it.cost = sp + 1 < r.n_s ? r.full_cost : r.last_cost;
+        it.row0 = r.row0;
+        it.L1u = r.L1u;
+        it.L2 = r.L2;
+        it.k_row0 = r.k_row0;
+        for (int i = 0; i < 6; ++i) it.pad[i] = 0;
+        return it;
+    };
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+
+    // ---- pass 1: cost histogram, one or two adds per query block ------------------------------
+    // Lanes of a warp whose last pieces cost the same add once, through their leader.
+    int32_t mine = 0;
+    for (int32_t g0 = 0; g0 < n_blocks; g0 += kMetaThreads) {
+        const int32_t gb = g0 + tid;
+        BlockItems r;
+        r.n_s = 0;
+        if (gb < n_blocks) r = block_items(gb);
+        const bool ok = r.n_s > 0;
+        if (ok && r.n_s > 1) atomicAdd(&hist[r.full_cost], r.n_s - 1);
+        const int key = ok ? r.last_cost : -1;
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
         if (ok && (peers & lt_mask) == 0) atomicAdd(&hist[key], __popc(peers));
-        mine += ok;
+        mine += r.n_s;
     }
     atomicAdd(&s_total, mine);
     __syncthreads();
 
     // ---- descending exclusive scan of the histogram: cursor[c] = items with cost > c ----------
-    if (tid < 32) {
-        // each lane owns kCostBins/32 consecutive bins; highest bins first
-        constexpr int per = kCostBins / 32;
-        int32_t local = 0;
-        for (int i = 0; i < per; ++i) local += hist[lane * per + i];
-        // suffix sum over lanes above this one
-        int32_t incl = local;
-        for (int o = 1; o < 32; o <<= 1) {
-            int32_t v = __shfl_down_sync(0xffffffffu, incl, o);
-            if (lane + o < 32) incl += v;
-        }
-        int32_t above = incl - local;
-        for (int i = per - 1; i >= 0; --i) {
-            const int bin = lane * per + i;
-            const int32_t c = hist[bin];
-            hist[bin] = above;
-            above += c;
-        }
+    // thread t holds bin kCostBins - 1 - t, so an inclusive scan in thread order counts the bins
+    // at or above each cost
+    static_assert(kCostBins == kMetaThreads, "one histogram bin per thread");
+    {
+        const int bin = kCostBins - 1 - tid;
+        const int32_t c = hist[bin];
+        const int32_t incl = block_inclusive_scan(c, warp_sums);
+        hist[bin] = incl - c;
     }
     __syncthreads();
 
-    // ---- pass 2: placement (one atomic per equal-cost lane group; lanes take ranks in it) ------
+    // ---- pass 2: placement -------------------------------------------------------------------
     const int32_t cap = s.max_items;
-    for (int64_t g0 = 0; g0 < n_pairs; g0 += kMetaThreads) {
-        WorkItem it;
-        const bool ok = pair_item(g0 + tid, &it);
-        const int key = ok ? it.cost : -1;
-        const uint32_t peers = __match_any_sync(0xffffffffu, key);
-        const int leader = __ffs(peers) - 1;
-        int32_t base = 0;
-        if (ok && lane == leader) base = atomicAdd(&hist[key], __popc(peers));
-        base = __shfl_sync(0xffffffffu, base, leader);
-        const int32_t slot = base + __popc(peers & lt_mask);
-        if (ok && slot < cap) items[slot] = it;
+    if (s.kc == 0) {
+        // one item per block: a thread per block, one atomic per equal-cost lane group
+        for (int32_t g0 = 0; g0 < n_blocks; g0 += kMetaThreads) {
+            const int32_t gb = g0 + tid;
+            BlockItems r;
+            r.n_s = 0;
+            if (gb < n_blocks) r = block_items(gb);
+            const bool ok = r.n_s > 0;
+            const int key = ok ? r.last_cost : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, key);
+            const int leader = __ffs(peers) - 1;
+            int32_t base = 0;
+            if (ok && lane == leader) base = atomicAdd(&hist[key], __popc(peers));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const int32_t slot = base + __popc(peers & lt_mask);
+            if (ok && slot < cap) store_item(&items[slot], make_item(r, 0));
+        }
+    } else {
+        // key splits (few query blocks, many pieces each): a warp per block; its lane 0 reserves
+        // the block's full-cost pieces and its last piece, the lanes write the items
+        for (int32_t gb = warp; gb < n_blocks; gb += kMetaThreads / 32) {
+            const BlockItems r = block_items(gb);
+            int32_t base_full = 0, base_last = 0;
+            if (lane == 0 && r.n_s > 0) {
+                if (r.n_s > 1) base_full = atomicAdd(&hist[r.full_cost], r.n_s - 1);
+                base_last = atomicAdd(&hist[r.last_cost], 1);
+            }
+            base_full = __shfl_sync(0xffffffffu, base_full, 0);
+            base_last = __shfl_sync(0xffffffffu, base_last, 0);
+            for (int32_t sp = lane; sp < r.n_s; sp += 32) {
+                const int32_t slot = sp + 1 < r.n_s ? base_full + sp : base_last;
+                if (slot < cap) store_item(&items[slot], make_item(r, sp));
+            }
+        }
     }
     __syncthreads();
 

@@ -52,7 +52,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 struct Slot {
     int32_t valid, b, q0, nq, j0, j1, row0, L1u, L2, k_row0;
     int32_t pad[6];
-    int32_t tbl[32];      // paged: block-table entries of the item's first 32 blocks
+    int32_t prow[32];     // paged: cache row of each of the item's first 32 key pieces
+                          // (-1: past the item's keys, -2: block-table entry out of range)
     float w[kNmax];
 };
 static_assert(sizeof(Slot) == 64 + 128 + 4 * kNmax, "Slot size");
@@ -257,51 +258,75 @@ __device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
     return (j1 - j0 + kKeyTile - 1) / kKeyTile;
 }
 
+// Paged keys: row in the key cache of piece pi of an item whose keys start at j0 (pieces of
+// piece_rows keys; j0 is a multiple of them). -1 past j1, -2 when the block-table entry is out
+// of range.
+__device__ __forceinline__ int32_t piece_row(const TcParams &P, int32_t b, int32_t j0, int32_t j1,
+                                             int32_t pi) {
+    const int32_t jp = j0 + pi * P.piece_rows;
+    if (jp >= j1) return -1;
+    const int32_t bs = P.p.block_size;
+    const int32_t blk = P.p.block_table[(int64_t)b * P.p.bt_stride + jp / bs];
+    if (blk < 0 || blk >= P.p.num_blocks) return -2;
+    return blk * bs + jp % bs;
+}
+
 // ---- roles ---------------------------------------------------------------------------------
-// Scheduler warp: takes tickets and stages each non-empty item (header, w, first block-table
-// entries) in the slot ring ahead of the producer, so item set-up latency stays off the
-// key-streaming path.
+// Scheduler warp: takes tickets and stages each non-empty item (header, w, cache rows of its
+// first 32 key pieces) in the slot ring ahead of the producer. The next item's loads go to
+// registers right after a slot is filled, so they complete while the warp waits for the next
+// free slot, and a ticket is taken only when the ring has moved on by one item.
 __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
                           volatile int *abort_flag, int n_items) {
+    constexpr int kWPerLane = kNmax / 32;
     const int lane = threadIdx.x & 31;
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
     const int N1 = P.p.n_heads;
-    bool ok = true;
-    for (int it = 0; ok; ++it) {
-        const int sl = it % kSlots;
-        if (!mbar_wait(bars.sl_empty(sl), ((it / kSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        // next non-empty item (the dense closed forms can yield items with an empty window)
-        int ticket = 0;
-        WorkItem wi{};
-        bool valid = false;
+    WorkItem cur{};
+    float wv[kWPerLane];
+    int32_t tv = -1;
+    // takes tickets up to the next item with a non-empty window (the dense closed forms can yield
+    // empty ones) and loads its weights (lane l holds entries l, l + 32, ...) and the cache row
+    // of its key piece l; false at the end of the list
+    auto fetch = [&]() -> bool {
         for (;;) {
+            int ticket = 0;
             if (lane == 0) ticket = atomicAdd(&P.ws->sched_next, 1);
             ticket = __shfl_sync(0xffffffffu, ticket, 0);
-            if (ticket >= n_items) break;
-            wi = P.view.item(P.p, ticket);
-            if (wi.j1 > wi.j0) { valid = true; break; }
+            if (ticket >= n_items) return false;
+            cur = P.view.item(P.p, ticket);
+            if (cur.j1 > cur.j0) break;
         }
+        const int64_t wbase = (int64_t)cur.row0 * N1;
+        const int nw = cur.nq * N1;
+#pragma unroll
+        for (int i = 0; i < kWPerLane; ++i) {
+            const int e = lane + 32 * i;
+            wv[i] = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+        }
+        if (P.piece_rows) tv = piece_row(P, cur.b, cur.j0, cur.j1, lane);
+        return true;
+    };
+    bool have = fetch();
+    bool ok = true;
+    for (int it = 0;; ++it) {
+        const int sl = it % kSlots;
+        if (!mbar_wait(bars.sl_empty(sl), ((it / kSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
         Slot &S = slots[sl];
-        if (valid) {
-            const BatchInfo bi = P.view.batch(P.p, wi.b);
-            const int64_t wbase = ((int64_t)bi.q_row0 + wi.q0) * N1;
-            const int nw = wi.nq * N1;
-            for (int e = lane; e < kNmax; e += 32)
-                S.w[e] = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
-            if (P.piece_rows) {
-                const int32_t bidx = wi.j0 / P.p.block_size + lane;
-                S.tbl[lane] = (int64_t)bidx * P.p.block_size < wi.j1
-                                  ? P.p.block_table[(int64_t)wi.b * P.p.bt_stride + bidx] : -1;
-            }
+        if (have) {
+#pragma unroll
+            for (int i = 0; i < kWPerLane; ++i) S.w[lane + 32 * i] = wv[i];
+            if (P.piece_rows) S.prow[lane] = tv;
             if (lane == 0) {
-                S.b = wi.b; S.q0 = wi.q0; S.nq = wi.nq; S.j0 = wi.j0; S.j1 = wi.j1;
-                S.row0 = bi.q_row0 + wi.q0; S.L1u = bi.L1u; S.L2 = bi.L2; S.k_row0 = bi.k_row0;
+                S.b = cur.b; S.q0 = cur.q0; S.nq = cur.nq; S.j0 = cur.j0; S.j1 = cur.j1;
+                S.row0 = cur.row0; S.L1u = cur.L1u; S.L2 = cur.L2; S.k_row0 = cur.k_row0;
             }
         }
-        if (lane == 0) S.valid = valid ? 1 : 0;
+        if (lane == 0) S.valid = have ? 1 : 0;
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.sl_full(sl));
-        if (!valid) break;
+        if (!have) break;
+        have = fetch();
     }
     if (!ok) *abort_flag = 1;
 }
@@ -323,7 +348,8 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
         const Slot &S = slots[sl];
         const int valid = S.valid;
         const int32_t b = S.b, q0 = S.q0, j0 = S.j0, j1 = S.j1, row0 = S.row0, k_row0 = S.k_row0;
-        int32_t tbl_val = S.tbl[lane];
+        int32_t pv = S.prow[lane];          // row of piece pbase + lane
+        int32_t pbase = 0;
         __syncwarp();
         if (!valid) {
             if (lane == 0) mbar_arrive(bars.sl_empty(sl));
@@ -340,56 +366,40 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
             tma_load_2d(qdst + P.q_half, tmq, bars.q_full(qb), 64, y);
         }
-        // K tiles of the item's key range. Paged keys: the warp keeps 32 block-table entries
-        // in registers (lane l holds entry tbl_base + l), the first 32 staged by the scheduler,
-        // later ones refilled 32 at a time.
+        // K tiles of the item's key range. Paged keys: lane l holds the cache row of piece
+        // pbase + l (the first 32 staged by the scheduler, later ones refilled 32 at a time) and
+        // lanes 0..pieces-1 each load one piece of the tile.
         const int32_t nt = n_tiles_of(j0, j1);
-        const int32_t bs = P.p.block_size;
-        int32_t tbl_base = P.piece_rows ? j0 / bs : 0;
+        const int pr = P.piece_rows;
+        const int pieces = pr ? kKeyTile / pr : 0;
         for (int32_t tile = 0; tile < nt; ++tile, kr.next(P.stages)) {
             const int st = kr.idx;
             if (!mbar_wait(bars.k_empty(st), kr.phase ^ 1u, abort_flag)) { ok = false; break; }
             const int32_t jt = j0 + tile * kKeyTile;
             const uint32_t kdst = sbase + P.k_off + st * kKStageBytes;
-            if (P.piece_rows == 0) {
+            if (pr == 0) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), kKStageBytes);
                     tma_load_2d(kdst, tmk, bars.k_full(st), 0, k_row0 + jt);
                     tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, k_row0 + jt);
                 }
             } else {
-                // one load per block piece: 128 / piece_rows pieces, consecutive blocks when
-                // blocks are at most 128 keys, else one piece inside block jt / bs
-                const int pr = P.piece_rows;
-                const int pieces = kKeyTile / pr;
-                const int32_t blk0 = jt / bs;
-                const int32_t nblk = bs <= kKeyTile ? pieces : 1;
-                if (blk0 < tbl_base || blk0 + nblk > tbl_base + 32) {
-                    tbl_base = blk0;
-                    const int32_t bidx = blk0 + lane;
-                    tbl_val = (int64_t)bidx * bs < j1
-                                  ? P.p.block_table[(int64_t)b * P.p.bt_stride + bidx] : -1;
+                const int32_t p0 = tile * pieces;
+                if (p0 + pieces > pbase + 32) {
+                    pbase = p0;
+                    pv = piece_row(P, b, j0, j1, pbase + lane);
                 }
-                int32_t rows[kKeyTile / 8];
-                int loads = 0;
-                for (int pc = 0; pc < pieces; ++pc) {
-                    const int32_t jp = jt + pc * pr;
-                    const int32_t blk = __shfl_sync(0xffffffffu, tbl_val,
-                                                    (bs <= kKeyTile ? blk0 + pc : blk0) - tbl_base);
-                    rows[pc] = -1;
-                    if (jp >= j1) continue;
-                    if (blk < 0 || blk >= P.p.num_blocks) { err |= LI_DEVERR_TABLE; continue; }
-                    rows[pc] = blk * bs + jp % bs;
-                    ++loads;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)loads * pr * 256u);
-                    for (int pc = 0; pc < pieces; ++pc) {
-                        if (rows[pc] < 0) continue;
-                        const uint32_t off = (uint32_t)pc * pr * 128u;
-                        tma_load_2d(kdst + off, tmk, bars.k_full(st), 0, rows[pc]);
-                        tma_load_2d(kdst + kKHalfBytes + off, tmk, bars.k_full(st), 64, rows[pc]);
-                    }
+                const int32_t row = __shfl_sync(0xffffffffu, pv, (p0 - pbase + lane) & 31);
+                const bool mine = lane < pieces && row >= 0;
+                const uint32_t loads = __ballot_sync(0xffffffffu, mine);
+                if (__ballot_sync(0xffffffffu, lane < pieces && row == -2)) err |= LI_DEVERR_TABLE;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)__popc(loads) * pr * 256u);
+                __syncwarp();
+                if (mine) {
+                    const uint32_t off = (uint32_t)lane * pr * 128u;
+                    tma_load_2d(kdst + off, tmk, bars.k_full(st), 0, row);
+                    tma_load_2d(kdst + kKHalfBytes + off, tmk, bars.k_full(st), 64, row);
                 }
             }
             __syncwarp();

@@ -338,8 +338,8 @@ constexpr int kRegKeys = 4096 / kThreads;   // keys per thread held in registers
 // Returns 1 when the outputs [0, m) are written, 3 when all scores tie (*vtie set), 2 when the
 // caller must take the exact radix path.
 __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *hist,
-                               uint64_t *buf, uint16_t *bufb, int32_t off, int32_t *oi, float *ov,
-                               Smem &sm, float *vtie) {
+                               uint64_t *buf, uint16_t *bufb, uint64_t *stage, int32_t off,
+                               int32_t *oi, float *ov, Smem &sm, float *vtie) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float kInf = __int_as_float(0x7f800000);
     int32_t nb = kThreads;
@@ -413,6 +413,8 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
         }
     }
     __syncthreads();
+    // rank within the bucket; the top m land in the stage at their output slots, and the row is
+    // then written out in slot order (contiguous stores instead of one scattered store per key)
     const int32_t filled = hist[cutb];
     for (int32_t p = tid; p < filled; p += kThreads) {
         const uint64_t x = buf[p];
@@ -422,10 +424,13 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
         int32_t rank = 0;
         for (int32_t a = beg; a < end; ++a) rank += buf[a] > x ? 1 : 0;
         const int32_t slot = beg + rank;
-        if (slot < m) {
-            oi[slot] = (int32_t)~(uint32_t)x + off;
-            if (ov) ov[slot] = key_score((uint32_t)(x >> 32));
-        }
+        if (slot < m) stage[slot] = x;
+    }
+    __syncthreads();
+    for (int32_t s = tid; s < m; s += kThreads) {
+        const uint64_t x = stage[s];
+        oi[s] = (int32_t)~(uint32_t)x + off;
+        if (ov) ov[s] = key_score((uint32_t)(x >> 32));
     }
     return 1;
 }
@@ -642,6 +647,8 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     int32_t *hist = reinterpret_cast<int32_t *>(dsm);                        // bucket path
     uint64_t *buf = reinterpret_cast<uint64_t *>(hist + kBucketsMax);
     uint16_t *bufb = reinterpret_cast<uint16_t *>(buf + topk + kBinCap);
+    uint64_t *stage = reinterpret_cast<uint64_t *>(                        // register path output
+        dsm + kBucketsMax * 4 + align_up((size_t)(topk + kBinCap) * 10, 16));
     uint32_t *keyA = reinterpret_cast<uint32_t *>(dsm);                      // exact path
     uint32_t *keyB = keyA + topk;
     int32_t *idxA = reinterpret_cast<int32_t *>(keyB + topk);
@@ -650,7 +657,9 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     uint64_t *cand = reinterpret_cast<uint64_t *>(hist + kBucketsMax);       // long-row path
     const uint32_t *rowc = nullptr;                                         // exact path reads global
 
-    const int32_t r = blockIdx.x;
+    // blocks start in index order; later rows of a causal window are the longer ones, so the
+    // rows are taken last to first (longest first)
+    const int32_t r = (int32_t)(gridDim.x - 1 - blockIdx.x);
     int32_t pos = 0;
     int32_t b = meta_ok ? row_batch(p, r, &pos) : -1;
     int32_t n = 0, off = 0;
@@ -677,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     float vtie = 0.0f;
     if (m > 0 && n <= kRegKeys * kThreads) {
         const float *src = sp.scores + (int64_t)r * sp.ld;
-        mode = reg_bucket_topk(src, n, m, hist, buf, bufb, off, oi, ov, sm, &vtie);
+        mode = reg_bucket_topk(src, n, m, hist, buf, bufb, stage, off, oi, ov, sm, &vtie);
         if (mode == 2) {
             uint32_t prefix = 0u, mask = 0u;
             int32_t need = m;
@@ -722,12 +731,13 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
 }
 
 // Bytes of the dynamic shared memory work area: the largest of the short-row bucket path
-// (histogram + scattered composites + their buckets), the long-row path (histogram +
-// candidates + scattered composites + their buckets) and the exact path (two key/index
-// buffers + digit counters).
+// (histogram + scattered composites + their buckets + the output stage), the long-row path
+// (histogram + candidates + scattered composites + their buckets) and the exact path (two
+// key/index buffers + digit counters).
 static size_t select_work_bytes(int topk, bool long_rows, int32_t *cand_cap) {
     const size_t scatter = (size_t)(topk + kBinCap) * 10;
-    const size_t shortp = (size_t)kBucketsMax * 4 + scatter;
+    const size_t staged = (size_t)(topk < kRegKeys * kThreads ? topk : kRegKeys * kThreads) * 8;
+    const size_t shortp = (size_t)kBucketsMax * 4 + align_up(scatter, 16) + staged;
     const size_t exact = (size_t)4 * topk * 4 + (size_t)kWarps * kDigits * 4;
     size_t work = shortp > exact ? shortp : exact;
     *cand_cap = 0;

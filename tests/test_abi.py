@@ -104,6 +104,11 @@ def test_valid_args_size_the_workspace(L):
           num_blocks=4, block_size=1025), 1),
     (dict(cu_seqlens_q=0x40000), 1), (dict(block_table=0x40000), 1), (dict(batch=-1), 1),
     (dict(max_seqlen_k=65), 1), (dict(return_value=2), 1),
+    # 32-bit row coordinates: query rows x heads and key rows beyond 2^31-1
+    (dict(batch=40000, q_len=1000, max_seqlen_q=1000, num_heads_q=64), 2),
+    (dict(batch=3, k_len=1 << 30, max_seqlen_k=64), 2),
+    (dict(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000, block_table_stride=4,
+          num_blocks=1 << 25, block_size=128), 2),
 ])
 def test_invalid_args_rejected_on_host(L, kw, status):
     st, _ = _ws_status(_args(**kw))
