@@ -97,6 +97,31 @@ def score_kernel_bytes(pb, pairs) -> int:
     return key_bytes(pb) + q + w + table + pairs * 4
 
 
+# DRAM traffic of one score-kernel launch (dram__bytes_read.sum + dram__bytes_write.sum from one
+# ncu capture of `python bench.py [--config NAME] --steps 3 --warmup 3 --cpu-seconds 0 --no-e2e`),
+# with the sha256 of the score-kernel sources the counters were taken on; reported only while the
+# sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
+SCORE_TRAFFIC = {
+    "causal_prefill": {"bytes": 68726784 + 10192384,
+                       "src_sha256": "5156ea82b96e4754f1df7401af48842689ecac4bab6180beaa36fc136930bf6b"},
+    "paged_decode": {"bytes": 286945024 + 7542016,
+                     "src_sha256": "5156ea82b96e4754f1df7401af48842689ecac4bab6180beaa36fc136930bf6b"},
+}
+SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
+                 "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")
+
+
+def score_traffic(config: str):
+    import hashlib
+    rec = SCORE_TRAFFIC.get(config)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for f in SCORE_SOURCES:
+        h.update((ROOT / f).read_bytes())
+    return rec["bytes"] if h.hexdigest() == rec["src_sha256"] else None
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -351,14 +376,16 @@ def main():
         achieved = nbytes / (sc / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": None, "algorithmic_bytes": nbytes,
+                    "frac": achieved / peak, "traffic": score_traffic(a.config),
+                    "algorithmic_bytes": nbytes,
                     "kernel": "score kernel (paged key gather + contraction + epilogue)",
                     "peak_source": f"{peaks['source']} HBM copy"}
     else:
         achieved = flops / (sc / 1e3) / 1e12
         peak = peaks["bf16_tflops"]
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": score_traffic(a.config),
+                    "algorithmic_bytes": score_kernel_bytes(pb_cpu, pairs),
                     "kernel": "score kernel (q.k contraction + ReLU/weight/head-sum epilogue)",
                     "peak_source": f"{peaks['source']} bf16 burst"}
 
