@@ -54,7 +54,7 @@ struct Slot {
     int32_t pad[6];
     int32_t prow[32];     // paged: cache row of each of the item's first 32 key pieces
                           // (-1: past the item's keys, -2: block-table entry out of range)
-    float w[kNmax];
+    float w[kNmax];       // weights of the item's columns, even columns halved (see epilogue)
 };
 static_assert(sizeof(Slot) == 64 + 128 + 4 * kNmax, "Slot size");
 
@@ -302,7 +302,9 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
 #pragma unroll
         for (int i = 0; i < kWPerLane; ++i) {
             const int e = lane + 32 * i;
-            wv[i] = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+            // even columns are staged halved: the epilogue takes their ReLU as x + |x|
+            const float we = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+            wv[i] = (e & 1) ? we : 0.5f * we;
         }
         if (P.piece_rows) tv = piece_row(P, cur.b, cur.j0, cur.j1, lane);
         return true;
@@ -496,16 +498,22 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                     float v[64];
                     tmem_ld64(acc + t * 64, v);
                     const float4 *w4 = reinterpret_cast<const float4 *>(S.w + t * 64);
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    // Even heads take the ReLU on the FMA pipe as x + |x| = 2 max(x, 0) with a
+                    // halved weight ((w/2)(2x) = w x exactly, so each FMA rounds the same value);
+                    // odd heads take max(x, 0) on the ALU pipe. The four partial sums (heads = 0,
+                    // 1, 2, 3 mod 4) are two packed pairs; a packed FMA is two round-to-nearest
+                    // fp32 FMAs.
+                    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int h4 = 0; h4 < 16; ++h4) {
                         const float4 ww = w4[h4];
-                        a0 = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), a0);
-                        a1 = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), a1);
-                        a2 = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), a2);
-                        a3 = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), a3);
+                        const float x0 = v[4 * h4 + 0], x2 = v[4 * h4 + 2];
+                        a01 = __ffma2_rn(make_float2(ww.x, ww.y),
+                                         make_float2(x0 + fabsf(x0), fmaxf(v[4 * h4 + 1], 0.f)), a01);
+                        a23 = __ffma2_rn(make_float2(ww.z, ww.w),
+                                         make_float2(x2 + fabsf(x2), fmaxf(v[4 * h4 + 3], 0.f)), a23);
                     }
-                    I = (a0 + a1) + (a2 + a3);
+                    I = (a01.x + a01.y) + (a23.x + a23.y);
                 } else {
                     const int c_lo = t * N1, c_hi = c_lo + N1;
                     float a = 0.f;
@@ -515,7 +523,8 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = ch + i;
-                            if (c >= c_lo && c < c_hi) a = fmaf(S.w[c], fmaxf(v[i], 0.f), a);
+                            if (c >= c_lo && c < c_hi)
+                                a = fmaf(S.w[c], (c & 1) ? fmaxf(v[i], 0.f) : v[i] + fabsf(v[i]), a);
                         }
                     }
                     I = a;
