@@ -63,6 +63,19 @@ SMALL = {
     "topk8192_n16": lambda: synthetic.bsnd(1, 4, 9000, 16, 8192, 0, seed=45),
     "offset_seqused": lambda: synthetic.tnd([10, 30], [60, 90], 4, 40, 3, seed=15,
                                             seqused_q=[7, 30], output_idx_offset=[1000, 5]),
+    # head counts that do not divide 256: tq = 5 / 10 rows, N = 240 (generic epilogue path)
+    "bsnd_n48": lambda: synthetic.bsnd(2, 130, 260, 48, 100, 3, seed=47),
+    "bsnd_n24_nomask": lambda: synthetic.bsnd(1, 50, 300, 24, 64, 0, seed=48),
+    # paged blocks of one full key tile, of two tiles, and without a mask
+    "paged_bs128": lambda: synthetic.paged([600, 300], 2, 64, 128, block_size=128, seed=49),
+    "paged_bs256_nomask": lambda: synthetic.paged([700, 90], 1, 32, 64, block_size=256,
+                                                  mask_mode=0, seed=50),
+    # small blocks over long windows: more than 32 key pieces per item (staged rows refilled)
+    "paged_bs16_long": lambda: synthetic.paged([1500, 700], 2, 16, 100, block_size=16, seed=52),
+    "paged_bs8_long": lambda: synthetic.paged([1900], 1, 8, 64, block_size=8, seed=53),
+    # few query blocks and long windows: key ranges split across work items
+    "paged_decode_split": lambda: synthetic.paged([5000, 3000, 100], 1, 64, 256, block_size=64,
+                                                  seed=51),
 }
 
 
