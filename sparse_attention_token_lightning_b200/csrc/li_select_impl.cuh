@@ -20,7 +20,10 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 constexpr int kBinCap = 128;          // largest bucket the per-bucket insertion sort takes
-constexpr int kBucketsMax = 4096;     // a power of two; at most 16 buckets per thread
+constexpr int kBucketsMax = 4096;     // a power of two
+// buckets per row: at most kBucketsMax and at most 16 per thread (the largest bucket scan)
+constexpr int kNbMax = kBucketsMax < 16 * kThreads ? kBucketsMax : 16 * kThreads;
+static_assert(kNbMax % kThreads == 0 && kNbMax / kThreads <= 16, "bucket scan covers 16 per thread");
 
 struct Smem {
     int32_t hist[kDigits];
@@ -343,7 +346,7 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float kInf = __int_as_float(0x7f800000);
     int32_t nb = kThreads;
-    while (nb < n && nb < kBucketsMax) nb <<= 1;
+    while (nb < n && nb < kNbMax) nb <<= 1;
     for (int i = tid; i < nb / 4; i += kThreads) reinterpret_cast<int4 *>(hist)[i] = make_int4(0, 0, 0, 0);
     if (tid == 0) { sm.s_cut = nb - 1; sm.s_maxbin = 0; }
     float v[kRegKeys];
@@ -457,7 +460,7 @@ __device__ int cand_bucket_topk(const uint64_t *cand, int32_t n_c, int32_t m, in
     }
     if (lane == 0) { sm.red_min[warp] = lo; sm.red_max[warp] = hi; }
     int32_t nb = kThreads;
-    while (nb < n_c && nb < kBucketsMax) nb <<= 1;
+    while (nb < n_c && nb < kNbMax) nb <<= 1;
     for (int i = tid; i < nb / 4; i += kThreads) reinterpret_cast<int4 *>(hist)[i] = make_int4(0, 0, 0, 0);
     if (tid == 0) { sm.s_cut = nb - 1; sm.s_maxbin = 0; }
     __syncthreads();
