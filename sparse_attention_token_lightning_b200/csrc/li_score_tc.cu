@@ -459,6 +459,44 @@ __device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
     if (!ok) *abort_flag = 1;
 }
 
+// Score of one key for one query row from its 64 head columns v (N1 = 64) and the row's staged
+// weights w: the sum over heads of w * ReLU(v). Even heads take the ReLU on the FMA pipe as
+// x + |x| = 2 max(x, 0) with a halved weight ((w/2)(2x) = w x exactly, so each FMA rounds the same
+// value); odd heads take max(x, 0) on the ALU pipe. The four partial sums (heads = 0, 1, 2, 3
+// mod 4) are two packed pairs; a packed FMA is two round-to-nearest fp32 FMAs.
+__device__ __forceinline__ float head_sum64(const float (&v)[64], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int h4 = 0; h4 < 16; ++h4) {
+        const float4 ww = w4[h4];
+        const float x0 = v[4 * h4 + 0], x2 = v[4 * h4 + 2];
+        a01 = __ffma2_rn(make_float2(ww.x, ww.y),
+                         make_float2(x0 + fabsf(x0), fmaxf(v[4 * h4 + 1], 0.f)), a01);
+        a23 = __ffma2_rn(make_float2(ww.z, ww.w),
+                         make_float2(x2 + fabsf(x2), fmaxf(v[4 * h4 + 3], 0.f)), a23);
+    }
+    return (a01.x + a01.y) + (a23.x + a23.y);
+}
+
+// The same sum for any N1: row t's columns [t*N1, (t+1)*N1) of the accumulator at acc, read 16
+// columns at a time; even columns carry halved weights.
+__device__ __forceinline__ float head_sum(uint32_t acc, const float *w, int t, int N1) {
+    const int c_lo = t * N1, c_hi = c_lo + N1;
+    float a = 0.f;
+    for (int ch = c_lo & ~15; ch < c_hi; ch += 16) {
+        float v[16];
+        tmem_ld16(acc + ch, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int c = ch + i;
+            if (c >= c_lo && c < c_hi)
+                a = fmaf(w[c], (c & 1) ? fmaxf(v[i], 0.f) : v[i] + fabsf(v[i]), a);
+        }
+    }
+    return a;
+}
+
 __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                          volatile int *abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -483,6 +521,11 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
         const int32_t q0 = S.q0, nq = S.nq, j0 = S.j0, j1 = S.j1, row0 = S.row0, L1u = S.L1u,
                       L2 = S.L2;
         const int32_t nt = n_tiles_of(j0, j1);
+        // At most one row per warp group (N1 >= 64): the row, its window end and its output
+        // row are fixed for the whole item.
+        const bool one_row = nq <= kEpiGroups;
+        const int32_t hi1 = one_row && group < nq ? min(window_hi(mask_mode, q0 + group, L1u, L2), j1) : 0;
+        float *const out1 = P.scores + (int64_t)(row0 + (one_row && group < nq ? group : 0)) * P.ld;
         for (int32_t tile = 0; tile < nt; ++tile, ar.next(P.n_acc)) {
             const int ab = ar.idx;
             if (!mbar_wait(bars.acc_full(ab), ar.phase, abort_flag)) { ok = false; break; }
@@ -490,46 +533,30 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
             const int32_t jt = j0 + tile * kKeyTile;
             const int32_t j = jt + 32 * quarter + lane;
             const uint32_t acc = tmem_base + lane_addr + ab * P.acc_stride;
-            for (int t = group; t < nq; t += kEpiGroups) {
-                const int32_t hi = min(window_hi(mask_mode, q0 + t, L1u, L2), j1);
-                if (jt >= hi) continue;                       // tile past this row's window
-                float I;
-                if (N1 == 64) {
+            if (one_row) {
+                if (N1 == 64 && jt < hi1) {
                     float v[64];
-                    tmem_ld64(acc + t * 64, v);
-                    const float4 *w4 = reinterpret_cast<const float4 *>(S.w + t * 64);
-                    // Even heads take the ReLU on the FMA pipe as x + |x| = 2 max(x, 0) with a
-                    // halved weight ((w/2)(2x) = w x exactly, so each FMA rounds the same value);
-                    // odd heads take max(x, 0) on the ALU pipe. The four partial sums (heads = 0,
-                    // 1, 2, 3 mod 4) are two packed pairs; a packed FMA is two round-to-nearest
-                    // fp32 FMAs.
-                    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int h4 = 0; h4 < 16; ++h4) {
-                        const float4 ww = w4[h4];
-                        const float x0 = v[4 * h4 + 0], x2 = v[4 * h4 + 2];
-                        a01 = __ffma2_rn(make_float2(ww.x, ww.y),
-                                         make_float2(x0 + fabsf(x0), fmaxf(v[4 * h4 + 1], 0.f)), a01);
-                        a23 = __ffma2_rn(make_float2(ww.z, ww.w),
-                                         make_float2(x2 + fabsf(x2), fmaxf(v[4 * h4 + 3], 0.f)), a23);
-                    }
-                    I = (a01.x + a01.y) + (a23.x + a23.y);
-                } else {
-                    const int c_lo = t * N1, c_hi = c_lo + N1;
-                    float a = 0.f;
-                    for (int ch = c_lo & ~15; ch < c_hi; ch += 16) {
-                        float v[16];
-                        tmem_ld16(acc + ch, v);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int c = ch + i;
-                            if (c >= c_lo && c < c_hi)
-                                a = fmaf(S.w[c], (c & 1) ? fmaxf(v[i], 0.f) : v[i] + fabsf(v[i]), a);
-                        }
-                    }
-                    I = a;
+                    tmem_ld64(acc + group * 64, v);
+                    const float I = head_sum64(v, S.w + group * 64);
+                    if (j < hi1) out1[j] = I;
+                } else if (jt < hi1) {
+                    const float I = head_sum(acc, S.w, group, N1);
+                    if (j < hi1) out1[j] = I;
                 }
-                if (j < hi) P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
+            } else {
+                for (int t = group; t < nq; t += kEpiGroups) {
+                    const int32_t hi = min(window_hi(mask_mode, q0 + t, L1u, L2), j1);
+                    if (jt >= hi) continue;                       // tile past this row's window
+                    float I;
+                    if (N1 == 64) {
+                        float v[64];
+                        tmem_ld64(acc + t * 64, v);
+                        I = head_sum64(v, S.w + t * 64);
+                    } else {
+                        I = head_sum(acc, S.w, t, N1);
+                    }
+                    if (j < hi) P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
+                }
             }
             tc_fence_before();
             __syncwarp();
