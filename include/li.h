@@ -140,7 +140,9 @@ li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *s
  *   tq            query rows per work item (tq x num_heads_q <= 256 MMA columns)
  *   kc            keys per work item, 0 when each item covers its rows' whole window
  *   max_items     capacity of the work list
- *   dense         1 when the work list is a closed form of the shapes and no schedule kernel runs
+ *   dense         0: a schedule kernel builds the work list; 1: dense BSND closed form; 2: closed
+ *                 form for one query block per batch with per-batch key lengths (decode); with
+ *                 1 or 2 no schedule kernel runs
  *   kernels       kernels one li_indexer call launches with metadata == NULL (0 when there are no
  *                 query rows); one fewer schedule kernel when a metadata buffer is passed
  *   score_tc      1 when the score step runs on the tcgen05 kernel, 0 on the CUDA-core kernel

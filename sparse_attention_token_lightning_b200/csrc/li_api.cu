@@ -192,6 +192,10 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     // dense BSND with no seqused and no key split: the work list has a closed form
     S.dense = (P.layout_q == LI_LAYOUT_BSND && P.layout_k == LI_LAYOUT_BSND && !P.seqused_q &&
                !P.seqused_k && S.kc == 0 && P.max_seqlen_k == P.k_len) ? 1 : 0;
+    // decode-shaped: one query block per batch, BSND or paged keys with per-batch lengths
+    if (!S.dense && P.layout_q == LI_LAYOUT_BSND && !P.seqused_q && P.q_len <= S.tq &&
+        (P.layout_k == LI_LAYOUT_BSND || P.layout_k == LI_LAYOUT_PA_BSND))
+        S.dense = 2;
     const int64_t splits = S.kc > 0 ? ((int64_t)P.max_seqlen_k + S.kc - 1) / S.kc : 1;
     const int64_t max_items = qblocks * splits;
     if (max_items > INT32_MAX / 2) return fail(LI_ERR_UNSUPPORTED, "schedule too large");
@@ -250,7 +254,7 @@ li_status li_plan(const li_args *args, li_plan_info *info) {
     info->tq = s.tq;
     info->kc = s.kc;
     info->max_items = s.max_items;
-    info->dense = s.dense ? 1 : 0;
+    info->dense = s.dense;
     info->kernels = p.rows > 0 ? (s.dense ? 2 : 3) : 0;
     info->score_tc = !use_simple_kernel() && li::score_tc_eligible(p, s) ? 1 : 0;
     return ok();

@@ -136,35 +136,86 @@ struct Schedule {
     int tq;          // query rows per item
     int kc;          // key-range split (0 = none)
     int max_items;   // capacity of the item list
-    int dense;       // 1: dense BSND without seqused and without key split; the work list is a
-                     //    closed-form function of the item number and needs no schedule kernel
+    int dense;       // work lists in closed form (no schedule kernel): 1 = dense BSND without
+                     // seqused and without key split; 2 = BSND queries, no seqused_q, all of a
+                     // batch's rows in one query block (decode), BSND or paged keys with
+                     // per-batch lengths; 0 = the schedule kernel builds the list
 };
 
+// Keys of batch b from the device-resident lengths, clamped the way the schedule kernel clamps
+// them (BSND or paged keys); sets LI_DEVERR_LENGTHS in *err when the stored length is out of
+// range.
+__device__ inline int32_t batch_keys(const Problem &p, int32_t b, uint32_t *err) {
+    int64_t L2;
+    if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        const int64_t u = p.seqused_k[b];
+        const int64_t cap = p.bt_stride * (int64_t)p.block_size;
+        if (u < 0 || u > cap) *err |= LI_DEVERR_LENGTHS;
+        L2 = u < 0 ? 0 : (u > cap ? cap : u);
+    } else {
+        L2 = p.k_len;
+        if (p.seqused_k) {
+            const int64_t u = p.seqused_k[b];
+            if (u < 0 || u > L2) *err |= LI_DEVERR_LENGTHS;
+            L2 = u < 0 ? 0 : (u < L2 ? u : L2);
+        }
+    }
+    if (L2 > p.max_seqlen_k) {
+        *err |= LI_DEVERR_LENGTHS;
+        L2 = p.max_seqlen_k;
+    }
+    return (int32_t)L2;
+}
+
 // Work list and per-batch lengths as the kernels see them: either the schedule built by
-// li_metadata (a MetaHeader in device memory) or, for dense BSND problems, closed forms.
+// li_metadata (a MetaHeader in device memory) or closed forms (Schedule::dense 1 or 2).
 struct SchedView {
-    const void *meta;      // nullptr: dense closed forms
+    const void *meta;      // nullptr: closed forms
     int32_t tq;
     int32_t n_items;
     int32_t nqb;           // dense: query blocks per batch
+    int32_t mode;          // closed form: 1 dense BSND, 2 one query block per batch
+    int32_t kc;            // mode 2: keys per item (0: the whole window)
+    int32_t splits;        // mode 2: item slots per batch (ceil(max_seqlen_k / kc), or 1)
 
     __device__ BatchInfo batch(const Problem &p, int32_t b) const {
         if (meta) return meta_batches(meta)[b];
         BatchInfo bi;
+        uint32_t err = 0;
         bi.L1 = bi.L1u = p.q_len;
-        bi.L2 = p.k_len;
+        bi.L2 = mode == 2 ? batch_keys(p, b, &err) : p.k_len;
         bi.q_row0 = b * p.q_len;
-        bi.k_row0 = b * p.k_len;
+        bi.k_row0 = p.layout_k == LI_LAYOUT_PA_BSND ? 0 : b * p.k_len;
         bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
         return bi;
     }
-    // Item t of the list (0 <= t < n_items). Dense: query blocks last-to-first (for the causal
-    // mask that is longest first), batches interleaved; an item whose window is empty has
-    // j1 <= j0 and is skipped by the caller.
+    // Item t of the list (0 <= t < n_items); an item whose window is empty has j1 <= j0 and is
+    // skipped by the caller. Mode 1: query blocks last-to-first (for the causal mask that is
+    // longest first), batches interleaved. Mode 2: key piece s = t / B of batch b = t % B, so
+    // every batch's first pieces come first; pieces past a batch's keys are empty.
     __device__ WorkItem item(const Problem &p, int32_t t) const {
         const int32_t hb = meta ? reinterpret_cast<const MetaHeader *>(meta)->batch : 0;
         if (meta) return meta_items(meta, hb)[t];
         WorkItem it;
+        if (mode == 2) {
+            const int32_t sp = t / p.batch;
+            uint32_t err = 0;
+            it.b = t - sp * p.batch;
+            it.q0 = 0;
+            it.nq = p.q_len;
+            it.L1u = p.q_len;
+            it.L2 = batch_keys(p, it.b, &err);
+            const int32_t jend = window_hi(p.mask_mode, p.q_len - 1, p.q_len, it.L2);
+            const int32_t span = kc > 0 ? kc : jend;
+            const int64_t j0 = (int64_t)sp * span;
+            it.j0 = j0 < jend ? (int32_t)j0 : jend;
+            it.j1 = j0 < jend ? min(jend, it.j0 + span) : jend;
+            it.cost = 0;
+            it.row0 = it.b * p.q_len;
+            it.k_row0 = p.layout_k == LI_LAYOUT_PA_BSND ? 0 : it.b * p.k_len;
+            for (int i = 0; i < 6; ++i) it.pad[i] = 0;
+            return it;
+        }
         const int32_t qb = nqb - 1 - t / p.batch;
         it.b = t % p.batch;
         it.q0 = qb * tq;
@@ -181,13 +232,27 @@ struct SchedView {
     }
 };
 
+// Closed form with per-batch key lengths (mode 2) has no schedule kernel to check the stored
+// lengths: threads tid0, tid0 + nthr, ... of one block check them and set the status bits.
+__device__ inline void check_batch_keys(const Problem &p, const SchedView &v, uint32_t *status,
+                                        int tid0, int nthr) {
+    if (v.meta || v.mode != 2) return;
+    uint32_t err = 0;
+    for (int32_t b = tid0; b < p.batch; b += nthr) (void)batch_keys(p, b, &err);
+    if (err) atomicOr(status, err);
+}
+
 // Builds the view for a kernel launch. meta == nullptr selects the dense closed forms.
 inline SchedView make_view(const Problem &p, const Schedule &s, const void *meta) {
     SchedView v;
     v.meta = meta;
     v.tq = s.tq;
     v.nqb = p.q_len > 0 ? (p.q_len + s.tq - 1) / s.tq : 0;
-    v.n_items = meta ? 0 : p.batch * v.nqb;   // with metadata the count is read on the device
+    v.mode = s.dense;
+    v.kc = s.kc;
+    v.splits = s.kc > 0 ? (p.max_seqlen_k + s.kc - 1) / s.kc : 1;
+    // with metadata the count is read on the device
+    v.n_items = meta ? 0 : (s.dense == 2 ? p.batch * v.splits : p.batch * v.nqb);
     return v;
 }
 

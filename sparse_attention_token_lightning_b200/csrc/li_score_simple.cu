@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
         n_items = hdr->n_items;
     }
     const int H = p.n_heads;
+    if (blockIdx.x == 0) check_batch_keys(p, view, &sp.ws->status, threadIdx.x, kThreads);
 
     __shared__ float qs[kMaxHeads][kHeadDim];
     __shared__ float ws_[kMaxHeads];

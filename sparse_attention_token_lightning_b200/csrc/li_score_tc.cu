@@ -627,6 +627,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     if (warp == 0) {
         producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
     } else if (warp == kSchedWarp) {
+        if (blockIdx.x == 0) check_batch_keys(P.p, P.view, &P.ws->status, lane, 32);
         scheduler(P, smem, bars, abort_flag, n_items);
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);

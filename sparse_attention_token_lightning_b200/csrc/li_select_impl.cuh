@@ -669,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     if (b >= 0) {
         const BatchInfo bi = sp.view.batch(p, b);
         n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2);
+
         if (p.output_idx_offset) {
             off = p.output_idx_offset[b];
             // the schedule kernel validates offsets; without it each row checks its own

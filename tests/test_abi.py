@@ -151,13 +151,13 @@ def test_plan_reports_schedule_and_kernel_count(L):
                           num_heads_q=64, seqused_k=0x40000, block_table=0x50000,
                           block_table_stride=512, num_blocks=64 * 512, block_size=64,
                           max_seqlen_k=32768, topk=2048))
-    assert pl["tq"] == 1 and pl["dense"] == 0 and pl["kernels"] == 3 and pl["score_tc"] == 1
+    assert pl["tq"] == 1 and pl["dense"] == 2 and pl["kernels"] == 2 and pl["score_tc"] == 1
     assert pl["kc"] > 0 and pl["max_items"] >= 64 * (32768 // pl["kc"])
     # block sizes the TMA pieces cannot tile go to the CUDA-core score kernel
     pl = li.li_plan(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
                           block_table_stride=64, num_blocks=64, block_size=12,
                           max_seqlen_k=512))
-    assert pl["score_tc"] == 0 and pl["kernels"] == 3
+    assert pl["score_tc"] == 0 and pl["kernels"] == 3 and pl["dense"] == 0
     # no query rows: nothing launches
     assert li.li_plan(_args(batch=0))["kernels"] == 0
     # argument errors come back as status codes

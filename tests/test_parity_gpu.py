@@ -128,6 +128,24 @@ def test_dense_closed_form_schedule_matches_metadata(shape):
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
 
 
+@pytest.mark.parametrize("make", [
+    lambda: synthetic.paged([5000, 3000, 100], 1, 64, 256, block_size=64, seed=54),
+    lambda: synthetic.paged([300, 45, 0], 2, 32, 64, block_size=16, seed=55),
+    lambda: synthetic.bsnd(3, 1, 3000, 64, 100, 3, seed=56, seqused_k=[3000, 10, 2500]),
+    lambda: synthetic.bsnd(2, 3, 700, 16, 40, 0, seed=57, seqused_k=[700, 0]),
+])
+def test_decode_closed_form_schedule_matches_metadata(orc, make):
+    """One query block per batch with per-batch key lengths: the work list is a closed form of
+    seqused_k (no schedule kernel); an explicit schedule must give bit-identical outputs, and
+    both must match the oracle."""
+    pb = make()
+    assert li.li_plan(li.make_args(pb))["dense"] == 2
+    a = run(pb, metadata=False)
+    b = run(pb, metadata=True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+    parity.check(orc, pb, a[0], a[1], label="decode closed form")
+
+
 def test_deterministic_reruns():
     pb = synthetic.bsnd(1, 1024, 1024, 64, 256, 3, seed=32).to("cuda")
     i1, v1 = li.indexer(pb)
