@@ -568,11 +568,12 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
     } else {
         __syncthreads();
     }
-    // pass 2: keys of bins 0..cut, 16 per thread per iteration, one atomic per warp
+    // pass 2: keys of bins 0..cut, 16 per thread per iteration: each thread packs its take flags
+    // into a mask, a warp scan of the counts gives every thread its write position, and one
+    // atomic per warp claims the warp's space
     auto takes = [&](float v) -> bool {
         return (int32_t)((kDigitBins - 1) - (int32_t)(score_key(v) >> 20)) <= cut;
     };
-    const uint32_t lt = lanemask_lt();
     for (int32_t c0 = 0; c0 < n4; c0 += kUnroll * kThreads) {
         float4 x[kUnroll];
 #pragma unroll
@@ -580,35 +581,39 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
             const int32_t i4 = c0 + k * kThreads + tid;
             x[k] = i4 < n4 ? __ldcg(src4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        uint32_t ball[4 * kUnroll];
-        int32_t total = 0;
+        uint32_t mask = 0;
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
-            const bool valid = c0 + k * kThreads + tid < n4;
-            ball[4 * k + 0] = __ballot_sync(0xffffffffu, valid && takes(x[k].x));
-            ball[4 * k + 1] = __ballot_sync(0xffffffffu, valid && takes(x[k].y));
-            ball[4 * k + 2] = __ballot_sync(0xffffffffu, valid && takes(x[k].z));
-            ball[4 * k + 3] = __ballot_sync(0xffffffffu, valid && takes(x[k].w));
+            if (c0 + k * kThreads + tid < n4) {
+                mask |= (takes(x[k].x) ? 1u : 0u) << (4 * k + 0);
+                mask |= (takes(x[k].y) ? 1u : 0u) << (4 * k + 1);
+                mask |= (takes(x[k].z) ? 1u : 0u) << (4 * k + 2);
+                mask |= (takes(x[k].w) ? 1u : 0u) << (4 * k + 3);
+            }
         }
+        const int32_t cnt = __popc(mask);
+        int32_t incl = cnt;
 #pragma unroll
-        for (int q = 0; q < 4 * kUnroll; ++q) total += __popc(ball[q]);
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const int32_t total = __shfl_sync(0xffffffffu, incl, 31);
         if (total == 0) continue;
         int32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sm.s_append, total);
-        base = __shfl_sync(0xffffffffu, base, 0);
+        if (lane == 31) base = atomicAdd(&sm.s_append, total);
+        int32_t pos = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
             const int32_t i4 = c0 + k * kThreads + tid;
             const float vals[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint32_t bl = ball[4 * k + c];
-                if (bl & (1u << lane)) {
-                    const int32_t pos = base + __popc(bl & lt);
+                if (mask & (1u << (4 * k + c))) {
                     if (pos < n_c)
                         cand[pos] = ((uint64_t)score_key(vals[c]) << 32) | (uint32_t)~(uint32_t)(4 * i4 + c);
+                    ++pos;
                 }
-                base += __popc(bl);
             }
         }
     }
@@ -621,7 +626,7 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
             int32_t base = 0;
             if (lane == 0) base = atomicAdd(&sm.s_append, __popc(bl));
             base = __shfl_sync(0xffffffffu, base, 0);
-            const int32_t pos = base + __popc(bl & lt);
+            const int32_t pos = base + __popc(bl & lanemask_lt());
             if (take && pos < n_c) cand[pos] = ((uint64_t)score_key(v) << 32) | (uint32_t)~(uint32_t)e;
         }
     }
