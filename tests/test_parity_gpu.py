@@ -133,6 +133,9 @@ def test_dense_closed_form_schedule_matches_metadata(shape):
     lambda: synthetic.paged([300, 45, 0], 2, 32, 64, block_size=16, seed=55),
     lambda: synthetic.bsnd(3, 1, 3000, 64, 100, 3, seed=56, seqused_k=[3000, 10, 2500]),
     lambda: synthetic.bsnd(2, 3, 700, 16, 40, 0, seed=57, seqused_k=[700, 0]),
+    # more batches than the score kernel's register-held work list takes (256)
+    lambda: synthetic.paged([(7 * b) % 400 + 1 for b in range(300)], 1, 8, 32, block_size=16,
+                            seed=58),
 ])
 def test_decode_closed_form_schedule_matches_metadata(orc, make):
     """One query block per batch with per-batch key lengths: the work list is a closed form of
