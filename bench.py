@@ -190,6 +190,19 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count (the oracle timing runs on one of them)."""
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu": model, "nproc": os.cpu_count()}
+
+
 def cpu_oracle_rate(pb, seconds: float, seed: int = 0):
     """Time the CPU oracle (as it stands, one thread) on seeded random rows of the workload for
     about `seconds`; returns (query rows per second, rows timed)."""
@@ -235,7 +248,8 @@ def run_reference(a):
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{rows} seeded-random query rows over {a.steps} steps "
                                        f"(~{step_seconds:.0f} s each), single-threaded C oracle; "
-                                       "per-row cost is unbiased so rows/s scales to the workload"},
+                                       "per-row cost is unbiased so rows/s scales to the workload",
+                             "host": host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -415,7 +429,9 @@ def main():
         rate, n, t = cpu_oracle_rate(pb_cpu, a.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
                                 "sample": f"{n} seeded-random query rows of the same workload, "
-                                          f"{t:.1f} s, single-threaded C oracle (fp64)"}
+                                          f"{t:.1f} s, single-threaded C oracle (fp64); rows/s "
+                                          "scales to the workload (row cost is unbiased)",
+                                "host": host_cpu()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
