@@ -149,6 +149,37 @@ def test_decode_closed_form_schedule_matches_metadata(orc, make):
     parity.check(orc, pb, a[0], a[1], label="decode closed form")
 
 
+@pytest.mark.parametrize("make", [
+    lambda seed: synthetic.bsnd(1, 300, 300, 64, 64, 3, seed=seed),
+    lambda seed: synthetic.paged([900, 300, 4100], 1, 64, 128, block_size=64, seed=seed),
+    lambda seed: synthetic.tnd([100, 3, 250], [100, 400, 260], 64, 64, 3, seed=seed),
+])
+def test_indexer_replays_in_a_cuda_graph(make):
+    """li_indexer launches stream-ordered work only, so a captured call replays: new data copied
+    into the same buffers gives the outputs of an eager call on that data, bit for bit."""
+    pb = make(60).to("cuda")
+    args = li.make_args(pb)
+    ws = li.empty_workspace(args, "cuda")
+    idx = torch.empty(li.out_shape(pb), dtype=torch.int32, device="cuda")
+    val = torch.empty(li.out_shape(pb), dtype=torch.float32, device="cuda")
+    li.li_indexer(args, None, ws, idx, val)        # first call outside capture
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        li.li_indexer(args, None, ws, idx, val, side)
+    fresh = make(61)
+    for f in synthetic.Problem.TENSORS:        # data, lengths and block table alike
+        if getattr(pb, f) is not None:
+            getattr(pb, f).copy_(getattr(fresh, f))
+    g.replay()
+    torch.cuda.synchronize()
+    st, bits = li.li_check_status(ws)
+    assert st == li.LI_OK, bits
+    ei, ev = li.indexer(fresh.to("cuda"))
+    assert torch.equal(idx, ei) and torch.equal(val.view(torch.int32), ev.view(torch.int32))
+
+
 def test_deterministic_reruns():
     pb = synthetic.bsnd(1, 1024, 1024, 64, 256, 3, seed=32).to("cuda")
     i1, v1 = li.indexer(pb)
