@@ -102,10 +102,10 @@ def score_kernel_bytes(pb, pairs) -> int:
 # with the sha256 of the score-kernel sources the counters were taken on; reported only while the
 # sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
 SCORE_TRAFFIC = {
-    "causal_prefill": {"bytes": 68724224 + 9434112,
-                       "src_sha256": "56c0d01832db8ae174a743d60053396abcbacaa6743526c036c0b9fc8fdd2f2b"},
-    "paged_decode": {"bytes": 286931712 + 7193344,
-                     "src_sha256": "56c0d01832db8ae174a743d60053396abcbacaa6743526c036c0b9fc8fdd2f2b"},
+    "causal_prefill": {"bytes": 68743680 + 9866752,
+                       "src_sha256": "77867c76e600c743c5b645f62403cecb65f0df2a57c04c4af0d86e71d8e3e0bb"},
+    "paged_decode": {"bytes": 286281728 + 6766592,
+                     "src_sha256": "77867c76e600c743c5b645f62403cecb65f0df2a57c04c4af0d86e71d8e3e0bb"},
 }
 SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
                  "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")
