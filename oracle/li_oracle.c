@@ -15,6 +15,13 @@
  *   2. The key window of query row i (custom_pypto.npu_lightning_indexer_pto, sparse_mode:
  *      0 = no mask, 3 = right-down causal, i.e. the lower triangle anchored at the bottom-right
  *      corner): mode 0 keeps 0 <= j < L2_b, mode 3 additionally keeps j <= i + L2_b - L1_b.
+ *      Compressed keys (lightning_indexer, "Prototype": cmp_ratio and cmp_residual_k;
+ *      "Constraints": cmp_residual_k[b] < cmp_ratio, required with cmp_ratio > 1 and mask 3):
+ *      [reading] key j of batch b stands for original tokens [j*r, (j+1)*r) of a sequence of
+ *      L2_b*r + cmp_residual_k[b] tokens, and under mode 3 it is kept when its last token is
+ *      visible: (j+1)*r - 1 <= i + L2_b*r + cmp_residual_k[b] - L1_b. The pages state no rule
+ *      and give no worked values for it: parity of this reading is unpinned beyond the
+ *      whole-block relation the pins check.
  *   3. The index score (custom_pypto.npu_lightning_indexer_pto, formula in the function
  *      description; lightning_indexer, "Function" steps 1-3 and "Formula"):
  *         I[i,j] = sum_h w[i,h] * ReLU( q[i,h,:] . k[j,:] )
@@ -67,6 +74,8 @@ typedef struct {
     int32_t num_blocks, block_size;
     int32_t n_heads, head_dim, topk;
     int32_t layout_q, layout_k, mask_mode;
+    const int32_t *cmp_residual_k;  /* [B] or NULL: tokens past the last whole compressed key */
+    int32_t cmp_ratio;              /* original tokens per key; 0 or 1 = keys not compressed  */
 } orc_problem;
 
 static double bf16_value(uint16_t bits)
@@ -87,6 +96,7 @@ typedef struct {
     int32_t b, i;          /* batch and row position within the batch                      */
     int64_t L1, L2;        /* query rows allocated / keys valid for the batch              */
     int64_t L1_used;       /* query rows in use (seqused_q), used for validity + alignment */
+    int64_t res;           /* compressed keys: residual original tokens of the batch           */
 } orc_row;
 
 static int orc_locate(const orc_problem *p, int64_t r, orc_row *o)
@@ -96,7 +106,7 @@ static int orc_locate(const orc_problem *p, int64_t r, orc_row *o)
         for (int bb = 0; bb < p->batch; ++bb)
             if (p->cu_seqlens_q[bb] <= r && r < p->cu_seqlens_q[bb + 1]) { b = bb; break; }
         if (b < 0) {            /* row not covered by any batch: no valid keys */
-            o->b = -1; o->i = 0; o->L1 = 0; o->L2 = 0; o->L1_used = 0;
+            o->b = -1; o->i = 0; o->L1 = 0; o->L2 = 0; o->L1_used = 0; o->res = 0;
             return ORC_OK;
         }
         o->b = b;
@@ -119,6 +129,7 @@ static int orc_locate(const orc_problem *p, int64_t r, orc_row *o)
     o->L1_used = o->L1;
     if (p->seqused_q && p->seqused_q[o->b] < o->L1_used)
         o->L1_used = p->seqused_q[o->b];
+    o->res = p->cmp_residual_k ? p->cmp_residual_k[o->b] : 0;
     return ORC_OK;
 }
 
@@ -127,6 +138,19 @@ static int64_t orc_window(const orc_problem *p, const orc_row *o)
 {
     if (o->b < 0 || o->i >= o->L1_used || o->L2 <= 0) return 0;
     int64_t hi = o->L2;
+    if (p->mask_mode == 3 && p->cmp_ratio > 1) {
+        /* compressed keys: count keys from the first while each one's last original token is
+           visible to row i (original tokens aligned right-down like uncompressed keys) */
+        const int64_t r = p->cmp_ratio;
+        const int64_t horizon = (int64_t)o->i + o->L2 * r + o->res - o->L1_used;
+        int64_t n = 0;
+#if ORC_MUTANT == 12
+        while (n < o->L2 && n * r <= horizon) ++n;           /* mistake: first token visible */
+#else
+        while (n < o->L2 && (n + 1) * r - 1 <= horizon) ++n;
+#endif
+        return n;
+    }
     if (p->mask_mode == 3) {
         /* [reading] right-down causal aligns the last used query row with the last key. */
 #if ORC_MUTANT == 3
@@ -241,6 +265,11 @@ static int orc_check(const orc_problem *p)
     if (p->layout_k == ORC_TND && !p->cu_seqlens_k) return ORC_EARG;
     if (p->layout_k == ORC_PA_BSND && (!p->seqused_k || !p->block_table || p->block_size < 1))
         return ORC_EARG;
+    if (p->cmp_ratio < 0) return ORC_EARG;
+    if (p->cmp_residual_k)
+        for (int b = 0; b < p->batch; ++b)
+            if (p->cmp_residual_k[b] < 0 || p->cmp_residual_k[b] >= (p->cmp_ratio > 1 ? p->cmp_ratio : 1))
+                return ORC_EDATA;
     return ORC_OK;
 }
 

@@ -48,6 +48,7 @@ class _Problem(ctypes.Structure):
         ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
         ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
+        ("cmp_residual_k", ctypes.c_void_p), ("cmp_ratio", ctypes.c_int32),
     ]
 
 
@@ -105,7 +106,7 @@ class Oracle:
         s.k = ptr("k", _bits16(pb.k))
         s.w = ptr("w", _bits16(pb.w))
         for f in ("cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k", "block_table",
-                  "output_idx_offset"):
+                  "output_idx_offset", "cmp_residual_k"):
             setattr(s, f, ptr(f, _i32(getattr(pb, f, None))))
         bt = keep.get("block_table")
         s.block_table_stride = int(bt.shape[-1]) if bt is not None and bt.ndim == 2 else 0
@@ -120,6 +121,7 @@ class Oracle:
         s.layout_q = LAYOUTS[pb.layout_q]
         s.layout_k = LAYOUTS[pb.layout_k]
         s.mask_mode = int(pb.mask_mode)
+        s.cmp_ratio = int(getattr(pb, "cmp_ratio", 1) or 1)
         return s, keep
 
     # -- entry points ----------------------------------------------------------------------

@@ -51,10 +51,12 @@ class Problem:
     output_idx_offset: Optional[torch.Tensor] = None
     num_blocks: int = 0
     block_size: int = 0
+    cmp_ratio: int = 1                 # original tokens per key (1: keys not compressed)
+    cmp_residual_k: Optional[torch.Tensor] = None   # [B] tokens past the last whole key
     meta: dict = field(default_factory=dict)
 
     TENSORS = ("q", "k", "w", "cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k",
-               "block_table", "output_idx_offset")
+               "block_table", "output_idx_offset", "cmp_residual_k")
 
     @property
     def rows(self) -> int:
@@ -110,6 +112,15 @@ def _qkw(g, q_shape, k_shape, w_shape, n_heads, integer):
 
 def _i32(x) -> torch.Tensor:
     return torch.as_tensor(x, dtype=torch.int32)
+
+
+def compressed(pb: Problem, cmp_ratio: int, residual) -> Problem:
+    """The same problem with its keys read as compressed keys: each stands for cmp_ratio
+    original tokens, and batch b's sequence has residual[b] (< cmp_ratio) more tokens than its
+    whole keys cover (lightning_indexer, "Prototype": cmp_ratio, cmp_residual_k)."""
+    return pb.replace(cmp_ratio=int(cmp_ratio),
+                      cmp_residual_k=None if residual is None else _i32(residual),
+                      name=f"{pb.name}_cmp{cmp_ratio}")
 
 
 def bsnd(B, S1, S2, N1, topk, mask_mode=3, seed=0, D=D_DEFAULT, integer=False, name="bsnd",

@@ -265,6 +265,32 @@ def pin_invariants_on_random_problems(orc):
         check_row_invariants(orc, pb, idx, val)
 
 
+def pin_compressed_window_counts_whole_blocks(orc):
+    """Compressed keys under the right-down mask: a row keeps exactly the keys whose r original
+    tokens all lie in the uncompressed window of the same row over the L2*r + res original
+    tokens, so its window is floor(uncompressed window / r). The uncompressed window comes from
+    the (separately pinned) uncompressed path on a problem with L2*r + res keys."""
+    cases = [(5, 7, 4, [2]), (9, 3, 2, [1]), (6, 11, 3, [0]), (12, 5, 5, [4]), (1, 6, 4, [3])]
+    for L1, L2c, r, res in cases:
+        comp = synthetic.compressed(synthetic.bsnd(1, L1, L2c, 2, 4, 3, seed=70), r, res)
+        full = synthetic.bsnd(1, L1, L2c * r + res[0], 2, 4, 3, seed=70)
+        bc, bf = orc.bind(comp), orc.bind(full)
+        for i in range(L1):
+            hc, _, _ = bc.row_info(i)
+            hf, _, _ = bf.row_info(i)
+            assert hc == hf // r, (L1, L2c, r, res, i, hc, hf)
+    # ratio 1 without residuals is the uncompressed problem, outputs included
+    pb = synthetic.bsnd(2, 30, 40, 4, 16, 3, seed=71)
+    a = orc.topk(pb)
+    b = orc.topk(synthetic.compressed(pb, 1, [0, 0]))
+    _assert_same(a[0], b[0], "indices")
+    _assert_same(_bits(a[1]), _bits(b[1]), "values")
+    # the unmasked window ignores the compression
+    pb0 = synthetic.bsnd(1, 8, 10, 2, 4, 0, seed=72)
+    for i in range(8):
+        assert orc.bind(synthetic.compressed(pb0, 4, [3])).row_info(i)[0] == 10
+
+
 def pin_pages_example_shape(orc):
     """The pages' worked example shape (B=2, S1=64, N1=16, topk=32) with 32 keys and mask 3:
     rows i < 32 see no key (i + S2 - S1 < 0) and row i >= 32 sees i - 31 keys."""
