@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define LI_ABI_VERSION 1
+#define LI_ABI_VERSION 2
 
 typedef enum li_layout {
     LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
@@ -107,6 +107,15 @@ typedef struct li_args {
     int32_t dtype_qk;                   /* li_dtype of q and k: LI_DTYPE_BF16                   */
     int32_t dtype_w;                    /* li_dtype of w: LI_DTYPE_BF16                         */
     int32_t return_value;               /* 1: write sparse_values too; 0: indices only          */
+    /* Compressed keys (lightning_indexer, "Prototype": cmp_ratio, cmp_residual_k; "Constraints":
+     * cmp_residual_k[b] < cmp_ratio, passed only with cmp_ratio > 1 and mask_mode 3). Each key
+     * stands for cmp_ratio original tokens and batch b's sequence has cmp_residual_k[b] tokens
+     * past its last whole key. The pages state no mask rule for them; the reading implemented:
+     * under mask_mode 3 key j is kept for query row i when its last original token is visible,
+     * (j+1)*cmp_ratio - 1 <= i + L2_b*cmp_ratio + cmp_residual_k[b] - L1_b. Device values outside
+     * [0, cmp_ratio) set LI_DEVERR_LENGTHS. */
+    const int32_t *cmp_residual_k;      /* [B] int32, or NULL                                   */
+    int32_t cmp_ratio;                  /* original tokens per key; 0 or 1 = not compressed     */
 } li_args;
 
 /*

@@ -72,6 +72,13 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
         return fail(LI_ERR_INVALID_ARG, "topk=%d outside [1, 8192]", a->topk);
     if (a->mask_mode != 0 && a->mask_mode != 3)
         return fail(LI_ERR_INVALID_ARG, "mask_mode=%d, must be 0 or 3", a->mask_mode);
+    // compressed keys: residuals are passed exactly when cmp_ratio > 1 under mask_mode 3
+    // (lightning_indexer / aclnnLightningIndexerV2 constraints)
+    if (a->cmp_ratio < 0)
+        return fail(LI_ERR_INVALID_ARG, "cmp_ratio=%d < 0", a->cmp_ratio);
+    if ((a->cmp_ratio > 1 && a->mask_mode == 3) != (a->cmp_residual_k != nullptr))
+        return fail(LI_ERR_INVALID_ARG,
+                    "cmp_residual_k is required with cmp_ratio > 1 and mask_mode 3, else absent");
     if (a->layout_q != LI_LAYOUT_BSND && a->layout_q != LI_LAYOUT_TND)
         return fail(LI_ERR_INVALID_ARG, "layout_q=%d, must be BSND or TND", a->layout_q);
     if (a->layout_k != LI_LAYOUT_BSND && a->layout_k != LI_LAYOUT_TND &&
@@ -164,6 +171,8 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     P.mask_mode = a->mask_mode;
     P.return_value = a->return_value;
     P.rows = (int32_t)rows;
+    P.cmp_ratio = a->cmp_ratio > 1 ? a->cmp_ratio : 1;
+    P.cmp_residual_k = a->cmp_residual_k;
 
     // Schedule: query blocks of tq rows (all N1 heads of tq rows fill one 256-column MMA tile),
     // split along the keys when there are too few blocks to fill the GPU.
@@ -196,6 +205,8 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     if (!S.dense && P.layout_q == LI_LAYOUT_BSND && !P.seqused_q && P.q_len <= S.tq &&
         (P.layout_k == LI_LAYOUT_BSND || P.layout_k == LI_LAYOUT_PA_BSND))
         S.dense = 2;
+    // per-batch residuals of compressed keys are read and checked by the schedule kernel
+    if (P.cmp_residual_k) S.dense = 0;
     const int64_t splits = S.kc > 0 ? ((int64_t)P.max_seqlen_k + S.kc - 1) / S.kc : 1;
     const int64_t max_items = qblocks * splits;
     if (max_items > INT32_MAX / 2) return fail(LI_ERR_UNSUPPORTED, "schedule too large");

@@ -44,7 +44,8 @@ struct BatchInfo {
     int32_t L2;            // keys of the batch
     int32_t q_row0;        // global query row of the batch's row 0
     int32_t k_row0;        // BSND: b*S2, TND: cu_seqlens_k[b], PA: 0
-    int32_t pad[3];
+    int32_t pad[3];        // schedule kernel: [0] query blocks, [1] first block; [2] residual
+                           // tokens of compressed keys (cmp_residual_k[b], else 0)
 };
 static_assert(sizeof(BatchInfo) == 32, "BatchInfo size");
 
@@ -59,7 +60,9 @@ struct alignas(16) WorkItem {
     int32_t cost;          // key tiles, for ordering
     int32_t row0;          // global query row of q0 (the batch's q_row0 + q0)
     int32_t L1u;           // the batch's query rows in use
-    int32_t L2;            // the batch's keys
+    int32_t L2;            // the batch's keys; compressed keys: j1 + L1u, so that the score
+                           // kernel's plain right-down window reaches j1 for every row of the item
+                           // (a superset of each row's window; the selection applies the exact one)
     int32_t k_row0;        // the batch's first key row
     int32_t pad[6];
 };
@@ -89,11 +92,15 @@ __host__ __device__ inline const WorkItem *meta_items(const void *meta, int batc
 }
 
 // Window of row i of a batch: keys [0, hi). mask 0: hi = L2. mask 3 (right-down causal):
-// hi = min(L2, i + L2 - L1u + 1), clipped at 0. Rows past L1u have no window.
-__host__ __device__ inline int32_t window_hi(int mask_mode, int32_t i, int32_t L1u, int32_t L2) {
+// hi = min(L2, i + L2 - L1u + 1), clipped at 0. Compressed keys (r > 1 original tokens each, res
+// tokens past the last whole key) under mask 3: the keys whose last original token is visible,
+// hi = floor((i + L2*r + res - L1u + 1) / r), clipped to [0, L2]. Rows past L1u have no window.
+__host__ __device__ inline int32_t window_hi(int mask_mode, int32_t i, int32_t L1u, int32_t L2,
+                                            int32_t r = 1, int32_t res = 0) {
     if (i >= L1u || L2 <= 0) return 0;
     if (mask_mode != 3) return L2;
-    int64_t lim = (int64_t)i + L2 - L1u + 1;
+    int64_t lim = r > 1 ? ((int64_t)i + (int64_t)L2 * r + res - L1u + 1) / r
+                        : (int64_t)i + L2 - L1u + 1;     // negative numerators clip to 0 below
     if (lim > L2) lim = L2;
     return lim < 0 ? 0 : (int32_t)lim;
 }
@@ -111,6 +118,8 @@ struct Problem {
     int32_t layout_q, layout_k, mask_mode;
     int32_t return_value;
     int32_t rows;                          // B*S1 or T1
+    const int32_t *cmp_residual_k;         // compressed keys: [B] residual tokens, or null
+    int32_t cmp_ratio;                     // original tokens per key (1: not compressed)
 };
 
 // fp32 elements per score row of the workspace (16-byte aligned rows).
@@ -128,6 +137,7 @@ __host__ __device__ inline uint32_t problem_signature(const Problem &p, int tq, 
     mix((uint32_t)p.max_seqlen_q); mix((uint32_t)p.max_seqlen_k); mix((uint32_t)p.n_heads);
     mix((uint32_t)p.layout_q); mix((uint32_t)p.layout_k); mix((uint32_t)p.mask_mode);
     mix((uint32_t)p.block_size); mix((uint32_t)tq); mix((uint32_t)kc);
+    mix((uint32_t)p.cmp_ratio); mix(p.cmp_residual_k ? 1u : 0u);
     return h;
 }
 

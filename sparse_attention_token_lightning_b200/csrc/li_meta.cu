@@ -64,7 +64,7 @@ __device__ inline void store_item(WorkItem *dst, const WorkItem &it) {
     for (int i = 0; i < (int)(sizeof(WorkItem) / sizeof(int4)); ++i) d[i] = src[i];
 }
 
-constexpr int kSmemBatches = 2048;     // batches whose lengths and block prefix stay in smem
+constexpr int kSmemBatches = 1024;     // batches whose lengths and block prefix stay in smem
 
 // Batch of global query block g: the last batch whose first block is <= g (qb0 holds each
 // batch's first block, in shared memory when the batch count allows, else in global memory).
@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
     // per-batch query rows in use, keys and first query block (B <= kSmemBatches)
     __shared__ int32_t s_L1u[kSmemBatches], s_L2[kSmemBatches], s_qb0[kSmemBatches];
     __shared__ int32_t s_qr0[kSmemBatches], s_kr0[kSmemBatches];   // first query / key rows
+    __shared__ int32_t s_res[kSmemBatches];          // residual tokens of compressed keys
     const bool in_smem = p.batch <= kSmemBatches;
     const int tid = threadIdx.x;
     for (int i = tid; i < kCostBins; i += kMetaThreads) hist[i] = 0;
@@ -141,18 +142,26 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
             const int64_t off = p.output_idx_offset[b];
             if (off < 0 || off + (L2 > 0 ? L2 - 1 : 0) > (int64_t)INT32_MAX) err |= LI_DEVERR_OFFSET;
         }
+        int32_t res = 0;
+        if (p.cmp_residual_k) {
+            const int32_t u = p.cmp_residual_k[b];
+            if (u < 0 || u >= p.cmp_ratio) err |= LI_DEVERR_LENGTHS;
+            res = u < 0 ? 0 : (u >= p.cmp_ratio ? p.cmp_ratio - 1 : u);
+        }
         bi.L1 = (int32_t)L1;
         bi.L1u = (int32_t)L1u;
         bi.L2 = (int32_t)L2;
         bi.q_row0 = (int32_t)q0;
         bi.k_row0 = (int32_t)k0;
-        bi.pad[0] = bi.pad[1] = bi.pad[2] = 0;
+        bi.pad[0] = bi.pad[1] = 0;
+        bi.pad[2] = res;
         binfo[b] = bi;
         if (in_smem) {
             s_L1u[b] = bi.L1u;
             s_L2[b] = bi.L2;
             s_qr0[b] = bi.q_row0;
             s_kr0[b] = bi.k_row0;
+            s_res[b] = res;
         }
         if (err) atomicOr(&s_status, err);
     }
@@ -189,6 +198,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
             bi.q_row0 = s_qr0[b];
             bi.k_row0 = s_kr0[b];
             bi.pad[1] = s_qb0[b];
+            bi.pad[2] = s_res[b];
         } else {
             bi = binfo[b];
         }
@@ -216,7 +226,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         r.q0 = (gb - bi.pad[1]) * s.tq;
         r.nq = min(s.tq, bi.L1u - r.q0);
         // windows are prefixes [0, hi) growing with the row, so the block's last row has the widest
-        r.jend = window_hi(p.mask_mode, r.q0 + r.nq - 1, bi.L1u, bi.L2);
+        r.jend = window_hi(p.mask_mode, r.q0 + r.nq - 1, bi.L1u, bi.L2, p.cmp_ratio, bi.pad[2]);
         r.kc = s.kc > 0 ? s.kc : r.jend;
         r.n_s = r.jend > 0 ? (r.jend + r.kc - 1) / r.kc : 0;
         r.full_cost = item_cost(0, r.kc);
@@ -239,6 +249,9 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(MetaParams mp) {
         it.L1u = r.L1u;
         it.L2 = r.L2;
         it.k_row0 = r.k_row0;
+        // compressed keys: a key count that makes the score kernel's plain window cover j1 for
+        // every row (it clips at j1; the selection applies each row's exact window)
+        if (p.cmp_residual_k) it.L2 = it.j1 + it.L1u;
         for (int i = 0; i < 6; ++i) it.pad[i] = 0;
         return it;
     };

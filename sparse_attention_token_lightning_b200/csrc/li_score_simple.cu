@@ -49,7 +49,8 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
         for (int r = 0; r < it.nq; ++r) {
             const int32_t i = it.q0 + r;
             const int64_t row = (int64_t)bi.q_row0 + i;
-            const int32_t hi = min(window_hi(p.mask_mode, i, bi.L1u, bi.L2), it.j1);
+            const int32_t hi =
+                min(window_hi(p.mask_mode, i, bi.L1u, bi.L2, p.cmp_ratio, bi.pad[2]), it.j1);
             __syncthreads();   // previous row's readers are done with qs / ws_
             for (int e = threadIdx.x; e < H * kHeadDim; e += kThreads) {
                 const int h = e / kHeadDim, d = e % kHeadDim;

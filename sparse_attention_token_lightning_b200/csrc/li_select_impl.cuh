@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     int32_t n = 0, off = 0;
     if (b >= 0) {
         const BatchInfo bi = sp.view.batch(p, b);
-        n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2);
+        n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2, p.cmp_ratio, bi.pad[2]);
 
         if (p.output_idx_offset) {
             off = p.output_idx_offset[b];

@@ -43,6 +43,7 @@ class LiArgs(ctypes.Structure):
         ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
         ("dtype_qk", ctypes.c_int32), ("dtype_w", ctypes.c_int32),
         ("return_value", ctypes.c_int32),
+        ("cmp_residual_k", ctypes.c_void_p), ("cmp_ratio", ctypes.c_int32),
     ]
 
 
@@ -154,6 +155,8 @@ def make_args(pb, return_value: int = 1) -> LiArgs:
     a.dtype_qk = 0
     a.dtype_w = 0
     a.return_value = int(return_value)
+    a.cmp_residual_k = _ptr(getattr(pb, "cmp_residual_k", None))
+    a.cmp_ratio = int(getattr(pb, "cmp_ratio", 1) or 1)
     return a
 
 

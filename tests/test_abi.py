@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert li.li_abi_version() == 1
+    assert li.li_abi_version() == 2
 
 
 @pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
@@ -104,6 +104,9 @@ def test_valid_args_size_the_workspace(L):
           num_blocks=4, block_size=1025), 1),
     (dict(cu_seqlens_q=0x40000), 1), (dict(block_table=0x40000), 1), (dict(batch=-1), 1),
     (dict(max_seqlen_k=65), 1), (dict(return_value=2), 1),
+    # compressed keys: residuals exactly with cmp_ratio > 1 under mask_mode 3
+    (dict(cmp_ratio=-1), 1), (dict(cmp_ratio=4), 1), (dict(cmp_residual_k=0x60000), 1),
+    (dict(cmp_ratio=4, mask_mode=0, cmp_residual_k=0x60000), 1),
     # 32-bit row coordinates: query rows x heads and key rows beyond 2^31-1
     (dict(batch=40000, q_len=1000, max_seqlen_q=1000, num_heads_q=64), 2),
     (dict(batch=3, k_len=1 << 30, max_seqlen_k=64), 2),
@@ -114,6 +117,14 @@ def test_invalid_args_rejected_on_host(L, kw, status):
     st, _ = _ws_status(_args(**kw))
     assert st == status, li.li_last_error_string()
     assert li.li_last_error_string()
+
+
+def test_compressed_key_args_accepted(L):
+    assert _ws_status(_args(cmp_ratio=4, cmp_residual_k=0x60000))[0] == 0
+    assert _ws_status(_args(cmp_ratio=4, mask_mode=0))[0] == 0
+    # residuals are per batch and read on the device: the schedule kernel always runs
+    pl = li.li_plan(_args(cmp_ratio=4, cmp_residual_k=0x60000))
+    assert pl["dense"] == 0 and pl["kernels"] == 3
 
 
 def test_topk_accepts_every_value_up_to_8192(L):

@@ -73,6 +73,17 @@ SMALL = {
     # small blocks over long windows: more than 32 key pieces per item (staged rows refilled)
     "paged_bs16_long": lambda: synthetic.paged([1500, 700], 2, 16, 100, block_size=16, seed=52),
     "paged_bs8_long": lambda: synthetic.paged([1900], 1, 8, 64, block_size=8, seed=53),
+    # compressed keys (cmp_ratio > 1, per-batch residuals) under the right-down mask
+    "cmp_pages_example": lambda: synthetic.compressed(
+        synthetic.bsnd(2, 64, 130 // 4, 16, 32, 3, seed=59), 4, [130 % 4, 130 % 4]),
+    "cmp_bsnd_ragged": lambda: synthetic.compressed(
+        synthetic.bsnd(2, 300, 120, 64, 64, 3, seed=60), 3, [2, 0]),
+    "cmp_tnd": lambda: synthetic.compressed(
+        synthetic.tnd([200, 40, 1], [60, 70, 5], 64, 32, 3, seed=61), 4, [3, 1, 0]),
+    "cmp_paged_decode": lambda: synthetic.compressed(
+        synthetic.paged([3000, 700], 1, 64, 128, block_size=64, seed=62), 8, [7, 2]),
+    "cmp_nomask": lambda: synthetic.compressed(synthetic.bsnd(1, 50, 90, 8, 40, 0, seed=63), 4,
+                                               None),
     # few query blocks and long windows: key ranges split across work items
     "paged_decode_split": lambda: synthetic.paged([5000, 3000, 100], 1, 64, 256, block_size=64,
                                                   seed=51),
@@ -238,6 +249,12 @@ def test_mismatched_metadata_reported():
     li.li_indexer(args, meta, ws, idx, val)
     st, bits = li.li_check_status(ws)
     assert st == 6 and bits & li.DEVERR_METADATA
+
+
+def test_compressed_residual_out_of_range_reported():
+    pb = synthetic.compressed(synthetic.bsnd(2, 8, 20, 4, 8, 3, seed=64), 4, [1, 4])
+    st, bits = _status_of(pb)
+    assert st == 6 and bits & li.DEVERR_LENGTHS
 
 
 def test_seqused_k_above_max_reported():
