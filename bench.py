@@ -46,6 +46,9 @@ WORKLOAD_TEXT = {
               "mask_mode=3",
     "long_2048": "long-context prefill: B=1, S1=S2=65536, N1=64, D=128, topk=2048, mask_mode=3",
     "long_8192": "long-context prefill: B=1, S1=S2=65536, N1=64, D=128, topk=8192, mask_mode=3",
+    "cmp_prefill": "compressed-key causal prefill: B=1, S1=4096 queries, 4096 original tokens "
+                   "compressed 4:1 into 1024 keys (cmp_ratio=4, residual 0), N1=64, D=128, "
+                   "topk=512, mask_mode=3, BSND",
 }
 
 
@@ -72,7 +75,14 @@ def valid_pairs(pb) -> int:
         if pb.mask_mode == 0:
             total += used * max(L2, 0)
             continue
-        # row i sees min(L2, max(0, i + L2 - used + 1)) keys
+        # row i sees min(L2, max(0, i + L2 - used + 1)) keys; compressed keys (r original tokens
+        # each, res past the last whole key): min(L2, max(0, (i + L2*r + res - used + 1) // r))
+        r = int(getattr(pb, "cmp_ratio", 1) or 1)
+        if r > 1 and pb.cmp_residual_k is not None:
+            res = int(pb.cmp_residual_k[b])
+            for i in range(used):
+                total += min(L2, max(0, (i + L2 * r + res - used + 1) // r))
+            continue
         lo = L2 - used + 1
         for i in range(used):
             total += min(L2, max(0, i + lo))

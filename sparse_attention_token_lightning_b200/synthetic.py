@@ -245,6 +245,10 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
         return bsnd(1, 65536, 65536, 64, 2048, 3, seed, integer=integer, name=name)
     if name == "long_8192":
         return bsnd(1, 65536, 65536, 64, 8192, 3, seed, integer=integer, name=name)
+    if name == "cmp_prefill":
+        # causal prefill over 4096 original tokens whose keys are compressed 4:1 (1024 keys)
+        return compressed(bsnd(1, 4096, 1024, 64, 512, 3, seed, integer=integer, name=name), 4,
+                          [0])
     if name == "pages_example":
         # The shape of the pages' worked example (B=2, S1=64, N1=16, topk=32) with the key
         # length it compresses to (130 // 4 = 32), taken uncompressed.
@@ -252,4 +256,5 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
     raise KeyError(name)
 
 
-CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192")
+CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192",
+           "cmp_prefill")

@@ -273,6 +273,7 @@ FULL = {
     "varlen": (16, (0, 32767)),
     "long_2048": (6, (0, 2047, 2048, 65535)),
     "long_8192": (4, (8191, 8192, 65535)),
+    "cmp_prefill": (16, (0, 3, 4, 2047, 4095)),
 }
 
 
