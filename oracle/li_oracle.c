@@ -33,8 +33,10 @@
  *      output_idx_offset (aclnnLightningIndexerV2 constraints: the shifted index must not exceed
  *      INT32_MAX).
  *
- * Precision. q, k and w arrive as bf16 bit patterns; every product and sum is taken in fp64, so
- * the score is the exact real value up to fp64 rounding. The selection decision is then taken on
+ * Precision. q and k arrive as bf16 or fp16 bit patterns (lightning_indexer, "Constraints": q
+ * and k share one type; the single-operator example passes fp16 q and k with fp32 w), w as bf16,
+ * fp16 or fp32; every product and sum is taken in fp64, so the score is the exact real value up
+ * to fp64 rounding. The selection decision is then taken on
  * the score rounded once to fp32, the precision the CUDA kernels decide in, and -0 is treated as
  * +0. Order: score descending, then key index ascending (the pages only say "deterministic").
  *
@@ -54,6 +56,7 @@
 #endif
 
 enum { ORC_BSND = 0, ORC_TND = 1, ORC_PA_BSND = 2 };
+enum { ORC_BF16 = 0, ORC_FP16 = 1, ORC_FP32 = 2 };
 enum { ORC_OK = 0, ORC_EARG = 1, ORC_EDATA = 2, ORC_ENOMEM = 3 };
 
 /* One problem. All arrays are host memory in the layouts the pages give:
@@ -62,7 +65,8 @@ enum { ORC_OK = 0, ORC_EARG = 1, ORC_EDATA = 2, ORC_ENOMEM = 3 };
  *   w: (B, S1, N1) or (T1, N1)
  * Optional arrays are NULL when absent. */
 typedef struct {
-    const uint16_t *q, *k, *w;
+    const uint16_t *q, *k;          /* bf16 or fp16 bit patterns (dtype_qk)                     */
+    const void *w;                  /* bf16 or fp16 bit patterns, or fp32 values (dtype_w)      */
     const int32_t *cu_seqlens_q, *cu_seqlens_k;
     const int32_t *seqused_q, *seqused_k;
     const int32_t *block_table;
@@ -76,6 +80,7 @@ typedef struct {
     int32_t layout_q, layout_k, mask_mode;
     const int32_t *cmp_residual_k;  /* [B] or NULL: tokens past the last whole compressed key */
     int32_t cmp_ratio;              /* original tokens per key; 0 or 1 = keys not compressed  */
+    int32_t dtype_qk, dtype_w;      /* ORC_BF16 / ORC_FP16 (q, k); also ORC_FP32 for w        */
 } orc_problem;
 
 static double bf16_value(uint16_t bits)
@@ -84,6 +89,40 @@ static double bf16_value(uint16_t bits)
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* IEEE 754 binary16: sign, 5 exponent bits (bias 15), 10 fraction bits. */
+static double fp16_value(uint16_t bits)
+{
+    const int sign = bits >> 15, e = (bits >> 10) & 0x1f, f = bits & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);                        /* subnormal: f * 2^-24        */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+#if ORC_MUTANT == 13
+        v = ldexp(1024.0 + f, e - 24);                    /* mistake: exponent bias 14   */
+#else
+        v = ldexp(1024.0 + f, e - 25);                    /* (1 + f/1024) * 2^(e - 15)   */
+#endif
+    return sign ? -v : v;
+}
+
+static double qk_value(const orc_problem *p, uint16_t bits)
+{
+    return p->dtype_qk == ORC_FP16 ? fp16_value(bits) : bf16_value(bits);
+}
+
+static double w_value(const orc_problem *p, int64_t idx)
+{
+    if (p->dtype_w == ORC_FP32) {
+        float f;
+        memcpy(&f, (const char *)p->w + 4 * idx, sizeof f);
+        return (double)f;
+    }
+    const uint16_t bits = ((const uint16_t *)p->w)[idx];
+    return p->dtype_w == ORC_FP16 ? fp16_value(bits) : bf16_value(bits);
 }
 
 static int64_t orc_num_rows(const orc_problem *p)
@@ -208,8 +247,8 @@ static double orc_score(const orc_problem *p, int64_t r, const orc_row *o, int64
         const uint16_t *qh = orc_query(p, r, h);
         double s = 0.0;
         for (int32_t d = 0; d < p->head_dim; ++d)
-            s += bf16_value(qh[d]) * bf16_value(kj[d]);
-        double wh = bf16_value(p->w[r * p->n_heads + h]);
+            s += qk_value(p, qh[d]) * qk_value(p, kj[d]);
+        double wh = w_value(p, r * p->n_heads + h);
 #if ORC_MUTANT == 1
         sum_ws += wh * s;                              /* mistake: ReLU after the head sum */
 #elif ORC_MUTANT == 2
@@ -266,6 +305,8 @@ static int orc_check(const orc_problem *p)
     if (p->layout_k == ORC_PA_BSND && (!p->seqused_k || !p->block_table || p->block_size < 1))
         return ORC_EARG;
     if (p->cmp_ratio < 0) return ORC_EARG;
+    if (p->dtype_qk != ORC_BF16 && p->dtype_qk != ORC_FP16) return ORC_EARG;
+    if (p->dtype_w != ORC_BF16 && p->dtype_w != ORC_FP16 && p->dtype_w != ORC_FP32) return ORC_EARG;
     if (p->cmp_residual_k)
         for (int b = 0; b < p->batch; ++b)
             if (p->cmp_residual_k[b] < 0 || p->cmp_residual_k[b] >= (p->cmp_ratio > 1 ? p->cmp_ratio : 1))

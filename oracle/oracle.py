@@ -49,17 +49,38 @@ class _Problem(ctypes.Structure):
         ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
         ("cmp_residual_k", ctypes.c_void_p), ("cmp_ratio", ctypes.c_int32),
+        ("dtype_qk", ctypes.c_int32), ("dtype_w", ctypes.c_int32),
     ]
 
 
+DTYPES = {"bf16": 0, "fp16": 1, "fp32": 2}
+
+
+def _dtype_name(x) -> str:
+    """bf16 / fp16 / fp32 of a tensor (uint16 arrays are bf16 bit patterns)."""
+    if isinstance(x, np.ndarray):
+        return "fp32" if x.dtype == np.float32 else "bf16"
+    import torch
+    return {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[x.dtype]
+
+
 def _bits16(x) -> np.ndarray:
-    """bf16 tensor or uint16 array -> contiguous uint16 numpy array of the bit patterns."""
+    """bf16/fp16 tensor or uint16 array -> contiguous uint16 numpy array of the bit patterns."""
     if isinstance(x, np.ndarray):
         assert x.dtype == np.uint16
         return np.ascontiguousarray(x)
     import torch  # local: the oracle does not need torch unless handed tensors
-    assert x.dtype == torch.bfloat16, x.dtype
+    assert x.dtype in (torch.bfloat16, torch.float16), x.dtype
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _weights(x) -> np.ndarray:
+    """w as 16-bit patterns, or fp32 values."""
+    if _dtype_name(x) == "fp32":
+        if not isinstance(x, np.ndarray):
+            x = x.detach().cpu().contiguous().numpy()
+        return np.ascontiguousarray(x, dtype=np.float32)
+    return _bits16(x)
 
 
 def _i32(x):
@@ -104,7 +125,9 @@ class Oracle:
         s = _Problem()
         s.q = ptr("q", _bits16(pb.q))
         s.k = ptr("k", _bits16(pb.k))
-        s.w = ptr("w", _bits16(pb.w))
+        s.w = ptr("w", _weights(pb.w))
+        s.dtype_qk = DTYPES[_dtype_name(pb.q)]
+        s.dtype_w = DTYPES[_dtype_name(pb.w)]
         for f in ("cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k", "block_table",
                   "output_idx_offset", "cmp_residual_k"):
             setattr(s, f, ptr(f, _i32(getattr(pb, f, None))))

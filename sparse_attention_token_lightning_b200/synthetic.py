@@ -123,6 +123,17 @@ def compressed(pb: Problem, cmp_ratio: int, residual) -> Problem:
                       name=f"{pb.name}_cmp{cmp_ratio}")
 
 
+_DT = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
+
+
+def with_dtypes(pb: Problem, qk: str = "bf16", w: str = "bf16") -> Problem:
+    """The same problem with q, k converted to qk (bf16 or fp16) and w to w (bf16, fp16 or fp32),
+    each value rounded once to the new type (lightning_indexer, "Constraints": q and k share a
+    type; the single-operator example uses fp16 q, k and fp32 w)."""
+    return pb.replace(q=pb.q.float().to(_DT[qk]), k=pb.k.float().to(_DT[qk]),
+                      w=pb.w.float().to(_DT[w]), name=f"{pb.name}_{qk}_{w}")
+
+
 def bsnd(B, S1, S2, N1, topk, mask_mode=3, seed=0, D=D_DEFAULT, integer=False, name="bsnd",
          seqused_q=None, seqused_k=None, output_idx_offset=None) -> Problem:
     """Dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)."""

@@ -291,6 +291,35 @@ def pin_compressed_window_counts_whole_blocks(orc):
         assert orc.bind(synthetic.compressed(pb0, 4, [3])).row_info(i)[0] == 10
 
 
+def pin_fp16_decoding(orc):
+    """fp16 queries decode as IEEE binary16 (numpy's float16 is the reference): with one head of
+    dimension 1, w = 1 and a single key k = 1, each row's only score is ReLU(q). The patterns
+    cover subnormals, normals of every exponent and negative values."""
+    pos = np.arange(0, 0x7C00, 5, dtype=np.uint16)              # +0 .. largest finite
+    bits = np.concatenate([pos, pos[::7] | np.uint16(0x8000)])   # and some negative ones
+    n = len(bits)
+    q = torch.from_numpy(bits.view(np.int16).copy()).view(torch.float16).reshape(1, n, 1, 1)
+    pb = synthetic.Problem(name="fp16_decode", q=q, k=torch.ones(1, 1, 1, 1, dtype=torch.float16),
+                           w=torch.ones(1, n, 1, dtype=torch.bfloat16), topk=1, batch=1, q_len=n,
+                           k_len=1, n_heads=1, head_dim=1, mask_mode=0, max_seqlen_q=n,
+                           max_seqlen_k=1)
+    idx, val, _ = orc.topk(pb)
+    want = np.maximum(bits.view(np.float16).astype(np.float32), np.float32(0))
+    assert np.array_equal(idx[:, 0], np.zeros(n, dtype=np.int32))
+    _assert_same(_bits(val[:, 0]), _bits(want), "fp16 decode")
+
+
+def pin_dtype_encodings_agree(orc):
+    """Integer-valued q, k (in -2..2) and w (in +-1/2, +-1, +-2) are exact in bf16, fp16 and
+    fp32, so every encoding of the same values gives the same outputs, bit for bit."""
+    base = synthetic.bsnd(2, 40, 70, 8, 24, 3, seed=73, integer=True)
+    ref = orc.topk(base)
+    for qk, w in [("fp16", "fp32"), ("fp16", "fp16"), ("bf16", "fp32"), ("fp16", "bf16")]:
+        got = orc.topk(synthetic.with_dtypes(base, qk, w))
+        _assert_same(ref[0], got[0], f"indices {qk}/{w}")
+        _assert_same(_bits(ref[1]), _bits(got[1]), f"values {qk}/{w}")
+
+
 def pin_pages_example_shape(orc):
     """The pages' worked example shape (B=2, S1=64, N1=16, topk=32) with 32 keys and mask 3:
     rows i < 32 see no key (i + S2 - S1 < 0) and row i >= 32 sees i - 31 keys."""

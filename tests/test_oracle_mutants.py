@@ -9,7 +9,7 @@ import pytest
 import oracle_pins
 from oracle import oracle as orc_mod
 
-MUTANTS = list(range(1, 13))
+MUTANTS = list(range(1, 14))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
