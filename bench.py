@@ -49,6 +49,8 @@ WORKLOAD_TEXT = {
     "cmp_prefill": "compressed-key causal prefill: B=1, S1=4096 queries, 4096 original tokens "
                    "compressed 4:1 into 1024 keys (cmp_ratio=4, residual 0), N1=64, D=128, "
                    "topk=512, mask_mode=3, BSND",
+    "fp16_prefill": "causal prefill in fp16: B=1, S1=S2=4096, N1=64, N2=1, D=128, topk=2048, "
+                    "mask_mode=3, BSND, q,k fp16 ~N(0,1), w fp32 ~N(0,1/64)",
 }
 
 
@@ -99,8 +101,8 @@ def key_bytes(pb) -> int:
 def score_kernel_bytes(pb, pairs) -> int:
     """Algorithmic DRAM bytes of one score-kernel launch: each valid key once (256 B), q and w
     of every query row, the block table rows in use, and the fp32 score of every valid pair."""
-    q = pb.q.numel() * 2
-    w = pb.w.numel() * 2
+    q = pb.q.numel() * pb.q.element_size()
+    w = pb.w.numel() * pb.w.element_size()
     table = 0
     if pb.layout_k == "PA_BSND":
         table = sum(-(-int(L) // pb.block_size) for L in pb.seqused_k.tolist()) * 4
@@ -397,6 +399,7 @@ def main():
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peaks = load_peaks()
+    dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[pb_cpu.q.dtype]
     pairs = valid_pairs(pb_cpu)
     flops = 2.0 * pairs * pb.n_heads * pb.head_dim
     sc = statistics.mean(score_ms)
@@ -417,11 +420,12 @@ def main():
                     "frac": achieved / peak, "traffic": score_traffic(a.config),
                     "algorithmic_bytes": score_kernel_bytes(pb_cpu, pairs),
                     "kernel": "score kernel (q.k contraction + ReLU/weight/head-sum epilogue)",
-                    "peak_source": f"{peaks['source']} bf16 burst"}
+                    "peak_source": f"{peaks['source']} bf16 burst"
+                                   + (" (fp16 runs at the bf16 rate)" if dtype == "fp16" else "")}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
                        "rows_per_step_per_gpu": rows, "valid_pairs": valid_pairs(pb_cpu),
                        "l2": "flushed before every step by a 256 MB write outside the step's "

@@ -62,7 +62,9 @@ typedef enum li_status {
 } li_status;
 
 typedef enum li_dtype {
-    LI_DTYPE_BF16 = 0
+    LI_DTYPE_BF16 = 0,
+    LI_DTYPE_FP16 = 1,
+    LI_DTYPE_FP32 = 2                   /* w only                                              */
 } li_dtype;
 
 /* Device status word bits, as reported through li_check_status(). */
@@ -104,8 +106,12 @@ typedef struct li_args {
     int32_t layout_q;                   /* li_layout: BSND or TND                               */
     int32_t layout_k;                   /* li_layout: BSND, TND or PA_BSND                      */
     int32_t mask_mode;                  /* 0 (no mask) or 3 (right-down causal)                 */
-    int32_t dtype_qk;                   /* li_dtype of q and k: LI_DTYPE_BF16                   */
-    int32_t dtype_w;                    /* li_dtype of w: LI_DTYPE_BF16                         */
+    int32_t dtype_qk;                   /* li_dtype of q and k (one type, lightning_indexer,
+                                           "Constraints"): LI_DTYPE_BF16 or LI_DTYPE_FP16;
+                                           products accumulate in fp32 either way          */
+    int32_t dtype_w;                    /* li_dtype of w: BF16, FP16 or FP32 (the pages'
+                                           single-operator example passes fp16 q, k and fp32
+                                           w); fp32 w must be 4-byte aligned               */
     int32_t return_value;               /* 1: write sparse_values too; 0: indices only          */
     /* Compressed keys (lightning_indexer, "Prototype": cmp_ratio, cmp_residual_k; "Constraints":
      * cmp_residual_k[b] < cmp_ratio, passed only with cmp_ratio > 1 and mask_mode 3). Each key

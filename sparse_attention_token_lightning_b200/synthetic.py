@@ -260,6 +260,11 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
         # causal prefill over 4096 original tokens whose keys are compressed 4:1 (1024 keys)
         return compressed(bsnd(1, 4096, 1024, 64, 512, 3, seed, integer=integer, name=name), 4,
                           [0])
+    if name == "fp16_prefill":
+        # the causal prefill in the types of the pages' single-operator example: fp16 q, k and
+        # fp32 w
+        return with_dtypes(bsnd(1, 4096, 4096, 64, 2048, 3, seed, integer=integer, name=name),
+                           "fp16", "fp32").replace(name=name)
     if name == "pages_example":
         # The shape of the pages' worked example (B=2, S1=64, N1=16, topk=32) with the key
         # length it compresses to (130 // 4 = 32), taken uncompressed.
@@ -268,4 +273,4 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
 
 
 CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192",
-           "cmp_prefill")
+           "cmp_prefill", "fp16_prefill")

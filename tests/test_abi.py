@@ -96,7 +96,8 @@ def test_valid_args_size_the_workspace(L):
 @pytest.mark.parametrize("kw,status", [
     (dict(num_heads_q=0), 1), (dict(num_heads_q=65), 1), (dict(num_heads_k=2), 1),
     (dict(head_dim=64), 1), (dict(topk=0), 1), (dict(topk=8193), 1), (dict(mask_mode=1), 1),
-    (dict(layout_q=2), 1), (dict(layout_k=5), 1), (dict(dtype_qk=1), 2), (dict(q=None), 1),
+    (dict(layout_q=2), 1), (dict(layout_k=5), 1), (dict(dtype_qk=2), 1), (dict(dtype_w=3), 1),
+    (dict(dtype_qk=-1), 1), (dict(dtype_w=2, w=0x30002), 1), (dict(w=0x30001), 1), (dict(q=None), 1),
     (dict(q=0x10008), 1), (dict(layout_q=1), 1), (dict(layout_k=1), 1), (dict(layout_k=2), 1),
     (dict(layout_k=2, seqused_k=0x40000, block_table=0x50000, block_table_stride=4,
           num_blocks=4, block_size=0), 1),
@@ -117,6 +118,14 @@ def test_invalid_args_rejected_on_host(L, kw, status):
     st, _ = _ws_status(_args(**kw))
     assert st == status, li.li_last_error_string()
     assert li.li_last_error_string()
+
+
+@pytest.mark.parametrize("qk,w", [(0, 0), (0, 1), (0, 2), (1, 0), (1, 1), (1, 2)])
+def test_every_dtype_pair_accepted(L, qk, w):
+    assert _ws_status(_args(dtype_qk=qk, dtype_w=w))[0] == 0
+    # a 16-bit w needs 2-byte alignment only
+    if w != 2:
+        assert _ws_status(_args(dtype_qk=qk, dtype_w=w, w=0x30002))[0] == 0
 
 
 def test_compressed_key_args_accepted(L):

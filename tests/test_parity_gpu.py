@@ -113,6 +113,49 @@ def test_integer_inputs_bit_exact(orc, name):
     parity.check(orc, pb, gi, gv, exact=True, label=name)
 
 
+# q and k in fp16 (one type for both), w in bf16, fp16 or fp32: the MMA takes fp16 operands and
+# the weights are staged as fp32, so the oracle decodes the same bits
+DT = synthetic.with_dtypes
+DTYPE_CASES = {
+    "pages_example_fp16_fp32": lambda: DT(synthetic.config("pages_example"), "fp16", "fp32"),
+    "bsnd_causal_ragged_fp16_fp16": lambda: DT(SMALL["bsnd_causal_ragged"](), "fp16", "fp16"),
+    "bsnd_n48_fp16_bf16": lambda: DT(SMALL["bsnd_n48"](), "fp16", "bf16"),
+    "tnd_varlen_bf16_fp32": lambda: DT(SMALL["tnd_varlen"](), "bf16", "fp32"),
+    "paged_bs64_fp16_fp32": lambda: DT(SMALL["paged_bs64"](), "fp16", "fp32"),
+    "paged_decode_split_fp16_fp32": lambda: DT(SMALL["paged_decode_split"](), "fp16", "fp32"),
+    "paged_bs16_long_bf16_fp16": lambda: DT(SMALL["paged_bs16_long"](), "bf16", "fp16"),
+    "cmp_tnd_fp16_fp32": lambda: DT(SMALL["cmp_tnd"](), "fp16", "fp32"),
+    "topk8192_n16_fp16_fp32": lambda: DT(SMALL["topk8192_n16"](), "fp16", "fp32"),
+}
+
+
+@pytest.mark.parametrize("name", list(DTYPE_CASES))
+def test_dtype_parity(orc, name):
+    pb = DTYPE_CASES[name]()
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
+    parity.check(orc, pb, gi, gv, label=name)
+    assert exact_rows == 0
+
+
+@pytest.mark.parametrize("qk,w", [("fp16", "fp32"), ("fp16", "fp16"), ("bf16", "fp32")])
+@pytest.mark.parametrize("name", ["bsnd_causal", "paged"])
+def test_integer_inputs_bit_exact_in_every_dtype(orc, name, qk, w):
+    pb = DT(EXACT[name](), qk, w)
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, exact=True, label=f"{name} {qk} {w}")
+
+
+def test_dtypes_change_only_the_rounding(orc):
+    """Integer-valued inputs are exact in every type: all six q/k and w type pairs must give
+    the same bits on the device."""
+    base = EXACT["tnd"]()
+    ref = run(base)
+    for qk in ("bf16", "fp16"):
+        for w in ("bf16", "fp16", "fp32"):
+            got = run(DT(base, qk, w))
+            assert np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1]), (qk, w)
+
+
 def test_indices_only(orc):
     pb = synthetic.bsnd(1, 64, 300, 8, 50, 3, seed=30)
     gi, gv = run(pb, return_value=False)
@@ -274,6 +317,7 @@ FULL = {
     "long_2048": (6, (0, 2047, 2048, 65535)),
     "long_8192": (4, (8191, 8192, 65535)),
     "cmp_prefill": (16, (0, 3, 4, 2047, 4095)),
+    "fp16_prefill": (16, (0, 2047, 4095)),
 }
 
 
@@ -319,11 +363,12 @@ def test_tie_heavy_rows_fall_back_correctly(orc):
 
 # ---- the two score kernels agree ------------------------------------------------------------------
 
-@pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "paged_bs64", "tnd_varlen"])
+@pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "paged_bs64", "tnd_varlen",
+                                  "pages_example_fp16_fp32", "paged_bs16_long_bf16_fp16"])
 def test_cuda_core_score_kernel_matches_tensor_core(orc, name, monkeypatch):
     """LI_SCORE_KERNEL=simple selects the CUDA-core score kernel (a debugging path); both
     kernels must produce outputs that agree under the parity tolerance."""
-    pb = SMALL[name]()
+    pb = SMALL[name]() if name in SMALL else DTYPE_CASES[name]()
     a = run(pb)
     monkeypatch.setenv("LI_SCORE_KERNEL", "simple")
     b = run(pb)
