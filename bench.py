@@ -114,10 +114,10 @@ def score_kernel_bytes(pb, pairs) -> int:
 # with the sha256 of the score-kernel sources the counters were taken on; reported only while the
 # sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
 SCORE_TRAFFIC = {
-    "causal_prefill": {"bytes": 68743680 + 9866752,
-                       "src_sha256": "77867c76e600c743c5b645f62403cecb65f0df2a57c04c4af0d86e71d8e3e0bb"},
-    "paged_decode": {"bytes": 286281728 + 6766592,
-                     "src_sha256": "77867c76e600c743c5b645f62403cecb65f0df2a57c04c4af0d86e71d8e3e0bb"},
+    "causal_prefill": {"bytes": 68768512 + 9410048,
+                       "src_sha256": "44dcb8cfdf287f173ac7b97450a1c9d9760e494944260dfb186494f39306d70f"},
+    "paged_decode": {"bytes": 286289408 + 6130432,
+                     "src_sha256": "44dcb8cfdf287f173ac7b97450a1c9d9760e494944260dfb186494f39306d70f"},
 }
 SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
                  "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")
