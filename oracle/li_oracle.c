@@ -32,6 +32,12 @@
  *      (aclnnLightningIndexerV2 and lightning_indexer, constraints), indices shifted by
  *      output_idx_offset (aclnnLightningIndexerV2 constraints: the shifted index must not exceed
  *      INT32_MAX).
+ *   5. Merge of key-range shards (the split-merge step that follows a key-range split of one
+ *      row): [reading] the pages select over the whole window of a row, so the top-k of a row
+ *      whose keys were split into disjoint ranges, each range selected on its own with its
+ *      keys' global indices, is the top-k of the union of the per-range lists under the same
+ *      order. orc_merge_topk writes out exactly that: all valid entries of all lists, one sort,
+ *      the first topk kept.
  *
  * Precision. q and k arrive as bf16 or fp16 bit patterns (lightning_indexer, "Constraints": q
  * and k share one type; the single-operator example passes fp16 q and k with fp32 w), w as bf16,
@@ -420,4 +426,42 @@ int orc_topk(const orc_problem *p, const int64_t *rows, int64_t n_rows,
     }
     free(e);
     return rc;
+}
+
+/* Step 5: top-k of the union of n_lists per-row lists. List l, row r, entry e is
+ * idx[(l*rows + r)*topk_in + e] / val[...]; an entry with a negative index is padding. Output row
+ * r holds the first topk_out of all valid entries of row r in step 4's order (score descending,
+ * index ascending), then -1 / -inf. The decision is taken on the fp32 values as given, -0 as
+ * +0. Returns ORC_EARG for bad sizes. */
+int orc_merge_topk(int64_t rows, int32_t n_lists, int32_t topk_in, const int32_t *idx,
+                   const float *val, int32_t topk_out, int32_t *out_idx, float *out_val)
+{
+    if (rows < 0 || n_lists < 1 || topk_in < 1 || topk_out < 1 || !idx || !val || !out_idx ||
+        !out_val)
+        return ORC_EARG;
+    int32_t lists = n_lists;
+#if ORC_MUTANT == 14
+    lists = n_lists - 1;                          /* mistake: the last list is dropped */
+#endif
+    orc_entry *e = (orc_entry *)malloc((size_t)lists * (size_t)topk_in * sizeof(orc_entry) + 1);
+    if (!e) return ORC_ENOMEM;
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t n = 0;
+        for (int32_t l = 0; l < lists; ++l) {
+            for (int32_t k = 0; k < topk_in; ++k) {
+                const int64_t at = ((int64_t)l * rows + r) * topk_in + k;
+                if (idx[at] < 0) continue;
+                e[n].v = val[at] == 0.0f ? 0.0f : val[at];
+                e[n].j = idx[at];
+                ++n;
+            }
+        }
+        qsort(e, (size_t)n, sizeof(orc_entry), orc_cmp);
+        for (int32_t s = 0; s < topk_out; ++s) {
+            out_idx[r * topk_out + s] = s < n ? (int32_t)e[s].j : -1;
+            out_val[r * topk_out + s] = s < n ? e[s].v : -INFINITY;
+        }
+    }
+    free(e);
+    return ORC_OK;
 }

@@ -110,6 +110,10 @@ class Oracle:
         lib.orc_score_at.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
         lib.orc_score_at.restype = ctypes.c_int
         lib.orc_topk.restype = ctypes.c_int
+        lib.orc_merge_topk.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+        lib.orc_merge_topk.restype = ctypes.c_int
         self.lib = lib
 
     # -- marshalling -----------------------------------------------------------------------
@@ -168,6 +172,21 @@ class Oracle:
 
     def row_info(self, pb, row: int):
         return self.bind(pb).row_info(row)
+
+    def merge_topk(self, idx_lists, val_lists, topk: int):
+        """Top-k of the union of per-row lists: idx_lists / val_lists are sequences of
+        (rows, topk_in) int32 / float32 arrays (one per key range); returns (idx, val) of shape
+        (rows, topk)."""
+        idx = np.ascontiguousarray(np.stack([np.asarray(x, dtype=np.int32) for x in idx_lists]))
+        val = np.ascontiguousarray(np.stack([np.asarray(x, dtype=np.float32) for x in val_lists]))
+        n_lists, rows, topk_in = idx.shape
+        out_i = np.empty((rows, topk), dtype=np.int32)
+        out_v = np.empty((rows, topk), dtype=np.float32)
+        rc = self.lib.orc_merge_topk(rows, n_lists, topk_in, idx.ctypes.data, val.ctypes.data,
+                                     topk, out_i.ctypes.data, out_v.ctypes.data)
+        if rc:
+            raise RuntimeError(f"oracle orc_merge_topk returned {rc}")
+        return out_i, out_v
 
 
 class Bound:

@@ -332,4 +332,57 @@ def pin_pages_example_shape(orc):
         assert valid == max(0, min(32, i - 31)), f"row {r}: {valid} valid entries"
 
 
+def _key_range(pb, s, e, mask_mode):
+    """Keys [s, e) of every batch of a dense BSND problem, indices shifted back to global by
+    output_idx_offset = s (written out here, independently of the library's shard helpers)."""
+    n = e - s
+    return pb.replace(name=f"{pb.name}[k{s}:{e}]", k=pb.k[:, s:e].contiguous(), k_len=n,
+                      max_seqlen_k=n, mask_mode=mask_mode,
+                      output_idx_offset=torch.full((pb.batch,), s, dtype=torch.int32))
+
+
+def pin_key_range_merge_equals_whole_row(orc):
+    """Selection is over the whole window of a row, so splitting the keys into disjoint ranges,
+    selecting in each with global indices and merging the lists must give the whole row's
+    top-k bit for bit: decode rows (one query row sees every key under mask 3), rows without a
+    mask, ranges shorter than topk (padded lists), and causal rows whose window covers every
+    range but the last."""
+    cases = [
+        (synthetic.bsnd(3, 1, 700, 16, 100, 3, seed=80), [0, 128, 333, 700], [0, 0, 3]),
+        (synthetic.bsnd(1, 5, 400, 8, 64, 0, seed=81), [0, 30, 250, 400], [0, 0, 0]),
+        (synthetic.bsnd(2, 4, 300, 4, 120, 3, seed=82, integer=True), [0, 100, 200, 300],
+         [0, 0, 3]),
+        (synthetic.bsnd(2, 6, 260, 8, 200, 3, seed=83), [0, 128, 250, 260], [0, 0, 3]),
+    ]
+    for pb, cuts, masks in cases:
+        whole = orc.topk(pb)
+        lists = [orc.topk(_key_range(pb, a, b, m)) for a, b, m in zip(cuts, cuts[1:], masks)]
+        got = orc.merge_topk([x[0] for x in lists], [x[1] for x in lists], pb.topk)
+        _assert_same(whole, got, pb.name)
+
+
+def pin_merge_brute_force(orc):
+    """Tiny lists with many equal scores across lists: the merge equals Python's sort of all
+    valid (score, index) pairs by score descending, then index ascending."""
+    g = np.random.default_rng(84)
+    for n_lists, rows, kin, kout in [(2, 3, 5, 4), (4, 5, 6, 9), (3, 2, 7, 30), (1, 4, 8, 3)]:
+        pool = g.permutation(1000)[: n_lists * rows * kin].reshape(n_lists, rows, kin)
+        idx = np.full((n_lists, rows, kin), -1, dtype=np.int32)
+        val = np.full((n_lists, rows, kin), -np.inf, dtype=np.float32)
+        for l in range(n_lists):
+            for r in range(rows):
+                n = int(g.integers(0, kin + 1))
+                ent = sorted(((float(g.integers(-3, 4)) / 2, int(pool[l, r, e])) for e in range(n)),
+                             key=lambda t: (-t[0], t[1]))
+                for e, (v, j) in enumerate(ent):
+                    idx[l, r, e], val[l, r, e] = j, v
+        got_i, got_v = orc.merge_topk(list(idx), list(val), kout)
+        for r in range(rows):
+            ent = sorted(((float(val[l, r, e]), int(idx[l, r, e])) for l in range(n_lists)
+                          for e in range(kin) if idx[l, r, e] >= 0), key=lambda t: (-t[0], t[1]))
+            ent = ent[:kout] + [(-np.inf, -1)] * max(0, kout - len(ent))
+            assert got_i[r].tolist() == [j for _, j in ent], (n_lists, r)
+            assert got_v[r].tolist() == [v for v, _ in ent], (n_lists, r)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -3,13 +3,14 @@
 This shows the pins are strong enough to catch a plausible slip anywhere in the oracle: ReLU
 after the head sum, weights dropped, top-left instead of right-down causal alignment, reversed
 tie order, -0 kept, head/row strides exchanged, block table ignored, TND keys offset by the
-query cumulative lengths, ReLU dropped, output offset dropped, wrong padding."""
+query cumulative lengths, ReLU dropped, output offset dropped, wrong padding, compressed keys kept
+when their first token is visible, a wrong fp16 exponent bias, a merge that drops a list."""
 import pytest
 
 import oracle_pins
 from oracle import oracle as orc_mod
 
-MUTANTS = list(range(1, 14))
+MUTANTS = list(range(1, 15))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
