@@ -10,8 +10,10 @@ roofline object reports the score kernel's tensor throughput against the measure
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
 Multi-GPU (torchrun): each rank runs its own independent problem (seed = rank); no data-path
-collective exists because query rows are independent (weak scaling). The reported time is the
-max over ranks of the device time of the K steps.
+collective exists because query rows are independent (weak scaling). The key-sharded workload
+(--config long_row_decode) splits one long row's keys across the ranks instead: every rank
+selects in its range, the lists are all-gathered (NCCL) and merged by li_merge_topk (strong
+scaling). The reported time is the max over ranks of the device time of the K steps.
 """
 from __future__ import annotations
 
@@ -30,7 +32,7 @@ import torch
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
-from sparse_attention_token_lightning_b200 import li, synthetic  # noqa: E402
+from sparse_attention_token_lightning_b200 import li, shard, synthetic  # noqa: E402
 
 METRIC = "indexer query-tokens/s; TFLOP/s as % bf16 tensor peak (N1=64,D=128,topk=2048)"
 UNIT = "query-tokens/s"
@@ -51,7 +53,12 @@ WORKLOAD_TEXT = {
                    "topk=512, mask_mode=3, BSND",
     "fp16_prefill": "causal prefill in fp16: B=1, S1=S2=4096, N1=64, N2=1, D=128, topk=2048, "
                     "mask_mode=3, BSND, q,k fp16 ~N(0,1), w fp32 ~N(0,1/64)",
+    "long_row_decode": "one decode row over a long context: B=1, S1=1, seqused_k=1048576, N1=64, "
+                       "D=128, topk=2048, mask_mode=3, PA_BSND block_size=64; on N GPUs each "
+                       "holds 1/N of the keys, selects in its range, then all-gather + merge",
 }
+# workloads whose keys (not rows) are split across GPUs: strong scaling, all-gather + merge
+KEY_SHARDED = ("long_row_decode",)
 
 
 def valid_pairs(pb) -> int:
@@ -267,6 +274,74 @@ def run_reference(a):
     return 0
 
 
+def run_emulated_ranges(a, dev):
+    """One GPU runs every key range of a key-sharded workload in turn (li_indexer per range,
+    into the slots an all-gather would fill), then li_merge_topk; reports the step and the merge
+    kernel's own time and bandwidth."""
+    G = a.emulate_ranges
+    pb_full = synthetic.config(a.config, seed=0)
+    parts = [shard.key_shard(pb_full, G, r, compact=True).to(dev) for r in range(G)]
+    argv = [li.make_args(p) for p in parts]
+    wss = [li.empty_workspace(x, dev) for x in argv]
+    shape = li.out_shape(parts[0])
+    gi = torch.empty((G,) + tuple(shape), dtype=torch.int32, device=dev)
+    gv = torch.empty((G,) + tuple(shape), dtype=torch.float32, device=dev)
+    out_i, out_v = torch.empty(shape, dtype=torch.int32, device=dev), torch.empty(
+        shape, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    m = li.LiMergeArgs()
+    for l in range(G):
+        m.idx_in[l], m.val_in[l] = gi[l].data_ptr(), gv[l].data_ptr()
+    m.idx_out, m.val_out, m.device_status = out_i.data_ptr(), out_v.data_ptr(), status.data_ptr()
+    m.rows, m.n_lists, m.topk_in, m.topk_out = parts[0].rows, G, pb_full.topk, pb_full.topk
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K = a.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def step(s=None):
+        for r in range(G):
+            li.li_indexer(argv[r], None, wss[r], gi[r], gv[r], stream)
+        if s is not None:
+            ev[s][1].record(stream)
+        li.li_merge_topk(m, stream)
+
+    for _ in range(a.warmup):
+        step()
+    for w in wss:
+        st, bits = li.li_check_status(w)
+        if st != li.LI_OK:
+            raise SystemExit(f"device status {st} bits {bits:#x}")
+    st, bits = li.li_check_status(status)
+    if st != li.LI_OK:
+        raise SystemExit(f"merge status {st} bits {bits:#x}")
+    torch.cuda.synchronize()
+    for s in range(K):
+        flush.zero_()
+        ev[s][0].record(stream)
+        step(s)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(ev[s][0].elapsed_time(ev[s][2]) for s in range(K))
+    merge_ms = statistics.mean(ev[s][1].elapsed_time(ev[s][2]) for s in range(K))
+    # merge traffic: every input entry read once (8 B), every output slot written once (8 B)
+    mbytes = G * gi[0].numel() * 8 + out_i.numel() * 8
+    peaks = load_peaks()
+    line = {"metric": METRIC, "value": pb_full.rows / (step_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+            "steps": K, "warmup": a.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
+                       "emulated_key_ranges": G,
+                       "l2": "flushed before every step by a 256 MB write outside the step's "
+                             "CUDA events"},
+            "merge": {"ms": merge_ms, "bytes": mbytes,
+                      "achieved_gbs": mbytes / (merge_ms / 1e3) / 1e9,
+                      "peak_gbs": peaks["hbm_gbs"], "lists": G},
+            "gpu_launches": (sum(li.li_plan(x)["kernels"] for x in argv) + 1) * K}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -278,6 +353,10 @@ def main():
                     help="CPU-oracle sample budget for cpu_baseline (0 = skip)")
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--emulate-ranges", type=int, default=0,
+                    help="split the workload's keys into this many ranges and, on one GPU, select "
+                         "in each range in turn, then merge (the N-GPU key-sharded data path "
+                         "without the gather)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -300,7 +379,19 @@ def main():
             torch.distributed.barrier()
 
     li.lib()
-    pb_cpu = synthetic.config(a.config, seed=rank)
+    keyshard = a.config in KEY_SHARDED
+    if a.emulate_ranges and (world > 1 or a.emulate_ranges > li.MERGE_MAX_LISTS):
+        ap.error("--emulate-ranges takes one GPU and at most 16 ranges")
+    if a.emulate_ranges:
+        return run_emulated_ranges(a, dev)
+    if keyshard:
+        # one problem; this rank holds its key range (and only the cache blocks it uses)
+        pb_full = synthetic.config(a.config, seed=0)
+        pb_cpu = shard.key_shard(pb_full, world, rank, compact=True)
+        rows_total = pb_full.rows
+    else:
+        pb_cpu = synthetic.config(a.config, seed=rank)
+        rows_total = pb_cpu.rows * world
     pb = pb_cpu.to(dev)
     args = li.make_args(pb)
     plan = li.li_plan(args)
@@ -310,8 +401,27 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    merged = keyshard and world > 1
+    if merged:
+        gi = torch.empty((world,) + tuple(idx.shape), dtype=torch.int32, device=dev)
+        gv = torch.empty((world,) + tuple(val.shape), dtype=torch.float32, device=dev)
+        out_i, out_v = torch.empty_like(idx), torch.empty_like(val)
+        margs = li.LiMergeArgs()
+        for l in range(world):
+            margs.idx_in[l], margs.val_in[l] = gi[l].data_ptr(), gv[l].data_ptr()
+        margs.idx_out, margs.val_out = out_i.data_ptr(), out_v.data_ptr()
+        margs.device_status = ws.data_ptr()
+        margs.rows, margs.n_lists = pb.rows, world
+        margs.topk_in = margs.topk_out = pb.topk
+    else:
+        out_i, out_v = idx, val
+
     def step():
         li.li_indexer(args, None, ws, idx, val, stream)
+        if merged:
+            torch.distributed.all_gather(list(gi.unbind(0)), idx)
+            torch.distributed.all_gather(list(gv.unbind(0)), val)
+            li.li_merge_topk(margs, stream)
 
     for _ in range(a.warmup):
         step()
@@ -359,25 +469,24 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
     ms_per_step = total_ms / K
-    rows = pb.rows
-    value = rows * world / (ms_per_step / 1e3)
+    value = rows_total / (ms_per_step / 1e3)
 
     # ---- end to end through the public API with host buffers ---------------------------------
     e2e = None
     if not a.no_e2e:
         host = {f: getattr(pb_cpu, f).pin_memory() for f in synthetic.Problem.TENSORS
                 if getattr(pb_cpu, f) is not None}
-        h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-        h_val = torch.empty(val.shape, dtype=val.dtype, pin_memory=True)
+        h_idx = torch.empty(out_i.shape, dtype=out_i.dtype, pin_memory=True)
+        h_val = torch.empty(out_v.shape, dtype=out_v.dtype, pin_memory=True)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = h_idx.numel() * 4 + h_val.numel() * 4
 
         def e2e_step():
             for f, t in host.items():
                 getattr(pb, f).copy_(t, non_blocking=True)
-            li.li_indexer(args, None, ws, idx, val, stream)
-            h_idx.copy_(idx, non_blocking=True)
-            h_val.copy_(val, non_blocking=True)
+            step()
+            h_idx.copy_(out_i, non_blocking=True)
+            h_val.copy_(out_v, non_blocking=True)
 
         for _ in range(3):
             e2e_step()
@@ -395,7 +504,7 @@ def main():
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             e2e_ms = float(t.item())
         barrier()
-        e2e = {"value": rows * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": rows_total / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peaks = load_peaks()
@@ -403,7 +512,7 @@ def main():
     pairs = valid_pairs(pb_cpu)
     flops = 2.0 * pairs * pb.n_heads * pb.head_dim
     sc = statistics.mean(score_ms)
-    if a.config == "paged_decode":
+    if pb_cpu.layout_k == "PA_BSND":
         # HBM-bound: every valid key (256 B) is read once; plus q, w and the fp32 score rows
         nbytes = score_kernel_bytes(pb_cpu, pairs)
         achieved = nbytes / (sc / 1e3) / 1e9
@@ -425,18 +534,21 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "scaling": "strong" if keyshard else "weak", "vs_baseline": None, "dtype": dtype,
+            "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
-                       "rows_per_step_per_gpu": rows, "valid_pairs": valid_pairs(pb_cpu),
+                       "rows_per_step": rows_total, "valid_pairs_per_gpu": valid_pairs(pb_cpu),
                        "l2": "flushed before every step by a 256 MB write outside the step's "
                              "CUDA events",
-                       "parallelism": f"{world} independent replicas (one problem per GPU)",
+                       "parallelism": (f"{world} key ranges of one problem (all-gather + merge)"
+                                       if merged else
+                                       f"{world} independent replicas (one problem per GPU)"),
                        "schedule": {k: plan[k] for k in ("tq", "kc", "dense", "score_tc")}},
             "roofline": roofline,
             "stages_ms": {"schedule": statistics.mean(meta_ms), "score": sc,
                           "select": statistics.mean(sel_ms)},
             "tflops_whole_step": flops / (ms_per_step / 1e3) / 1e12,
-            "clocks": clk, "gpu_launches": plan["kernels"] * K}
+            "clocks": clk, "gpu_launches": (plan["kernels"] + (1 if merged else 0)) * K}
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and a.cpu_seconds > 0:

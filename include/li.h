@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define LI_ABI_VERSION 2
+#define LI_ABI_VERSION 3
 
 typedef enum li_layout {
     LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
@@ -72,6 +72,8 @@ typedef enum li_dtype {
 #define LI_DEVERR_LENGTHS   0x2u   /* cu_seqlens not monotone, or a length above its maximum  */
 #define LI_DEVERR_TABLE     0x4u   /* a block_table entry in use is outside [0, num_blocks)    */
 #define LI_DEVERR_OFFSET    0x8u   /* output_idx_offset < 0, or index + offset > INT32_MAX     */
+#define LI_DEVERR_MERGE_ORDER 0x10u /* li_merge_topk: an input row out of order, or a valid entry
+                                       after padding                                          */
 
 /*
  * Arguments of one indexer call. Mirrors the pages' prototypes (lightning_indexer, "Prototype":
@@ -162,6 +164,10 @@ li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *s
  *                 query rows); one fewer schedule kernel when a metadata buffer is passed
  *   score_tc      1 when the score step runs on the tcgen05 kernel, 0 on the CUDA-core kernel
  *                 (paged caches whose block_size the TMA pieces cannot tile)
+ *   select_pieces key pieces each row's selection is cut into (1: one CTA per row). Few very long
+ *                 rows (decode over a long context) are split so that more SMs work on them;
+ *                 the pieces' lists are merged as li_merge_topk merges key ranges, one more
+ *                 kernel, and the workspace holds the partial lists
  * Returns LI_OK and fills *info, or an argument error.
  */
 typedef struct li_plan_info {
@@ -171,6 +177,7 @@ typedef struct li_plan_info {
     int32_t dense;
     int32_t kernels;
     int32_t score_tc;
+    int32_t select_pieces;
 } li_plan_info;
 li_status li_plan(const li_args *args, li_plan_info *info);
 
@@ -248,6 +255,48 @@ li_status li_set_stage_events(void *const *events, int32_t n_events);
 #define LI_NOALLOC_SCRATCH_BYTES (32u << 20)
 li_status li_indexer_noalloc(const li_args *args, int32_t *sparse_indices, float *sparse_values,
                              uint32_t *device_status, void *stream);
+
+/*
+ * li_merge_topk -- the split-merge step after a key-range split: the top-k of the union of
+ * several per-row top-k lists. A row whose keys are split into disjoint ranges (one range per GPU,
+ * or per piece of a very long row), each range selected by li_indexer with output_idx_offset set
+ * to the range's first key (so the indices are global), is merged back here. [reading] The pages
+ * select over a row's whole window (lightning_indexer, "Function" step 3; aclnnLightningIndexerV2,
+ * "主要计算过程"); the first topk of the union under the same order is that selection.
+ *
+ *   idx_in[l], val_in[l]  list l < n_lists: [rows, topk_in] int32 / fp32, row-major, as li_indexer
+ *                         writes them: each row ordered by score descending, then index ascending,
+ *                         with its padding (index < 0) after the valid entries. Indices must be
+ *                         distinct across lists. Device memory, or a peer GPU's memory that the
+ *                         current device can load from (plain loads, nothing else).
+ *   idx_out, val_out      [rows, topk_out]: the first topk_out valid entries of the union in that
+ *                         order, then -1 / -inf. val_out may be NULL (indices only).
+ *   device_status         device uint32 or NULL: LI_DEVERR_MERGE_ORDER is OR-ed in when an input
+ *                         row (its first topk_out entries) is out of order or has a valid entry
+ *                         after padding; the output is then unspecified. Read it with
+ *                         li_check_status(device_status, stream, &bits).
+ *
+ * Entries equal in score and index found in two lists (not a valid input) both appear, the lower
+ * list first. Only the first topk_out entries of an input row are read. Returns LI_ERR_INVALID_ARG
+ * for n_lists outside [1, LI_MERGE_MAX_LISTS], rows < 0, topk_in or topk_out outside [1, 8192], a
+ * NULL list or idx_out, or a pointer not 4-byte aligned; LI_ERR_UNSUPPORTED for rows > 2^31-1;
+ * LI_ERR_CUDA when the launch fails. Stream-ordered, allocates nothing, graph-capturable, and
+ * deterministic.
+ */
+#define LI_MERGE_MAX_LISTS 16
+typedef struct li_merge_args {
+    const int32_t *idx_in[LI_MERGE_MAX_LISTS];
+    const float *val_in[LI_MERGE_MAX_LISTS];
+    int32_t *idx_out;
+    float *val_out;
+    uint32_t *device_status;
+    int64_t rows;
+    int32_t n_lists;
+    int32_t topk_in;
+    int32_t topk_out;
+    int32_t reserved;                   /* must be 0 */
+} li_merge_args;
+li_status li_merge_topk(const li_merge_args *args, void *stream);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *li_last_error_string(void);

@@ -10,6 +10,8 @@
 #include <string>
 
 #include "li_internal.cuh"
+#include "li_merge.cuh"
+#include "li_select.cuh"
 
 namespace {
 
@@ -223,9 +225,20 @@ size_t scores_ld(const li::Problem &p) {
     return (size_t)li::scores_row_floats(p.max_seqlen_k, p.topk);
 }
 
+// Partial top-k lists of a row-split selection: [pieces][rows][topk] indices, then values.
+size_t piece_bytes(const li::Problem &p, int pieces) {
+    if (pieces <= 1) return 0;
+    const size_t n = (size_t)pieces * (size_t)p.rows * (size_t)p.topk;
+    return (n * sizeof(int32_t) + 255) / 256 * 256 + n * sizeof(float);
+}
+
+size_t scores_bytes(const li::Problem &p) {
+    return ((size_t)p.rows * scores_ld(p) * sizeof(float) + 255) / 256 * 256;
+}
+
 size_t indexer_ws_bytes(const li::Problem &p, const li::Schedule &s) {
-    return sizeof(li::WsHeader) + li::meta_bytes(p.batch, s.max_items) +
-           (size_t)p.rows * scores_ld(p) * sizeof(float);
+    return sizeof(li::WsHeader) + li::meta_bytes(p.batch, s.max_items) + scores_bytes(p) +
+           piece_bytes(p, li::select_pieces(p));
 }
 
 }  // namespace
@@ -271,7 +284,9 @@ li_status li_plan(const li_args *args, li_plan_info *info) {
     info->kc = s.kc;
     info->max_items = s.max_items;
     info->dense = s.dense;
-    info->kernels = p.rows > 0 ? (s.dense ? 2 : 3) : 0;
+    const int pieces = li::select_pieces(p);
+    info->kernels = p.rows > 0 ? (s.dense ? 2 : 3) + (pieces > 1 ? 1 : 0) : 0;
+    info->select_pieces = pieces;
     info->score_tc = !use_simple_kernel() && li::score_tc_eligible(p, s) ? 1 : 0;
     return ok();
 }
@@ -340,9 +355,34 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
     }
     stage_mark(3, cs);
     stage_mark(4, cs);
-    e = li::launch_select(p, s, meta, ws, scores, ld, sparse_indices,
-                          p.return_value ? sparse_values : nullptr, cs);
-    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+    const int pieces = li::select_pieces(p);
+    if (pieces > 1) {
+        // few very long rows: one CTA per key piece, then the split merge of the pieces' lists
+        const size_t n = (size_t)pieces * (size_t)p.rows * (size_t)p.topk;
+        char *pbase = reinterpret_cast<char *>(scores) + scores_bytes(p);
+        auto *part_idx = reinterpret_cast<int32_t *>(pbase);
+        auto *part_val = reinterpret_cast<float *>(pbase + (n * sizeof(int32_t) + 255) / 256 * 256);
+        e = li::launch_select_pieces(p, s, meta, ws, scores, ld, pieces, part_idx, part_val, cs);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+        li_merge_args m{};
+        const size_t list = (size_t)p.rows * (size_t)p.topk;
+        for (int c = 0; c < pieces; ++c) {
+            m.idx_in[c] = part_idx + c * list;
+            m.val_in[c] = part_val + c * list;
+        }
+        m.idx_out = sparse_indices;
+        m.val_out = p.return_value ? sparse_values : nullptr;
+        m.device_status = &ws->status;
+        m.rows = p.rows;
+        m.n_lists = pieces;
+        m.topk_in = m.topk_out = p.topk;
+        e = li::launch_merge(m, cs);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+    } else {
+        e = li::launch_select(p, s, meta, ws, scores, ld, sparse_indices,
+                              p.return_value ? sparse_values : nullptr, cs);
+        if (e != cudaSuccess) return fail(LI_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+    }
     stage_mark(5, cs);
     return ok();
 }
@@ -370,6 +410,32 @@ li_status li_set_stage_events(void *const *events, int32_t n_events) {
     if (n_events != 6 || !events) return fail(LI_ERR_INVALID_ARG, "li_set_stage_events wants 0 or 6 events");
     for (int i = 0; i < 6; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_stage_events_on = true;
+    return ok();
+}
+
+li_status li_merge_topk(const li_merge_args *a, void *stream) {
+    if (!a) return fail(LI_ERR_INVALID_ARG, "args is NULL");
+    if (a->n_lists < 1 || a->n_lists > LI_MERGE_MAX_LISTS)
+        return fail(LI_ERR_INVALID_ARG, "n_lists=%d outside [1, %d]", a->n_lists, LI_MERGE_MAX_LISTS);
+    if (a->rows < 0) return fail(LI_ERR_INVALID_ARG, "rows=%lld < 0", (long long)a->rows);
+    if (a->topk_in < 1 || a->topk_in > 8192 || a->topk_out < 1 || a->topk_out > 8192)
+        return fail(LI_ERR_INVALID_ARG, "topk_in=%d / topk_out=%d outside [1, 8192]", a->topk_in,
+                    a->topk_out);
+    if (a->reserved != 0) return fail(LI_ERR_INVALID_ARG, "reserved field must be 0");
+    if (!a->idx_out) return fail(LI_ERR_INVALID_ARG, "idx_out is NULL");
+    for (int l = 0; l < a->n_lists; ++l) {
+        if (!a->idx_in[l] || !a->val_in[l])
+            return fail(LI_ERR_INVALID_ARG, "list %d: idx_in / val_in is NULL", l);
+        if (!aligned(a->idx_in[l], 4) || !aligned(a->val_in[l], 4))
+            return fail(LI_ERR_INVALID_ARG, "list %d: pointers must be 4-byte aligned", l);
+    }
+    if (!aligned(a->idx_out, 4) || !aligned(a->val_out, 4) || !aligned(a->device_status, 4))
+        return fail(LI_ERR_INVALID_ARG, "outputs and device_status must be 4-byte aligned");
+    if (a->rows > INT32_MAX)
+        return fail(LI_ERR_UNSUPPORTED, "rows=%lld above 2^31-1", (long long)a->rows);
+    if (a->rows == 0) return ok();
+    cudaError_t e = li::launch_merge(*a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

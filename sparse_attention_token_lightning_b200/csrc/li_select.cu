@@ -23,6 +23,7 @@
 // take two streaming passes: a 12-bit key-digit histogram that bounds the selection, then a
 // gather of the candidates into shared memory, which the bucket sort orders.
 #include "li_internal.cuh"
+#include "li_select.cuh"
 
 namespace li {
 namespace {
@@ -37,6 +38,13 @@ struct Params {
     float *out_val;
     uint32_t signature;
     int32_t cand_cap;       // long-row candidates that fit in shared memory
+};
+
+struct PieceParams {
+    int32_t *idx;           // [pieces][rows][topk] partial lists
+    float *val;
+    int32_t pieces;
+    int32_t piece_len;
 };
 
 // Short rows: 256 threads per row, 16 keys per thread held in registers.
@@ -102,6 +110,45 @@ cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta,
     const size_t smem = sel512::select_work_bytes(p.topk, true, &cand_cap);
     return launch_one<512, true, sel512::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val, smem,
                                                cand_cap, sel512::select_kernel<true>, st);
+}
+
+int select_pieces(const Problem &p) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        sms = 148;
+    }
+    // only rows long enough that one CTA streaming the whole row is the bottleneck, and few
+    // enough rows that the GPU would otherwise sit mostly idle
+    if (p.rows <= 0 || p.max_seqlen_k < kPieceMinKeys || p.rows * 4 > sms) return 1;
+    int pieces = sms / (int)p.rows;
+    const int by_len = (p.max_seqlen_k + kPieceMinKeys / 2 - 1) / (kPieceMinKeys / 2);
+    if (pieces > by_len) pieces = by_len;
+    if (pieces > kMaxPieces) pieces = kMaxPieces;
+    while (pieces > 1 && !merge_fits_smem(pieces, p.topk, p.topk)) --pieces;
+    return pieces < 2 ? 1 : pieces;
+}
+
+int32_t piece_len(const Problem &p, int pieces) {
+    const int64_t len = ((int64_t)p.max_seqlen_k + pieces - 1) / pieces;
+    return (int32_t)((len + 127) / 128 * 128);
+}
+
+cudaError_t launch_select_pieces(const Problem &p, const Schedule &s, const void *meta,
+                                 WsHeader *ws, const float *scores, int64_t ld, int pieces,
+                                 int32_t *part_idx, float *part_val, cudaStream_t st) {
+    int32_t cand_cap = 0;
+    const size_t smem = sel1024::select_work_bytes(p.topk, true, &cand_cap);
+    if (smem + sizeof(sel1024::Smem) > 227 * 1024) return cudaErrorInvalidConfiguration;
+    auto kern = sel1024::select_piece_kernel<true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    Params sp{p, make_view(p, s, meta), ws, scores, ld, nullptr, nullptr,
+              problem_signature(p, s.tq, s.kc), cand_cap};
+    PieceParams pp{part_idx, part_val, pieces, piece_len(p, pieces)};
+    kern<<<(unsigned)(p.rows * pieces), 1024, smem, st>>>(sp, pp);
+    return cudaGetLastError();
 }
 
 }  // namespace li

@@ -634,22 +634,14 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
     return cand_bucket_topk(cand, n_c, m, hist, sbuf, sbufb, off, oi, ov, sm);
 }
 
-// kLong: the problem may have rows longer than kRegKeys * kThreads keys (long-row path compiled
-// in; two CTAs per SM). Otherwise only the register path and the exact fallback exist.
+// Selection of one row (or one key piece of a row): keys [0, n) of the fp32 row `src`, output
+// indices shifted by `off`, topk slots written to oi / ov (ov may be null).
 template <bool kLong>
-__global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) : 4) select_kernel(Params sp) {
+__device__ __forceinline__ void select_body(const Params &sp, int32_t n, int32_t off,
+                                            const float *src, int32_t *oi, float *ov,
+                                            unsigned char *dsm, Smem &sm) {
     const Problem &p = sp.p;
     const int tid = threadIdx.x;
-    bool meta_ok = true;
-    if (sp.view.meta) {
-        const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(sp.view.meta);
-        meta_ok = hdr->magic == kMetaMagic && hdr->signature == sp.signature;
-        if (blockIdx.x == 0 && tid == 0)
-            set_status(&sp.ws->status, meta_ok ? hdr->status : kDevErrMetadata);
-    }
-
-    extern __shared__ __align__(16) unsigned char dsm[];
-    __shared__ Smem sm;
     const int32_t topk = p.topk;
     // work area shared by the two paths, then the row cache
     int32_t *hist = reinterpret_cast<int32_t *>(dsm);                        // bucket path
@@ -665,27 +657,7 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     uint64_t *cand = reinterpret_cast<uint64_t *>(hist + kBucketsMax);       // long-row path
     const uint32_t *rowc = nullptr;                                         // exact path reads global
 
-    // blocks start in index order; later rows of a causal window are the longer ones, so the
-    // rows are taken last to first (longest first)
-    const int32_t r = (int32_t)(gridDim.x - 1 - blockIdx.x);
-    int32_t pos = 0;
-    int32_t b = meta_ok ? row_batch(p, r, &pos) : -1;
-    int32_t n = 0, off = 0;
-    if (b >= 0) {
-        const BatchInfo bi = sp.view.batch(p, b);
-        n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2, p.cmp_ratio, bi.pad[2]);
-
-        if (p.output_idx_offset) {
-            off = p.output_idx_offset[b];
-            // the schedule kernel validates offsets; without it each row checks its own
-            if (!sp.view.meta && tid == 0 &&
-                (off < 0 || (int64_t)off + (bi.L2 > 0 ? bi.L2 - 1 : 0) > (int64_t)INT32_MAX))
-                set_status(&sp.ws->status, LI_DEVERR_OFFSET);
-        }
-    }
     const int32_t m = min(n, topk);
-    int32_t *oi = sp.out_idx + (int64_t)r * topk;
-    float *ov = sp.out_val ? sp.out_val + (int64_t)r * topk : nullptr;
     const float kNegInf = -__int_as_float(0x7f800000);
 
     // 0: all padding, 1: bucket path (outputs written), 2: exact path (A or B buffers),
@@ -694,7 +666,6 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     bool inB = false;
     float vtie = 0.0f;
     if (m > 0 && n <= kRegKeys * kThreads) {
-        const float *src = sp.scores + (int64_t)r * sp.ld;
         mode = reg_bucket_topk(src, n, m, hist, buf, bufb, stage, off, oi, ov, sm, &vtie);
         if (mode == 2) {
             uint32_t prefix = 0u, mask = 0u;
@@ -705,7 +676,6 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
             inB = sort_desc(m, keyA, idxA, keyB, idxB, cnt, sm);
         }
     } else if (kLong && m > 0) {
-        const float *src = sp.scores + (int64_t)r * sp.ld;
         uint64_t *sbuf = cand + sp.cand_cap;
         uint16_t *sbufb = reinterpret_cast<uint16_t *>(sbuf + topk + kBinCap);
         mode = long_row_topk(src, n, m, hist, cand, sp.cand_cap, sbuf, sbufb, off, oi, ov, sm);
@@ -737,6 +707,74 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
         oi[s] = id;
         if (ov) ov[s] = v;
     }
+}
+
+// Window and output offset of query row r: *n keys, *off added to the indices. Checks the
+// schedule's signature (block 0 reports it) and, without a schedule kernel, the row's offset.
+__device__ __forceinline__ void row_window(const Params &sp, int32_t r, int32_t *n, int32_t *off) {
+    const Problem &p = sp.p;
+    const int tid = threadIdx.x;
+    bool meta_ok = true;
+    if (sp.view.meta) {
+        const MetaHeader *hdr = reinterpret_cast<const MetaHeader *>(sp.view.meta);
+        meta_ok = hdr->magic == kMetaMagic && hdr->signature == sp.signature;
+        if (blockIdx.x == 0 && tid == 0)
+            set_status(&sp.ws->status, meta_ok ? hdr->status : kDevErrMetadata);
+    }
+    int32_t pos = 0;
+    int32_t b = meta_ok ? row_batch(p, r, &pos) : -1;
+    *n = 0;
+    *off = 0;
+    if (b >= 0) {
+        const BatchInfo bi = sp.view.batch(p, b);
+        *n = window_hi(p.mask_mode, pos, bi.L1u, bi.L2, p.cmp_ratio, bi.pad[2]);
+
+        if (p.output_idx_offset) {
+            *off = p.output_idx_offset[b];
+            // the schedule kernel validates offsets; without it each row checks its own
+            if (!sp.view.meta && tid == 0 &&
+                (*off < 0 || (int64_t)*off + (bi.L2 > 0 ? bi.L2 - 1 : 0) > (int64_t)INT32_MAX))
+                set_status(&sp.ws->status, LI_DEVERR_OFFSET);
+        }
+    }
+}
+
+// kLong: the problem may have rows longer than kRegKeys * kThreads keys (long-row path compiled
+// in; two CTAs per SM). Otherwise only the register path and the exact fallback exist.
+template <bool kLong>
+__global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) : 4) select_kernel(Params sp) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ Smem sm;
+    // blocks start in index order; later rows of a causal window are the longer ones, so the
+    // rows are taken last to first (longest first)
+    const int32_t r = (int32_t)(gridDim.x - 1 - blockIdx.x);
+    int32_t n, off;
+    row_window(sp, r, &n, &off);
+    const int32_t topk = sp.p.topk;
+    select_body<kLong>(sp, n, off, sp.scores + (int64_t)r * sp.ld, sp.out_idx + (int64_t)r * topk,
+                       sp.out_val ? sp.out_val + (int64_t)r * topk : nullptr, dsm, sm);
+}
+
+// Few very long rows: each row's keys are cut into `pieces` consecutive pieces of piece_len keys
+// (a multiple of 128, so every piece starts 16-byte aligned), one CTA per (row, piece). Piece
+// c of row r selects among keys [c*piece_len, min(n, (c+1)*piece_len)) with their row indices
+// and writes a full top-k list (sorted, padded) to list c of the partial buffers
+// [pieces][rows][topk]; the split merge turns the lists into the row's output.
+template <bool kLong>
+__global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) : 4)
+select_piece_kernel(Params sp, PieceParams pp) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ Smem sm;
+    const int32_t rows = (int32_t)(gridDim.x / pp.pieces);
+    const int32_t r = rows - 1 - (int32_t)(blockIdx.x / pp.pieces);
+    const int32_t c = (int32_t)(blockIdx.x % pp.pieces);
+    int32_t n, off;
+    row_window(sp, r, &n, &off);
+    const int64_t start = (int64_t)c * pp.piece_len;
+    const int32_t len = n > start ? (int32_t)min((int64_t)pp.piece_len, (int64_t)n - start) : 0;
+    const int64_t slot = ((int64_t)c * rows + r) * sp.p.topk;
+    select_body<kLong>(sp, len, off + (int32_t)start, sp.scores + (int64_t)r * sp.ld + start,
+                       pp.idx + slot, pp.val + slot, dsm, sm);
 }
 
 // Bytes of the dynamic shared memory work area: the largest of the short-row bucket path

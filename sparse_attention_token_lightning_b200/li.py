@@ -55,14 +55,26 @@ class LiPlanInfo(ctypes.Structure):
 
     _fields_ = [("tq", ctypes.c_int32), ("kc", ctypes.c_int32), ("max_items", ctypes.c_int32),
                 ("dense", ctypes.c_int32), ("kernels", ctypes.c_int32),
-                ("score_tc", ctypes.c_int32)]
+                ("score_tc", ctypes.c_int32), ("select_pieces", ctypes.c_int32)]
 
 
 _lib = None
 
 EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
            "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
-           "li_abi_version", "li_indexer_noalloc", "li_plan")
+           "li_abi_version", "li_indexer_noalloc", "li_plan", "li_merge_topk")
+
+MERGE_MAX_LISTS = 16          # LI_MERGE_MAX_LISTS
+
+
+class LiMergeArgs(ctypes.Structure):
+    """Mirror of li_merge_args (include/li.h)."""
+    _fields_ = [
+        ("idx_in", ctypes.c_void_p * MERGE_MAX_LISTS), ("val_in", ctypes.c_void_p * MERGE_MAX_LISTS),
+        ("idx_out", ctypes.c_void_p), ("val_out", ctypes.c_void_p),
+        ("device_status", ctypes.c_void_p), ("rows", ctypes.c_int64), ("n_lists", ctypes.c_int32),
+        ("topk_in", ctypes.c_int32), ("topk_out", ctypes.c_int32), ("reserved", ctypes.c_int32),
+    ]
 
 
 def lib_path() -> Path:
@@ -97,6 +109,8 @@ def lib():
     L.li_set_stage_events.restype = ctypes.c_int
     L.li_last_error_string.argtypes = []
     L.li_last_error_string.restype = ctypes.c_char_p
+    L.li_merge_topk.argtypes = [ctypes.POINTER(LiMergeArgs), vp]
+    L.li_merge_topk.restype = ctypes.c_int
     L.li_abi_version.argtypes = []
     L.li_abi_version.restype = ctypes.c_int32
     _lib = L
@@ -219,6 +233,51 @@ def li_set_stage_events(events):
     assert len(events) == 6
     arr = (ctypes.c_void_p * 6)(*[int(e.cuda_event) for e in events])
     _check(lib().li_set_stage_events(arr, 6))
+
+
+def li_merge_topk(args: LiMergeArgs, stream=None):
+    _check(lib().li_merge_topk(ctypes.byref(args), _stream_handle(stream)))
+
+
+def merge_topk(idx_lists, val_lists, topk: int, return_value: bool = True, device_status=None,
+               stream=None, check: bool = True):
+    """Top-k of the union of per-row lists from key-range shards (li_merge_topk).
+
+    idx_lists / val_lists: sequences of device tensors whose last dimension is topk_in and whose
+    other dimensions flatten to the same row count (li_indexer outputs, indices already global),
+    or one stacked tensor of shape (n_lists, ...). Returns (indices, values) shaped like one
+    input list with topk as the last dimension; values is None when return_value is False."""
+    if isinstance(idx_lists, torch.Tensor):
+        idx_lists, val_lists = list(idx_lists.unbind(0)), list(val_lists.unbind(0))
+    n = len(idx_lists)
+    if n != len(val_lists) or not 1 <= n <= MERGE_MAX_LISTS:
+        raise ValueError(f"{n} index lists and {len(val_lists)} value lists")
+    ref = idx_lists[0]
+    topk_in = int(ref.shape[-1])
+    rows = ref.numel() // max(topk_in, 1)
+    for i, v in zip(idx_lists, val_lists):
+        if (i.dtype != torch.int32 or v.dtype != torch.float32 or i.shape != ref.shape or
+                v.shape != ref.shape or not i.is_contiguous() or not v.is_contiguous()):
+            raise ValueError("lists must be contiguous int32 / float32 tensors of one shape")
+    out_shape_ = tuple(ref.shape[:-1]) + (int(topk),)
+    idx = torch.empty(out_shape_, dtype=torch.int32, device=ref.device)
+    val = torch.empty(out_shape_, dtype=torch.float32, device=ref.device) if return_value else None
+    own_status = device_status is None and check
+    if own_status:
+        device_status = torch.zeros(1, dtype=torch.int32, device=ref.device)
+    a = LiMergeArgs()
+    for l in range(n):
+        a.idx_in[l] = idx_lists[l].data_ptr()
+        a.val_in[l] = val_lists[l].data_ptr()
+    a.idx_out, a.val_out = idx.data_ptr(), _ptr(val)
+    a.device_status = _ptr(device_status)
+    a.rows, a.n_lists, a.topk_in, a.topk_out = rows, n, topk_in, int(topk)
+    li_merge_topk(a, stream)
+    if own_status:
+        st, bits = li_check_status(device_status, stream)
+        if st != LI_OK:
+            raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
+    return idx, val
 
 
 def out_shape(pb):

@@ -265,6 +265,10 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
         # fp32 w
         return with_dtypes(bsnd(1, 4096, 4096, 64, 2048, 3, seed, integer=integer, name=name),
                            "fp16", "fp32").replace(name=name)
+    if name == "long_row_decode":
+        # one decode row over 2^20 keys (256 MB of keys); split by key range across GPUs
+        return paged([1 << 20], 1, 64, 2048, block_size=64, mask_mode=3, seed=seed + 1,
+                     integer=integer, name=name)
     if name == "pages_example":
         # The shape of the pages' worked example (B=2, S1=64, N1=16, topk=32) with the key
         # length it compresses to (130 // 4 = 32), taken uncompressed.
@@ -273,4 +277,4 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
 
 
 CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192",
-           "cmp_prefill", "fp16_prefill")
+           "cmp_prefill", "fp16_prefill", "long_row_decode")

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert li.li_abi_version() == 2
+    assert li.li_abi_version() == 3
 
 
 @pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
@@ -128,6 +128,43 @@ def test_every_dtype_pair_accepted(L, qk, w):
         assert _ws_status(_args(dtype_qk=qk, dtype_w=w, w=0x30002))[0] == 0
 
 
+def _merge_args(**kw):
+    a = li.LiMergeArgs()
+    n = kw.pop("n_lists", 2)
+    for l in range(min(n, li.MERGE_MAX_LISTS)):
+        a.idx_in[l] = 0x10000 + 0x1000 * l
+        a.val_in[l] = 0x40000 + 0x1000 * l
+    a.idx_out, a.val_out, a.device_status = 0x80000, 0x90000, 0xA0000
+    a.rows, a.n_lists, a.topk_in, a.topk_out = 0, n, 64, 64
+    for k, v in kw.items():
+        if k.startswith("idx_in_"):
+            a.idx_in[int(k[7:])] = v
+        else:
+            setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n_lists=0), dict(n_lists=17), dict(rows=-1), dict(topk_in=0), dict(topk_out=8193),
+    dict(topk_in=8193), dict(reserved=1), dict(idx_out=None), dict(idx_in_1=None),
+    dict(idx_in_1=0x11002), dict(val_out=0x90002), dict(device_status=0xA0001)])
+def test_invalid_merge_args_rejected_on_host(L, kw):
+    assert L.li_merge_topk(ctypes.byref(_merge_args(**kw)), None) == 1
+    assert li.li_last_error_string()
+
+
+def test_merge_rows_limit_and_empty_call(L):
+    assert L.li_merge_topk(ctypes.byref(_merge_args(rows=1 << 31)), None) == 2
+    # no rows: validated, nothing launched (no device needed)
+    assert L.li_merge_topk(ctypes.byref(_merge_args(rows=0, val_out=None, device_status=None,
+                                                    n_lists=16)), None) == 0
+
+
+def test_merge_args_struct_matches_the_header(L):
+    # 16 + 16 list pointers, 3 more pointers, int64 rows, four int32
+    assert ctypes.sizeof(li.LiMergeArgs) == 35 * 8 + 8 + 16
+
+
 def test_compressed_key_args_accepted(L):
     assert _ws_status(_args(cmp_ratio=4, cmp_residual_k=0x60000))[0] == 0
     assert _ws_status(_args(cmp_ratio=4, mask_mode=0))[0] == 0
@@ -165,7 +202,8 @@ def test_plan_reports_schedule_and_kernel_count(L):
     # dense causal BSND: closed-form work list, score + select kernels only
     pl = li.li_plan(_args(q_len=4096, k_len=4096, max_seqlen_q=4096, max_seqlen_k=4096,
                           num_heads_q=64, topk=2048))
-    assert pl == dict(tq=4, kc=0, max_items=1024, dense=1, kernels=2, score_tc=1)
+    assert pl == dict(tq=4, kc=0, max_items=1024, dense=1, kernels=2, score_tc=1,
+                      select_pieces=1)
     # one query row per batch (decode): tq capped by max_seqlen_q, schedule kernel needed
     pl = li.li_plan(_args(layout_k=2, k_len=0, q_len=1, max_seqlen_q=1, batch=64,
                           num_heads_q=64, seqused_k=0x40000, block_table=0x50000,
@@ -173,6 +211,18 @@ def test_plan_reports_schedule_and_kernel_count(L):
                           max_seqlen_k=32768, topk=2048))
     assert pl["tq"] == 1 and pl["dense"] == 2 and pl["kernels"] == 2 and pl["score_tc"] == 1
     assert pl["kc"] > 0 and pl["max_items"] >= 64 * (32768 // pl["kc"])
+    # one very long decode row: its selection is cut into key pieces plus one merge kernel,
+    # and the workspace grows by the pieces' lists
+    long_row = dict(layout_k=2, k_len=0, q_len=1, max_seqlen_q=1, batch=1, num_heads_q=64,
+                    seqused_k=0x40000, block_table=0x50000, block_table_stride=16384,
+                    num_blocks=16384, block_size=64, topk=2048)
+    pl = li.li_plan(_args(max_seqlen_k=1 << 20, **long_row))
+    assert pl["select_pieces"] > 1 and pl["kernels"] == 3
+    one = li.li_plan(_args(max_seqlen_k=16384, **long_row))
+    assert one["select_pieces"] == 1 and one["kernels"] == 2
+    st_a, n_split = _ws_status(_args(max_seqlen_k=1 << 20, **long_row))
+    st_b, n_whole = _ws_status(_args(max_seqlen_k=(1 << 20) - 128, **long_row))
+    assert st_a == st_b == 0
     # block sizes the TMA pieces cannot tile go to the CUDA-core score kernel
     pl = li.li_plan(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
                           block_table_stride=64, num_blocks=64, block_size=12,

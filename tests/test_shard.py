@@ -71,6 +71,95 @@ def test_sub_problem_rows_equal_whole_problem_rows(orc, mask):
         assert np.array_equal(v.view(np.uint32), whole_v[a:b].view(np.uint32))
 
 
+# ---- key-range sharding ---------------------------------------------------------------------------
+
+def test_key_ranges_partition_the_keys():
+    for L2, parts, align, cap in [(1000, 3, 1, None), (1000, 8, 64, None), (100, 4, 1, 50),
+                                  (5, 8, 1, None), (0, 3, 1, None), (4097, 2, 64, 4000)]:
+        rng = shard.key_ranges(L2, parts, align, cap)
+        assert len(rng) == parts and rng[0][0] == 0 and rng[-1][1] == L2
+        assert all(a <= b for a, b in rng)
+        assert all(rng[i][1] == rng[i + 1][0] for i in range(parts - 1))
+        assert all(a % align == 0 for a, _ in rng)
+        if cap is not None:
+            assert rng[-1][0] <= cap
+
+
+KEY_SHARD_CASES = {
+    "paged_decode": lambda: synthetic.paged([3000, 700, 65, 1], 1, 16, 128, block_size=64,
+                                            seed=90, spare_blocks=3),
+    "paged_decode_bs16": lambda: synthetic.paged([900, 40], 1, 8, 300, block_size=16, seed=91),
+    "paged_causal_rows": lambda: synthetic.paged([1000, 500], 3, 8, 100, block_size=64, seed=92),
+    "paged_tnd_q_nomask": lambda: synthetic.paged([700, 300], 0, 8, 64, block_size=32, seed=93,
+                                                  mask_mode=0, layout_q="TND", lens_q=[4, 2]),
+    "bsnd_causal_seqused": lambda: synthetic.bsnd(2, 6, 500, 8, 150, 3, seed=94,
+                                                  seqused_k=[500, 321]),
+    "bsnd_nomask_offset": lambda: synthetic.bsnd(2, 5, 400, 4, 64, 0, seed=95,
+                                                 output_idx_offset=[7, 1000]),
+}
+
+
+@pytest.mark.parametrize("compact", [False, True])
+@pytest.mark.parametrize("parts", [1, 2, 3, 5])
+@pytest.mark.parametrize("name", list(KEY_SHARD_CASES))
+def test_key_shards_merge_to_the_whole_problem(orc, name, parts, compact):
+    """Selecting in every key range with global indices and merging the lists gives the whole
+    problem's output bit for bit (oracle on both sides, so this checks the range algebra)."""
+    pb = KEY_SHARD_CASES[name]()
+    whole = orc.topk(pb)
+    lists = [orc.topk(shard.key_shard(pb, parts, r, compact)) for r in range(parts)]
+    got = orc.merge_topk([x[0] for x in lists], [x[1] for x in lists], pb.topk)
+    assert np.array_equal(got[0], whole[0]), name
+    assert np.array_equal(got[1].view(np.uint32), whole[1].view(np.uint32)), name
+
+
+def test_key_shard_rejects_what_it_cannot_split():
+    with pytest.raises(ValueError):
+        shard.key_shard(synthetic.tnd([5], [90], 4, 8, 3, seed=96), 2, 0)
+    with pytest.raises(ValueError):
+        shard.key_shard(KEY_SHARD_CASES["paged_decode"](), 2, 2)
+
+
+def _oracle_run(pb):
+    from oracle import oracle as orc_mod
+    i, v, rc = orc_mod.default().topk(pb)
+    assert rc == 0
+    return torch.from_numpy(i), torch.from_numpy(v)
+
+
+def _oracle_merge(gi, gv, topk):
+    from oracle import oracle as orc_mod
+    i, v = orc_mod.default().merge_topk(list(gi.numpy()), list(gv.numpy()), topk)
+    return torch.from_numpy(i), torch.from_numpy(v)
+
+
+def _key_rank_main(rank, world, init_file, result_file):
+    dist.init_process_group("gloo", init_method=f"file://{init_file}", rank=rank,
+                            world_size=world)
+    try:
+        pb = KEY_SHARD_CASES["paged_decode"]()
+        part = shard.key_shard(pb, world, rank)
+        idx, val = shard.key_sharded_indexer(part, run=_oracle_run, merge=_oracle_merge)
+        if rank == 0:
+            torch.save((idx, val), result_file)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_merge_key_ranges(orc):
+    """Two ranks each hold half of every sequence's keys, select with the oracle, all-gather the
+    lists and merge: every rank ends with the whole rows' top-k."""
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        init_file = os.path.join(d, "init")
+        result_file = os.path.join(d, "out.pt")
+        mp.spawn(_key_rank_main, args=(world, init_file, result_file), nprocs=world, join=True)
+        idx, val = torch.load(result_file)
+    whole = orc.topk(KEY_SHARD_CASES["paged_decode"]())
+    assert np.array_equal(idx.numpy(), whole[0])
+    assert np.array_equal(val.numpy().view(np.uint32), whole[1].view(np.uint32))
+
+
 @pytest.mark.gpu
 def test_sharded_gpu_runs_are_bit_identical_to_the_whole_run():
     if not torch.cuda.is_available():
