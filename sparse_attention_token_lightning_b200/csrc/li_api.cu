@@ -376,7 +376,7 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
         m.rows = p.rows;
         m.n_lists = pieces;
         m.topk_in = m.topk_out = p.topk;
-        e = li::launch_merge(m, cs);
+        e = li::launch_merge(m, cs, false);     // the pieces' lists are sorted by construction
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     } else {
         e = li::launch_select(p, s, meta, ws, scores, ld, sparse_indices,

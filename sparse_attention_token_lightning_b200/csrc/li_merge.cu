@@ -38,6 +38,7 @@ struct MergeParams {
     uint32_t *status;
     int32_t n_lists, topk_in, topk_out;
     int32_t lim;          // entries of an input row that can reach the output: min(topk_in, topk_out)
+    int32_t check;        // verify the input order (lists from outside the library)
 };
 
 // Larger key = earlier in the order. The score is mapped to an order-preserving unsigned
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const __grid_constant__
 }
 
 constexpr int kTreeThreads = 512;
-constexpr int kStageUnroll = 8;                  // entries each thread has in flight while staging
+constexpr int kStageUnroll = 16;                 // entries each thread has in flight while staging
 
 __device__ __forceinline__ float key_value(uint64_t k) {
     const uint32_t u = (uint32_t)(k >> 32);
@@ -174,35 +175,48 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
     const int G = P.n_lists, lim = P.lim;
     const int64_t base = r * (int64_t)P.topk_in;
     if (tid == 0) s_bad = 0;
+    // flat position f = l * lim + e over all lists, kept as (l, e) and advanced by the block
+    // size without a division; kStageUnroll independent loads per thread
     const int32_t total_in = G * lim;
+    int sl = 0;
+    int32_t se = tid;
+    while (se >= lim && sl < G) { se -= lim; ++sl; }
+    const int sl0 = sl;
+    const int32_t se0 = se;
     for (int32_t f0 = 0; f0 < total_in; f0 += kTreeThreads * kStageUnroll) {
-        int32_t iv[kStageUnroll];
+        // loads only in this loop (no branch on a loaded value), so all of them are in flight
+        int32_t iv[kStageUnroll], fe[kStageUnroll];
         float vv[kStageUnroll];
 #pragma unroll
         for (int u = 0; u < kStageUnroll; ++u) {
-            const int32_t f = f0 + u * kTreeThreads + tid;
             iv[u] = -1;
             vv[u] = 0.0f;
-            if (f < total_in) {
-                const int l = f / lim;
-                const int64_t at = base + (f - l * lim);
-                iv[u] = __ldg(P.idx[l] + at);
-                vv[u] = __ldg(P.val[l] + at);
+            fe[u] = -1;
+            if (sl < G) {
+                const int64_t at = base + se;
+                iv[u] = __ldg(P.idx[sl] + at);
+                vv[u] = __ldg(P.val[sl] + at);
+                fe[u] = sl * lim + se;
+                se += kTreeThreads;
+                while (se >= lim && sl < G) { se -= lim; ++sl; }
             }
         }
 #pragma unroll
-        for (int u = 0; u < kStageUnroll; ++u) {
-            const int32_t f = f0 + u * kTreeThreads + tid;
-            if (f < total_in) s_mem[f] = iv[u] >= 0 ? order_key(iv[u], vv[u]) : 0ull;
-        }
+        for (int u = 0; u < kStageUnroll; ++u)
+            if (fe[u] >= 0) s_mem[fe[u]] = iv[u] >= 0 ? order_key(iv[u], vv[u]) : 0ull;
     }
     __syncthreads();
-    // input contract: strictly decreasing keys, then padding (key 0); valid prefix of each list
+    // input contract: within a list, keys strictly decrease until the padding (key 0) starts
     bool bad = false;
-    for (int32_t f = tid; f < total_in; f += kTreeThreads) {
-        const int32_t e = f % lim;
-        if (e + 1 < lim && s_mem[f + 1] != 0 && !(s_mem[f] > s_mem[f + 1])) bad = true;
+    for (sl = P.check ? sl0 : G, se = se0; sl < G;) {
+        if (se + 1 < lim) {
+            const uint64_t k0 = s_mem[sl * lim + se], k1 = s_mem[sl * lim + se + 1];
+            if (k1 != 0 && !(k0 > k1)) bad = true;
+        }
+        se += kTreeThreads;
+        while (se >= lim && sl < G) { se -= lim; ++sl; }
     }
+    // valid prefix of each list
     if (tid < G) {
         const uint64_t *k = s_mem + tid * lim;
         int32_t lo = 0, hi = lim;
@@ -219,8 +233,7 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
     int32_t *oi = P.idx_out + r * (int64_t)P.topk_out;
     float *ov = P.val_out ? P.val_out + r * (int64_t)P.topk_out : nullptr;
     int cur = 0, count = G;
-    const uint64_t *src = s_mem;
-    uint64_t *dst = s_mem + y_off;
+    int32_t src = 0, dst = y_off;              // word offsets of this level's input and output
     for (;;) {
         const int pairs = (count + 1) >> 1;
         const bool last = pairs == 1;
@@ -239,13 +252,14 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
         const int tpp = kTreeThreads / pairs;
         const int q = tid / tpp, tt = tid - q * tpp;
         if (q < pairs) {
-            const uint64_t *A = src + s_off[cur][2 * q];
+            const uint64_t *A = s_mem + src + s_off[cur][2 * q];
             const int32_t na = s_len[cur][2 * q];
             const bool hasB = 2 * q + 1 < count;
-            const uint64_t *B = hasB ? src + s_off[cur][2 * q + 1] : A;
+            const uint64_t *B = hasB ? s_mem + src + s_off[cur][2 * q + 1] : A;
             const int32_t nb = hasB ? s_len[cur][2 * q + 1] : 0;
             const int32_t n_out = s_len[cur ^ 1][q];
-            const int32_t k = (n_out + tpp - 1) / tpp;
+            // an odd run length keeps the lanes of a warp (k entries apart) on different banks
+            const int32_t k = ((n_out + tpp - 1) / tpp) | 1;
             const int32_t d = tt * k;
             if (d < n_out) {
                 // merge path: i entries of A are among the first d outputs
@@ -258,7 +272,7 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
                 int32_t i = lo, j = d - lo;
                 uint64_t a = i < na ? A[i] : 0ull;
                 uint64_t b = j < nb ? B[j] : 0ull;
-                uint64_t *out = dst + s_off[cur ^ 1][q];
+                uint64_t *out = s_mem + dst + s_off[cur ^ 1][q];
                 const int32_t end = min(d + k, n_out);
                 for (int32_t pos = d; pos < end; ++pos) {
                     const bool takeA = j >= nb || (i < na && a >= b);
@@ -281,8 +295,8 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
         }
         if (last) break;
         __syncthreads();
-        const uint64_t *nsrc = dst;
-        dst = const_cast<uint64_t *>(src);
+        const int32_t nsrc = dst;
+        dst = src;
         src = nsrc;
         cur ^= 1;
         count = pairs;
@@ -323,7 +337,7 @@ bool merge_fits_smem(int n_lists, int topk_in, int topk_out) {
     return tree_smem_words(n_lists, lim, topk_out, &y_off) * sizeof(uint64_t) <= kSmemMergeMax;
 }
 
-cudaError_t launch_merge(const li_merge_args &a, cudaStream_t stream) {
+cudaError_t launch_merge(const li_merge_args &a, cudaStream_t stream, bool check) {
     MergeParams P{};
     for (int l = 0; l < a.n_lists; ++l) {
         P.idx[l] = a.idx_in[l];
@@ -336,6 +350,7 @@ cudaError_t launch_merge(const li_merge_args &a, cudaStream_t stream) {
     P.topk_in = a.topk_in;
     P.topk_out = a.topk_out;
     P.lim = a.topk_in < a.topk_out ? a.topk_in : a.topk_out;
+    P.check = check ? 1 : 0;
     int32_t y_off = 0;
     const size_t smem = tree_smem_words(a.n_lists, P.lim, a.topk_out, &y_off) * sizeof(uint64_t);
     if (smem <= kSmemMergeMax) {
