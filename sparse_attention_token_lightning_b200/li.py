@@ -280,6 +280,65 @@ def merge_topk(idx_lists, val_lists, topk: int, return_value: bool = True, devic
     return idx, val
 
 
+class HostPipeline:
+    """li_indexer over a series of host-resident problems of one shape: inputs copied in from
+    pinned host memory, outputs read back to pinned host memory, with the copies overlapping the
+    kernels. Three streams (copy in, kernels, copy out) and `depth` sets of device buffers let
+    step i's host-to-device copy, step i-1's kernels and step i-2's device-to-host copy run at
+    the same time; events keep a buffer set from being refilled before its kernels have read it
+    or overwritten before its outputs have been copied out.
+
+    template: a problem giving the shapes, types and scalar arguments (its tensors are copied
+    once to size the device buffers). run(inputs, outputs): inputs[i] maps the problem's tensor
+    fields (q, k, w and the side arrays) to pinned host tensors of the template's shapes;
+    outputs[i] is a pair of pinned host tensors (indices, values) of li.out_shape. Returns when
+    the work is queued; synchronize() waits for it."""
+
+    def __init__(self, template, device, depth: int = 2):
+        from .synthetic import Problem
+        self.fields = [f for f in Problem.TENSORS if getattr(template, f) is not None]
+        self.sets = []
+        for _ in range(depth):
+            pb = template.to(device)
+            args = make_args(pb)
+            self.sets.append(dict(
+                pb=pb, args=args, ws=empty_workspace(args, device),
+                idx=torch.empty(out_shape(pb), dtype=torch.int32, device=device),
+                val=torch.empty(out_shape(pb), dtype=torch.float32, device=device),
+                loaded=torch.cuda.Event(), ran=torch.cuda.Event(), saved=torch.cuda.Event()))
+        self.s_in = torch.cuda.Stream(device)
+        self.s_run = torch.cuda.Stream(device)
+        self.s_out = torch.cuda.Stream(device)
+
+    def run(self, inputs, outputs):
+        for i, (h, (hi, hv)) in enumerate(zip(inputs, outputs)):
+            S = self.sets[i % len(self.sets)]
+            self.s_in.wait_event(S["ran"])          # the set's previous kernels are done with it
+            with torch.cuda.stream(self.s_in):
+                for f in self.fields:
+                    getattr(S["pb"], f).copy_(h[f], non_blocking=True)
+                S["loaded"].record(self.s_in)
+            self.s_run.wait_event(S["loaded"])
+            self.s_run.wait_event(S["saved"])       # its previous outputs are back on the host
+            li_indexer(S["args"], None, S["ws"], S["idx"], S["val"], self.s_run)
+            S["ran"].record(self.s_run)
+            self.s_out.wait_event(S["ran"])
+            with torch.cuda.stream(self.s_out):
+                hi.copy_(S["idx"], non_blocking=True)
+                hv.copy_(S["val"], non_blocking=True)
+                S["saved"].record(self.s_out)
+
+    def check(self):
+        """Device status of every buffer set (raises LiError on a data error)."""
+        for S in self.sets:
+            st, bits = li_check_status(S["ws"], self.s_run)
+            if st != LI_OK:
+                raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
+
+    def synchronize(self):
+        self.s_out.synchronize()
+
+
 def out_shape(pb):
     return (pb.batch, pb.q_len, 1, pb.topk) if pb.layout_q == "BSND" else (pb.q_len, 1, pb.topk)
 

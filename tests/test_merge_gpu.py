@@ -152,3 +152,20 @@ def test_split_row_selection_integer_inputs_bit_exact(orc):
     torch.cuda.synchronize()
     parity.check(orc, pb, parity.as_rows(gi, pb.topk), parity.as_rows(gv, pb.topk), exact=True,
                  label="integer split rows")
+
+
+def test_host_pipeline_matches_single_calls():
+    """The pipelined host-to-host runner gives every step the same outputs as one li.indexer call
+    on that step's problem (different inputs per step, more steps than buffer sets)."""
+    probs = [synthetic.bsnd(2, 300, 459, 64, 200, 3, seed=120 + i) for i in range(5)]
+    pipe = li.HostPipeline(probs[0], "cuda")
+    inputs = [{f: getattr(pb, f).pin_memory() for f in pipe.fields} for pb in probs]
+    shape = li.out_shape(probs[0])
+    outputs = [(torch.empty(shape, dtype=torch.int32).pin_memory(),
+                torch.empty(shape, dtype=torch.float32).pin_memory()) for _ in probs]
+    pipe.run(inputs, outputs)
+    pipe.synchronize()
+    pipe.check()
+    for pb, (hi, hv) in zip(probs, outputs):
+        ri, rv = li.indexer(pb.to("cuda"))
+        assert torch.equal(hi, ri.cpu()) and torch.equal(hv, rv.cpu())
