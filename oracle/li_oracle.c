@@ -40,9 +40,12 @@
  *      the first topk kept.
  *
  * Precision. q and k arrive as bf16 or fp16 bit patterns (lightning_indexer, "Constraints": q
- * and k share one type; the single-operator example passes fp16 q and k with fp32 w), w as bf16,
- * fp16 or fp32; every product and sum is taken in fp64, so the score is the exact real value up
- * to fp64 rounding. The selection decision is then taken on
+ * and k share one type; the single-operator example passes fp16 q and k with fp32 w), or as fp8
+ * e4m3 codes with q_descale and k_descale (aclnnLightningIndexerV2, parameter dimensions: the
+ * pages name these two arguments and nothing more; [reading] dequantized q = code x
+ * q_descale[row, head], k = code x k_descale[key]; parity of this reading is unpinned beyond the
+ * fp8 decoding and the scaling laws the pins check). w arrives as bf16, fp16 or fp32; every
+ * product and sum is taken in fp64, so the score is the exact real value up to fp64 rounding. The selection decision is then taken on
  * the score rounded once to fp32, the precision the CUDA kernels decide in, and -0 is treated as
  * +0. Order: score descending, then key index ascending (the pages only say "deterministic").
  *
@@ -62,7 +65,7 @@
 #endif
 
 enum { ORC_BSND = 0, ORC_TND = 1, ORC_PA_BSND = 2 };
-enum { ORC_BF16 = 0, ORC_FP16 = 1, ORC_FP32 = 2 };
+enum { ORC_BF16 = 0, ORC_FP16 = 1, ORC_FP32 = 2, ORC_FP8_E4M3 = 3 };
 enum { ORC_OK = 0, ORC_EARG = 1, ORC_EDATA = 2, ORC_ENOMEM = 3 };
 
 /* One problem. All arrays are host memory in the layouts the pages give:
@@ -71,7 +74,7 @@ enum { ORC_OK = 0, ORC_EARG = 1, ORC_EDATA = 2, ORC_ENOMEM = 3 };
  *   w: (B, S1, N1) or (T1, N1)
  * Optional arrays are NULL when absent. */
 typedef struct {
-    const uint16_t *q, *k;          /* bf16 or fp16 bit patterns (dtype_qk)                     */
+    const void *q, *k;              /* bf16 / fp16 bit patterns (2 bytes) or fp8 e4m3 (1 byte)  */
     const void *w;                  /* bf16 or fp16 bit patterns, or fp32 values (dtype_w)      */
     const int32_t *cu_seqlens_q, *cu_seqlens_k;
     const int32_t *seqused_q, *seqused_k;
@@ -86,7 +89,10 @@ typedef struct {
     int32_t layout_q, layout_k, mask_mode;
     const int32_t *cmp_residual_k;  /* [B] or NULL: tokens past the last whole compressed key */
     int32_t cmp_ratio;              /* original tokens per key; 0 or 1 = keys not compressed  */
-    int32_t dtype_qk, dtype_w;      /* ORC_BF16 / ORC_FP16 (q, k); also ORC_FP32 for w        */
+    int32_t dtype_qk, dtype_w;      /* ORC_BF16 / ORC_FP16 / ORC_FP8_E4M3 (q, k); ORC_BF16 /
+                                       ORC_FP16 / ORC_FP32 (w)                                  */
+    const float *q_descale;         /* fp8 q, k: [rows * N1] (laid out like w) and one value  */
+    const float *k_descale;         /* per key row (laid out like k without D); NULL otherwise */
 } orc_problem;
 
 static double bf16_value(uint16_t bits)
@@ -115,8 +121,26 @@ static double fp16_value(uint16_t bits)
     return sign ? -v : v;
 }
 
-static double qk_value(const orc_problem *p, uint16_t bits)
+/* OCP 8-bit float E4M3 (the "fn" variant: no infinities): sign, 4 exponent bits (bias 7),
+ * 3 fraction bits; exponent 15 with fraction 7 is NaN, so the largest value is 448. */
+static double fp8_e4m3_value(uint8_t bits)
 {
+    const int sign = bits >> 7, e = (bits >> 3) & 0xf, f = bits & 0x7;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -9);                         /* subnormal: (f/8) * 2^-6     */
+    else if (e == 15 && f == 7)
+        v = NAN;
+    else
+        v = ldexp(8.0 + f, e - 10);                       /* (1 + f/8) * 2^(e - 7)       */
+    return sign ? -v : v;
+}
+
+/* Element i of q or k (a 2-byte or 1-byte array by dtype_qk) as a real number. */
+static double qk_value(const orc_problem *p, const void *arr, int64_t i)
+{
+    if (p->dtype_qk == ORC_FP8_E4M3) return fp8_e4m3_value(((const uint8_t *)arr)[i]);
+    const uint16_t bits = ((const uint16_t *)arr)[i];
     return p->dtype_qk == ORC_FP16 ? fp16_value(bits) : bf16_value(bits);
 }
 
@@ -208,52 +232,61 @@ static int64_t orc_window(const orc_problem *p, const orc_row *o)
     return hi < 0 ? 0 : hi;
 }
 
-/* Key j of batch b (logical position within the batch's key sequence). */
-static const uint16_t *orc_key(const orc_problem *p, int32_t b, int64_t j)
+/* Row of k (in units of D elements) holding key j of batch b (logical position within the
+ * batch's key sequence). */
+static int64_t orc_key_row(const orc_problem *p, int32_t b, int64_t j)
 {
-    const int64_t D = p->head_dim;
     if (p->layout_k == ORC_TND) {
 #if ORC_MUTANT == 8
-        return p->k + ((int64_t)p->cu_seqlens_q[b] + j) * D;   /* mistake: query offsets */
+        return (int64_t)p->cu_seqlens_q[b] + j;   /* mistake: query offsets */
 #else
-        return p->k + ((int64_t)p->cu_seqlens_k[b] + j) * D;
+        return (int64_t)p->cu_seqlens_k[b] + j;
 #endif
     }
     if (p->layout_k == ORC_PA_BSND) {
 #if ORC_MUTANT == 7
         (void)b;
-        return p->k + j * D;                      /* mistake: block table ignored */
+        return j;                                 /* mistake: block table ignored */
 #else
         int64_t blk = p->block_table[(int64_t)b * p->block_table_stride + j / p->block_size];
-        return p->k + (blk * p->block_size + j % p->block_size) * D;
+        return blk * p->block_size + j % p->block_size;
 #endif
     }
-    return p->k + ((int64_t)b * p->k_len + j) * D;
+    return (int64_t)b * p->k_len + j;
 }
 
-static const uint16_t *orc_query(const orc_problem *p, int64_t r, int32_t h)
+/* Row of q (in units of D elements) holding head h of query row r. */
+static int64_t orc_query_row(const orc_problem *p, int64_t r, int32_t h)
 {
 #if ORC_MUTANT == 6
-    /* mistake: head and row strides exchanged */
-    return p->q + ((int64_t)h * orc_num_rows(p) + r) * p->head_dim;
+    return (int64_t)h * orc_num_rows(p) + r;      /* mistake: head and row strides exchanged */
 #else
-    return p->q + (r * p->n_heads + h) * p->head_dim;
+    return r * p->n_heads + h;
 #endif
 }
 
 /* Step 3: the exact score of row r against key j, in fp64. */
 static double orc_score(const orc_problem *p, int64_t r, const orc_row *o, int64_t j)
 {
-    const uint16_t *kj = orc_key(p, o->b, j);
+    const int64_t D = p->head_dim;
+    const int64_t kr = orc_key_row(p, o->b, j);
     double I = 0.0;
 #if ORC_MUTANT == 1
     double sum_ws = 0.0;
 #endif
     for (int32_t h = 0; h < p->n_heads; ++h) {
-        const uint16_t *qh = orc_query(p, r, h);
+        const int64_t qr = orc_query_row(p, r, h);
         double s = 0.0;
         for (int32_t d = 0; d < p->head_dim; ++d)
-            s += qk_value(p, qh[d]) * qk_value(p, kj[d]);
+            s += qk_value(p, p->q, qr * D + d) * qk_value(p, p->k, kr * D + d);
+        /* [reading] fp8 q and k are quantized values: q_descale[r, h] and k_descale[key row]
+         * scale them back (the pages name q_descale and k_descale and their dimensions only) */
+        if (p->dtype_qk == ORC_FP8_E4M3)
+#if ORC_MUTANT == 15
+            s *= (double)p->q_descale[r * p->n_heads + h];    /* mistake: k_descale dropped */
+#else
+            s *= (double)p->q_descale[r * p->n_heads + h] * (double)p->k_descale[kr];
+#endif
         double wh = w_value(p, r * p->n_heads + h);
 #if ORC_MUTANT == 1
         sum_ws += wh * s;                              /* mistake: ReLU after the head sum */
@@ -311,7 +344,9 @@ static int orc_check(const orc_problem *p)
     if (p->layout_k == ORC_PA_BSND && (!p->seqused_k || !p->block_table || p->block_size < 1))
         return ORC_EARG;
     if (p->cmp_ratio < 0) return ORC_EARG;
-    if (p->dtype_qk != ORC_BF16 && p->dtype_qk != ORC_FP16) return ORC_EARG;
+    if (p->dtype_qk != ORC_BF16 && p->dtype_qk != ORC_FP16 && p->dtype_qk != ORC_FP8_E4M3)
+        return ORC_EARG;
+    if (p->dtype_qk == ORC_FP8_E4M3 && (!p->q_descale || !p->k_descale)) return ORC_EARG;
     if (p->dtype_w != ORC_BF16 && p->dtype_w != ORC_FP16 && p->dtype_w != ORC_FP32) return ORC_EARG;
     if (p->cmp_residual_k)
         for (int b = 0; b < p->batch; ++b)

@@ -50,18 +50,20 @@ class _Problem(ctypes.Structure):
         ("layout_q", ctypes.c_int32), ("layout_k", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
         ("cmp_residual_k", ctypes.c_void_p), ("cmp_ratio", ctypes.c_int32),
         ("dtype_qk", ctypes.c_int32), ("dtype_w", ctypes.c_int32),
+        ("q_descale", ctypes.c_void_p), ("k_descale", ctypes.c_void_p),
     ]
 
 
-DTYPES = {"bf16": 0, "fp16": 1, "fp32": 2}
+DTYPES = {"bf16": 0, "fp16": 1, "fp32": 2, "fp8_e4m3": 3}
 
 
 def _dtype_name(x) -> str:
-    """bf16 / fp16 / fp32 of a tensor (uint16 arrays are bf16 bit patterns)."""
+    """bf16 / fp16 / fp32 / fp8_e4m3 of a tensor (uint16 arrays are bf16 bit patterns)."""
     if isinstance(x, np.ndarray):
         return "fp32" if x.dtype == np.float32 else "bf16"
     import torch
-    return {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[x.dtype]
+    return {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32",
+            torch.float8_e4m3fn: "fp8_e4m3"}[x.dtype]
 
 
 def _bits16(x) -> np.ndarray:
@@ -72,6 +74,22 @@ def _bits16(x) -> np.ndarray:
     import torch  # local: the oracle does not need torch unless handed tensors
     assert x.dtype in (torch.bfloat16, torch.float16), x.dtype
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _qk_codes(x) -> np.ndarray:
+    """q or k as stored: 16-bit patterns (bf16 / fp16) or 8-bit codes (fp8 e4m3)."""
+    if not isinstance(x, np.ndarray) and _dtype_name(x) == "fp8_e4m3":
+        import torch
+        return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.uint8).numpy())
+    return _bits16(x)
+
+
+def _f32(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().contiguous().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
 
 
 def _weights(x) -> np.ndarray:
@@ -127,8 +145,10 @@ class Oracle:
             return arr.ctypes.data
 
         s = _Problem()
-        s.q = ptr("q", _bits16(pb.q))
-        s.k = ptr("k", _bits16(pb.k))
+        s.q = ptr("q", _qk_codes(pb.q))
+        s.k = ptr("k", _qk_codes(pb.k))
+        s.q_descale = ptr("q_descale", _f32(getattr(pb, "q_descale", None)))
+        s.k_descale = ptr("k_descale", _f32(getattr(pb, "k_descale", None)))
         s.w = ptr("w", _weights(pb.w))
         s.dtype_qk = DTYPES[_dtype_name(pb.q)]
         s.dtype_w = DTYPES[_dtype_name(pb.w)]

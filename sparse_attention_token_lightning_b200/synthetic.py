@@ -53,10 +53,12 @@ class Problem:
     block_size: int = 0
     cmp_ratio: int = 1                 # original tokens per key (1: keys not compressed)
     cmp_residual_k: Optional[torch.Tensor] = None   # [B] tokens past the last whole key
+    q_descale: Optional[torch.Tensor] = None   # fp8 q: fp32, shaped like w
+    k_descale: Optional[torch.Tensor] = None   # fp8 k: fp32, one per key row (k without D)
     meta: dict = field(default_factory=dict)
 
     TENSORS = ("q", "k", "w", "cu_seqlens_q", "cu_seqlens_k", "seqused_q", "seqused_k",
-               "block_table", "output_idx_offset", "cmp_residual_k")
+               "block_table", "output_idx_offset", "cmp_residual_k", "q_descale", "k_descale")
 
     @property
     def rows(self) -> int:
@@ -132,6 +134,27 @@ def with_dtypes(pb: Problem, qk: str = "bf16", w: str = "bf16") -> Problem:
     type; the single-operator example uses fp16 q, k and fp32 w)."""
     return pb.replace(q=pb.q.float().to(_DT[qk]), k=pb.k.float().to(_DT[qk]),
                       w=pb.w.float().to(_DT[w]), name=f"{pb.name}_{qk}_{w}")
+
+
+def quantized(pb: Problem, unit_scales: bool = False) -> Problem:
+    """The same problem with q and k as fp8 e4m3 codes plus q_descale (per row and head, shaped
+    like w) and k_descale (per key row): each q head row and each key row is divided by its own
+    scale, max|x| / 448 (the largest e4m3 value), and rounded once to e4m3. unit_scales keeps
+    every scale at 1 (integer-valued inputs are exact in e4m3)."""
+    q = pb.q.float()
+    k = pb.k.float()
+    if unit_scales:
+        qs = torch.ones(q.shape[:-1])
+        ks = torch.ones(k.shape[:-1])
+    else:
+        qs = (q.abs().amax(dim=-1) / 448.0).clamp_min(1e-12)
+        ks = (k.abs().amax(dim=-1) / 448.0).clamp_min(1e-12)
+    qc = (q / qs.unsqueeze(-1)).to(torch.float8_e4m3fn)
+    kc = (k / ks.unsqueeze(-1)).to(torch.float8_e4m3fn)
+    return pb.replace(q=qc, k=kc, q_descale=qs.reshape(pb.w.shape).contiguous(),
+                      k_descale=ks.reshape(k.shape[:-2] if k.dim() == 4 and k.shape[-2] == 1
+                                           else k.shape[:-1]).contiguous(),
+                      name=f"{pb.name}_fp8")
 
 
 def bsnd(B, S1, S2, N1, topk, mask_mode=3, seed=0, D=D_DEFAULT, integer=False, name="bsnd",

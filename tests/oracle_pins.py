@@ -332,6 +332,51 @@ def pin_pages_example_shape(orc):
         assert valid == max(0, min(32, i - 31)), f"row {r}: {valid} valid entries"
 
 
+def pin_fp8_decoding(orc):
+    """fp8 e4m3 codes decode as the OCP E4M3 format (torch's float8_e4m3fn is the reference): one
+    head of dimension 1, w = 1, one key of value 1 and unit scales, so each row's only score is
+    ReLU(q). Every code but the two NaNs is covered."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    n = len(codes)
+    q = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).reshape(1, n, 1, 1)
+    one = torch.ones(1, 1, 1, 1).to(torch.float8_e4m3fn)
+    pb = synthetic.Problem(name="fp8_decode", q=q, k=one, w=torch.ones(1, n, 1, dtype=torch.bfloat16),
+                           topk=1, batch=1, q_len=n, k_len=1, n_heads=1, head_dim=1, mask_mode=0,
+                           max_seqlen_q=n, max_seqlen_k=1, q_descale=torch.ones(1, n, 1),
+                           k_descale=torch.ones(1, 1))
+    idx, val, _ = orc.topk(pb)
+    want = np.maximum(q.reshape(-1).float().numpy(), np.float32(0))
+    assert np.array_equal(idx[:, 0], np.zeros(n, dtype=np.int32))
+    _assert_same(_bits(val[:, 0]), _bits(want), "fp8 decode")
+
+
+def pin_fp8_unit_scales_match_bf16(orc):
+    """Integer-valued q and k are exact in e4m3; with every scale 1 the fp8 problem is the bf16
+    problem, bit for bit (dense, varlen and paged keys)."""
+    for base in (synthetic.bsnd(2, 40, 70, 8, 24, 3, seed=74, integer=True),
+                 synthetic.tnd([5, 30], [40, 64], 4, 16, 3, seed=75, integer=True),
+                 synthetic.paged([90, 20], 2, 8, 32, block_size=16, seed=76, integer=True)):
+        _assert_same(orc.topk(base)[:2], orc.topk(synthetic.quantized(base, unit_scales=True))[:2],
+                     base.name)
+
+
+def pin_fp8_scales_act_as_dequantization(orc):
+    """Small integer codes times power-of-two scales are exact in fp16, so an fp8 problem with
+    per-(row, head) q scales and per-key k scales must equal, bit for bit, the fp16 problem that
+    holds the products: the scales multiply the codes, q's by row and head, k's by key row."""
+    g = torch.Generator().manual_seed(77)
+    for base in (synthetic.bsnd(2, 30, 50, 4, 20, 3, seed=78, integer=True),
+                 synthetic.paged([70, 33], 2, 4, 16, block_size=16, seed=79, integer=True)):
+        qs = 2.0 ** torch.randint(-2, 3, base.w.shape, generator=g).float()
+        ks = 2.0 ** torch.randint(-2, 3, base.k.shape[:-2] if base.k.dim() == 4 else
+                                  base.k.shape[:-1], generator=g).float()
+        fp8 = base.replace(q=base.q.float().to(torch.float8_e4m3fn),
+                           k=base.k.float().to(torch.float8_e4m3fn), q_descale=qs, k_descale=ks)
+        fp16 = base.replace(q=(base.q.float() * qs.unsqueeze(-1)).half(),
+                            k=(base.k.float() * ks.reshape(base.k.shape[:-1]).unsqueeze(-1)).half())
+        _assert_same(orc.topk(fp16)[:2], orc.topk(fp8)[:2], base.name)
+
+
 def _key_range(pb, s, e, mask_mode):
     """Keys [s, e) of every batch of a dense BSND problem, indices shifted back to global by
     output_idx_offset = s (written out here, independently of the library's shard helpers)."""

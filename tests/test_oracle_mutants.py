@@ -4,13 +4,14 @@ This shows the pins are strong enough to catch a plausible slip anywhere in the 
 after the head sum, weights dropped, top-left instead of right-down causal alignment, reversed
 tie order, -0 kept, head/row strides exchanged, block table ignored, TND keys offset by the
 query cumulative lengths, ReLU dropped, output offset dropped, wrong padding, compressed keys kept
-when their first token is visible, a wrong fp16 exponent bias, a merge that drops a list."""
+when their first token is visible, a wrong fp16 exponent bias, a merge that drops a list, fp8 keys
+without their scale."""
 import pytest
 
 import oracle_pins
 from oracle import oracle as orc_mod
 
-MUTANTS = list(range(1, 15))
+MUTANTS = list(range(1, 16))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
