@@ -53,6 +53,10 @@ WORKLOAD_TEXT = {
                    "topk=512, mask_mode=3, BSND",
     "fp16_prefill": "causal prefill in fp16: B=1, S1=S2=4096, N1=64, N2=1, D=128, topk=2048, "
                     "mask_mode=3, BSND, q,k fp16 ~N(0,1), w fp32 ~N(0,1/64)",
+    "fp8_prefill": "causal prefill, fp8: B=1, S1=S2=4096, N1=64, D=128, topk=2048, mask_mode=3, "
+                   "BSND, q and k e4m3 with per-(row, head) and per-key fp32 scales, w bf16",
+    "fp8_decode": "paged decode, fp8: B=64, S1=1, N1=64, D=128, topk=2048, mask_mode=3, PA_BSND "
+                  "block_size=64, seqused_k~U[4096,32768], q and k e4m3 with fp32 scales",
     "long_row_decode": "one decode row over a long context: B=1, S1=1, seqused_k=1048576, N1=64, "
                        "D=128, topk=2048, mask_mode=3, PA_BSND block_size=64; on N GPUs each "
                        "holds 1/N of the keys, selects in its range, then all-gather + merge",
@@ -99,17 +103,19 @@ def valid_pairs(pb) -> int:
 
 
 def key_bytes(pb) -> int:
-    """Bytes of keys the path must read once: 256 B per valid key per batch."""
+    """Bytes of keys the path must read once: one key row (256 B in 16-bit types, 128 B in fp8,
+    plus its 4-byte scale) per valid key per batch."""
+    row = pb.head_dim * pb.k.element_size() + (4 if pb.k_descale is not None else 0)
     if pb.layout_k == "PA_BSND":
-        return int(pb.seqused_k.sum()) * pb.head_dim * 2
-    return pb.k.numel() * 2
+        return int(pb.seqused_k.sum()) * row
+    return pb.k.numel() // pb.head_dim * row
 
 
 def score_kernel_bytes(pb, pairs) -> int:
     """Algorithmic DRAM bytes of one score-kernel launch: each valid key once (256 B), q and w
     of every query row, the block table rows in use, and the fp32 score of every valid pair."""
     q = pb.q.numel() * pb.q.element_size()
-    w = pb.w.numel() * pb.w.element_size()
+    w = pb.w.numel() * pb.w.element_size() * (2 if pb.q_descale is not None else 1)
     table = 0
     if pb.layout_k == "PA_BSND":
         table = sum(-(-int(L) // pb.block_size) for L in pb.seqused_k.tolist()) * 4
@@ -530,7 +536,8 @@ def main():
                "serial_ms_per_step": serial_ms}
 
     peaks = load_peaks()
-    dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[pb_cpu.q.dtype]
+    dtype = {torch.bfloat16: "bf16", torch.float16: "fp16",
+             torch.float8_e4m3fn: "fp8_e4m3"}[pb_cpu.q.dtype]
     pairs = valid_pairs(pb_cpu)
     flops = 2.0 * pairs * pb.n_heads * pb.head_dim
     sc = statistics.mean(score_ms)
@@ -546,13 +553,16 @@ def main():
                     "peak_source": f"{peaks['source']} HBM copy"}
     else:
         achieved = flops / (sc / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
+        # fp8 contractions run at twice the bf16 rate (nominal dense 4.5 vs 2.25 PFLOP/s)
+        peak = peaks["bf16_tflops"] * (2.0 if dtype == "fp8_e4m3" else 1.0)
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": score_traffic(a.config),
                     "algorithmic_bytes": score_kernel_bytes(pb_cpu, pairs),
                     "kernel": "score kernel (q.k contraction + ReLU/weight/head-sum epilogue)",
                     "peak_source": f"{peaks['source']} bf16 burst"
-                                   + (" (fp16 runs at the bf16 rate)" if dtype == "fp16" else "")}
+                                   + (" (fp16 runs at the bf16 rate)" if dtype == "fp16" else "")
+                                   + (" x 2, the nominal fp8/bf16 ratio" if dtype == "fp8_e4m3"
+                                      else "")}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

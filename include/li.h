@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define LI_ABI_VERSION 3
+#define LI_ABI_VERSION 4
 
 typedef enum li_layout {
     LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
@@ -64,7 +64,8 @@ typedef enum li_status {
 typedef enum li_dtype {
     LI_DTYPE_BF16 = 0,
     LI_DTYPE_FP16 = 1,
-    LI_DTYPE_FP32 = 2                   /* w only                                              */
+    LI_DTYPE_FP32 = 2,                  /* w only                                              */
+    LI_DTYPE_FP8_E4M3 = 3               /* q and k only, with q_descale and k_descale          */
 } li_dtype;
 
 /* Device status word bits, as reported through li_check_status(). */
@@ -72,8 +73,12 @@ typedef enum li_dtype {
 #define LI_DEVERR_LENGTHS   0x2u   /* cu_seqlens not monotone, or a length above its maximum  */
 #define LI_DEVERR_TABLE     0x4u   /* a block_table entry in use is outside [0, num_blocks)    */
 #define LI_DEVERR_OFFSET    0x8u   /* output_idx_offset < 0, or index + offset > INT32_MAX     */
-#define LI_DEVERR_MERGE_ORDER 0x10u /* li_merge_topk: an input row out of order, or a valid entry
+#define LI_DEVERR_METADATA  0x10u   /* the metadata passed was built for other arguments        */
+#define LI_DEVERR_INTERNAL  0x20u   /* the score kernel's shared memory came misaligned         */
+#define LI_DEVERR_MERGE_ORDER 0x40u /* li_merge_topk: an input row out of order, or a valid entry
                                        after padding                                          */
+#define LI_DEVERR_DESCALE   0x80u   /* fp8 q/k: a q_descale or k_descale in use is not a positive
+                                       finite number                                          */
 
 /*
  * Arguments of one indexer call. Mirrors the pages' prototypes (lightning_indexer, "Prototype":
@@ -124,6 +129,15 @@ typedef struct li_args {
      * [0, cmp_ratio) set LI_DEVERR_LENGTHS. */
     const int32_t *cmp_residual_k;      /* [B] int32, or NULL                                   */
     int32_t cmp_ratio;                  /* original tokens per key; 0 or 1 = not compressed     */
+    /* Quantized q and k (aclnnLightningIndexerV2, parameter dimensions: q_descale and k_descale
+     * are named with q, k and w and nothing more is said). The reading implemented: with
+     * dtype_qk = LI_DTYPE_FP8_E4M3, q and k hold OCP E4M3 codes (1 byte per element, rows of
+     * 128 bytes, 16-byte aligned) and the values they stand for are code x q_descale[row, head]
+     * and code x k_descale[key row]. Both arrays are fp32, 4-byte aligned, required with fp8
+     * and NULL otherwise. Scales in use must be positive and finite (LI_DEVERR_DESCALE). */
+    const float *q_descale;             /* [rows x num_heads_q], laid out like w                */
+    const float *k_descale;             /* one per key row, laid out like k without D: BSND
+                                           (B, S2), TND (T2), PA_BSND (num_blocks, block_size)  */
 } li_args;
 
 /*

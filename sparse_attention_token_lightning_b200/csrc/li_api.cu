@@ -86,8 +86,14 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     if (a->layout_k != LI_LAYOUT_BSND && a->layout_k != LI_LAYOUT_TND &&
         a->layout_k != LI_LAYOUT_PA_BSND)
         return fail(LI_ERR_INVALID_ARG, "layout_k=%d, must be BSND, TND or PA_BSND", a->layout_k);
-    if (a->dtype_qk != LI_DTYPE_BF16 && a->dtype_qk != LI_DTYPE_FP16)
-        return fail(LI_ERR_INVALID_ARG, "dtype_qk=%d, must be bf16 or fp16", a->dtype_qk);
+    if (a->dtype_qk != LI_DTYPE_BF16 && a->dtype_qk != LI_DTYPE_FP16 &&
+        a->dtype_qk != LI_DTYPE_FP8_E4M3)
+        return fail(LI_ERR_INVALID_ARG, "dtype_qk=%d, must be bf16, fp16 or fp8 e4m3", a->dtype_qk);
+    if ((a->dtype_qk == LI_DTYPE_FP8_E4M3) != (a->q_descale != nullptr) ||
+        (a->dtype_qk == LI_DTYPE_FP8_E4M3) != (a->k_descale != nullptr))
+        return fail(LI_ERR_INVALID_ARG, "q_descale and k_descale go with fp8 q/k, and only with it");
+    if (!aligned(a->q_descale, 4) || !aligned(a->k_descale, 4))
+        return fail(LI_ERR_INVALID_ARG, "q_descale and k_descale must be 4-byte aligned");
     if (a->dtype_w != LI_DTYPE_BF16 && a->dtype_w != LI_DTYPE_FP16 && a->dtype_w != LI_DTYPE_FP32)
         return fail(LI_ERR_INVALID_ARG, "dtype_w=%d, must be bf16, fp16 or fp32", a->dtype_w);
     if (a->return_value != 0 && a->return_value != 1)
@@ -344,13 +350,16 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
         meta = inline_meta;
     }
     bool launched = false;
+    li::Quant quant;
+    quant.q_descale = args->q_descale;
+    quant.k_descale = args->k_descale;
     stage_mark(2, cs);
     if (!use_simple_kernel()) {
-        e = li::launch_score_tc(p, s, meta, ws, scores, ld, cs, &launched);
+        e = li::launch_score_tc(p, quant, s, meta, ws, scores, ld, cs, &launched);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
     }
     if (!launched) {
-        e = li::launch_score_simple(p, s, meta, ws, scores, ld, cs);
+        e = li::launch_score_simple(p, quant, s, meta, ws, scores, ld, cs);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
     }
     stage_mark(3, cs);

@@ -302,6 +302,19 @@ __device__ inline const uint16_t *key_ptr(const Problem &p, const BatchInfo &bi,
     return p.k + ((int64_t)bi.k_row0 + j) * kHeadDim;
 }
 
+// Row of the key cache holding key j of batch b (-1: block-table entry out of range).
+__device__ inline int64_t key_row(const Problem &p, const BatchInfo &bi, int32_t b, int32_t j) {
+    if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        int32_t blk = p.block_table[(int64_t)b * p.bt_stride + j / p.block_size];
+        if (blk < 0 || blk >= p.num_blocks) return -1;
+        return (int64_t)blk * p.block_size + j % p.block_size;
+    }
+    return (int64_t)bi.k_row0 + j;
+}
+
+// A scale of fp8 q/k is usable when it is a positive finite number.
+__device__ inline bool good_scale(float x) { return x > 0.0f && x < __int_as_float(0x7f800000); }
+
 __device__ inline float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ inline float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
@@ -330,15 +343,24 @@ __device__ inline void set_status(uint32_t *status, uint32_t bits) {
 // Sets the message li_last_error_string() returns on this host thread.
 void set_last_error(const char *msg);
 
+// fp8 q/k scales (li_args q_descale / k_descale), null for 16-bit q/k. Kept out of Problem so
+// that the kernels' parameter blocks keep their layout.
+struct Quant {
+    const float *q_descale = nullptr;     // [rows * N1], laid out like w
+    const float *k_descale = nullptr;     // one per key row
+};
+
 // ---- launchers implemented in the .cu files --------------------------------------------------
 cudaError_t launch_metadata(const Problem &p, const Schedule &s, void *meta, cudaStream_t st);
-cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
-                                WsHeader *ws, float *scores, int64_t ld, cudaStream_t st);
+cudaError_t launch_score_simple(const Problem &p, const Quant &qd, const Schedule &s,
+                                const void *meta, WsHeader *ws, float *scores, int64_t ld,
+                                cudaStream_t st);
 // Tensor-core score kernel: whether the problem fits it, and its launcher (*launched = false
 // when it does not, leaving the step to launch_score_simple).
 bool score_tc_eligible(const Problem &p, const Schedule &s);
-cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
-                            float *scores, int64_t ld, cudaStream_t st, bool *launched);
+cudaError_t launch_score_tc(const Problem &p, const Quant &qd, const Schedule &s, const void *meta,
+                            WsHeader *ws, float *scores, int64_t ld, cudaStream_t st,
+                            bool *launched);
 // (meta == nullptr in the score and select launchers selects the dense closed-form schedule)
 cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
                           const float *scores, int64_t ld, int32_t *out_idx, float *out_val,

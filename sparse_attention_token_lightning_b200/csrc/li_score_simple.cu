@@ -7,6 +7,8 @@
 // workspace (custom_pypto.npu_lightning_indexer_pto, function description formula;
 // lightning_indexer, "Function" steps 1-3). Keys are fetched per layout: BSND / TND rows, or the
 // paged cache through the block table (custom_pypto.npu_lightning_indexer_pto, block_table).
+#include <cuda_fp8.h>
+
 #include "li_internal.cuh"
 
 namespace li {
@@ -21,7 +23,14 @@ struct Params {
     float *scores;
     int64_t ld;
     uint32_t signature;
+    Quant qd;
 };
+
+__device__ inline float fp8_to_f32(uint8_t c) {
+    __nv_fp8_e4m3 x;
+    x.__x = c;
+    return (float)x;
+}
 
 __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
     const Problem &p = sp.p;
@@ -37,6 +46,7 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
     }
     const int H = p.n_heads;
     const bool fp16 = p.dtype_qk == LI_DTYPE_FP16;
+    const bool fp8 = p.dtype_qk == LI_DTYPE_FP8_E4M3;
     if (blockIdx.x == 0) check_batch_keys(p, view, &sp.ws->status, threadIdx.x, kThreads);
 
     __shared__ float qs[kMaxHeads][kHeadDim];
@@ -55,7 +65,15 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
             __syncthreads();   // previous row's readers are done with qs / ws_
             for (int e = threadIdx.x; e < H * kHeadDim; e += kThreads) {
                 const int h = e / kHeadDim, d = e % kHeadDim;
-                qs[h][d] = half16_to_f32(p.q[(row * H + h) * kHeadDim + d], fp16);
+                const int64_t qi = (row * H + h) * kHeadDim + d;
+                if (fp8) {
+                    // [reading] the code times its row-and-head scale
+                    const float sc = sp.qd.q_descale[row * H + h];
+                    if (!good_scale(sc)) err |= LI_DEVERR_DESCALE;
+                    qs[h][d] = fp8_to_f32(reinterpret_cast<const uint8_t *>(p.q)[qi]) * sc;
+                } else {
+                    qs[h][d] = half16_to_f32(p.q[qi], fp16);
+                }
             }
             for (int h = threadIdx.x; h < H; h += kThreads)
                 ws_[h] = weight_f32(p, row * H + h);
@@ -65,6 +83,20 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
                 float I = 0.0f;
                 if (kp == nullptr) {
                     err |= LI_DEVERR_TABLE;
+                } else if (fp8) {
+                    const int64_t kr = key_row(p, bi, it.b, j);
+                    const uint8_t *k8 = reinterpret_cast<const uint8_t *>(p.k) + kr * kHeadDim;
+                    const float ks = sp.qd.k_descale[kr];
+                    if (!good_scale(ks)) err |= LI_DEVERR_DESCALE;
+                    float kv[kHeadDim];
+#pragma unroll
+                    for (int d = 0; d < kHeadDim; ++d) kv[d] = fp8_to_f32(k8[d]) * ks;
+                    for (int h = 0; h < H; ++h) {
+                        float s = 0.0f;
+#pragma unroll
+                        for (int d = 0; d < kHeadDim; ++d) s = fmaf(qs[h][d], kv[d], s);
+                        I = fmaf(ws_[h], fmaxf(s, 0.0f), I);
+                    }
                 } else {
                     uint32_t kr[kHeadDim / 2];
                     const uint4 *k4 = reinterpret_cast<const uint4 *>(kp);
@@ -93,9 +125,10 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
 
 }  // namespace
 
-cudaError_t launch_score_simple(const Problem &p, const Schedule &s, const void *meta,
-                                WsHeader *ws, float *scores, int64_t ld, cudaStream_t st) {
-    Params sp{p, make_view(p, s, meta), ws, scores, ld, problem_signature(p, s.tq, s.kc)};
+cudaError_t launch_score_simple(const Problem &p, const Quant &qd, const Schedule &s,
+                                const void *meta, WsHeader *ws, float *scores, int64_t ld,
+                                cudaStream_t st) {
+    Params sp{p, make_view(p, s, meta), ws, scores, ld, problem_signature(p, s.tq, s.kc), qd};
     int grid = s.max_items < 148 * 8 ? s.max_items : 148 * 8;
     if (grid < 1) grid = 1;
     score_simple_kernel<<<grid, kThreads, 0, st>>>(sp);

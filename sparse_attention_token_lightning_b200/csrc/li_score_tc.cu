@@ -87,6 +87,7 @@ struct TcParams {
     uint32_t acc_stride;  // TMEM columns per accumulator (power of two >= N)
     uint32_t q_half;      // bytes of one 64-wide half of a Q buffer (N x 128)
     uint32_t k_off;       // start of the K ring (after the two Q buffers)
+    Quant qd;             // fp8 q/k: the scales (null otherwise)
 };
 
 // ---- PTX wrappers --------------------------------------------------------------------------
@@ -158,6 +159,17 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// fp8 (E4M3 x E4M3, fp32 accumulate) MMA, K = 32, with a compile-time accumulate flag.
+template <bool kAccumulate>
+__device__ __forceinline__ void umma_f8_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "n"(kAccumulate ? 1 : 0)
+        : "memory");
+}
+
 // MMA with a compile-time accumulate flag (no predicate set-up on the issue path).
 template <bool kAccumulate>
 __device__ __forceinline__ void umma_bf16_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -276,7 +288,7 @@ __device__ __forceinline__ int32_t piece_row(const TcParams &P, int32_t b, int32
 // first 32 key pieces) in the slot ring ahead of the producer. The next item's loads go to
 // registers right after a slot is filled, so they complete while the warp waits for the next
 // free slot, and a ticket is taken only when the ring has moved on by one item.
-template <int kW>
+template <int kW, bool kQ8>
 __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
                           volatile int *abort_flag, int n_items) {
     constexpr int kWPerLane = kNmax / 32;
@@ -286,6 +298,7 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
     WorkItem cur{};
     float wv[kWPerLane];
     int32_t tv = -1;
+    bool scale_err = false;
     // takes tickets up to the next item with a non-empty window (the dense closed forms can yield
     // empty ones) and loads its weights (lane l holds entries l, l + 32, ...) and the cache row
     // of its key piece l; false at the end of the list
@@ -304,7 +317,13 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
         for (int i = 0; i < kWPerLane; ++i) {
             const int e = lane + 32 * i;
             // even columns are staged halved: the epilogue takes their ReLU as x + |x|
-            const float we = e < nw ? weight_f32<kW>(P.p, wbase + e) : 0.0f;
+            float we = e < nw ? weight_f32<kW>(P.p, wbase + e) : 0.0f;
+            if constexpr (kQ8) {
+                // a positive q scale passes through the ReLU: w ReLU(s q) = (w s) ReLU(q)
+                const float sc = e < nw ? P.qd.q_descale[wbase + e] : 1.0f;
+                if (!good_scale(sc)) scale_err = true;
+                we *= sc;
+            }
             wv[i] = (e & 1) ? we : 0.5f * we;
         }
         if (P.piece_rows) tv = piece_row(P, cur.b, cur.j0, cur.j1, lane);
@@ -332,12 +351,20 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
         have = fetch();
     }
     if (!ok) *abort_flag = 1;
+    if constexpr (kQ8) {
+        if (__any_sync(0xffffffffu, scale_err) && lane == 0) set_status(&P.ws->status, LI_DEVERR_DESCALE);
+    }
 }
 
 // TMA producer warp: per staged item, the Q tile (double buffered) and the K tiles of its key
 // range through the ring; paged keys block by block through the block table.
+// kQ8: fp8 q/k, whose 128-element rows are one 128-byte box (two 64-element halves for 16-bit
+// types), so a Q tile and a K stage are half as many bytes and loads.
+template <bool kQ8>
 __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
                          uint8_t *smem, const Bars &bars, volatile int *abort_flag) {
+    constexpr uint32_t kStage = kQ8 ? kKHalfBytes : kKStageBytes;
+    constexpr uint32_t kRowBytes = kQ8 ? 128u : 256u;
     const int lane = threadIdx.x & 31;
     const uint32_t sbase = smem_u32(smem);
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
@@ -365,9 +392,14 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
         if (lane == 0) {
             const uint32_t qdst = sbase + qb * 2u * P.q_half;
             const int32_t y = row0 * N1;
-            mbar_arrive_expect_tx(bars.q_full(qb), 2u * P.q_half);
-            tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
-            tma_load_2d(qdst + P.q_half, tmq, bars.q_full(qb), 64, y);
+            if constexpr (kQ8) {
+                mbar_arrive_expect_tx(bars.q_full(qb), P.q_half);
+                tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
+            } else {
+                mbar_arrive_expect_tx(bars.q_full(qb), 2u * P.q_half);
+                tma_load_2d(qdst, tmq, bars.q_full(qb), 0, y);
+                tma_load_2d(qdst + P.q_half, tmq, bars.q_full(qb), 64, y);
+            }
         }
         // K tiles of the item's key range. Paged keys: lane l holds the cache row of piece
         // pbase + l (the first 32 staged by the scheduler, later ones refilled 32 at a time) and
@@ -379,12 +411,13 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             const int st = kr.idx;
             if (!mbar_wait(bars.k_empty(st), kr.phase ^ 1u, abort_flag)) { ok = false; break; }
             const int32_t jt = j0 + tile * kKeyTile;
-            const uint32_t kdst = sbase + P.k_off + st * kKStageBytes;
+            const uint32_t kdst = sbase + P.k_off + st * kStage;
             if (pr == 0) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(bars.k_full(st), kKStageBytes);
+                    mbar_arrive_expect_tx(bars.k_full(st), kStage);
                     tma_load_2d(kdst, tmk, bars.k_full(st), 0, k_row0 + jt);
-                    tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, k_row0 + jt);
+                    if constexpr (!kQ8)
+                        tma_load_2d(kdst + kKHalfBytes, tmk, bars.k_full(st), 64, k_row0 + jt);
                 }
             } else {
                 const int32_t p0 = tile * pieces;
@@ -397,12 +430,13 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
                 const uint32_t loads = __ballot_sync(0xffffffffu, mine);
                 if (__ballot_sync(0xffffffffu, lane < pieces && row == -2)) err |= LI_DEVERR_TABLE;
                 if (lane == 0)
-                    mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)__popc(loads) * pr * 256u);
+                    mbar_arrive_expect_tx(bars.k_full(st), (uint32_t)__popc(loads) * pr * kRowBytes);
                 __syncwarp();
                 if (mine) {
                     const uint32_t off = (uint32_t)lane * pr * 128u;
                     tma_load_2d(kdst + off, tmk, bars.k_full(st), 0, row);
-                    tma_load_2d(kdst + kKHalfBytes + off, tmk, bars.k_full(st), 64, row);
+                    if constexpr (!kQ8)
+                        tma_load_2d(kdst + kKHalfBytes + off, tmk, bars.k_full(st), 64, row);
                 }
             }
             __syncwarp();
@@ -414,8 +448,10 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
     if (lane == 0 && err) set_status(&P.ws->status, err);
 }
 
+template <bool kQ8>
 __device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
                            volatile int *abort_flag, uint32_t tmem_base) {
+    constexpr uint32_t kStage = kQ8 ? kKHalfBytes : kKStageBytes;
     const uint32_t sbase = smem_u32(smem);
     Slot *slots = reinterpret_cast<Slot *>(smem + kSlotOff);
     RingPos kr, ar;
@@ -442,14 +478,22 @@ __device__ void mma_issuer(const TcParams &P, uint8_t *smem, const Bars &bars,
             tc_fence_after();
             // descriptors advance by the byte offset / 16 in their address field (no carry:
             // shared addresses stay below 2^18 bytes)
-            const uint64_t a0 = sw128_desc(sbase + P.k_off + st * kKStageBytes);
+            const uint64_t a0 = sw128_desc(sbase + P.k_off + st * kStage);
             const uint32_t d = tmem_base + ab * P.acc_stride;
-            umma_bf16_c<false>(d, a0, b0, P.idesc);
+            if constexpr (kQ8) {
+                // one 128-byte row holds all 128 elements: four K = 32 steps of 32 bytes
+                umma_f8_c<false>(d, a0, b0, P.idesc);
 #pragma unroll
-            for (int kk = 1; kk < kHeadDim / 16; ++kk) {
-                const uint64_t a_off = ((kk >> 2) * kKHalfBytes + (kk & 3) * 32u) >> 4;
-                const uint64_t b_off = ((uint64_t)(kk >> 2) * b_half16) + (uint64_t)((kk & 3) * 2);
-                umma_bf16_c<true>(d, a0 + a_off, b0 + b_off, P.idesc);
+                for (int kk = 1; kk < kHeadDim / 32; ++kk)
+                    umma_f8_c<true>(d, a0 + 2 * kk, b0 + 2 * kk, P.idesc);
+            } else {
+                umma_bf16_c<false>(d, a0, b0, P.idesc);
+#pragma unroll
+                for (int kk = 1; kk < kHeadDim / 16; ++kk) {
+                    const uint64_t a_off = ((kk >> 2) * kKHalfBytes + (kk & 3) * 32u) >> 4;
+                    const uint64_t b_off = ((uint64_t)(kk >> 2) * b_half16) + (uint64_t)((kk & 3) * 2);
+                    umma_bf16_c<true>(d, a0 + a_off, b0 + b_off, P.idesc);
+                }
             }
             umma_commit(bars.k_empty(st));
             umma_commit(bars.acc_full(ab));
@@ -498,6 +542,9 @@ __device__ __forceinline__ float head_sum(uint32_t acc, const float *w, int t, i
     return a;
 }
 
+// kQ8: fp8 q/k. The q scales were folded into the staged weights; a key's positive scale passes
+// through the ReLU of every head, so each key's sum is multiplied by its k scale.
+template <bool kQ8>
 __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                          volatile int *abort_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -509,6 +556,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
     RingPos ar;
     bool ok = true;
+    bool scale_err = false;
     for (int it = 0; ok; ++it) {
         const int sl = it % kSlots;
         if (!mbar_wait(bars.sl_full(sl), (it / kSlots) & 1, abort_flag)) { ok = false; break; }
@@ -527,21 +575,65 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
         const bool one_row = nq <= kEpiGroups;
         const int32_t hi1 = one_row && group < nq ? min(window_hi(mask_mode, q0 + group, L1u, L2), j1) : 0;
         float *const out1 = P.scores + (int64_t)(row0 + (one_row && group < nq ? group : 0)) * P.ld;
+        // fp8: this thread's key scale of tile t (-1 row: none), loaded kKdAhead tiles early and
+        // carried in registers so the load is in flight while earlier tiles are summed; paged
+        // rows come from the rows the scheduler staged
+        constexpr int kKdAhead = 3;
+        auto kd_load = [&](int32_t t, bool &has) -> float {
+            has = false;
+            const int32_t jj = j0 + t * kKeyTile + 32 * quarter + lane;
+            if (t >= nt || jj >= j1) return 0.0f;
+            int64_t kr = (int64_t)S.k_row0 + jj;
+            if (P.piece_rows) {
+                const int32_t pc = (jj - j0) / P.piece_rows;
+                int32_t prow = pc < 32 ? S.prow[pc] : -1;
+                if (pc >= 32) {
+                    const int32_t bs = P.p.block_size;
+                    const int32_t blk = P.p.block_table[(int64_t)S.b * P.p.bt_stride + jj / bs];
+                    prow = blk >= 0 && blk < P.p.num_blocks ? blk * bs + (jj - jj % P.piece_rows) % bs
+                                                            : -2;
+                }
+                if (prow < 0) return 0.0f;
+                kr = (int64_t)prow + (jj - j0) % P.piece_rows;
+            }
+            has = true;
+            return __ldg(P.qd.k_descale + kr);
+        };
+        float kq0 = 0.f, kq1 = 0.f, kq2 = 0.f;
+        bool hq0 = false, hq1 = false, hq2 = false;
+        if constexpr (kQ8) {
+            static_assert(kKdAhead == 3, "three scales in flight");
+            kq0 = kd_load(0, hq0);
+            kq1 = kd_load(1, hq1);
+            kq2 = kd_load(2, hq2);
+        }
         for (int32_t tile = 0; tile < nt; ++tile, ar.next(P.n_acc)) {
             const int ab = ar.idx;
-            if (!mbar_wait(bars.acc_full(ab), ar.phase, abort_flag)) { ok = false; break; }
-            tc_fence_after();
             const int32_t jt = j0 + tile * kKeyTile;
             const int32_t j = jt + 32 * quarter + lane;
+            float kd = 1.0f;
+            if constexpr (kQ8) {
+                bool hn = false;
+                const float kn = kd_load(tile + kKdAhead, hn);
+                kd = kq0;
+                if (hq0 && !good_scale(kd)) scale_err = true;
+                kq0 = kq1; hq0 = hq1;
+                kq1 = kq2; hq1 = hq2;
+                kq2 = kn; hq2 = hn;
+            }
+            if (!mbar_wait(bars.acc_full(ab), ar.phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
             const uint32_t acc = tmem_base + lane_addr + ab * P.acc_stride;
             if (one_row) {
                 if (N1 == 64 && jt < hi1) {
                     float v[64];
                     tmem_ld64(acc + group * 64, v);
-                    const float I = head_sum64(v, S.w + group * 64);
+                    float I = head_sum64(v, S.w + group * 64);
+                    if constexpr (kQ8) I *= kd;
                     if (j < hi1) out1[j] = I;
                 } else if (jt < hi1) {
-                    const float I = head_sum(acc, S.w, group, N1);
+                    float I = head_sum(acc, S.w, group, N1);
+                    if constexpr (kQ8) I *= kd;
                     if (j < hi1) out1[j] = I;
                 }
             } else {
@@ -556,6 +648,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                     } else {
                         I = head_sum(acc, S.w, t, N1);
                     }
+                    if constexpr (kQ8) I *= kd;
                     if (j < hi) P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
                 }
             }
@@ -567,10 +660,14 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
         if (lane == 0) mbar_arrive(bars.sl_empty(sl));
     }
     if (!ok) *abort_flag = 1;
+    if constexpr (kQ8) {
+        if (__any_sync(0xffffffffu, scale_err) && lane == 0) set_status(&P.ws->status, LI_DEVERR_DESCALE);
+    }
 }
 
-// kW: li_dtype of w (the weights are staged as fp32; q and k go to the MMA as they are)
-template <int kW>
+// kW: li_dtype of w (the weights are staged as fp32; q and k go to the MMA as they are);
+// kQ8: fp8 q/k with scales.
+template <int kW, bool kQ8>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const TcParams P) {
@@ -628,15 +725,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
+        producer<kQ8>(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
     } else if (warp == kSchedWarp) {
         if (blockIdx.x == 0) check_batch_keys(P.p, P.view, &P.ws->status, lane, 32);
-        scheduler<kW>(P, smem, bars, abort_flag, n_items);
+        scheduler<kW, kQ8>(P, smem, bars, abort_flag, n_items);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(P, smem, bars, abort_flag, tmem_base);
+        if (lane == 0) mma_issuer<kQ8>(P, smem, bars, abort_flag, tmem_base);
         __syncwarp();
     } else {
-        epilogue(P, smem, bars, abort_flag, tmem_base);
+        epilogue<kQ8>(P, smem, bars, abort_flag, tmem_base);
     }
 
     tc_fence_before();
@@ -664,15 +761,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows, bool fp16) {
+// Rows of 128 elements; 16-bit types are loaded as two 64-element (128-byte) boxes, fp8 as one.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows, int dtype) {
     auto fn = encode_fn();
     if (!fn || rows == 0) return false;
+    const bool b8 = dtype == LI_DTYPE_FP8_E4M3;
     cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * (b8 ? 1 : 2)};
+    cuuint32_t box[2] = {b8 ? 128u : 64u, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                    const_cast<void *>(ptr), dims, strides,
+    const CUtensorMapDataType t = b8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                  : dtype == LI_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(m, t, 2, const_cast<void *>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -708,8 +809,9 @@ bool score_tc_eligible(const Problem &p, const Schedule &s) {
 
 // Launches the tensor-core kernel when the problem fits it; *launched = false leaves the call
 // to the CUDA-core kernel (see score_tc_eligible, and a tensor map the driver refuses).
-cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *meta, WsHeader *ws,
-                            float *scores, int64_t ld, cudaStream_t st, bool *launched) {
+cudaError_t launch_score_tc(const Problem &p, const Quant &qd, const Schedule &s, const void *meta,
+                            WsHeader *ws, float *scores, int64_t ld, cudaStream_t st,
+                            bool *launched) {
     *launched = false;
     if (!score_tc_eligible(p, s)) return cudaSuccess;
     TcParams P{};
@@ -722,8 +824,11 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     P.tq = s.tq;
     P.N = (s.tq * p.n_heads + 15) / 16 * 16;
     if (P.N > kNmax || P.N < 16) return cudaSuccess;
-    // D fp32; A and B both bf16 (format 1) or both fp16 (format 0); N, M
-    const uint32_t ab_format = p.dtype_qk == LI_DTYPE_FP16 ? 0u : 1u;
+    const bool q8 = p.dtype_qk == LI_DTYPE_FP8_E4M3;
+    P.qd = qd;
+    // D fp32; A and B both bf16 (format 1) or both fp16 (format 0) for kind::f16, both E4M3
+    // (format 0) for kind::f8f6f4; N, M
+    const uint32_t ab_format = p.dtype_qk == LI_DTYPE_BF16 ? 1u : 0u;
     P.idesc = (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((uint32_t)(P.N >> 3) << 17) |
               ((uint32_t)(128 >> 4) << 24);
     P.q_half = (uint32_t)P.N * 128u;               // N is a multiple of 16: 1 KB aligned halves
@@ -732,7 +837,7 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     while (P.acc_stride < (uint32_t)P.N) P.acc_stride <<= 1;
     P.n_acc = (int)(kTmemCols / P.acc_stride);
     if (P.n_acc > kMaxAcc) P.n_acc = kMaxAcc;
-    P.stages = (int)((kTailOff - P.k_off) / kKStageBytes);
+    P.stages = (int)((kTailOff - P.k_off) / (q8 ? kKHalfBytes : kKStageBytes));
     if (P.stages > kMaxStages) P.stages = kMaxStages;
     if (P.stages < 2) return cudaSuccess;
     uint64_t k_rows = 0;
@@ -753,14 +858,16 @@ cudaError_t launch_score_tc(const Problem &p, const Schedule &s, const void *met
     const uint64_t q_rows = (uint64_t)(p.layout_q == LI_LAYOUT_TND ? p.q_len : p.batch * p.q_len) *
                             p.n_heads;
     CUtensorMap mq, mk;
-    const bool fp16 = p.dtype_qk == LI_DTYPE_FP16;
-    if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N, fp16)) return cudaSuccess;
+    if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N, p.dtype_qk)) return cudaSuccess;
     if (!make_map(&mk, p.k, k_rows, P.piece_rows ? (uint32_t)P.piece_rows : (uint32_t)kKeyTile,
-                  fp16))
+                  p.dtype_qk))
         return cudaSuccess;
-    auto kern = p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32>
-                : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16>
-                                             : score_tc_kernel<LI_DTYPE_BF16>;
+    auto kern = q8 ? (p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32, true>
+                      : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16, true>
+                                                   : score_tc_kernel<LI_DTYPE_BF16, true>)
+                   : (p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32, false>
+                      : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16, false>
+                                                   : score_tc_kernel<LI_DTYPE_BF16, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;

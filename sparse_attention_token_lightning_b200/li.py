@@ -44,10 +44,12 @@ class LiArgs(ctypes.Structure):
         ("dtype_qk", ctypes.c_int32), ("dtype_w", ctypes.c_int32),
         ("return_value", ctypes.c_int32),
         ("cmp_residual_k", ctypes.c_void_p), ("cmp_ratio", ctypes.c_int32),
+        ("q_descale", ctypes.c_void_p), ("k_descale", ctypes.c_void_p),
     ]
 
 
-DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}   # li_dtype
+DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2,
+          torch.float8_e4m3fn: 3}                                   # li_dtype
 
 
 class LiPlanInfo(ctypes.Structure):
@@ -174,6 +176,8 @@ def make_args(pb, return_value: int = 1) -> LiArgs:
     a.return_value = int(return_value)
     a.cmp_residual_k = _ptr(getattr(pb, "cmp_residual_k", None))
     a.cmp_ratio = int(getattr(pb, "cmp_ratio", 1) or 1)
+    a.q_descale = _ptr(getattr(pb, "q_descale", None))
+    a.k_descale = _ptr(getattr(pb, "k_descale", None))
     return a
 
 

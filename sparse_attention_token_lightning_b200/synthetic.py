@@ -288,6 +288,10 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
         # fp32 w
         return with_dtypes(bsnd(1, 4096, 4096, 64, 2048, 3, seed, integer=integer, name=name),
                            "fp16", "fp32").replace(name=name)
+    if name == "fp8_prefill":
+        return quantized(config("causal_prefill", seed, integer)).replace(name=name)
+    if name == "fp8_decode":
+        return quantized(config("paged_decode", seed, integer)).replace(name=name)
     if name == "long_row_decode":
         # one decode row over 2^20 keys (256 MB of keys); split by key range across GPUs
         return paged([1 << 20], 1, 64, 2048, block_size=64, mask_mode=3, seed=seed + 1,
@@ -300,4 +304,4 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
 
 
 CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192",
-           "cmp_prefill", "fp16_prefill", "long_row_decode")
+           "cmp_prefill", "fp16_prefill", "long_row_decode", "fp8_prefill", "fp8_decode")

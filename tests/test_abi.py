@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert li.li_abi_version() == 3
+    assert li.li_abi_version() == 4
 
 
 @pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
@@ -96,7 +96,7 @@ def test_valid_args_size_the_workspace(L):
 @pytest.mark.parametrize("kw,status", [
     (dict(num_heads_q=0), 1), (dict(num_heads_q=65), 1), (dict(num_heads_k=2), 1),
     (dict(head_dim=64), 1), (dict(topk=0), 1), (dict(topk=8193), 1), (dict(mask_mode=1), 1),
-    (dict(layout_q=2), 1), (dict(layout_k=5), 1), (dict(dtype_qk=2), 1), (dict(dtype_w=3), 1),
+    (dict(layout_q=2), 1), (dict(layout_k=5), 1), (dict(dtype_qk=2), 1), (dict(dtype_qk=4), 1), (dict(dtype_w=3), 1),
     (dict(dtype_qk=-1), 1), (dict(dtype_w=2, w=0x30002), 1), (dict(w=0x30001), 1), (dict(q=None), 1),
     (dict(q=0x10008), 1), (dict(layout_q=1), 1), (dict(layout_k=1), 1), (dict(layout_k=2), 1),
     (dict(layout_k=2, seqused_k=0x40000, block_table=0x50000, block_table_stride=4,
@@ -118,6 +118,15 @@ def test_invalid_args_rejected_on_host(L, kw, status):
     st, _ = _ws_status(_args(**kw))
     assert st == status, li.li_last_error_string()
     assert li.li_last_error_string()
+
+
+def test_fp8_requires_both_scales(L):
+    fp8 = dict(dtype_qk=3, q_descale=0x70000, k_descale=0x74000)
+    assert _ws_status(_args(**fp8))[0] == 0
+    assert _ws_status(_args(dtype_qk=3))[0] == 1                        # no scales
+    assert _ws_status(_args(dtype_qk=3, q_descale=0x70000))[0] == 1     # one scale
+    assert _ws_status(_args(q_descale=0x70000, k_descale=0x74000))[0] == 1   # scales without fp8
+    assert _ws_status(_args(**dict(fp8, k_descale=0x74002)))[0] == 1    # misaligned
 
 
 @pytest.mark.parametrize("qk,w", [(0, 0), (0, 1), (0, 2), (1, 0), (1, 1), (1, 2)])

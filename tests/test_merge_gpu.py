@@ -58,7 +58,7 @@ def test_merge_reports_an_unsorted_list():
     val[1, 2, [3, 4]] = val[1, 2, [4, 3]]
     with pytest.raises(li.LiError) as e:
         li.merge_topk(torch.from_numpy(idx).cuda(), torch.from_numpy(val).cuda(), 50)
-    assert "0x10" in str(e.value)
+    assert "0x40" in str(e.value)
 
 
 def test_merge_reports_a_valid_entry_after_padding():

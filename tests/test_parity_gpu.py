@@ -156,6 +156,60 @@ def test_dtypes_change_only_the_rounding(orc):
             assert np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1]), (qk, w)
 
 
+# fp8 e4m3 q and k with per-(row, head) and per-key scales (kind::f8f6f4 MMA)
+Q8 = synthetic.quantized
+FP8_CASES = {
+    "pages_example_fp8": lambda: Q8(synthetic.config("pages_example")),
+    "bsnd_causal_ragged_fp8": lambda: Q8(SMALL["bsnd_causal_ragged"]()),
+    "bsnd_n48_fp8": lambda: Q8(SMALL["bsnd_n48"]()),
+    "bsnd_n16_fp8_fp32w": lambda: (lambda pb: pb.replace(w=pb.w.float()))(
+        Q8(SMALL["bsnd_n16_q_longer"]())),
+    "tnd_varlen_fp8": lambda: Q8(SMALL["tnd_varlen"]()),
+    "paged_bs64_fp8": lambda: Q8(SMALL["paged_bs64"]()),
+    "paged_bs16_long_fp8": lambda: Q8(SMALL["paged_bs16_long"]()),
+    "paged_decode_split_fp8": lambda: Q8(SMALL["paged_decode_split"]()),
+    "paged_bs256_nomask_fp8": lambda: Q8(SMALL["paged_bs256_nomask"]()),
+}
+
+
+@pytest.mark.parametrize("name", list(FP8_CASES))
+def test_fp8_parity(orc, name):
+    pb = FP8_CASES[name]()
+    assert li.li_plan(li.make_args(pb))["score_tc"] == 1
+    gi, gv, exact_rows = run_counting_fallbacks(pb)
+    parity.check(orc, pb, gi, gv, label=name)
+
+
+@pytest.mark.parametrize("name", list(EXACT))
+def test_fp8_unit_scales_bit_exact(orc, name):
+    pb = Q8(EXACT[name](), unit_scales=True)
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, exact=True, label=f"{name} fp8")
+
+
+@pytest.mark.parametrize("name", ["bsnd_causal", "paged"])
+def test_fp8_power_of_two_scales_bit_exact(orc, name):
+    """Integer codes with power-of-two scales: every product and partial sum is exact in fp32,
+    so the device must match the oracle bit for bit, which checks where each scale applies."""
+    base = EXACT[name]()
+    g = torch.Generator().manual_seed(130)
+    qs = 2.0 ** torch.randint(-2, 3, base.w.shape, generator=g).float()
+    ks = 2.0 ** torch.randint(-2, 3, base.k.shape[:-2], generator=g).float()
+    pb = base.replace(q=base.q.float().to(torch.float8_e4m3fn),
+                      k=base.k.float().to(torch.float8_e4m3fn), q_descale=qs, k_descale=ks)
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, exact=True, label=f"{name} fp8 scaled")
+
+
+def test_fp8_bad_scale_reported():
+    pb = Q8(synthetic.bsnd(1, 20, 60, 8, 16, 3, seed=131))
+    ks = pb.k_descale.clone()
+    ks[0, 5] = 0.0
+    with pytest.raises(li.LiError) as e:
+        li.indexer(pb.replace(k_descale=ks).to("cuda"))
+    assert "0x80" in str(e.value)
+
+
 def test_indices_only(orc):
     pb = synthetic.bsnd(1, 64, 300, 8, 50, 3, seed=30)
     gi, gv = run(pb, return_value=False)
@@ -318,6 +372,8 @@ FULL = {
     "long_8192": (4, (8191, 8192, 65535)),
     "cmp_prefill": (16, (0, 3, 4, 2047, 4095)),
     "fp16_prefill": (16, (0, 2047, 4095)),
+    "fp8_prefill": (16, (0, 2047, 4095)),
+    "fp8_decode": (8, (0, 63)),
 }
 
 
@@ -364,11 +420,13 @@ def test_tie_heavy_rows_fall_back_correctly(orc):
 # ---- the two score kernels agree ------------------------------------------------------------------
 
 @pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "paged_bs64", "tnd_varlen",
-                                  "pages_example_fp16_fp32", "paged_bs16_long_bf16_fp16"])
+                                  "pages_example_fp16_fp32", "paged_bs16_long_bf16_fp16",
+                                  "bsnd_causal_ragged_fp8", "paged_bs64_fp8"])
 def test_cuda_core_score_kernel_matches_tensor_core(orc, name, monkeypatch):
     """LI_SCORE_KERNEL=simple selects the CUDA-core score kernel (a debugging path); both
     kernels must produce outputs that agree under the parity tolerance."""
-    pb = SMALL[name]() if name in SMALL else DTYPE_CASES[name]()
+    pb = (SMALL[name]() if name in SMALL else DTYPE_CASES[name]() if name in DTYPE_CASES
+          else FP8_CASES[name]())
     a = run(pb)
     monkeypatch.setenv("LI_SCORE_KERNEL", "simple")
     b = run(pb)
