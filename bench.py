@@ -127,10 +127,10 @@ def score_kernel_bytes(pb, pairs) -> int:
 # with the sha256 of the score-kernel sources the counters were taken on; reported only while the
 # sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
 SCORE_TRAFFIC = {
-    "causal_prefill": {"bytes": 68768512 + 9410048,
-                       "src_sha256": "44dcb8cfdf287f173ac7b97450a1c9d9760e494944260dfb186494f39306d70f"},
-    "paged_decode": {"bytes": 286289408 + 6130432,
-                     "src_sha256": "44dcb8cfdf287f173ac7b97450a1c9d9760e494944260dfb186494f39306d70f"},
+    "causal_prefill": {"bytes": 68752128 + 9507840,
+                       "src_sha256": "99f45778113cd656381f5cce8f3ce584cc78533a5fefa7a93a9d50d559b1bf39"},
+    "paged_decode": {"bytes": 286280704 + 6545152,
+                     "src_sha256": "99f45778113cd656381f5cce8f3ce584cc78533a5fefa7a93a9d50d559b1bf39"},
 }
 SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
                  "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")
