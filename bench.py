@@ -4,8 +4,10 @@
 One step = one li_indexer call on one batch of synthetic input: schedule build, score kernel
 (ReLU, weights, head sum, mask fused), top-k selection and padding, i.e. the whole hot path.
 Default workload: causal prefill, B=1, S1=S2=4096, N1=64, D=128, topk=2048, right-down causal
-mask, BSND, bf16 inputs (fp32 accumulation). The metric is query tokens per second; the
-roofline object reports the score kernel's tensor throughput against the measured bf16 peak.
+mask, BSND, bf16 inputs (fp32 accumulation); other workloads by --config (paged decode,
+varlen, long context, compressed keys, fp16 and fp8 inputs, one long row). The metric is query
+tokens per second; the roofline object reports the score kernel's tensor throughput against the
+measured bf16 peak (the HBM bandwidth for paged keys).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 

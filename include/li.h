@@ -19,7 +19,8 @@
  * sequence, plus output_idx_offset[b] when given.
  *
  * Conventions shared by every entry point
- *   - All data pointers are DEVICE pointers of the current CUDA device; NULL means "absent".
+ *   - All data pointers are DEVICE pointers of the current CUDA device (li_merge_topk's input
+ *     lists may also be a peer GPU's memory); NULL means "absent".
  *   - The caller owns every buffer; the library never allocates device or pinned memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every launch
  *     is stream-ordered; no entry point except li_check_status synchronizes or reads device
@@ -86,10 +87,11 @@ typedef enum li_dtype {
  * layout_q/k, mask_mode, return_value) with the tensor shapes made explicit.
  */
 typedef struct li_args {
-    const void *q;                      /* bf16, BSND (B,S1,N1,128) or TND (T1,N1,128), dense  */
-    const void *k;                      /* bf16, BSND (B,S2,1,128), TND (T2,1,128) or
+    const void *q;                      /* dtype_qk, BSND (B,S1,N1,128) or TND (T1,N1,128),
+                                           dense                                               */
+    const void *k;                      /* dtype_qk, BSND (B,S2,1,128), TND (T2,1,128) or
                                            PA_BSND (num_blocks, block_size, 1, 128), dense     */
-    const void *w;                      /* bf16, (B,S1,N1) or (T1,N1), dense                    */
+    const void *w;                      /* dtype_w, (B,S1,N1) or (T1,N1), dense                 */
     const int32_t *cu_seqlens_q;        /* [B+1], non-decreasing; required iff layout_q == TND  */
     const int32_t *cu_seqlens_k;        /* [B+1], non-decreasing; required iff layout_k == TND  */
     const int32_t *seqused_q;           /* [B] or NULL: query rows in use per batch; rows past
@@ -114,8 +116,9 @@ typedef struct li_args {
     int32_t layout_k;                   /* li_layout: BSND, TND or PA_BSND                      */
     int32_t mask_mode;                  /* 0 (no mask) or 3 (right-down causal)                 */
     int32_t dtype_qk;                   /* li_dtype of q and k (one type, lightning_indexer,
-                                           "Constraints"): LI_DTYPE_BF16 or LI_DTYPE_FP16;
-                                           products accumulate in fp32 either way          */
+                                           "Constraints"): LI_DTYPE_BF16, LI_DTYPE_FP16 or
+                                           LI_DTYPE_FP8_E4M3 (with q_descale / k_descale,
+                                           below); products accumulate in fp32 in every case */
     int32_t dtype_w;                    /* li_dtype of w: BF16, FP16 or FP32 (the pages'
                                            single-operator example passes fp16 q, k and fp32
                                            w); fp32 w must be 4-byte aligned               */
