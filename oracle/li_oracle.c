@@ -1,5 +1,6 @@
 /*
- * Lightning Indexer forward pass: plain CPU oracle.
+ * Lightning Indexer forward pass (and, at the end of the file, its backward with the KL loss):
+ * plain CPU oracle.
  *
  * TEST INFRASTRUCTURE. This file is the slow, obviously correct reference that the CUDA library
  * is checked against. Only the tests, the package's smoke check and the benchmark's CPU-baseline
@@ -499,4 +500,125 @@ int orc_merge_topk(int64_t rows, int32_t n_lists, int32_t topk_in, const int32_t
     }
     free(e);
     return ORC_OK;
+}
+
+/* ---- Indexer backward with the KL loss ------------------------------------------------------
+ *
+ * torch_npu.npu_sparse_lightning_indexer_grad_kl_loss, "计算公式" 1-4. For query row r (batch b)
+ * and its selected keys s (sparse_indices[r, :], positions inside batch b's keys, -1 = padding):
+ *   1. I[s]   = sum_h w[r,h] ReLU(qi[r,h,:] . ki[s,:])                   (the indexer score)
+ *   2. P_g[s] = exp(scale (q[r,g,:] . k[s,:] + q_rope[r,g,:] . k_rope[s,:]) - max[r,g]) / sum[r,g]
+ *      (the main attention softmax, rebuilt from its forward statistics softmax_max/_sum)
+ *   3. p[s]   = sum_g P_g[s] / sum_{s'} sum_g P_g[s']   [reading] the head sum of the main
+ *      attention scores normalised to 1 over the selected keys ("L1 normalisation along the
+ *      context direction"); loss_r = sum_s p[s] log(p[s] / softmax(I)[s]) with 0 log 0 = 0, and
+ *      the loss returned is the sum over rows [reading: the formula's sum over t].
+ *   4. dI[s] = softmax(I)[s] - p[s];  dw[r,h] = sum_s dI[s] ReLU(S[h,s]) with S = qi . ki;
+ *      dS[h,s] = dI[s] w[r,h] [S[h,s] > 0];  dqi[r,h,:] = sum_s dS[h,s] ki[s,:];
+ *      dki[s,:] += sum_h dS[h,s] qi[r,h,:]  (summed over every row that selected key s).
+ * Inputs are real values (the wrapper decodes bf16/fp16 exactly); everything is fp64. Rows with
+ * no selected key add nothing. */
+typedef struct {
+    const double *q, *k;            /* main attention: q [rows, G, Dm], k [key rows, Dm]        */
+    const double *q_rope, *k_rope;  /* [rows, G, Dr] / [key rows, Dr], or NULL when Dr == 0    */
+    const double *qi, *ki, *w;      /* indexer: qi [rows, H, Di], ki [key rows, Di], w [rows, H]*/
+    const int32_t *sparse_indices;  /* [rows, topk]                                            */
+    const int64_t *key_base;        /* [rows]: key row of position 0 of the row's batch        */
+    const double *softmax_max, *softmax_sum;   /* [rows, G]                                    */
+    double scale;
+    int64_t rows, key_rows;
+    int32_t G, Dm, Dr, H, Di, topk;
+} orc_kl;
+
+static double dot(const double *a, const double *b, int32_t n)
+{
+    double s = 0.0;
+    for (int32_t d = 0; d < n; ++d) s += a[d] * b[d];
+    return s;
+}
+
+/* loss (scalar), d_qi [rows, H, Di], d_ki [key rows, Di], d_w [rows, H]; the gradient arrays are
+ * overwritten. Returns ORC_EARG for bad sizes, ORC_EDATA for a selected key outside the keys. */
+int orc_kl_grad(const orc_kl *a, double *loss, double *d_qi, double *d_ki, double *d_w)
+{
+    if (!a || !loss || !d_qi || !d_ki || !d_w || a->rows < 0 || a->G < 1 || a->Dm < 1 ||
+        a->Dr < 0 || a->H < 1 || a->Di < 1 || a->topk < 1 || (a->Dr > 0 && (!a->q_rope || !a->k_rope)))
+        return ORC_EARG;
+    const int32_t K = a->topk, H = a->H, G = a->G, Di = a->Di;
+    memset(d_qi, 0, sizeof(double) * (size_t)a->rows * H * Di);
+    memset(d_ki, 0, sizeof(double) * (size_t)a->key_rows * Di);
+    memset(d_w, 0, sizeof(double) * (size_t)a->rows * H);
+    double *I = (double *)malloc(sizeof(double) * K), *p = (double *)malloc(sizeof(double) * K);
+    double *sig = (double *)malloc(sizeof(double) * K), *S = (double *)malloc(sizeof(double) * K * H);
+    int64_t *kr = (int64_t *)malloc(sizeof(int64_t) * K);
+    if (!I || !p || !sig || !S || !kr) {
+        free(I); free(p); free(sig); free(S); free(kr);
+        return ORC_ENOMEM;
+    }
+    double total = 0.0;
+    int rc = ORC_OK;
+    for (int64_t r = 0; r < a->rows && rc == ORC_OK; ++r) {
+        int32_t n = 0;
+        for (int32_t e = 0; e < K; ++e) {
+            const int32_t j = a->sparse_indices[r * K + e];
+            if (j < 0) continue;
+            const int64_t row = a->key_base[r] + j;
+            if (row >= a->key_rows) { rc = ORC_EDATA; break; }
+            kr[n++] = row;
+        }
+        if (rc != ORC_OK || n == 0) continue;
+        /* 1. indexer scores */
+        for (int32_t s = 0; s < n; ++s) {
+            I[s] = 0.0;
+            for (int32_t h = 0; h < H; ++h) {
+                const double v = dot(a->qi + (r * H + h) * Di, a->ki + kr[s] * Di, Di);
+                S[s * H + h] = v;
+                I[s] += a->w[r * H + h] * (v > 0.0 ? v : 0.0);
+            }
+        }
+        /* 2-3. target distribution from the main attention */
+        double psum = 0.0;
+        for (int32_t s = 0; s < n; ++s) {
+            p[s] = 0.0;
+            for (int32_t g = 0; g < G; ++g) {
+                double x = dot(a->q + (r * G + g) * a->Dm, a->k + kr[s] * a->Dm, a->Dm);
+                if (a->Dr > 0) x += dot(a->q_rope + (r * G + g) * a->Dr, a->k_rope + kr[s] * a->Dr, a->Dr);
+                p[s] += exp(a->scale * x - a->softmax_max[r * G + g]) / a->softmax_sum[r * G + g];
+            }
+            psum += p[s];
+        }
+#if ORC_MUTANT != 17
+        for (int32_t s = 0; s < n; ++s) p[s] /= psum;          /* mutant 17 skips the L1 norm */
+#else
+        (void)psum;
+#endif
+        /* softmax of the indexer scores */
+        double imax = I[0], ssum = 0.0;
+        for (int32_t s = 1; s < n; ++s) imax = I[s] > imax ? I[s] : imax;
+        for (int32_t s = 0; s < n; ++s) ssum += exp(I[s] - imax);
+        for (int32_t s = 0; s < n; ++s) sig[s] = exp(I[s] - imax) / ssum;
+        for (int32_t s = 0; s < n; ++s)
+            if (p[s] > 0.0) total += p[s] * (log(p[s]) - log(sig[s]));
+        /* 4. gradients */
+        for (int32_t s = 0; s < n; ++s) {
+#if ORC_MUTANT == 16
+            const double dI = p[s] - sig[s];                    /* mistake: sign of dI */
+#else
+            const double dI = sig[s] - p[s];
+#endif
+            for (int32_t h = 0; h < H; ++h) {
+                const double v = S[s * H + h];
+                if (v <= 0.0) continue;
+                d_w[r * H + h] += dI * v;
+                const double dS = dI * a->w[r * H + h];
+                for (int32_t d = 0; d < Di; ++d) {
+                    d_qi[(r * H + h) * Di + d] += dS * a->ki[kr[s] * Di + d];
+                    d_ki[kr[s] * Di + d] += dS * a->qi[(r * H + h) * Di + d];
+                }
+            }
+        }
+    }
+    free(I); free(p); free(sig); free(S); free(kr);
+    *loss = total;
+    return rc;
 }

@@ -109,6 +109,26 @@ def _i32(x):
     return np.ascontiguousarray(x, dtype=np.int32)
 
 
+class _KL(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_rope", ctypes.c_void_p),
+        ("k_rope", ctypes.c_void_p), ("qi", ctypes.c_void_p), ("ki", ctypes.c_void_p),
+        ("w", ctypes.c_void_p), ("sparse_indices", ctypes.c_void_p), ("key_base", ctypes.c_void_p),
+        ("softmax_max", ctypes.c_void_p), ("softmax_sum", ctypes.c_void_p),
+        ("scale", ctypes.c_double), ("rows", ctypes.c_int64), ("key_rows", ctypes.c_int64),
+        ("G", ctypes.c_int32), ("Dm", ctypes.c_int32), ("Dr", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("Di", ctypes.c_int32), ("topk", ctypes.c_int32),
+    ]
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
 class Oracle:
     """One loaded build of the oracle (the normal one, or a planted mutant)."""
 
@@ -132,6 +152,8 @@ class Oracle:
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p]
         lib.orc_merge_topk.restype = ctypes.c_int
+        lib.orc_kl_grad.argtypes = [ctypes.POINTER(_KL)] + [ctypes.c_void_p] * 4
+        lib.orc_kl_grad.restype = ctypes.c_int
         self.lib = lib
 
     # -- marshalling -----------------------------------------------------------------------
@@ -192,6 +214,44 @@ class Oracle:
 
     def row_info(self, pb, row: int):
         return self.bind(pb).row_info(row)
+
+    def kl_grad(self, kp):
+        """Indexer backward with the KL loss (orc_kl_grad) of a problem carrying q, k, q_rope,
+        k_rope (main attention), qi, ki, w (indexer), sparse_indices, key_base, softmax_max,
+        softmax_sum and scale. Arrays may be tensors of any float type (decoded exactly) or
+        numpy arrays. Returns (loss, d_qi, d_ki, d_w) in float64 with the shapes of qi, ki, w."""
+        keep = {}
+
+        def ptr(name, arr):
+            if arr is None:
+                return None
+            keep[name] = arr
+            return arr.ctypes.data
+
+        a = _KL()
+        q, k = _f64(kp.q), _f64(kp.k)
+        qi, ki, w = _f64(kp.qi), _f64(kp.ki), _f64(kp.w)
+        qr, kr = _f64(getattr(kp, "q_rope", None)), _f64(getattr(kp, "k_rope", None))
+        rows, G = w.shape[0] if w.ndim == 2 else w.shape[0] * w.shape[1], q.shape[-2]
+        a.q, a.k, a.qi, a.ki, a.w = (ptr(n, v) for n, v in
+                                     (("q", q), ("k", k), ("qi", qi), ("ki", ki), ("w", w)))
+        a.q_rope, a.k_rope = ptr("qr", qr), ptr("kr", kr)
+        si = _i32(kp.sparse_indices)
+        kb = np.ascontiguousarray(np.asarray(kp.key_base, dtype=np.int64))
+        a.sparse_indices, a.key_base = ptr("si", si), ptr("kb", kb)
+        a.softmax_max = ptr("smax", _f64(kp.softmax_max))
+        a.softmax_sum = ptr("ssum", _f64(kp.softmax_sum))
+        a.scale = float(kp.scale)
+        a.rows, a.key_rows = rows, ki.size // ki.shape[-1]
+        a.G, a.Dm, a.Dr = G, q.shape[-1], 0 if qr is None else qr.shape[-1]
+        a.H, a.Di, a.topk = qi.shape[-2], qi.shape[-1], si.shape[-1]
+        loss = ctypes.c_double(0.0)
+        d_qi, d_ki, d_w = np.empty_like(qi), np.empty_like(ki), np.empty_like(w)
+        rc = self.lib.orc_kl_grad(ctypes.byref(a), ctypes.addressof(loss), d_qi.ctypes.data,
+                                  d_ki.ctypes.data, d_w.ctypes.data)
+        if rc:
+            raise RuntimeError(f"oracle orc_kl_grad returned {rc}")
+        return loss.value, d_qi, d_ki, d_w
 
     def merge_topk(self, idx_lists, val_lists, topk: int):
         """Top-k of the union of per-row lists: idx_lists / val_lists are sequences of

@@ -305,3 +305,78 @@ def config(name: str, seed: int = 0, integer: bool = False) -> Problem:
 
 CONFIGS = ("tiny", "causal_prefill", "paged_decode", "varlen", "long_2048", "long_8192",
            "cmp_prefill", "fp16_prefill", "long_row_decode", "fp8_prefill", "fp8_decode")
+
+
+# ---- indexer backward with the KL loss ------------------------------------------------------------
+
+@dataclass
+class KLProblem:
+    """Inputs of the indexer backward with the KL loss (torch_npu.npu_sparse_lightning_indexer_
+    grad_kl_loss): the main attention's query and key (one key head, optional rope parts), the
+    indexer's query_index, key_index and weights, the selected keys of every row (positions in
+    the row's batch, -1 padded), and the main attention's softmax statistics over those keys."""
+
+    name: str
+    q: torch.Tensor                 # (B, S1, G, Dm)
+    k: torch.Tensor                 # (B, S2, 1, Dm)
+    q_rope: Optional[torch.Tensor]  # (B, S1, G, Dr) or None
+    k_rope: Optional[torch.Tensor]  # (B, S2, 1, Dr) or None
+    qi: torch.Tensor                # (B, S1, H, Di)
+    ki: torch.Tensor                # (B, S2, 1, Di)
+    w: torch.Tensor                 # (B, S1, H)
+    sparse_indices: torch.Tensor    # (B, S1, 1, topk) int32
+    key_base: torch.Tensor          # (B * S1,) int64: key row of position 0 of the row's batch
+    softmax_max: torch.Tensor       # (B, 1, S1, G) fp32
+    softmax_sum: torch.Tensor       # (B, 1, S1, G) fp32
+    scale: float
+
+    TENSORS = ("q", "k", "q_rope", "k_rope", "qi", "ki", "w", "sparse_indices", "key_base",
+               "softmax_max", "softmax_sum")
+
+    def to(self, device) -> "KLProblem":
+        kw = {f: (None if getattr(self, f) is None else getattr(self, f).to(device))
+              for f in self.TENSORS}
+        return dataclasses.replace(self, **kw)
+
+    def replace(self, **kw) -> "KLProblem":
+        return dataclasses.replace(self, **kw)
+
+
+def kl_bsnd(B, S, G, Dm, Dr, H, topk, seed=0, Di=D_DEFAULT, dtype=torch.bfloat16,
+            name="kl") -> KLProblem:
+    """A causal BSND problem (S1 = S2 = S): inputs N(0, 1) (w N(0, 1/H)) rounded to `dtype`;
+    row i selects min(topk, i + 1) distinct keys of its causal window at random (in random
+    order, -1 padded); softmax_max / softmax_sum are the main attention's forward statistics
+    over the selected keys, per head, taken in fp64 and rounded to fp32: the max of
+    scale * (q . k + q_rope . k_rope) and the sum of exp(x - max); scale = 1 / sqrt(Dm + Dr)."""
+    g = _gen(seed)
+    q = torch.randn(B, S, G, Dm, generator=g).to(dtype)
+    k = torch.randn(B, S, 1, Dm, generator=g).to(dtype)
+    q_rope = torch.randn(B, S, G, Dr, generator=g).to(dtype) if Dr else None
+    k_rope = torch.randn(B, S, 1, Dr, generator=g).to(dtype) if Dr else None
+    qi = torch.randn(B, S, H, Di, generator=g).to(dtype)
+    ki = torch.randn(B, S, 1, Di, generator=g).to(dtype)
+    w = (torch.randn(B, S, H, generator=g) / math.sqrt(H)).to(dtype)
+    idx = torch.full((B, S, 1, topk), -1, dtype=torch.int32)
+    for b in range(B):
+        for i in range(S):
+            m = min(topk, i + 1)
+            idx[b, i, 0, :m] = torch.randperm(i + 1, generator=g)[:m].to(torch.int32)
+    scale = 1.0 / math.sqrt(Dm + Dr)
+    smax = torch.zeros(B, 1, S, G, dtype=torch.float32)
+    ssum = torch.zeros(B, 1, S, G, dtype=torch.float32)
+    for b in range(B):
+        for i in range(S):
+            sel = idx[b, i, 0]
+            sel = sel[sel >= 0].long()
+            x = q[b, i].double() @ k[b, sel, 0].double().T
+            if Dr:
+                x = x + q_rope[b, i].double() @ k_rope[b, sel, 0].double().T
+            x = x * scale
+            mx = x.max(dim=1).values
+            smax[b, 0, i] = mx.float()
+            ssum[b, 0, i] = torch.exp(x - mx[:, None]).sum(dim=1).float()
+    key_base = (torch.arange(B, dtype=torch.int64) * S).repeat_interleave(S)
+    return KLProblem(name=name, q=q, k=k, q_rope=q_rope, k_rope=k_rope, qi=qi, ki=ki, w=w,
+                     sparse_indices=idx, key_base=key_base, softmax_max=smax, softmax_sum=ssum,
+                     scale=scale)

@@ -377,6 +377,94 @@ def pin_fp8_scales_act_as_dequantization(orc):
         _assert_same(orc.topk(fp16)[:2], orc.topk(fp8)[:2], base.name)
 
 
+class _KLArrays:
+    """A backward-with-KL-loss problem held as float64 numpy arrays (shapes as KLProblem)."""
+
+    def __init__(self, rng, B=1, S=5, G=2, Dm=6, Dr=3, H=3, Di=4, topk=3):
+        r = lambda *sh: rng.standard_normal(sh)
+        self.q, self.k = r(B, S, G, Dm), r(B, S, 1, Dm)
+        self.q_rope, self.k_rope = r(B, S, G, Dr), r(B, S, 1, Dr)
+        self.qi, self.ki, self.w = r(B, S, H, Di), r(B, S, 1, Di), r(B, S, H)
+        idx = np.full((B, S, 1, topk), -1, dtype=np.int32)
+        for b in range(B):
+            for i in range(S):
+                m = min(topk, i + 1)
+                idx[b, i, 0, :m] = rng.permutation(i + 1)[:m]
+        self.sparse_indices = idx
+        self.key_base = np.repeat(np.arange(B, dtype=np.int64) * S, S)
+        self.softmax_max = rng.uniform(0.5, 2.0, (B, 1, S, G))
+        self.softmax_sum = rng.uniform(1.0, 3.0, (B, 1, S, G))
+        self.scale = 0.3
+
+
+def pin_kl_gradients_match_finite_differences(orc):
+    """The backward's gradients are the derivatives of its loss: central differences of the
+    loss in every element of query_index, key_index and weights (a key selected by several rows
+    included) match d_query_index, d_key_index and d_weights."""
+    rng = np.random.default_rng(90)
+    for kw in (dict(), dict(B=2, S=4, G=1, Dr=0, H=2, topk=4)):
+        kp = _KLArrays(rng, **kw)
+        if kw.get("Dr") == 0:
+            kp.q_rope = kp.k_rope = None
+        _loss, dqi, dki, dw = orc.kl_grad(kp)
+        eps = 1e-6
+        for name, grad in (("qi", dqi), ("ki", dki), ("w", dw)):
+            arr = getattr(kp, name)
+            for pos in np.ndindex(arr.shape):
+                keep = arr[pos]
+                arr[pos] = keep + eps
+                lp = orc.kl_grad(kp)[0]
+                arr[pos] = keep - eps
+                lm = orc.kl_grad(kp)[0]
+                arr[pos] = keep
+                fd = (lp - lm) / (2 * eps)
+                assert abs(fd - grad[pos]) <= 1e-6 + 1e-5 * abs(fd), (name, pos, fd, grad[pos])
+
+
+def pin_kl_target_is_the_attention_softmax(orc):
+    """With one main-attention head, its true softmax statistics and zero weights (so the
+    indexer's distribution is uniform over the n selected keys), each row's loss is the KL
+    divergence of the attention softmax over the selected keys from uniform: log n - H(p), p
+    computed by scipy's softmax and H by scipy's entropy."""
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    kp = synthetic.kl_bsnd(1, 9, 1, 16, 4, 2, 5, seed=91, Di=8)
+    kp = kp.replace(w=torch.zeros_like(kp.w))
+    want = 0.0
+    for i in range(9):
+        sel = kp.sparse_indices[0, i, 0]
+        sel = sel[sel >= 0].long()
+        x = (kp.q[0, i].double() @ kp.k[0, sel, 0].double().T +
+             kp.q_rope[0, i].double() @ kp.k_rope[0, sel, 0].double().T)[0].numpy() * kp.scale
+        p = softmax(x)
+        want += np.log(len(p)) - entropy(p)
+    loss, dqi, dki, dw = orc.kl_grad(kp)
+    # the forward statistics were rounded to fp32: the head's P sums to 1 within ~1e-7
+    assert abs(loss - want) <= 1e-6 * max(1.0, abs(want)), (loss, want)
+
+
+def pin_kl_target_normalised_over_selected_keys(orc):
+    """p is renormalised over each row's selected keys, so scaling every head's softmax_sum of a
+    row by one factor changes nothing, while scaling one head's alone reweights the heads."""
+    rng = np.random.default_rng(92)
+    kp = _KLArrays(rng)
+    base = orc.kl_grad(kp)
+    kp.softmax_sum[0, 0, 2, :] *= 3.0
+    same = orc.kl_grad(kp)
+    assert abs(same[0] - base[0]) <= 1e-9 * abs(base[0])
+    for a, b in zip(base[1:], same[1:]):
+        assert np.allclose(a, b, rtol=1e-9, atol=1e-12)
+    kp.softmax_sum[0, 0, 2, 0] *= 5.0
+    assert abs(orc.kl_grad(kp)[0] - base[0]) > 1e-6
+
+
+def pin_kl_loss_is_nonnegative(orc):
+    """A sum of KL divergences is never negative (bf16 problems of several sizes)."""
+    for seed, (S, G, H, topk) in enumerate([(12, 4, 8, 6), (30, 2, 4, 16), (7, 8, 1, 3)]):
+        loss = orc.kl_grad(synthetic.kl_bsnd(1, S, G, 32, 8, H, topk, seed=93 + seed, Di=16))[0]
+        assert loss >= 0.0, loss
+
+
 def _key_range(pb, s, e, mask_mode):
     """Keys [s, e) of every batch of a dense BSND problem, indices shifted back to global by
     output_idx_offset = s (written out here, independently of the library's shard helpers)."""
