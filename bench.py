@@ -63,6 +63,14 @@ WORKLOAD_TEXT = {
                        "D=128, topk=2048, mask_mode=3, PA_BSND block_size=64; on N GPUs each "
                        "holds 1/N of the keys, selects in its range, then all-gather + merge",
 }
+WORKLOAD_TEXT["kl_backward"] = (
+    "indexer backward with the KL loss: B=1, S1=S2=2048 causal, 1024 selected keys per row, main "
+    "attention G=16 heads of Dm=512 + Dr=64, indexer H=64 heads of 128, bf16 inputs, fp32 "
+    "outputs")
+# fp32 CUDA-core peak of the first backward version: 148 SMs x 128 fp32 lanes x 2 flops per FMA
+# x 1965 MHz (the maximum SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
 # workloads whose keys (not rows) are split across GPUs: strong scaling, all-gather + merge
 KEY_SHARDED = ("long_row_decode",)
 
@@ -250,11 +258,41 @@ def cpu_oracle_rate(pb, seconds: float, seed: int = 0):
     return done / t_total, done, t_total
 
 
+def run_reference_kl(a):
+    """The reference arm of the backward workload: the oracle on the 16 longest rows per step."""
+    from oracle import oracle as orc
+    kp = synthetic.kl_config(a.config)
+    rows = kp.w.shape[0] * kp.w.shape[1]
+    part = synthetic.kl_rows(kp, rows - 16, rows)
+    o = orc.default()
+    for _ in range(a.warmup):
+        o.kl_grad(part)
+    times = []
+    for _ in range(a.steps):
+        t0 = time.perf_counter()
+        o.kl_grad(part)
+        times.append(time.perf_counter() - t0)
+    t = statistics.mean(times)
+    line = {"metric": "indexer backward query-rows/s", "value": 16 / t, "unit": "query-rows/s",
+            "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config},
+            "cpu_baseline": {"value": 16 / t, "unit": "query-rows/s", "cores": 1,
+                             "kind": "oracle", "sample": "the 16 longest rows per step"},
+            "e2e": {"value": 16 / t, "unit": "query-rows/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(a):
     """The CPU oracle as the reference arm: each step times a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if a.config == "kl_backward":
+        return run_reference_kl(a)
     pb = synthetic.config(a.config)
     step_seconds = a.ref_step_seconds
     for s in range(a.warmup):
@@ -350,6 +388,96 @@ def run_emulated_ranges(a, dev):
     return 0
 
 
+def kl_flops(kp) -> float:
+    """Algorithmic flops of one backward step: per selected (row, key), the main-attention dot
+    products 2 G (Dm + Dr), the indexer score 2 H Di, its recomputation 2 H Di and the two
+    gradient products 4 H Di."""
+    n = int((kp.sparse_indices >= 0).sum())
+    G, Dm = kp.q.shape[-2], kp.q.shape[-1]
+    Dr = 0 if kp.q_rope is None else kp.q_rope.shape[-1]
+    H, Di = kp.qi.shape[-2], kp.qi.shape[-1]
+    return n * (2.0 * G * (Dm + Dr) + 8.0 * H * Di)
+
+
+def run_kl(a, dev, world, rank):
+    """The indexer backward with the KL loss (li_kl_grad): one step = one call over every row."""
+    kp_cpu = synthetic.kl_config(a.config, seed=rank)
+    kp = kp_cpu.to(dev)
+    args = li.make_kl_args(kp)
+    n = li.ctypes.c_size_t(0)
+    L = li.lib()
+    li._check(L.li_kl_grad_workspace_size(li.ctypes.byref(args), li.ctypes.byref(n)))
+    ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    d_qi = torch.empty(kp.qi.shape, dtype=torch.float32, device=dev)
+    d_ki = torch.empty(kp.ki.shape, dtype=torch.float32, device=dev)
+    d_w = torch.empty(kp.w.shape, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        li._check(L.li_kl_grad(li.ctypes.byref(args), ws.data_ptr(), n.value, loss.data_ptr(),
+                               d_qi.data_ptr(), d_ki.data_ptr(), d_w.data_ptr(),
+                               li._stream_handle(stream)))
+
+    for _ in range(a.warmup):
+        step()
+    st, bits = li.li_check_status(ws)
+    if st != li.LI_OK:
+        raise SystemExit(f"device status {st} bits {bits:#x}")
+    K = a.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for s in range(K):
+        flush.zero_()
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / K
+    rows = kp_cpu.w.shape[0] * kp_cpu.w.shape[1]
+    flops = kl_flops(kp_cpu)
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {"metric": "indexer backward query-rows/s", "value": rows * world / (ms / 1e3),
+            "unit": "query-rows/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in, fp32 compute", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
+                       "l2": "flushed before every step by a 256 MB write outside the step's "
+                             "CUDA events",
+                       "parallelism": f"{world} independent replicas (one problem per GPU)"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
+                         "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS, "traffic": None,
+                         "kernel": "kl_row_kernel (CUDA cores, fp32; first version)",
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+            "clocks": clk, "gpu_launches": 3 * K}
+    if rank == 0 and world == 1 and a.cpu_seconds > 0:
+        from oracle import oracle as orc
+        R = 64
+        part = synthetic.kl_rows(kp_cpu, rows - R, rows)
+        t0 = time.perf_counter()
+        orc.default().kl_grad(part)
+        t = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": R / t, "unit": "query-rows/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"the last {R} rows (the longest), {t:.1f} s, "
+                                          "single-threaded C oracle (fp64)",
+                                "host": host_cpu()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -388,6 +516,11 @@ def main():
 
     li.lib()
     keyshard = a.config in KEY_SHARDED
+    if a.config == "kl_backward":
+        rc = run_kl(a, dev, world, rank)
+        if dist:
+            torch.distributed.destroy_process_group()
+        return rc
     if a.emulate_ranges and (world > 1 or a.emulate_ranges > li.MERGE_MAX_LISTS):
         ap.error("--emulate-ranges takes one GPU and at most 16 ranges")
     if a.emulate_ranges:

@@ -315,6 +315,42 @@ typedef struct li_merge_args {
 } li_merge_args;
 li_status li_merge_topk(const li_merge_args *args, void *stream);
 
+/*
+ * li_kl_grad -- the indexer's backward with the KL loss (torch_npu.npu_sparse_lightning_indexer_
+ * grad_kl_loss, formulas 1-4). For every query row r and its selected keys s (sparse_indices,
+ * positions in the row's batch, -1 padded):
+ *     I[s] = sum_h w[r,h] ReLU(qi[r,h,:] . ki[s,:])
+ *     p[s] ~ sum_g exp(scale (q[r,g,:] . k[s,:] + q_rope[r,g,:] . k_rope[s,:]) - softmax_max[r,g])
+ *            / softmax_sum[r,g], normalised to 1 over the row's selected keys
+ *     loss = sum_r sum_s p[s] log(p[s] / softmax(I)[s]),   dI = softmax(I) - p
+ *     d_w[r,h] = sum_s dI[s] ReLU(S[h,s]),  dS[h,s] = dI[s] w[r,h] [S[h,s] > 0]  (S = qi . ki)
+ *     d_qi[r,h,:] = sum_s dS[h,s] ki[s,:],   d_ki[s,:] = sum over rows of sum_h dS[h,s] qi[r,h,:]
+ * [reading] the sums over keys run over the selected keys; p is the head sum of the main
+ * attention softmax rebuilt from its forward statistics and renormalised; the loss sums the rows.
+ * Layout BSND: q (B,S1,G,Dm), k (B,S2,1,Dm), q_rope (B,S1,G,Dr) / k_rope (B,S2,1,Dr) or both NULL
+ * (Dr = 0), qi (B,S1,H,128), ki (B,S2,1,128), w (B,S1,H), all bf16; sparse_indices
+ * (B,S1,1,topk) int32; softmax_max / softmax_sum (B,1,S1,G) fp32. Outputs, fp32: *loss (one
+ * value), d_qi like qi, d_ki like ki (zeroed by the call, then accumulated), d_w like w.
+ * G in [1, 128], Dm in [1, 576] and Dr in [0, 64] multiples of 8, H in [1, 64], topk in
+ * [1, 2048]. Selected positions must lie in [0, S2); others set LI_DEVERR_LENGTHS and are
+ * skipped. The workspace holds one fp32 per row plus the status word: li_kl_grad_workspace_size.
+ * Stream-ordered, no allocation. d_ki is accumulated with atomic adds, so its rounding (not its
+ * value beyond that) may differ from run to run; the loss is summed in a fixed order.
+ */
+typedef struct li_kl_args {
+    const void *q, *k, *q_rope, *k_rope;     /* bf16 main attention                          */
+    const void *qi, *ki, *w;                 /* bf16 indexer query, key and weights          */
+    const int32_t *sparse_indices;
+    const float *softmax_max, *softmax_sum;
+    float scale;
+    int32_t batch, s1, s2;                   /* B, S1 (query rows per batch), S2 (keys)      */
+    int32_t G, Dm, Dr, H, topk;
+    int32_t reserved;                        /* must be 0                                    */
+} li_kl_args;
+li_status li_kl_grad_workspace_size(const li_kl_args *args, size_t *bytes);
+li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_bytes, float *loss,
+                     float *d_qi, float *d_ki, float *d_w, void *stream);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char *li_last_error_string(void);
 

@@ -10,6 +10,7 @@
 #include <string>
 
 #include "li_internal.cuh"
+#include "li_kl.cuh"
 #include "li_merge.cuh"
 #include "li_select.cuh"
 
@@ -445,6 +446,71 @@ li_status li_merge_topk(const li_merge_args *a, void *stream) {
     if (a->rows == 0) return ok();
     cudaError_t e = li::launch_merge(*a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+namespace {
+li_status validate_kl(const li_kl_args *a) {
+    if (!a) return fail(LI_ERR_INVALID_ARG, "args is NULL");
+    if (a->reserved != 0) return fail(LI_ERR_INVALID_ARG, "reserved field must be 0");
+    if (a->batch < 0 || a->s1 < 0 || a->s2 < 0)
+        return fail(LI_ERR_INVALID_ARG, "batch / s1 / s2 must be >= 0");
+    if (a->G < 1 || a->G > 128 || a->H < 1 || a->H > 64 || a->topk < 1 || a->topk > 2048)
+        return fail(LI_ERR_INVALID_ARG, "G=%d (1..128), H=%d (1..64), topk=%d (1..2048)", a->G,
+                    a->H, a->topk);
+    if (a->Dm < 8 || a->Dm > 576 || a->Dm % 8 || a->Dr < 0 || a->Dr > 64 || a->Dr % 8)
+        return fail(LI_ERR_INVALID_ARG, "Dm=%d (8..576) and Dr=%d (0..64) must be multiples of 8",
+                    a->Dm, a->Dr);
+    if ((int64_t)a->G * (a->Dm + a->Dr) > 40960)
+        return fail(LI_ERR_INVALID_ARG, "G x (Dm + Dr) = %lld above 40960",
+                    (long long)a->G * (a->Dm + a->Dr));
+    if ((int64_t)a->batch * a->s1 > INT32_MAX || (int64_t)a->batch * a->s2 > INT32_MAX)
+        return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 query or key rows");
+    if (!a->q || !a->k || !a->qi || !a->ki || !a->w || !a->sparse_indices || !a->softmax_max ||
+        !a->softmax_sum)
+        return fail(LI_ERR_INVALID_ARG, "a required input is NULL");
+    if ((a->Dr > 0) != (a->q_rope != nullptr) || (a->Dr > 0) != (a->k_rope != nullptr))
+        return fail(LI_ERR_INVALID_ARG, "q_rope and k_rope go with Dr > 0, and only with it");
+    if (!(a->scale > 0.0f)) return fail(LI_ERR_INVALID_ARG, "scale must be positive");
+    const void *ptrs[] = {a->q, a->k, a->q_rope, a->k_rope, a->qi, a->ki, a->w, a->sparse_indices,
+                          a->softmax_max, a->softmax_sum};
+    for (const void *p : ptrs)
+        if (!aligned(p, 4)) return fail(LI_ERR_INVALID_ARG, "inputs must be 4-byte aligned");
+    return LI_OK;
+}
+size_t kl_ws_bytes(const li_kl_args *a) {
+    return 256 + ((size_t)a->batch * a->s1 * sizeof(float) + 255) / 256 * 256;
+}
+}  // namespace
+
+li_status li_kl_grad_workspace_size(const li_kl_args *args, size_t *bytes) {
+    li_status st = validate_kl(args);
+    if (st != LI_OK) return st;
+    if (!bytes) return fail(LI_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = kl_ws_bytes(args);
+    return ok();
+}
+
+li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_bytes, float *loss,
+                     float *d_qi, float *d_ki, float *d_w, void *stream) {
+    li_status st = validate_kl(args);
+    if (st != LI_OK) return st;
+    if (!workspace || !aligned(workspace, 256))
+        return fail(LI_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+    if (workspace_bytes < kl_ws_bytes(args))
+        return fail(LI_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                    kl_ws_bytes(args));
+    const bool rows = (int64_t)args->batch * args->s1 > 0;
+    if (!loss || !aligned(loss, 4) || (rows && (!d_qi || !d_w || !aligned(d_qi, 4) || !aligned(d_w, 4))) ||
+        ((int64_t)args->batch * args->s2 > 0 && (!d_ki || !aligned(d_ki, 4))))
+        return fail(LI_ERR_INVALID_ARG, "outputs must be 4-byte aligned device buffers");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, 256, cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "workspace clear: %s", cudaGetErrorString(e));
+    auto *status = static_cast<uint32_t *>(workspace);
+    auto *row_loss = reinterpret_cast<float *>(static_cast<char *>(workspace) + 256);
+    e = li::launch_kl_grad(*args, row_loss, status, loss, d_qi, d_ki, d_w, cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

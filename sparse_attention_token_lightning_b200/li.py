@@ -64,9 +64,24 @@ _lib = None
 
 EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
            "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
-           "li_abi_version", "li_indexer_noalloc", "li_plan", "li_merge_topk")
+           "li_abi_version", "li_indexer_noalloc", "li_plan", "li_merge_topk",
+           "li_kl_grad_workspace_size", "li_kl_grad")
 
 MERGE_MAX_LISTS = 16          # LI_MERGE_MAX_LISTS
+
+
+class LiKlArgs(ctypes.Structure):
+    """Mirror of li_kl_args (include/li.h)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_rope", ctypes.c_void_p),
+        ("k_rope", ctypes.c_void_p), ("qi", ctypes.c_void_p), ("ki", ctypes.c_void_p),
+        ("w", ctypes.c_void_p), ("sparse_indices", ctypes.c_void_p),
+        ("softmax_max", ctypes.c_void_p), ("softmax_sum", ctypes.c_void_p),
+        ("scale", ctypes.c_float), ("batch", ctypes.c_int32), ("s1", ctypes.c_int32),
+        ("s2", ctypes.c_int32), ("G", ctypes.c_int32), ("Dm", ctypes.c_int32),
+        ("Dr", ctypes.c_int32), ("H", ctypes.c_int32), ("topk", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
 
 
 class LiMergeArgs(ctypes.Structure):
@@ -111,6 +126,10 @@ def lib():
     L.li_set_stage_events.restype = ctypes.c_int
     L.li_last_error_string.argtypes = []
     L.li_last_error_string.restype = ctypes.c_char_p
+    L.li_kl_grad_workspace_size.argtypes = [ctypes.POINTER(LiKlArgs), sz]
+    L.li_kl_grad_workspace_size.restype = ctypes.c_int
+    L.li_kl_grad.argtypes = [ctypes.POINTER(LiKlArgs), vp, ctypes.c_size_t, vp, vp, vp, vp, vp]
+    L.li_kl_grad.restype = ctypes.c_int
     L.li_merge_topk.argtypes = [ctypes.POINTER(LiMergeArgs), vp]
     L.li_merge_topk.restype = ctypes.c_int
     L.li_abi_version.argtypes = []
@@ -282,6 +301,42 @@ def merge_topk(idx_lists, val_lists, topk: int, return_value: bool = True, devic
         if st != LI_OK:
             raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
     return idx, val
+
+
+def make_kl_args(kp) -> LiKlArgs:
+    """li_kl_args of a device-resident backward problem (synthetic.KLProblem)."""
+    a = LiKlArgs()
+    B, S1, G, Dm = kp.q.shape
+    a.q, a.k, a.qi, a.ki, a.w = (t.data_ptr() for t in (kp.q, kp.k, kp.qi, kp.ki, kp.w))
+    a.q_rope, a.k_rope = _ptr(kp.q_rope), _ptr(kp.k_rope)
+    a.sparse_indices = kp.sparse_indices.data_ptr()
+    a.softmax_max, a.softmax_sum = kp.softmax_max.data_ptr(), kp.softmax_sum.data_ptr()
+    a.scale = float(kp.scale)
+    a.batch, a.s1, a.s2 = B, S1, kp.k.shape[1]
+    a.G, a.Dm, a.Dr = G, Dm, 0 if kp.q_rope is None else kp.q_rope.shape[-1]
+    a.H, a.topk = kp.qi.shape[2], kp.sparse_indices.shape[-1]
+    return a
+
+
+def kl_grad(kp, stream=None, check: bool = True):
+    """The indexer backward with the KL loss on a device-resident problem: returns (loss,
+    d_query_index, d_key_index, d_weights) as fp32 device tensors (loss of shape (1,))."""
+    a = make_kl_args(kp)
+    n = ctypes.c_size_t(0)
+    _check(lib().li_kl_grad_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    dev = kp.q.device
+    ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    d_qi = torch.empty(kp.qi.shape, dtype=torch.float32, device=dev)
+    d_ki = torch.empty(kp.ki.shape, dtype=torch.float32, device=dev)
+    d_w = torch.empty(kp.w.shape, dtype=torch.float32, device=dev)
+    _check(lib().li_kl_grad(ctypes.byref(a), ws.data_ptr(), n.value, loss.data_ptr(),
+                            d_qi.data_ptr(), d_ki.data_ptr(), d_w.data_ptr(), _stream_handle(stream)))
+    if check:
+        st, bits = li_check_status(ws, stream)
+        if st != LI_OK:
+            raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
+    return loss, d_qi, d_ki, d_w
 
 
 class HostPipeline:

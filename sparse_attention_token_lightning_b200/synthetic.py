@@ -380,3 +380,21 @@ def kl_bsnd(B, S, G, Dm, Dr, H, topk, seed=0, Di=D_DEFAULT, dtype=torch.bfloat16
     return KLProblem(name=name, q=q, k=k, q_rope=q_rope, k_rope=k_rope, qi=qi, ki=ki, w=w,
                      sparse_indices=idx, key_base=key_base, softmax_max=smax, softmax_sum=ssum,
                      scale=scale)
+
+
+def kl_config(name: str, seed: int = 0) -> KLProblem:
+    if name == "kl_backward":
+        # causal rows over 2048 tokens, 1024 selected keys per row, a 16-head main attention of
+        # 512 + 64 dims and a 64-head indexer
+        return kl_bsnd(1, 2048, 16, 512, 64, 64, 1024, seed=seed, name=name)
+    raise KeyError(name)
+
+
+def kl_rows(kp: KLProblem, a: int, b: int) -> KLProblem:
+    """Rows [a, b) of a one-batch backward problem (all keys kept)."""
+    assert kp.q.shape[0] == 1
+    sl = lambda t: None if t is None else t[:, a:b].contiguous()
+    return kp.replace(q=sl(kp.q), q_rope=sl(kp.q_rope), qi=sl(kp.qi), w=sl(kp.w),
+                      sparse_indices=sl(kp.sparse_indices), key_base=kp.key_base[a:b].contiguous(),
+                      softmax_max=kp.softmax_max[:, :, a:b].contiguous(),
+                      softmax_sum=kp.softmax_sum[:, :, a:b].contiguous())

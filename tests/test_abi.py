@@ -174,6 +174,36 @@ def test_merge_args_struct_matches_the_header(L):
     assert ctypes.sizeof(li.LiMergeArgs) == 35 * 8 + 8 + 16
 
 
+def _kl_args(**kw):
+    a = li.LiKlArgs()
+    a.q, a.k, a.qi, a.ki, a.w = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    a.sparse_indices, a.softmax_max, a.softmax_sum = 0x60000, 0x70000, 0x80000
+    a.scale, a.batch, a.s1, a.s2 = 0.05, 2, 64, 64
+    a.G, a.Dm, a.Dr, a.H, a.topk = 16, 512, 0, 64, 32
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw", [
+    dict(G=0), dict(G=129), dict(H=65), dict(topk=0), dict(topk=2049), dict(Dm=0), dict(Dm=580),
+    dict(Dm=100), dict(Dr=64), dict(Dr=12, q_rope=0x90000, k_rope=0xA0000), dict(G=128, Dm=512),
+    dict(q=None), dict(softmax_sum=None), dict(scale=0.0), dict(reserved=1), dict(batch=-1),
+    dict(q_rope=0x90000, k_rope=0xA0000), dict(w=0x50002)])
+def test_invalid_kl_args_rejected_on_host(L, kw):
+    n = ctypes.c_size_t(0)
+    assert L.li_kl_grad_workspace_size(ctypes.byref(_kl_args(**kw)), ctypes.byref(n)) == 1
+    assert li.li_last_error_string()
+
+
+def test_kl_workspace_holds_a_loss_per_row(L):
+    n = ctypes.c_size_t(0)
+    assert L.li_kl_grad_workspace_size(ctypes.byref(_kl_args()), ctypes.byref(n)) == 0
+    assert n.value >= 256 + 2 * 64 * 4
+    ok = _kl_args(Dr=64, q_rope=0x90000, k_rope=0xA0000)
+    assert L.li_kl_grad_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == 0
+
+
 def test_compressed_key_args_accepted(L):
     assert _ws_status(_args(cmp_ratio=4, cmp_residual_k=0x60000))[0] == 0
     assert _ws_status(_args(cmp_ratio=4, mask_mode=0))[0] == 0
