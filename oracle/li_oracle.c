@@ -622,3 +622,72 @@ int orc_kl_grad(const orc_kl *a, double *loss, double *d_qi, double *d_ki, doubl
     *loss = total;
     return rc;
 }
+
+/* ---- Sparse attention over the selected keys ---------------------------------------------------
+ *
+ * The consumer of the indexer's output (aclnnLightningIndexerV2, "主要计算过程" step 3: the
+ * selected indices are the attention's input; aclnnSparseFlashAttentionGrad, "Calculation formula":
+ * the selected keys and values are gathered by the top-k indices, and only value = key is
+ * supported). For query row r, head g and the row's selected keys s:
+ *     x[s]  = scale (q[r,g,:] . k[s,:] + q_rope[r,g,:] . k_rope[s,:])
+ *     m     = max_s x[s],   l = sum_s exp(x[s] - m)
+ *     o[r,g,:] = sum_s exp(x[s] - m) / l * k[s,:]          [reading] the value rows are the key rows
+ * and the forward statistics softmax_max = m, softmax_sum = l that the backward takes. A row with
+ * no selected key gets o = 0, m = -inf, l = 0. fp64 from real-valued inputs. */
+typedef struct {
+    const double *q, *k, *q_rope, *k_rope;   /* q [rows, G, Dm], k [key rows, Dm], rope or NULL */
+    const int32_t *sparse_indices;           /* [rows, topk], positions in the row's batch       */
+    const int64_t *key_base;                 /* [rows]                                           */
+    double scale;
+    int64_t rows, key_rows;
+    int32_t G, Dm, Dr, topk;
+} orc_attn;
+
+int orc_sparse_attention(const orc_attn *a, double *out, double *smax, double *ssum)
+{
+    if (!a || !out || !smax || !ssum || a->rows < 0 || a->G < 1 || a->Dm < 1 || a->Dr < 0 ||
+        a->topk < 1 || (a->Dr > 0 && (!a->q_rope || !a->k_rope)))
+        return ORC_EARG;
+    const int32_t K = a->topk, G = a->G, Dm = a->Dm;
+    double *x = (double *)malloc(sizeof(double) * K);
+    int64_t *kr = (int64_t *)malloc(sizeof(int64_t) * K);
+    if (!x || !kr) { free(x); free(kr); return ORC_ENOMEM; }
+    int rc = ORC_OK;
+    for (int64_t r = 0; r < a->rows && rc == ORC_OK; ++r) {
+        int32_t n = 0;
+        for (int32_t e = 0; e < K; ++e) {
+            const int32_t j = a->sparse_indices[r * K + e];
+            if (j < 0) continue;
+            if (a->key_base[r] + j >= a->key_rows) { rc = ORC_EDATA; break; }
+            kr[n++] = a->key_base[r] + j;
+        }
+        for (int32_t g = 0; g < G && rc == ORC_OK; ++g) {
+            double *o = out + (r * G + g) * Dm;
+            for (int32_t d = 0; d < Dm; ++d) o[d] = 0.0;
+            if (n == 0) {
+                smax[r * G + g] = -INFINITY;
+                ssum[r * G + g] = 0.0;
+                continue;
+            }
+            double m = -INFINITY, l = 0.0;
+            for (int32_t s = 0; s < n; ++s) {
+                x[s] = dot(a->q + (r * G + g) * Dm, a->k + kr[s] * Dm, Dm);
+#if ORC_MUTANT != 18
+                if (a->Dr > 0)
+                    x[s] += dot(a->q_rope + (r * G + g) * a->Dr, a->k_rope + kr[s] * a->Dr, a->Dr);
+#endif
+                x[s] *= a->scale;
+                if (x[s] > m) m = x[s];
+            }
+            for (int32_t s = 0; s < n; ++s) l += exp(x[s] - m);
+            for (int32_t s = 0; s < n; ++s) {
+                const double pw = exp(x[s] - m) / l;
+                for (int32_t d = 0; d < Dm; ++d) o[d] += pw * a->k[kr[s] * Dm + d];
+            }
+            smax[r * G + g] = m;
+            ssum[r * G + g] = l;
+        }
+    }
+    free(x); free(kr);
+    return rc;
+}

@@ -129,6 +129,16 @@ def _f64(x):
     return np.ascontiguousarray(x, dtype=np.float64)
 
 
+class _Attn(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_rope", ctypes.c_void_p),
+        ("k_rope", ctypes.c_void_p), ("sparse_indices", ctypes.c_void_p),
+        ("key_base", ctypes.c_void_p), ("scale", ctypes.c_double), ("rows", ctypes.c_int64),
+        ("key_rows", ctypes.c_int64), ("G", ctypes.c_int32), ("Dm", ctypes.c_int32),
+        ("Dr", ctypes.c_int32), ("topk", ctypes.c_int32),
+    ]
+
+
 class Oracle:
     """One loaded build of the oracle (the normal one, or a planted mutant)."""
 
@@ -154,6 +164,8 @@ class Oracle:
         lib.orc_merge_topk.restype = ctypes.c_int
         lib.orc_kl_grad.argtypes = [ctypes.POINTER(_KL)] + [ctypes.c_void_p] * 4
         lib.orc_kl_grad.restype = ctypes.c_int
+        lib.orc_sparse_attention.argtypes = [ctypes.POINTER(_Attn)] + [ctypes.c_void_p] * 3
+        lib.orc_sparse_attention.restype = ctypes.c_int
         self.lib = lib
 
     # -- marshalling -----------------------------------------------------------------------
@@ -252,6 +264,33 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle orc_kl_grad returned {rc}")
         return loss.value, d_qi, d_ki, d_w
+
+    def sparse_attention(self, kp):
+        """Attention of each row's query heads over its selected keys, values = keys
+        (orc_sparse_attention), for a problem carrying q, k, q_rope, k_rope, sparse_indices,
+        key_base and scale (e.g. synthetic.KLProblem). Returns (out [rows, G, Dm],
+        softmax_max [rows, G], softmax_sum [rows, G]) in float64."""
+        q, k = _f64(kp.q), _f64(kp.k)
+        qr, kr = _f64(getattr(kp, "q_rope", None)), _f64(getattr(kp, "k_rope", None))
+        si = _i32(kp.sparse_indices)
+        kb = np.ascontiguousarray(np.asarray(kp.key_base, dtype=np.int64))
+        G, Dm = q.shape[-2], q.shape[-1]
+        rows = q.size // (G * Dm)
+        a = _Attn()
+        a.q, a.k = q.ctypes.data, k.ctypes.data
+        a.q_rope = None if qr is None else qr.ctypes.data
+        a.k_rope = None if kr is None else kr.ctypes.data
+        a.sparse_indices, a.key_base = si.ctypes.data, kb.ctypes.data
+        a.scale = float(kp.scale)
+        a.rows, a.key_rows = rows, k.size // Dm
+        a.G, a.Dm, a.Dr, a.topk = G, Dm, 0 if qr is None else qr.shape[-1], si.shape[-1]
+        out = np.empty((rows, G, Dm))
+        smax, ssum = np.empty((rows, G)), np.empty((rows, G))
+        rc = self.lib.orc_sparse_attention(ctypes.byref(a), out.ctypes.data, smax.ctypes.data,
+                                           ssum.ctypes.data)
+        if rc:
+            raise RuntimeError(f"oracle orc_sparse_attention returned {rc}")
+        return out, smax, ssum
 
     def merge_topk(self, idx_lists, val_lists, topk: int):
         """Top-k of the union of per-row lists: idx_lists / val_lists are sequences of

@@ -465,6 +465,37 @@ def pin_kl_loss_is_nonnegative(orc):
         assert loss >= 0.0, loss
 
 
+def pin_attention_matches_scipy_softmax(orc):
+    """Attention over the selected keys: for every row and head, scipy's softmax of the scaled
+    dot products (with the rope parts) weights the selected key rows (values = keys), its max
+    and sum of exponentials are the forward statistics, and one selected key returns that key."""
+    from scipy.special import logsumexp, softmax
+    kp = synthetic.kl_bsnd(2, 12, 3, 16, 8, 2, 5, seed=95, Di=8)
+    out, smax, ssum = orc.sparse_attention(kp)
+    q, k = kp.q.double().numpy(), kp.k.double().numpy()
+    qr, kr = kp.q_rope.double().numpy(), kp.k_rope.double().numpy()
+    for b in range(2):
+        for i in range(12):
+            sel = kp.sparse_indices[b, i, 0].numpy()
+            sel = sel[sel >= 0]
+            x = (q[b, i] @ k[b, sel, 0].T + qr[b, i] @ kr[b, sel, 0].T) * kp.scale
+            r = b * 12 + i
+            assert np.allclose(out[r], softmax(x, axis=1) @ k[b, sel, 0], rtol=1e-12, atol=1e-12)
+            assert np.allclose(smax[r], x.max(axis=1), rtol=1e-14, atol=0)
+            assert np.allclose(np.log(ssum[r]) + smax[r], logsumexp(x, axis=1), rtol=1e-12)
+            if len(sel) == 1:
+                assert np.allclose(out[r], np.repeat(k[b, sel, 0], 3, axis=0))
+
+
+def pin_attention_statistics_feed_the_backward(orc):
+    """The backward's generator takes the main attention's statistics over the selected keys (in
+    torch, fp64, rounded to fp32); the oracle's attention gives the same statistics."""
+    kp = synthetic.kl_bsnd(1, 20, 4, 32, 8, 2, 6, seed=96, Di=8)
+    _out, smax, ssum = orc.sparse_attention(kp)
+    assert np.allclose(smax, kp.softmax_max.reshape(20, 4).double().numpy(), rtol=1e-6, atol=1e-6)
+    assert np.allclose(ssum, kp.softmax_sum.reshape(20, 4).double().numpy(), rtol=1e-6)
+
+
 def _key_range(pb, s, e, mask_mode):
     """Keys [s, e) of every batch of a dense BSND problem, indices shifted back to global by
     output_idx_offset = s (written out here, independently of the library's shard helpers)."""

@@ -5,13 +5,14 @@ after the head sum, weights dropped, top-left instead of right-down causal align
 tie order, -0 kept, head/row strides exchanged, block table ignored, TND keys offset by the
 query cumulative lengths, ReLU dropped, output offset dropped, wrong padding, compressed keys kept
 when their first token is visible, a wrong fp16 exponent bias, a merge that drops a list, fp8 keys
-without their scale, the backward's dI with the wrong sign, its target left unnormalised."""
+without their scale, the backward's dI with the wrong sign, its target left unnormalised, the attention's rope
+term dropped."""
 import pytest
 
 import oracle_pins
 from oracle import oracle as orc_mod
 
-MUTANTS = list(range(1, 18))
+MUTANTS = list(range(1, 19))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
