@@ -113,6 +113,19 @@ def test_key_shards_merge_to_the_whole_problem(orc, name, parts, compact):
     assert np.array_equal(got[1].view(np.uint32), whole[1].view(np.uint32)), name
 
 
+def test_key_ranges_empty_for_every_sequence(orc):
+    """More ranges than blocks: some ranges hold no key of any sequence (the compacted cache then
+    keeps one placeholder block), select nothing, and the merge is still the whole selection."""
+    pb = synthetic.paged([100, 40], 1, 4, 16, block_size=64, seed=97)
+    whole = orc.topk(pb)
+    parts = [shard.key_shard(pb, 6, r, compact=True) for r in range(6)]
+    assert any(int(p.seqused_k.sum()) == 0 for p in parts)
+    lists = [orc.topk(p) for p in parts]
+    got = orc.merge_topk([x[0] for x in lists], [x[1] for x in lists], pb.topk)
+    assert np.array_equal(got[0], whole[0])
+    assert np.array_equal(got[1].view(np.uint32), whole[1].view(np.uint32))
+
+
 def test_key_shard_rejects_what_it_cannot_split():
     with pytest.raises(ValueError):
         shard.key_shard(synthetic.tnd([5], [90], 4, 8, 3, seed=96), 2, 0)
