@@ -10,12 +10,11 @@
 // the number of valid entries is written exactly once, and the rest is padded. Only the first
 // topk_out entries of an input row can reach the output, so nothing past them is read.
 //
-// Two kernels. merge_smem_kernel (one CTA per row) copies the row's lists into shared memory as
-// 64-bit order keys with coalesced loads, so every probe is a shared-memory load, and hands out
-// runs in waves of increasing position: run c of every list in one wave, c + 1 in the next.
-// Ranks grow with position, so once a whole wave lands at or past topk_out the row is done; with
-// n lists about topk_out / n entries of each list survive, and the waves stop there.
-// merge_kernel (one CTA per (row, list)) probes global memory and serves rows whose lists do
+// Two kernels. merge_tree_kernel (one CTA per row, the fast path) copies the row's lists into
+// shared memory as 64-bit order keys with many loads in flight, then merges them pairwise, level
+// by level, each result cut to topk_out entries; a pair's output positions are split evenly over
+// its threads, each finding its start on the merge path by binary search. merge_kernel (one CTA
+// per (row, list), the ranking scheme above) probes global memory and serves rows whose lists do
 // not fit in shared memory.
 //
 // HBM traffic: every input entry that can reach the output is read once (8 B) and every output
