@@ -138,9 +138,9 @@ def score_kernel_bytes(pb, pairs) -> int:
 # sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
 SCORE_TRAFFIC = {
     "causal_prefill": {"bytes": 68752128 + 9507840,
-                       "src_sha256": "99f45778113cd656381f5cce8f3ce584cc78533a5fefa7a93a9d50d559b1bf39"},
+                       "src_sha256": "b623c5865b8927a7cbd1c63a806547438de94eb902870e84c685e067617a720f"},
     "paged_decode": {"bytes": 286280704 + 6545152,
-                     "src_sha256": "99f45778113cd656381f5cce8f3ce584cc78533a5fefa7a93a9d50d559b1bf39"},
+                     "src_sha256": "b623c5865b8927a7cbd1c63a806547438de94eb902870e84c685e067617a720f"},
 }
 SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
                  "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")

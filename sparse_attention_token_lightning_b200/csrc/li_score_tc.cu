@@ -13,17 +13,17 @@
 // registers; no cross-lane reduction is needed and w is a per-row broadcast.
 //
 // Warp roles (one CTA per SM, persistent, work items pulled from a global ticket counter):
-//   warp 0      scheduler + TMA producer: takes a ticket, stages the item's header and w in a
-//               shared-memory slot, loads the item's Q tile (double buffered) and streams its
-//               K tiles through a 3-stage ring. Paged keys come block by block through the
-//               block table.
-//   warp 1      allocates TMEM (512 columns = two 256-column accumulators); one thread issues
-//               the tcgen05.mma chain (8 x K16 per tile) and commits to the barriers.
-//   warps 2-9   epilogue: two warps per TMEM lane quarter, each taking every other query row of
-//               the item; tcgen05.ld of a row's N1 columns, ReLU, weight, head sum, causal mask,
-//               coalesced fp32 stores.
-// Every wait on an mbarrier is bounded in time; on expiry the kernel records LI_DEVERR_TIMEOUT,
-// the roles leave their loops, TMEM is freed and the kernel returns.
+//   warp 18     scheduler: takes tickets, stages each item's header, weights and paged cache rows
+//   warp 0      TMA producer: the item's Q tile (double buffered), its K tiles through a ring of
+//               as many stages as fit; paged keys piece by piece through the staged rows
+//   warp 1      allocates TMEM (512 columns); one thread issues the tcgen05.mma chain per tile
+//               (8 x kind::f16 K16 for bf16/fp16, 4 x kind::f8f6f4 K32 for fp8) and commits
+//   warps 2-17  epilogue: four warps per TMEM lane quarter, warp group g taking rows g, g+4, ..;
+//               tcgen05.ld of a row's N1 columns, ReLU, weight, head sum (fp8: times the key's
+//               scale), causal mask, coalesced fp32 stores
+// Instantiated per w type and for fp8 q/k. Every wait on an mbarrier is bounded in time; on
+// expiry the kernel records LI_DEVERR_TIMEOUT, the roles leave their loops, TMEM is freed and the
+// kernel returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
