@@ -14,14 +14,17 @@
 //      atomic histogram, and a warp-striped exclusive scan give each bucket its output range;
 //      the bucket holding output position m-1 is the last one needed.
 //   3. The keys of the needed buckets are scattered to their ranges as 64-bit composites
-//      (score key << 32 | ~index), in any order, then each bucket (about one key on average) is
-//      insertion-sorted descending, which fixes the exact order including ties.
+//      (score key << 32 | ~index), in any order; each key then counts the larger composites of
+//      its bucket (about one or two keys) and lands in an output stage at its exact slot,
+//      which fixes the order including ties; the stage is written out in slot order.
 // Exact fallback, for rows whose needed buckets hold more than kBinCap keys (heavy exact ties)
 // or whose score range overflows: radix select of the m-th key (most significant byte first),
 // gather in index order, stable LSD radix sort.
 // Rows of up to kRegKeys*kThreads keys are held in registers (one read of the row); longer rows
 // take two streaming passes: a 12-bit key-digit histogram that bounds the selection, then a
 // gather of the candidates into shared memory, which the bucket sort orders.
+// Few very long rows (rows x 4 <= SMs, at least kPieceMinKeys keys) are cut into key pieces, one
+// CTA each (select_piece_kernel), whose sorted lists the split merge joins into the row's output.
 #include "li_internal.cuh"
 #include "li_select.cuh"
 
