@@ -496,6 +496,25 @@ def pin_attention_statistics_feed_the_backward(orc):
     assert np.allclose(ssum, kp.softmax_sum.reshape(20, 4).double().numpy(), rtol=1e-6)
 
 
+def pin_selected_key_order_does_not_matter(orc):
+    """Sums over the selected keys cannot depend on the order of sparse_indices: shuffling every
+    row's entries (padding included) leaves the attention, its statistics, the loss and all
+    gradients unchanged up to fp64 rounding."""
+    kp = synthetic.kl_bsnd(2, 10, 3, 16, 8, 4, 6, seed=98, Di=8)
+    g = torch.Generator().manual_seed(99)
+    si = kp.sparse_indices.clone()
+    for b in range(2):
+        for i in range(10):
+            si[b, i, 0] = si[b, i, 0][torch.randperm(6, generator=g)]
+    sh = kp.replace(sparse_indices=si)
+    for a, b in zip(orc.sparse_attention(kp), orc.sparse_attention(sh)):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+    la, lb = orc.kl_grad(kp), orc.kl_grad(sh)
+    assert abs(la[0] - lb[0]) <= 1e-12 * abs(la[0])
+    for a, b in zip(la[1:], lb[1:]):
+        assert np.allclose(a, b, rtol=1e-10, atol=1e-12)
+
+
 def _key_range(pb, s, e, mask_mode):
     """Keys [s, e) of every batch of a dense BSND problem, indices shifted back to global by
     output_idx_offset = s (written out here, independently of the library's shard helpers)."""
