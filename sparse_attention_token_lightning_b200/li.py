@@ -1,9 +1,11 @@
 """Thin ctypes binding over ``libli.so`` (C ABI in include/li.h).
 
 Argument marshalling only: every step of the indexer runs in the library's CUDA kernels. The
-functions keep the C names (``li_metadata``, ``li_indexer``, ...). ``indexer()`` is a convenience
-that allocates the outputs and the workspace with torch and calls ``li_indexer`` on the current
-stream. There is no fallback: if the library is missing, loading raises.
+functions keep the C names (``li_metadata``, ``li_indexer``, ``li_merge_topk``, ``li_kl_grad``,
+...). ``indexer()``, ``merge_topk()`` and ``kl_grad()`` are conveniences that allocate outputs and
+workspaces with torch and call the library on the current stream; ``HostPipeline`` runs the
+indexer over host-resident problems with the copies overlapping the kernels. There is no
+fallback: if the library is missing, loading raises.
 """
 from __future__ import annotations
 
@@ -18,6 +20,7 @@ STATUS = {0: "LI_OK", 1: "LI_ERR_INVALID_ARG", 2: "LI_ERR_UNSUPPORTED", 3: "LI_E
           4: "LI_ERR_CUDA", 5: "LI_ERR_DEVICE_TIMEOUT", 6: "LI_ERR_DEVICE_DATA"}
 LI_OK = 0
 DEVERR_TIMEOUT, DEVERR_LENGTHS, DEVERR_TABLE, DEVERR_OFFSET, DEVERR_METADATA = 1, 2, 4, 8, 16
+DEVERR_INTERNAL, DEVERR_MERGE_ORDER, DEVERR_DESCALE = 32, 64, 128        # LI_DEVERR_* of li.h
 
 
 class LiError(RuntimeError):

@@ -73,3 +73,20 @@ def test_oracle_mirrors_match_the_oracle_source(tmp_path):
         assert ctypes.sizeof(mirror) == table[(cname, "size")], cname
         for fname, _t in mirror._fields_:
             assert getattr(mirror, fname).offset == table[(cname, fname)], (cname, fname)
+
+
+def test_python_constants_match_the_header():
+    """Status codes, device error bits and type codes named in li.py equal the header's."""
+    text = (ROOT / "include" / "li.h").read_text()
+    import re
+    defs = dict(re.findall(r"#define (LI_DEVERR_\w+)\s+(0x[0-9a-fA-F]+)u", text))
+    for name, val in [("TIMEOUT", li.DEVERR_TIMEOUT), ("LENGTHS", li.DEVERR_LENGTHS),
+                      ("TABLE", li.DEVERR_TABLE), ("OFFSET", li.DEVERR_OFFSET),
+                      ("METADATA", li.DEVERR_METADATA), ("INTERNAL", li.DEVERR_INTERNAL),
+                      ("MERGE_ORDER", li.DEVERR_MERGE_ORDER), ("DESCALE", li.DEVERR_DESCALE)]:
+        assert int(defs["LI_DEVERR_" + name], 16) == val, name
+    enum = dict((k, int(v)) for k, v in re.findall(r"(LI_(?:ERR_\w+|OK)) = (\d+)", text))
+    assert {v: k for k, v in enum.items()} == li.STATUS
+    dt = dict((k, int(v)) for k, v in re.findall(r"LI_DTYPE_(\w+) = (\d+)", text))
+    assert dt == {"BF16": 0, "FP16": 1, "FP32": 2, "FP8_E4M3": 3}
+    assert sorted(li.DTYPES.values()) == [0, 1, 2, 3]
