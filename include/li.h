@@ -254,7 +254,9 @@ li_status li_set_stage_events(void *const *events, int32_t n_events);
  * array compiled into the library (a static device array of LI_NOALLOC_SCRATCH_BYTES). The
  * caller passes the inputs in `args` and the outputs as with li_indexer, plus `device_status`:
  * a device uint32 (or NULL) that receives the call's device status word, stream-ordered, so
- * li_check_status(device_status, stream, &bits) reports data errors of this call.
+ * li_check_status(device_status, stream, &bits) reports data errors of this call. It is written
+ * only when the call returns LI_OK; on any error return it keeps its previous contents, and the
+ * returned status (with li_last_error_string) is the call's result.
  *
  *   - Problems whose workspace (li_indexer_workspace_size) exceeds LI_NOALLOC_SCRATCH_BYTES are
  *     rejected on the host with LI_ERR_WORKSPACE and a message giving both sizes.

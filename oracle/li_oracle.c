@@ -50,8 +50,8 @@
  * the score rounded once to fp32, the precision the CUDA kernels decide in, and -0 is treated as
  * +0. Order: score descending, then key index ascending (the pages only say "deterministic").
  *
- * Readings of points the pages leave open are listed in the design notes; each is marked
- * [reading] below where it is applied.
+ * Every point the pages leave open is taken with the plainest reading the rest of the pages
+ * support, and each such reading is marked [reading] below where it is applied.
  *
  * Planted mistakes. Building with -DORC_MUTANT=n plants mistake n (see the ORC_MUTANT blocks).
  * A test builds each mutant and checks that the pins catch it. A normal build has none.

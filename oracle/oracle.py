@@ -23,7 +23,7 @@ LAYOUTS = {"BSND": 0, "TND": 1, "PA_BSND": 2}
 ORC_OK, ORC_EARG, ORC_EDATA, ORC_ENOMEM = 0, 1, 2, 3
 
 
-def build(mutant: int = 0, out_dir: Path | None = None, openmp: bool = False) -> Path:
+def build(mutant: int = 0, out_dir: Path | None = None) -> Path:
     """Compile the oracle with gcc. ``mutant`` > 0 plants the numbered mistake (for tests)."""
     out_dir = Path(out_dir) if out_dir is not None else BUILD_DIR
     out_dir.mkdir(parents=True, exist_ok=True)

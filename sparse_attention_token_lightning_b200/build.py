@@ -34,18 +34,31 @@ def headers():
     return sorted(CSRC.glob("*.cuh")) + sorted(INCLUDE.glob("*.h"))
 
 
-def up_to_date() -> bool:
-    if not LIB.exists():
+# Test build: every bounded device wait gives up after 1 ms, and the score kernel's TMA producer
+# issues no load (so no bulk copy is ever in flight and the MMA warp's first wait runs out). The
+# tests load it beside libli.so to drive the timeout exit; nothing else uses it.
+WAIT_TEST_LIB = PKG / "libli_waittest.so"
+WAIT_TEST_FLAGS = ("-DLI_WAIT_LIMIT_NS=1000000ull", "-DLI_TEST_NO_LOADS=1")
+
+
+def up_to_date(lib: Path = LIB) -> bool:
+    if not lib.exists():
         return False
-    t = LIB.stat().st_mtime
+    t = lib.stat().st_mtime
     return all(f.stat().st_mtime <= t for f in sources() + headers())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> Path:
-    if not force and up_to_date():
-        return LIB
-    obj_dir = PKG / "_build"
-    obj_dir.mkdir(exist_ok=True)
+def build_wait_test(force: bool = False, verbose: bool = False) -> Path:
+    """libli_waittest.so (see WAIT_TEST_FLAGS)."""
+    return build(force, verbose, WAIT_TEST_FLAGS, lib=WAIT_TEST_LIB, obj_sub="waittest")
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), lib: Path = LIB,
+          obj_sub: str = "") -> Path:
+    if not force and up_to_date(lib):
+        return lib
+    obj_dir = PKG / "_build" / obj_sub if obj_sub else PKG / "_build"
+    obj_dir.mkdir(parents=True, exist_ok=True)
     objs = []
     procs = []
     common = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -66,13 +79,14 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> Path:
             failed.append(src.name)
     if failed:
         raise RuntimeError(f"nvcc failed for {failed}")
-    tmp = LIB.with_suffix(".so.tmp")
+    tmp = lib.with_suffix(".so.tmp")
     link = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *map(str, objs)]
     subprocess.run(link, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
+    build_wait_test(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)

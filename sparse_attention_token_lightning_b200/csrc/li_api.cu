@@ -3,6 +3,7 @@
 // (aclnnLightningIndexerV2: a first call validates the arguments and sizes the workspace, a
 // second call runs on a stream) and their metadata-then-indexer order (lightning_indexer,
 // "Prototype").
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -31,19 +32,6 @@ li_status fail(li_status st, const char *fmt, ...) {
 li_status ok() {
     g_err.clear();
     return LI_OK;
-}
-
-int sm_count() {
-    static int cached = 0;
-    if (cached) return cached;
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) {
-        cached = n;
-        return n;
-    }
-    (void)cudaGetLastError();
-    return 148;
 }
 
 cudaEvent_t g_stage_events[6] = {};
@@ -205,8 +193,8 @@ li_status validate(const li_args *a, li::Problem *p, li::Schedule *s) {
     S.kc = 0;
     // too few query blocks to fill the GPU (decode): split the key ranges so that there are
     // about 32 items per SM, small enough for the dynamic scheduler to end all SMs together
-    const int64_t target = 32LL * sm_count();
-    if (qblocks < 2LL * sm_count() && P.max_seqlen_k >= 2048) {
+    const int64_t target = 32LL * li::device_sm_count();
+    if (qblocks < 2LL * li::device_sm_count() && P.max_seqlen_k >= 2048) {
         int64_t kc = ((int64_t)P.max_seqlen_k * (qblocks > 0 ? qblocks : 1) + target - 1) / target;
         kc = (kc + li::kKeyTile - 1) / li::kKeyTile * li::kKeyTile;
         if (kc < 512) kc = 512;
@@ -252,6 +240,28 @@ size_t indexer_ws_bytes(const li::Problem &p, const li::Schedule &s) {
 
 namespace li {
 void set_last_error(const char *msg) { g_err = msg; }
+
+int device_sm_count() {
+    constexpr int kMaxDevices = 128;
+    static std::atomic<int> cache[kMaxDevices];      // 0 = not looked up yet
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    const bool slot = dev >= 0 && dev < kMaxDevices;
+    if (slot) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    if (slot) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 }  // namespace li
 
 extern "C" {

@@ -343,6 +343,10 @@ __device__ inline void set_status(uint32_t *status, uint32_t bits) {
 // Sets the message li_last_error_string() returns on this host thread.
 void set_last_error(const char *msg);
 
+// Streaming multiprocessors of the current device, looked up once per device (148, the B200's
+// count, when the query fails).
+int device_sm_count();
+
 // fp8 q/k scales (li_args q_descale / k_descale), null for 16-bit q/k. Kept out of Problem so
 // that the kernels' parameter blocks keep their layout.
 struct Quant {

@@ -47,7 +47,19 @@ constexpr uint32_t kKStageBytes = 2 * kKHalfBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxAcc = 8;                               // TMEM accumulators (512 / stride)
 constexpr uint32_t kDevErrInternal = 0x20u;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+// Limit of every bounded wait. The library is built with 2 s; a test build lowers it to 1 ms
+// and defines LI_TEST_NO_LOADS, under which the producer issues no TMA load and never arrives on
+// the full barriers, so the MMA warp's first wait runs out with no bulk copy in flight: that
+// build exercises the timeout exit (status bit, every role leaving its loop, TMEM freed).
+#ifndef LI_WAIT_LIMIT_NS
+#define LI_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = LI_WAIT_LIMIT_NS;
+#ifdef LI_TEST_NO_LOADS
+constexpr bool kIssueLoads = false;
+#else
+constexpr bool kIssueLoads = true;
+#endif
 
 struct Slot {
     int32_t valid, b, q0, nq, j0, j1, row0, L1u, L2, k_row0;
@@ -389,7 +401,7 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
         // Q tile of the item (all heads of tq rows): two TMA loads, one per 64-wide K half.
         const int qb = it & 1;
         if (!mbar_wait(bars.q_empty(qb), ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) {
+        if (kIssueLoads && lane == 0) {
             const uint32_t qdst = sbase + qb * 2u * P.q_half;
             const int32_t y = row0 * N1;
             if constexpr (kQ8) {
@@ -412,7 +424,9 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             if (!mbar_wait(bars.k_empty(st), kr.phase ^ 1u, abort_flag)) { ok = false; break; }
             const int32_t jt = j0 + tile * kKeyTile;
             const uint32_t kdst = sbase + P.k_off + st * kStage;
-            if (pr == 0) {
+            if (!kIssueLoads) {
+                // test build: no load and no arrive; the MMA warp's wait on k_full runs out
+            } else if (pr == 0) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), kStage);
                     tma_load_2d(kdst, tmk, bars.k_full(st), 0, k_row0 + jt);
@@ -779,17 +793,6 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows,
     return r == CUDA_SUCCESS;
 }
 
-int sm_count_cached() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            n = 148;
-    }
-    return n;
-}
-
 }  // namespace
 
 // Shape checks of the tensor-core kernel: MMA width 16..256, at least two key stages in shared
@@ -871,7 +874,7 @@ cudaError_t launch_score_tc(const Problem &p, const Quant &qd, const Schedule &s
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    int grid = sm_count_cached();
+    int grid = device_sm_count();
     if (s.max_items < grid) grid = s.max_items;
     kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, P);
     e = cudaGetLastError();

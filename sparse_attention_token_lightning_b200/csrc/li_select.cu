@@ -98,12 +98,7 @@ cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta,
         return launch_one<256, false, sel256::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val,
                                                     smem, cand_cap, sel256::select_kernel<false>, st);
     }
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        (void)cudaGetLastError();
-        sms = 148;
-    }
+    const int sms = device_sm_count();
     if (p.rows < 2 * sms) {
         const size_t smem = sel1024::select_work_bytes(p.topk, true, &cand_cap);
         return launch_one<1024, true, sel1024::Smem>(p, s, meta, ws, scores, ld, out_idx, out_val,
@@ -116,12 +111,7 @@ cudaError_t launch_select(const Problem &p, const Schedule &s, const void *meta,
 }
 
 int select_pieces(const Problem &p) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        (void)cudaGetLastError();
-        sms = 148;
-    }
+    const int sms = device_sm_count();
     // only rows long enough that one CTA streaming the whole row is the bottleneck, and few
     // enough rows that the GPU would otherwise sit mostly idle
     if (p.rows <= 0 || p.max_seqlen_k < kPieceMinKeys || p.rows * 4 > sms) return 1;

@@ -109,7 +109,14 @@ def lib():
     if not _LIB_PATH.exists():
         raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
                            "`python -m sparse_attention_token_lightning_b200.build`")
-    L = ctypes.CDLL(str(_LIB_PATH))
+    _lib = load(_LIB_PATH)
+    return _lib
+
+
+def load(path) -> ctypes.CDLL:
+    """A separately loaded build of the library at `path` (same C ABI), with the argument types
+    set; used for the test build whose device waits give up after 1 ms."""
+    L = ctypes.CDLL(str(path))
     P = ctypes.POINTER(LiArgs)
     sz = ctypes.POINTER(ctypes.c_size_t)
     vp = ctypes.c_void_p
@@ -137,7 +144,6 @@ def lib():
     L.li_merge_topk.restype = ctypes.c_int
     L.li_abi_version.argtypes = []
     L.li_abi_version.restype = ctypes.c_int32
-    _lib = L
     return L
 
 

@@ -387,6 +387,34 @@ def test_full_size_sampled(orc, name):
     assert exact_rows == 0, f"{exact_rows} rows left the bucket selection paths"
 
 
+FULL_EXACT = {
+    # name: (problem, rows to sample, rows that must be checked). Integer-valued inputs make every
+    # score exact in fp32, so these compare bit for bit, tie order included, at the benchmark's
+    # shapes: the headline causal prefill (rows around the topk = 2048 boundary and the longest
+    # row), topk 8192 over rows of more than 8192 keys, and paged decode rows of up to 32K keys.
+    "causal_prefill": (lambda: synthetic.config("causal_prefill", integer=True), 16,
+                       (0, 1, 127, 2046, 2047, 2048, 2049, 4094, 4095)),
+    "topk8192_long_rows": (lambda: synthetic.bsnd(1, 48, 12000, 16, 8192, 3, seed=73,
+                                                  integer=True, name="topk8192_long_rows"),
+                           48, ()),
+    "paged_decode": (lambda: synthetic.config("paged_decode", integer=True), 8, ()),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_EXACT))
+def test_full_size_integer_inputs_bit_exact(orc, name):
+    make, n, must = FULL_EXACT[name]
+    pb = make()
+    if name == "paged_decode":
+        # the longest and the shortest decode rows, plus a seeded sample
+        lens = pb.seqused_k.tolist()
+        must = (int(np.argmax(lens)), int(np.argmin(lens)))
+        assert max(lens) > 32000
+    rows = parity.sample_rows(pb, n, seed=2, must=must)
+    gi, gv = run(pb)
+    parity.check(orc, pb, gi, gv, rows=rows, exact=True, label=f"{name} integer")
+
+
 @pytest.mark.parametrize("name", ["tiny", "bsnd_causal_ragged", "tnd_varlen", "paged_bs64",
                                   "topk8192_n16", "paged_bs16_tnd_q", "offset_seqused"])
 def test_tie_free_rows_use_the_bucket_paths(orc, name):
