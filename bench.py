@@ -67,6 +67,10 @@ WORKLOAD_TEXT["kl_backward"] = (
     "indexer backward with the KL loss: B=1, S1=S2=2048 causal, 1024 selected keys per row, main "
     "attention G=16 heads of Dm=512 + Dr=64, indexer H=64 heads of 128, bf16 inputs, fp32 "
     "outputs")
+WORKLOAD_TEXT["sparse_attention"] = (
+    "sparse attention over the selected keys: B=1, S1=S2=4096 causal, each row min(2048, i+1) "
+    "selected keys (random, indexer-shaped), G=16 heads of Dm=512 + Dr=64, values = keys, bf16 "
+    "inputs, fp32 outputs and statistics")
 # fp32 CUDA-core peak of the first backward version: 148 SMs x 128 fp32 lanes x 2 flops per FMA
 # x 1965 MHz (the maximum SM clock)
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -464,6 +468,100 @@ def kl_flops(kp) -> float:
     return n * (2.0 * G * (Dm + Dr) + 8.0 * H * Di)
 
 
+def attn_flops(ap) -> float:
+    """Algorithmic flops of one attention step: per selected (row, key), the scores 2 G (Dm + Dr)
+    and the value product 2 G Dm."""
+    n = int(((ap.sparse_indices >= 0) & (ap.sparse_indices < ap.k.shape[1])).sum())
+    G, Dm = ap.q.shape[-2], ap.q.shape[-1]
+    Dr = 0 if ap.q_rope is None else ap.q_rope.shape[-1]
+    return n * (2.0 * G * (Dm + Dr) + 2.0 * G * Dm), n
+
+
+def run_attn(a, dev, world, rank):
+    """Sparse attention over the selected keys (li_sparse_attention): one step = every row."""
+    ap_cpu = synthetic.attn_config(a.config, seed=rank)
+    ap = ap_cpu.to(dev)
+    args = li.make_attn_args(ap)
+    B, S1, G, Dm = ap.q.shape
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    out = torch.empty((B, S1, G, Dm), dtype=torch.float32, device=dev)
+    smax = torch.empty((B, 1, S1, G), dtype=torch.float32, device=dev)
+    ssum = torch.empty((B, 1, S1, G), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        li.li_sparse_attention(args, ws, out, smax, ssum, stream)
+
+    for _ in range(a.warmup):
+        step()
+    st, bits = li.li_check_status(ws)
+    if st != li.LI_OK:
+        raise SystemExit(f"device status {st} bits {bits:#x}")
+    K = a.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for s in range(K):
+        flush.zero_()
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / K
+    rows = B * S1
+    flops, pairs = attn_flops(ap_cpu)
+    achieved = flops / (ms / 1e3) / 1e12
+    peaks = load_peaks()
+    Dr = 0 if ap_cpu.q_rope is None else ap_cpu.q_rope.shape[-1]
+    gathered = pairs * (Dm + Dr) * 2
+    line = {"metric": "sparse attention query-tokens/s", "value": rows * world / (ms / 1e3),
+            "unit": "query-tokens/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
+                       "selected_pairs": pairs,
+                       "l2": "flushed before every step by a 256 MB write outside the step's "
+                             "CUDA events",
+                       "parallelism": f"{world} independent replicas (one problem per GPU)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": None,
+                         "kernel": "sparse_attn_kernel (gather + tcgen05 scores, softmax, "
+                                   "value product)",
+                         "peak_source": f"{peaks['source']} bf16 burst"},
+            "gather": {"bytes": gathered, "achieved_gbs": gathered / (ms / 1e3) / 1e9,
+                       "note": "selected key rows copied into shared memory once per (row, key)"},
+            "clocks": clk, "gpu_launches": K}
+    if rank == 0 and world == 1 and a.cpu_seconds > 0:
+        from oracle import oracle as orc
+        import numpy as np
+        R = 16
+        pick = np.random.default_rng(1).choice(rows, R, replace=False)
+        part = ap_cpu.rows(pick)
+        with one_core():
+            t0 = time.perf_counter()
+            orc.default().sparse_attention(part)
+            t = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": R / t, "unit": "query-tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{R} seeded-random rows, {t:.1f} s, single-threaded C "
+                                          "oracle (fp64), one pinned core",
+                                "host": host_cpu()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_kl(a, dev, world, rank):
     """The indexer backward with the KL loss (li_kl_grad): one step = one call over every row."""
     kp_cpu = synthetic.kl_config(a.config, seed=rank)
@@ -582,8 +680,8 @@ def main():
 
     li.lib()
     keyshard = a.config in KEY_SHARDED
-    if a.config == "kl_backward":
-        rc = run_kl(a, dev, world, rank)
+    if a.config in ("kl_backward", "sparse_attention"):
+        rc = (run_kl if a.config == "kl_backward" else run_attn)(a, dev, world, rank)
         if dist:
             torch.distributed.destroy_process_group()
         return rc

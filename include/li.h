@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LI_ABI_VERSION 4
+#define LI_ABI_VERSION 5
 
 typedef enum li_layout {
     LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
@@ -352,6 +352,43 @@ typedef struct li_kl_args {
 li_status li_kl_grad_workspace_size(const li_kl_args *args, size_t *bytes);
 li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_bytes, float *loss,
                      float *d_qi, float *d_ki, float *d_w, void *stream);
+
+/*
+ * li_sparse_attention -- attention of every query row over the keys the indexer selected for it,
+ * the indexer's consumer (aclnnLightningIndexerV2, main computation steps: the selected indices
+ * are the attention's input; aclnnSparseFlashAttentionGrad, calculation formula: the selected keys
+ * and values are gathered by the top-k indices, and value = key is the supported case). For query
+ * row r of batch b, head g and the row's selected keys s:
+ *     x[s]     = scale * (q[r,g,:] . k[s,:] + q_rope[r,g,:] . k_rope[s,:])
+ *     o[r,g,:] = sum_s exp(x[s] - m) k[s,:] / l,   m = max_s x[s],   l = sum_s exp(x[s] - m)
+ * [reading] the value rows are the key rows (all Dm dims; the rope dims only enter the scores).
+ * The statistics m and l are the inputs li_kl_grad takes as softmax_max / softmax_sum.
+ *
+ * Layout BSND, all bf16 and dense: q (B,S1,G,Dm), k (B,S2,1,Dm), q_rope (B,S1,G,Dr) and k_rope
+ * (B,S2,1,Dr) or both NULL (Dr = 0); sparse_indices (B,S1,1,topk) int32, positions in the row's
+ * batch (as li_indexer writes them without output_idx_offset); a negative entry selects nothing,
+ * an entry >= S2 selects nothing and sets LI_DEVERR_LENGTHS. Entries may repeat (each counts).
+ * Outputs, fp32: out (B,S1,G,Dm); softmax_max and softmax_sum (B,1,S1,G). A row that selects no
+ * key gets out = 0, softmax_max = -inf, softmax_sum = 0.
+ * Limits: G in [1, 32], Dm in {128, 256, 384, 512}, Dr in {0, 64}, topk in [1, 8192], S2 >= 1
+ * when there are rows, scale > 0; q, k, q_rope, k_rope 16-byte aligned, the rest 4-byte aligned.
+ * Numerics: products and sums in fp32 on the tensor cores; the softmax weights enter the value
+ * product rounded to bf16 (the normaliser l is the fp32 sum of the unrounded weights).
+ * The workspace (li_sparse_attention_workspace_size: 256 bytes) holds the device status word
+ * (read it with li_check_status) and a row counter; its contents on entry are ignored.
+ * Stream-ordered, no allocation, deterministic (bit-identical reruns).
+ */
+typedef struct li_attn_args {
+    const void *q, *k, *q_rope, *k_rope;    /* bf16, see above                                   */
+    const int32_t *sparse_indices;
+    float scale;
+    int32_t batch, s1, s2;                  /* B, S1 (query rows per batch), S2 (keys per batch) */
+    int32_t G, Dm, Dr, topk;
+    int32_t reserved;                       /* must be 0                                         */
+} li_attn_args;
+li_status li_sparse_attention_workspace_size(const li_attn_args *args, size_t *bytes);
+li_status li_sparse_attention(const li_attn_args *args, void *workspace, size_t workspace_bytes,
+                              float *out, float *softmax_max, float *softmax_sum, void *stream);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *li_last_error_string(void);

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <string>
 
+#include "li_attn.cuh"
 #include "li_internal.cuh"
 #include "li_kl.cuh"
 #include "li_merge.cuh"
@@ -521,6 +522,69 @@ li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_b
     auto *row_loss = reinterpret_cast<float *>(static_cast<char *>(workspace) + 256);
     e = li::launch_kl_grad(*args, row_loss, status, loss, d_qi, d_ki, d_w, cs);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+namespace {
+li_status validate_attn(const li_attn_args *a, li::AttnLayout *L) {
+    if (!a) return fail(LI_ERR_INVALID_ARG, "args is NULL");
+    if (a->reserved != 0) return fail(LI_ERR_INVALID_ARG, "reserved field must be 0");
+    if (a->batch < 0 || a->s1 < 0 || a->s2 < 0)
+        return fail(LI_ERR_INVALID_ARG, "batch / s1 / s2 must be >= 0");
+    if (a->G < 1 || a->G > 32) return fail(LI_ERR_INVALID_ARG, "G=%d outside [1, 32]", a->G);
+    if (a->Dm < 128 || a->Dm > 512 || a->Dm % 128)
+        return fail(LI_ERR_INVALID_ARG, "Dm=%d must be 128, 256, 384 or 512", a->Dm);
+    if (a->Dr != 0 && a->Dr != 64) return fail(LI_ERR_INVALID_ARG, "Dr=%d must be 0 or 64", a->Dr);
+    if (a->topk < 1 || a->topk > li::kMaxTopk)
+        return fail(LI_ERR_INVALID_ARG, "topk=%d outside [1, 8192]", a->topk);
+    if (!(a->scale > 0.0f) || !(a->scale < 3.0e38f))
+        return fail(LI_ERR_INVALID_ARG, "scale must be a positive finite number");
+    const int64_t rows = (int64_t)a->batch * a->s1;
+    if (rows > 0 && a->s2 < 1) return fail(LI_ERR_INVALID_ARG, "S2=0 with query rows");
+    if (rows * a->G > INT32_MAX || (int64_t)a->batch * a->s2 > INT32_MAX)
+        return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 query-head rows or key rows");
+    if (rows > 0 && (!a->q || !a->k || !a->sparse_indices))
+        return fail(LI_ERR_INVALID_ARG, "q, k and sparse_indices are required");
+    if ((a->Dr > 0) != (a->q_rope != nullptr) || (a->Dr > 0) != (a->k_rope != nullptr))
+        return fail(LI_ERR_INVALID_ARG, "q_rope and k_rope go with Dr > 0, and only with it");
+    if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->q_rope, 16) ||
+        !aligned(a->k_rope, 16) || !aligned(a->sparse_indices, 4))
+        return fail(LI_ERR_INVALID_ARG, "q, k and the rope parts must be 16-byte aligned");
+    if (!li::attn_layout(*a, L))
+        return fail(LI_ERR_UNSUPPORTED, "G=%d with Dm=%d does not fit the kernel's shared memory",
+                    a->G, a->Dm);
+    return LI_OK;
+}
+}  // namespace
+
+li_status li_sparse_attention_workspace_size(const li_attn_args *args, size_t *bytes) {
+    li::AttnLayout L;
+    li_status st = validate_attn(args, &L);
+    if (st != LI_OK) return st;
+    if (!bytes) return fail(LI_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = 256;
+    return ok();
+}
+
+li_status li_sparse_attention(const li_attn_args *args, void *workspace, size_t workspace_bytes,
+                              float *out, float *softmax_max, float *softmax_sum, void *stream) {
+    li::AttnLayout L;
+    li_status st = validate_attn(args, &L);
+    if (st != LI_OK) return st;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < 256)
+        return fail(LI_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer of >= 256 bytes");
+    const bool rows = (int64_t)args->batch * args->s1 > 0;
+    if (rows && (!out || !softmax_max || !softmax_sum || !aligned(out, 4) ||
+                 !aligned(softmax_max, 4) || !aligned(softmax_sum, 4)))
+        return fail(LI_ERR_INVALID_ARG, "out, softmax_max and softmax_sum must be 4-byte aligned");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, 256, cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "workspace clear: %s", cudaGetErrorString(e));
+    if (!rows) return ok();
+    auto *hdr = static_cast<uint32_t *>(workspace);
+    e = li::launch_sparse_attention(*args, hdr, reinterpret_cast<int32_t *>(hdr + 1), out,
+                                    softmax_max, softmax_sum, cs);
+    if (e != cudaSuccess) return fail(LI_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

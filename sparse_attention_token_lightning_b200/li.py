@@ -68,7 +68,8 @@ _lib = None
 EXPORTS = ("li_metadata_workspace_size", "li_metadata", "li_indexer_workspace_size",
            "li_indexer", "li_check_status", "li_set_stage_events", "li_last_error_string",
            "li_abi_version", "li_indexer_noalloc", "li_plan", "li_merge_topk",
-           "li_kl_grad_workspace_size", "li_kl_grad")
+           "li_kl_grad_workspace_size", "li_kl_grad", "li_sparse_attention_workspace_size",
+           "li_sparse_attention")
 
 MERGE_MAX_LISTS = 16          # LI_MERGE_MAX_LISTS
 
@@ -84,6 +85,17 @@ class LiKlArgs(ctypes.Structure):
         ("s2", ctypes.c_int32), ("G", ctypes.c_int32), ("Dm", ctypes.c_int32),
         ("Dr", ctypes.c_int32), ("H", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+    ]
+
+
+class LiAttnArgs(ctypes.Structure):
+    """Mirror of li_attn_args (include/li.h)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_rope", ctypes.c_void_p),
+        ("k_rope", ctypes.c_void_p), ("sparse_indices", ctypes.c_void_p),
+        ("scale", ctypes.c_float), ("batch", ctypes.c_int32), ("s1", ctypes.c_int32),
+        ("s2", ctypes.c_int32), ("G", ctypes.c_int32), ("Dm", ctypes.c_int32),
+        ("Dr", ctypes.c_int32), ("topk", ctypes.c_int32), ("reserved", ctypes.c_int32),
     ]
 
 
@@ -140,6 +152,10 @@ def load(path) -> ctypes.CDLL:
     L.li_kl_grad_workspace_size.restype = ctypes.c_int
     L.li_kl_grad.argtypes = [ctypes.POINTER(LiKlArgs), vp, ctypes.c_size_t, vp, vp, vp, vp, vp]
     L.li_kl_grad.restype = ctypes.c_int
+    L.li_sparse_attention_workspace_size.argtypes = [ctypes.POINTER(LiAttnArgs), sz]
+    L.li_sparse_attention_workspace_size.restype = ctypes.c_int
+    L.li_sparse_attention.argtypes = [ctypes.POINTER(LiAttnArgs), vp, ctypes.c_size_t, vp, vp, vp, vp]
+    L.li_sparse_attention.restype = ctypes.c_int
     L.li_merge_topk.argtypes = [ctypes.POINTER(LiMergeArgs), vp]
     L.li_merge_topk.restype = ctypes.c_int
     L.li_abi_version.argtypes = []
@@ -346,6 +362,49 @@ def kl_grad(kp, stream=None, check: bool = True):
         if st != LI_OK:
             raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
     return loss, d_qi, d_ki, d_w
+
+
+def make_attn_args(ap) -> LiAttnArgs:
+    """li_attn_args of a device-resident attention problem (q, k, q_rope, k_rope,
+    sparse_indices, scale: synthetic.AttnProblem or synthetic.KLProblem)."""
+    a = LiAttnArgs()
+    B, S1, G, Dm = ap.q.shape
+    a.q, a.k = ap.q.data_ptr(), ap.k.data_ptr()
+    a.q_rope, a.k_rope = _ptr(ap.q_rope), _ptr(ap.k_rope)
+    a.sparse_indices = ap.sparse_indices.data_ptr()
+    a.scale = float(ap.scale)
+    a.batch, a.s1, a.s2 = B, S1, ap.k.shape[1]
+    a.G, a.Dm, a.Dr = G, Dm, 0 if ap.q_rope is None else ap.q_rope.shape[-1]
+    a.topk = ap.sparse_indices.shape[-1]
+    return a
+
+
+def li_sparse_attention(args: LiAttnArgs, workspace: torch.Tensor, out: torch.Tensor,
+                        softmax_max: torch.Tensor, softmax_sum: torch.Tensor, stream=None):
+    _check(lib().li_sparse_attention(ctypes.byref(args), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), out.data_ptr(),
+                                     softmax_max.data_ptr(), softmax_sum.data_ptr(),
+                                     _stream_handle(stream)))
+
+
+def sparse_attention(ap, stream=None, check: bool = True):
+    """Attention of every row over its selected keys (values = keys) on a device-resident
+    problem: returns (out (B,S1,G,Dm), softmax_max (B,1,S1,G), softmax_sum (B,1,S1,G)), fp32."""
+    a = make_attn_args(ap)
+    n = ctypes.c_size_t(0)
+    _check(lib().li_sparse_attention_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    dev = ap.q.device
+    B, S1, G, Dm = ap.q.shape
+    ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    out = torch.empty((B, S1, G, Dm), dtype=torch.float32, device=dev)
+    smax = torch.empty((B, 1, S1, G), dtype=torch.float32, device=dev)
+    ssum = torch.empty((B, 1, S1, G), dtype=torch.float32, device=dev)
+    li_sparse_attention(a, ws, out, smax, ssum, stream)
+    if check:
+        st, bits = li_check_status(ws, stream)
+        if st != LI_OK:
+            raise LiError(st, f"{li_last_error_string()} (device bits 0x{bits:x})")
+    return out, smax, ssum
 
 
 class HostPipeline:

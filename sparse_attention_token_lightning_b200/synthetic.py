@@ -398,3 +398,77 @@ def kl_rows(kp: KLProblem, a: int, b: int) -> KLProblem:
                       sparse_indices=sl(kp.sparse_indices), key_base=kp.key_base[a:b].contiguous(),
                       softmax_max=kp.softmax_max[:, :, a:b].contiguous(),
                       softmax_sum=kp.softmax_sum[:, :, a:b].contiguous())
+
+
+# ---- sparse attention over the selected keys ------------------------------------------------------
+
+@dataclass
+class AttnProblem:
+    """Inputs of the attention over each row's selected keys (values = keys): the main attention's
+    query and key (one key head, optional rope parts) and the selected keys of every row
+    (positions in the row's batch, -1 = none)."""
+
+    name: str
+    q: torch.Tensor                 # (B, S1, G, Dm)
+    k: torch.Tensor                 # (B, S2, 1, Dm)
+    q_rope: Optional[torch.Tensor]  # (B, S1, G, Dr) or None
+    k_rope: Optional[torch.Tensor]  # (B, S2, 1, Dr) or None
+    sparse_indices: torch.Tensor    # (B, S1, 1, topk) int32
+    key_base: torch.Tensor          # (B * S1,) int64: key row of position 0 of the row's batch
+    scale: float
+
+    TENSORS = ("q", "k", "q_rope", "k_rope", "sparse_indices", "key_base")
+
+    def to(self, device) -> "AttnProblem":
+        kw = {f: (None if getattr(self, f) is None else getattr(self, f).to(device))
+              for f in self.TENSORS}
+        return dataclasses.replace(self, **kw)
+
+    def replace(self, **kw) -> "AttnProblem":
+        return dataclasses.replace(self, **kw)
+
+    def rows(self, rows) -> "AttnProblem":
+        """The same problem restricted to the given global query rows (all keys kept), as one
+        batch of len(rows) rows; key_base keeps each row's batch."""
+        B, S1 = self.q.shape[:2]
+        r = torch.as_tensor(rows, dtype=torch.int64)
+        take = lambda t: None if t is None else t.reshape(B * S1, *t.shape[2:])[r].unsqueeze(0)
+        return self.replace(q=take(self.q), q_rope=take(self.q_rope),
+                            sparse_indices=take(self.sparse_indices),
+                            key_base=self.key_base[r].contiguous())
+
+
+def attn_bsnd(B, S1, S2, G, Dm, Dr, topk, seed=0, causal=True, scale=None, name="attn",
+              dtype=torch.bfloat16) -> AttnProblem:
+    """q, k (and rope parts) N(0, 1) rounded to `dtype`. Row i of a batch selects
+    min(topk, window) distinct keys of its window at random (causal: keys 0..i + S2 - S1; else
+    all S2 keys), listed in random order and followed by -1 padding, as the indexer's output
+    would be; scale = 1 / sqrt(Dm + Dr) unless given."""
+    g = _gen(seed)
+    q = torch.randn(B, S1, G, Dm, generator=g).to(dtype)
+    k = torch.randn(B, S2, 1, Dm, generator=g).to(dtype)
+    q_rope = torch.randn(B, S1, G, Dr, generator=g).to(dtype) if Dr else None
+    k_rope = torch.randn(B, S2, 1, Dr, generator=g).to(dtype) if Dr else None
+    # random keys of each row's window: the first topk of a random score over the window
+    u = torch.rand(B, S1, S2, generator=g)
+    if causal:
+        i = torch.arange(S1).view(1, S1, 1)
+        j = torch.arange(S2).view(1, 1, S2)
+        u = torch.where(j <= i + (S2 - S1), u, torch.full_like(u, -1.0))
+    kk = min(topk, S2)
+    val, idx = torch.topk(u, kk, dim=-1)
+    idx = torch.where(val >= 0, idx, torch.full_like(idx, -1)).to(torch.int32)
+    sel = torch.full((B, S1, 1, topk), -1, dtype=torch.int32)
+    sel[:, :, 0, :kk] = idx
+    key_base = (torch.arange(B, dtype=torch.int64) * S2).repeat_interleave(S1)
+    return AttnProblem(name=name, q=q, k=k, q_rope=q_rope, k_rope=k_rope, sparse_indices=sel,
+                       key_base=key_base,
+                       scale=float(scale) if scale is not None else 1.0 / math.sqrt(Dm + Dr))
+
+
+def attn_config(name: str, seed: int = 0) -> AttnProblem:
+    if name == "sparse_attention":
+        # the causal prefill's selection shape (4096 rows, 2048 keys each once the window allows)
+        # consumed by a 16-head main attention of 512 + 64 dims
+        return attn_bsnd(1, 4096, 4096, 16, 512, 64, 2048, seed=seed, name=name)
+    raise KeyError(name)

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert li.li_abi_version() == 4
+    assert li.li_abi_version() == 5
 
 
 @pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
@@ -273,3 +273,33 @@ def test_plan_reports_schedule_and_kernel_count(L):
     a = _args(num_heads_q=0)
     assert L.li_plan(ctypes.byref(a), ctypes.byref(li.LiPlanInfo())) == 1
     assert L.li_plan(ctypes.byref(_args()), None) == 1
+
+
+def _attn_args(**kw):
+    a = li.LiAttnArgs()
+    a.q, a.k, a.sparse_indices = 0x10000, 0x20000, 0x30000
+    a.scale, a.batch, a.s1, a.s2 = 0.04, 2, 64, 64
+    a.G, a.Dm, a.Dr, a.topk = 16, 512, 0, 32
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw", [
+    dict(G=0), dict(G=33), dict(Dm=64), dict(Dm=576), dict(Dm=200), dict(Dr=32),
+    dict(Dr=64), dict(q_rope=0x40000, k_rope=0x50000), dict(topk=0), dict(topk=8193),
+    dict(scale=0.0), dict(scale=float("inf")), dict(reserved=1), dict(batch=-1), dict(s2=0),
+    dict(q=None), dict(sparse_indices=None), dict(q=0x10008), dict(sparse_indices=0x30002)])
+def test_invalid_attention_args_rejected_on_host(L, kw):
+    n = ctypes.c_size_t(0)
+    assert L.li_sparse_attention_workspace_size(ctypes.byref(_attn_args(**kw)), ctypes.byref(n)) == 1
+    assert li.li_last_error_string()
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(Dr=64, q_rope=0x40000, k_rope=0x50000),
+                                dict(G=32, Dm=512, Dr=64, q_rope=0x40000, k_rope=0x50000),
+                                dict(G=1, Dm=128), dict(batch=0, s2=0)])
+def test_attention_args_accepted(L, kw):
+    n = ctypes.c_size_t(0)
+    assert L.li_sparse_attention_workspace_size(ctypes.byref(_attn_args(**kw)), ctypes.byref(n)) == 0
+    assert n.value == 256

@@ -13,7 +13,7 @@ from sparse_attention_token_lightning_b200 import li
 
 ROOT = Path(__file__).resolve().parents[1]
 MIRRORS = {"li_args": li.LiArgs, "li_plan_info": li.LiPlanInfo, "li_merge_args": li.LiMergeArgs,
-           "li_kl_args": li.LiKlArgs}
+           "li_kl_args": li.LiKlArgs, "li_attn_args": li.LiAttnArgs}
 
 
 @pytest.fixture(scope="module")
