@@ -12,22 +12,29 @@
 // backward). A row with no selected key gets o = 0, m = -inf, l = 0.
 //
 // One persistent CTA per SM takes query rows from a ticket counter. Per row the selected keys are
-// processed in tiles of 128:
-//   warp 4      scheduler: takes a ticket, finds the row's last selected position (the tile
+// processed in tiles of 64:
+//   warp 8      scheduler: takes a ticket, finds the row's last selected position (the tile
 //               count), publishes the row, and loads the row's Q tile (all heads, Dm + Dr dims)
 //               with TMA into a 128-byte swizzled buffer
-//   warps 6-9   gather: each tile's 128 key rows are copied with cp.async (16 bytes per thread and
+//   warps 11-14 gather: each tile's 64 key rows are copied with cp.async (16 bytes per thread and
 //               copy, eight threads per 128-byte segment) into 128-byte swizzled chunks of 64 dims;
-//               two chunks form a 32 KB pair slot, the rope dims a 16 KB rope slot
-//   warp 5      allocates TMEM; one thread issues tcgen05.mma:
-//                 S[key, g]  = sum over chunks  K_chunk . Q_chunk^T   (keys on M = 128, heads on N)
-//                 O^T[d, g] += V^T . P^T       per pair of chunks (dims on M, keys on K; the key
-//                                              tile is read MN-major, P from shared memory)
-//   warps 0-3   softmax (thread = key = TMEM lane): S from TMEM, per-head tile max over the 128
-//               keys, an online softmax against a reference max that moves only when the tile max
-//               exceeds it by more than ln(256) (so every p <= 256; O and the sums are rescaled
-//               then), p to shared memory as bf16 for the MMA, fp32 sums kept per thread; at the
-//               end of the row the output rows O / l and the statistics
+//               two chunks form a 16 KB pair slot, the rope dims an 8 KB rope slot; one barrier
+//               per tile signals its arrival
+//   warp 9      allocates TMEM; one thread issues the scores S = sum over chunks K_chunk Q_chunk^T
+//               (keys on M = 64, heads on N; row m of S sits in TMEM lane m % 16 + 32 (m / 16))
+//   warp 10     one thread issues the values O_g^T += V^T P^T per pair of chunks (dims on M = 128,
+//               keys on K; the key tile read MN-major, P from shared memory); a tcgen05.mma
+//               costs about the same to issue whatever its N, so the two products are issued
+//               from two threads
+//   warps 0-7   softmax, two groups of four warps: group g takes the row's tiles j = g, g + 2, ...
+//               with its own S and P buffers, its own O accumulator and its own online softmax,
+//               so the two groups work on consecutive tiles at once; lanes 0-15 of a warp hold
+//               the first half of a key's heads, lanes 16-31 the second half. The reference max
+//               of a group moves only when a tile max exceeds it by more than ln(256) (so every
+//               p <= 256; O and the sums are rescaled then); p goes to shared memory as bf16 for
+//               the MMA and the sums stay in fp32. At the end of the row group 1 hands its
+//               statistics to group 0, which combines the two partial outputs and writes the
+//               output rows and the statistics.
 // Every wait is bounded in time; on expiry the kernel records LI_DEVERR_TIMEOUT and returns.
 #include <cuda_bf16.h>
 
@@ -40,14 +47,19 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kKeys = 128;                          // keys per tile (MMA M of S = K Q^T)
-constexpr uint32_t kChunk = kKeys * 128;            // 64 dims of 128 keys: 16 KB
-constexpr uint32_t kPair = 2 * kChunk;              // 128 dims: 32 KB
-constexpr int kSoftWarps = 4, kSchedWarp = 4, kMmaWarp = 5, kGatherWarp0 = 6, kGatherWarps = 4;
-constexpr int kThreads = 32 * 10;
+constexpr int kKeys = 64;                           // keys per tile (MMA M of S = K Q^T)
+constexpr uint32_t kChunk = kKeys * 128;            // 64 dims of 64 keys: 8 KB
+constexpr uint32_t kPair = 2 * kChunk;              // 128 dims: 16 KB
+// warps 0-7 softmax (group = warp / 4 takes the row's tiles j with j % 2 == group; quarter =
+// warp % 4), 8 scheduler, 9 scores MMA (and TMEM), 10 values MMA, 11-14 gather
+constexpr int kSoftWarps = 8, kSchedWarp = 8, kQkWarp = 9, kPvWarp = 10, kGatherWarp0 = 11;
+constexpr int kGatherWarps = 4;
+constexpr int kThreads = 32 * 15;
 constexpr int kGatherThreads = 32 * kGatherWarps;
+constexpr int kGroupThreads = 128;
 constexpr uint32_t kSmemBytes = 232448;
-constexpr int kMaxPairSlots = 8, kMaxRopeSlots = 2;
+constexpr int kMaxPairSlots = 16, kMaxRopeSlots = 2, kTileRing = 8;
+constexpr int kMaxHeads = 32;
 constexpr float kLog2e = 1.4426950408889634f;
 // the reference max moves when a tile max exceeds it by more than this (natural log units):
 // every p = exp(x - ref) stays <= 256
@@ -63,36 +75,36 @@ struct RowSlot {
 // Barrier layout in the shared-memory tail.
 struct Bars {
     uint32_t base;
-    __device__ uint32_t rs_full(int i) const { return base + 8 * (0 + i); }
-    __device__ uint32_t rs_empty(int i) const { return base + 8 * (2 + i); }
-    __device__ uint32_t q_full(int i) const { return base + 8 * (4 + i); }
-    __device__ uint32_t q_empty(int i) const { return base + 8 * (6 + i); }
-    __device__ uint32_t s_full(int i) const { return base + 8 * (8 + i); }
-    __device__ uint32_t s_empty(int i) const { return base + 8 * (10 + i); }
-    __device__ uint32_t p_full(int i) const { return base + 8 * (12 + i); }
-    __device__ uint32_t p_empty(int i) const { return base + 8 * (14 + i); }
-    __device__ uint32_t o_done() const { return base + 8 * 16; }
-    __device__ uint32_t o_full() const { return base + 8 * 17; }
-    __device__ uint32_t o_empty() const { return base + 8 * 18; }
-    __device__ uint32_t pair_full(int i) const { return base + 8 * (19 + i); }
-    __device__ uint32_t pair_empty(int i) const { return base + 8 * (19 + kMaxPairSlots + i); }
-    __device__ uint32_t rope_full(int i) const { return base + 8 * (19 + 2 * kMaxPairSlots + i); }
-    __device__ uint32_t rope_empty(int i) const {
-        return base + 8 * (19 + 2 * kMaxPairSlots + kMaxRopeSlots + i);
-    }
-    // exchange of the softmax warps' per-head partial results (tile max, row sums)
-    __device__ uint32_t red_full(int i) const { return base + 8 * (19 + 2 * kMaxPairSlots + 2 * kMaxRopeSlots + i); }
-    __device__ uint32_t sum_full(int i) const { return base + 8 * (21 + 2 * kMaxPairSlots + 2 * kMaxRopeSlots + i); }
+    __device__ uint32_t at(int i) const { return base + 8 * i; }
+    __device__ uint32_t rs_full(int i) const { return at(0 + i); }
+    __device__ uint32_t rs_empty(int i) const { return at(2 + i); }
+    __device__ uint32_t q_full(int i) const { return at(4 + i); }
+    __device__ uint32_t q_empty(int i) const { return at(6 + i); }
+    __device__ uint32_t s_full(int g) const { return at(8 + g); }          // per softmax group
+    __device__ uint32_t s_empty(int g) const { return at(10 + g); }
+    __device__ uint32_t p_full(int g) const { return at(12 + g); }
+    __device__ uint32_t p_empty(int g) const { return at(14 + g); }
+    __device__ uint32_t o_done(int g) const { return at(16 + g); }
+    __device__ uint32_t o_full() const { return at(18); }
+    __device__ uint32_t o_empty() const { return at(19); }
+    __device__ uint32_t stat_full(int i) const { return at(20 + i); }
+    __device__ uint32_t stat_empty(int i) const { return at(22 + i); }
+    __device__ uint32_t red_full(int g, int b) const { return at(24 + 2 * g + b); }
+    __device__ uint32_t sum_full(int g, int b) const { return at(28 + 2 * g + b); }
+    __device__ uint32_t tile_full(int i) const { return at(32 + i); }
+    __device__ uint32_t rope_empty(int i) const { return at(32 + kTileRing + i); }
+    __device__ uint32_t pair_empty(int i) const { return at(32 + kTileRing + kMaxRopeSlots + i); }
 };
-constexpr int kNumBars = 23 + 2 * kMaxPairSlots + 2 * kMaxRopeSlots;
-// tail: barriers | row slots | max and sum exchange, [2][4 warps][32] floats each | TMEM slot,
-// abort flag
-constexpr uint32_t kTailBytes = 3072;
+constexpr int kNumBars = 32 + kTileRing + kMaxRopeSlots + kMaxPairSlots;
+// tail: barriers | row slots | per group: tile-max and row-sum exchange [2 groups][2][32 heads]
+// [4 warps] floats | group-1 statistics [2][3][32] | TMEM slot, abort flag
+constexpr uint32_t kTailBytes = 6144;
 constexpr uint32_t kTailOff = kSmemBytes - kTailBytes;
 constexpr uint32_t kRowSlotOff = kTailOff + 8 * kNumBars;
 constexpr uint32_t kRedOff = (kRowSlotOff + 2 * sizeof(RowSlot) + 15) / 16 * 16;
-constexpr uint32_t kSumOff = kRedOff + 2 * 4 * 32 * 4;
-constexpr uint32_t kFlagOff = kSumOff + 2 * 4 * 32 * 4;
+constexpr uint32_t kSumOff = kRedOff + 2 * 2 * kMaxHeads * 4 * 4;
+constexpr uint32_t kStatOff = kSumOff + 2 * 2 * kMaxHeads * 4 * 4;
+constexpr uint32_t kFlagOff = kStatOff + 2 * 3 * kMaxHeads * 4;
 static_assert(kFlagOff + 16 <= kSmemBytes, "shared memory tail");
 static_assert(kTailOff % 1024 == 0, "tail alignment");
 
@@ -127,6 +139,11 @@ __device__ __forceinline__ bool wait_(uint32_t bar, uint32_t parity, volatile in
 // complete and one that gave up on the abort flag at the same moment agree on giving up).
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+// TMEM columns: S of group g at g N; O of group g, pair b at 2 N + (g npairs + b) N.
+__device__ __forceinline__ uint32_t o_col(const AttnParams &P, int g, int b) {
+    return (uint32_t)(2 * P.N + (g * P.npairs + b) * P.N);
 }
 
 // ---- scheduler: rows and their Q tiles --------------------------------------------------------
@@ -188,11 +205,11 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
                             volatile int *abort_flag) {
     const int t = threadIdx.x - 32 * kGatherWarp0;      // 0..127
     const int lane = t & 31;
-    const int key0 = t >> 3, piece = t & 7;              // keys key0 + 16 i, 16-byte piece
+    const int key0 = t >> 3, piece = t & 7;              // keys key0 + 16 i (i < 4), 16-byte piece
     const uint32_t sbase = smem_u32(smem);
     const uint32_t swz = (uint32_t)((piece ^ (key0 & 7)) << 4);   // (key0 + 16 i) & 7 == key0 & 7
     const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
-    Ring pr, rr;
+    Ring pr, rr, tr;
     uint32_t err = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -204,11 +221,11 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
         if (lane == 0) mbar_arrive(bars.rs_empty(sl));
         if (row < 0) break;
         const int32_t *ir = P.indices + (int64_t)row * P.topk;
-        for (int j = 0; j < tiles && ok; ++j) {
-            const uint16_t *krow[8];
-            const uint16_t *rrow[8];
+        for (int j = 0; j < tiles && ok; ++j, tr.next(kTileRing)) {
+            const uint16_t *krow[4];
+            const uint16_t *rrow[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const int pos = kKeys * j + key0 + 16 * i;
                 const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
                 if (v >= P.s2) err |= LI_DEVERR_LENGTHS;
@@ -223,19 +240,19 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
+                    for (int i = 0; i < 4; ++i)
                         cp_async16(base + h * kChunk + i * 16u * 128u, krow[i] + 64 * (2 * b + h));
-                cp_async_arrive(bars.pair_full(pr.idx));
             }
             if (!ok) break;
             if (P.Dr > 0) {
                 if (!wait_warp(bars.rope_empty(rr.idx), rr.phase ^ 1u, abort_flag)) { ok = false; break; }
                 const uint32_t base = sbase + P.rope_off + rr.idx * kChunk + key0 * 128u + swz;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) cp_async16(base + i * 16u * 128u, rrow[i]);
-                cp_async_arrive(bars.rope_full(rr.idx));
+                for (int i = 0; i < 4; ++i) cp_async16(base + i * 16u * 128u, rrow[i]);
                 rr.next(P.rope_slots);
             }
+            // one arrival per thread once every copy of the tile has landed
+            cp_async_arrive(bars.tile_full(tr.idx));
         }
     }
     // no copy may still be writing shared memory when the CTA leaves
@@ -244,15 +261,70 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
     if (err) atomicOr(P.status, err);
 }
 
-// ---- MMA issuer ----------------------------------------------------------------------------
-__device__ void mma_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
-                         volatile int *abort_flag, uint32_t tmem) {
+// ---- scores MMA: S(j) = K(j) Q^T into the S buffer of tile j's softmax group -------------------
+__device__ void qk_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
+                        volatile int *abort_flag, uint32_t tmem) {
     const uint32_t sbase = smem_u32(smem);
     const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
     const uint32_t N = (uint32_t)P.N;
-    const uint32_t cb = N * 128u;                        // one Q chunk / one P atom column
-    Ring qr, pr, rr, sr;
-    uint32_t tile = 0, nrow = 0;
+    const uint32_t cb = N * 128u;
+    Ring qr, pq, rr, tr;
+    uint32_t kg[2] = {0u, 0u};                           // tiles of each group so far
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+        const int sl = it & 1;
+        if (!wait_(bars.rs_full(sl), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int row = slots[sl].row, tiles = slots[sl].tiles;
+        mbar_arrive(bars.rs_empty(sl));
+        if (row < 0) break;
+        if (tiles == 0) continue;
+        if (!wait_(bars.q_full(qr.idx), qr.phase, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qa = sbase + P.q_off + qr.idx * P.q_bytes;
+        for (int j = 0; j < tiles; ++j, tr.next(kTileRing)) {
+            const int g = j & 1;
+            if (!wait_(bars.s_empty(g), (kg[g] & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            if (!wait_(bars.tile_full(tr.idx), tr.phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_s = tmem + g * N;
+            for (int b = 0; b < P.npairs; ++b, pq.next(P.pair_slots)) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint64_t a = sw128_desc(sbase + P.pair_off + pq.idx * kPair + h * kChunk);
+                    const uint64_t bq = sw128_desc(qa + (2 * b + h) * cb);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(d_s, a + 2 * kk, bq + 2 * kk, P.idesc_qk, (b | h | kk) != 0);
+                }
+            }
+            if (P.Dr > 0) {
+                const uint64_t a = sw128_desc(sbase + P.rope_off + rr.idx * kChunk);
+                const uint64_t bq = sw128_desc(qa + 2 * P.npairs * cb);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) umma_f16(d_s, a + 2 * kk, bq + 2 * kk, P.idesc_qk, 1u);
+                umma_commit(bars.rope_empty(rr.idx));
+                rr.next(P.rope_slots);
+            }
+            umma_commit(bars.s_full(g));
+            ++kg[g];
+        }
+        if (!ok) break;
+        umma_commit(bars.q_empty(qr.idx));
+        qr.next(P.q_bufs);
+    }
+    if (!ok) *abort_flag = 1;
+}
+
+// ---- values MMA: O_g^T += V(j)^T P(j)^T for tile j of group g --------------------------------
+__device__ void pv_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
+                        volatile int *abort_flag, uint32_t tmem) {
+    const uint32_t sbase = smem_u32(smem);
+    const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
+    const uint32_t N = (uint32_t)P.N;
+    const uint32_t cb = N * 128u;
+    Ring pv;
+    uint32_t kg[2] = {0u, 0u};
+    uint32_t nrow = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it & 1;
@@ -261,99 +333,62 @@ __device__ void mma_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
         mbar_arrive(bars.rs_empty(sl));
         if (row < 0) break;
         const uint32_t this_row = nrow++;
-        if (tiles > 0) {
-            if (!wait_(bars.q_full(qr.idx), qr.phase, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t qa = sbase + P.q_off + qr.idx * P.q_bytes;
-            for (int j = 0; j < tiles; ++j, ++tile, sr.next(2)) {
-                if (!wait_(bars.s_empty(sr.idx), sr.phase ^ 1u, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_s = tmem + sr.idx * N;
-                Ring p0 = pr;
-                for (int b = 0; b < P.npairs; ++b, p0.next(P.pair_slots)) {
-                    if (!wait_(bars.pair_full(p0.idx), p0.phase, abort_flag)) { ok = false; break; }
-                    fence_async_smem();
-                    tc_fence_after();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint64_t a = sw128_desc(sbase + P.pair_off + p0.idx * kPair + h * kChunk);
-                        const uint64_t bq = sw128_desc(qa + (2 * b + h) * cb);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_f16(d_s, a + 2 * kk, bq + 2 * kk, P.idesc_qk, (b | h | kk) != 0);
-                    }
-                }
-                if (!ok) break;
-                if (P.Dr > 0) {
-                    if (!wait_(bars.rope_full(rr.idx), rr.phase, abort_flag)) { ok = false; break; }
-                    fence_async_smem();
-                    tc_fence_after();
-                    const uint64_t a = sw128_desc(sbase + P.rope_off + rr.idx * kChunk);
-                    const uint64_t bq = sw128_desc(qa + 2 * P.npairs * cb);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) umma_f16(d_s, a + 2 * kk, bq + 2 * kk, P.idesc_qk, 1u);
-                    umma_commit(bars.rope_empty(rr.idx));
-                    rr.next(P.rope_slots);
-                }
-                umma_commit(bars.s_full(sr.idx));
-                // O is overwritten by the row's first tile: the previous row's output must have been
-                // read out of TMEM (one o_empty phase per row, completed in order)
-                if (j == 0 && this_row > 0 &&
-                    !wait_(bars.o_empty(), (this_row - 1) & 1u, abort_flag)) { ok = false; break; }
-                // P of this tile, then O^T += V^T P^T pair by pair
-                if (!wait_(bars.p_full(sr.idx), sr.phase, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t pa = sbase + P.p_off + sr.idx * 2u * cb;
-                for (int b = 0; b < P.npairs; ++b, pr.next(P.pair_slots)) {
-                    const uint32_t va = sbase + P.pair_off + pr.idx * kPair;
-                    const uint32_t d_o = tmem + 2u * N + b * N;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t a = sw128_desc_mn(va + kk * 16u * 128u, kChunk);
-                        const uint64_t bp = sw128_desc(pa + (kk >> 2) * cb) + 2 * (kk & 3);
-                        umma_f16(d_o, a, bp, P.idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(bars.pair_empty(pr.idx));
-                }
-                umma_commit(bars.p_empty(sr.idx));
-                umma_commit(bars.o_done());
+        for (int j = 0; j < tiles; ++j) {
+            const int g = j & 1;
+            // both groups' O are overwritten by the row's first two tiles: the previous row's
+            // output must have been read out of TMEM (one o_empty phase per row, in order)
+            if (j == 0 && this_row > 0 && !wait_(bars.o_empty(), (this_row - 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
             }
-            if (!ok) break;
-            umma_commit(bars.q_empty(qr.idx));
-            qr.next(P.q_bufs);
+            if (!wait_(bars.p_full(g), kg[g] & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t pa = sbase + P.p_off + g * cb;
+            for (int b = 0; b < P.npairs; ++b, pv.next(P.pair_slots)) {
+                const uint32_t va = sbase + P.pair_off + pv.idx * kPair;
+                const uint32_t d_o = tmem + o_col(P, g, b);
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    const uint64_t a = sw128_desc_mn(va + kk * 16u * 128u, kChunk);
+                    umma_f16(d_o, a, sw128_desc(pa) + 2 * kk, P.idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bars.pair_empty(pv.idx));
+            }
+            umma_commit(bars.p_empty(g));
+            umma_commit(bars.o_done(g));
+            ++kg[g];
         }
+        if (!ok) break;
         umma_commit(bars.o_full());
     }
     if (!ok) *abort_flag = 1;
 }
 
 // ---- softmax and output ----------------------------------------------------------------------
-// Per-head reduction of NH values over the 32 lanes of a warp, transposed: afterwards lane l
-// holds the result for head head_of_lane<NH>(l) (lanes l and l ^ 1 share a head when NH = 16).
-template <int NH>
-__device__ __forceinline__ int head_of_lane(int lane) {
-    // the halving steps keep the upper half on lanes whose bit (16, 8, 4, 2[, 1]) is set
-    if constexpr (NH == 32)
-        return ((lane >> 4) & 1) * 16 + ((lane >> 3) & 1) * 8 + ((lane >> 2) & 1) * 4 +
-               ((lane >> 1) & 1) * 2 + (lane & 1);
+// Per-head reduction of HH values over the 16 lanes of a half-warp, transposed: afterwards lane l
+// holds the result for head (l >> 4) * HH + half_head<HH>(l) (with HH = 8, lanes l and l ^ 1
+// share a head).
+template <int HH>
+__device__ __forceinline__ int half_head(int lane) {
+    if constexpr (HH == 16)
+        return ((lane >> 3) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 1) & 1) * 2 + (lane & 1);
     else
-        return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-               ((lane >> 1) & 1);
+        return ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
-template <int NH, bool kMax>
-__device__ __forceinline__ float warp_reduce_heads(const float (&v)[NH], int lane) {
-    float a[NH];
+template <int HH, bool kMax>
+__device__ __forceinline__ float half_reduce(const float (&v)[HH], int lane) {
+    float a[HH];
 #pragma unroll
-    for (int i = 0; i < NH; ++i) a[i] = v[i];
-    // step s halves the values held: lanes with bit (16 >> s) set keep the upper half
-    constexpr int kSteps = NH == 32 ? 5 : 4;
+    for (int i = 0; i < HH; ++i) a[i] = v[i];
+    // step s halves the values held: lanes with bit (8 >> s) set keep the upper half
+    constexpr int kSteps = HH == 16 ? 4 : 3;
 #pragma unroll
     for (int s = 0; s < kSteps; ++s) {
-        const int bit = 16 >> s;
-        const int half = NH >> (s + 1);
+        const int bit = 8 >> s;
+        const int half = HH >> (s + 1);
         const bool up = (lane & bit) != 0;
 #pragma unroll
-        for (int i = 0; i < NH / 2; ++i) {
+        for (int i = 0; i < HH / 2; ++i) {
             if (i < half) {
                 const float keep = up ? a[i + half] : a[i];
                 const float send = up ? a[i] : a[i + half];
@@ -362,26 +397,11 @@ __device__ __forceinline__ float warp_reduce_heads(const float (&v)[NH], int lan
             }
         }
     }
-    // NH = 16 leaves lane bit 0 unreduced
-    if constexpr (NH == 16) {
+    if constexpr (HH == 8) {
         const float o = __shfl_xor_sync(0xffffffffu, a[0], 1);
         a[0] = kMax ? fmaxf(a[0], o) : a[0] + o;
     }
     return a[0];
-}
-
-// S of this thread's key: NH columns of its TMEM lane.
-template <int NH>
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[NH]) {
-    float a[16];
-    tmem_ld16(taddr, a);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = a[i];
-    if constexpr (NH == 32) {
-        tmem_ld16(taddr + 16, a);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 + i] = a[i];
-    }
 }
 
 // bf16 bits of x, round to nearest even (x is finite and non-negative here)
@@ -389,26 +409,35 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// Softmax group g (warps 4 g .. 4 g + 3) over the row's tiles j = g, g + 2, ...: each thread owns
+// key 16 q + (lane % 16) of the tile (q = warp % 4, the TMEM lanes of M = 64 scores) and heads
+// (lane / 16) HH .. + HH - 1 of it. Group 1 hands its statistics to group 0, which combines the
+// two partial outputs and writes the row.
 template <int NH>
 __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
                              volatile int *abort_flag, uint32_t tmem) {
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int key = 32 * w + lane;                        // TMEM lane: key of the tile / dim of O
-    const uint32_t lane_addr = (uint32_t)(32 * w) << 16;
+    constexpr int HH = NH / 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = warp >> 2, q = warp & 3;
+    const int key = 16 * q + (lane & 15);
+    const int half = lane >> 4;
+    const int hb = half * HH;
+    const int dlane = 32 * q + lane;                     // dim of a 128-dim block of O
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const uint32_t N = (uint32_t)P.N;
     const uint32_t cb = N * 128u;
-    const uint32_t sbase = smem_u32(smem);
     const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
-    float *red = reinterpret_cast<float *>(smem + kRedOff);      // [2][4 warps][32]
-    float *sumx = reinterpret_cast<float *>(smem + kSumOff);     // [2][4 warps][32]
+    float *red = reinterpret_cast<float *>(smem + kRedOff) + g * 2 * kMaxHeads * 4;
+    float *sumx = reinterpret_cast<float *>(smem + kSumOff) + g * 2 * kMaxHeads * 4;
+    float *stat = reinterpret_cast<float *>(smem + kStatOff);    // [2][3][kMaxHeads]
     const float kInf = __int_as_float(0x7f800000);
-    const int my_head = head_of_lane<NH>(lane);
-    // P element (head h, this key) in the K-major 128-byte swizzled tile: atom column key / 64,
-    // row h, 16-byte chunk ((key % 64) / 8) ^ (h % 8)
-    const uint32_t p_key = (uint32_t)(key >> 6) * cb + (uint32_t)((key & 7) << 1);
-    const uint32_t p_chunk = (uint32_t)((key & 63) >> 3);
-    Ring sr;
-    uint32_t tile = 0, nrow = 0;
+    const int my_head = hb + half_head<HH>(lane);
+    const bool writer = HH == 16 || (lane & 1) == 0;
+    // P element (head h, this key) in the K-major 128-byte swizzled tile of N rows x 64 keys:
+    // row h, 16-byte chunk (key / 8) ^ (h % 8)
+    const uint32_t p_key = (uint32_t)((key & 7) << 1);
+    const uint32_t p_chunk = (uint32_t)(key >> 3);
+    uint32_t kg = 0, nrow = 0;                           // this group's tiles, rows
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it & 1;
@@ -418,54 +447,75 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
         if (lane == 0) mbar_arrive(bars.rs_empty(sl));
         if (row < 0) break;
         const int32_t *ir = P.indices + (int64_t)row * P.topk;
-        float m_ref[NH], m_true[NH], l_part[NH];
+        float m_ref[NH], m_true[NH], l_part[HH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) { m_ref[h] = -kInf; m_true[h] = -kInf; l_part[h] = 0.f; }
-        for (int j = 0; j < tiles; ++j, ++tile, sr.next(2)) {
+        for (int h = 0; h < NH; ++h) { m_ref[h] = -kInf; m_true[h] = -kInf; }
+#pragma unroll
+        for (int i = 0; i < HH; ++i) l_part[i] = 0.f;
+        int mine = 0;                                    // tiles of this group in the row
+        for (int j = g; j < tiles; j += 2, ++kg, ++mine) {
             const int pos = kKeys * j + key;
             const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
             const bool valid = v >= 0 && v < P.s2;
-            if (!wait_warp(bars.s_full(sr.idx), sr.phase, abort_flag)) { ok = false; break; }
+            if (!wait_warp(bars.s_full(g), kg & 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            float x[NH];
-            tmem_ld_row<NH>(tmem + lane_addr + sr.idx * N, x);
+            float x[16];
+            float y[HH];
+            tmem_ld16(tmem + lane_addr + g * N, x);      // lanes 0-15: heads 0-15 of the key
+            if constexpr (NH == 16) {
+#pragma unroll
+                for (int i = 0; i < HH; ++i) {
+                    const float up = __shfl_sync(0xffffffffu, x[HH + i], lane & 15);
+                    y[i] = half ? up : x[i];
+                }
+            } else {
+                float x2[16];
+                tmem_ld16(tmem + lane_addr + g * N + 16, x2);
+#pragma unroll
+                for (int i = 0; i < HH; ++i) {
+                    const float up = __shfl_sync(0xffffffffu, x2[i], lane & 15);
+                    y[i] = half ? up : x[i];
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars.s_empty(sr.idx));
+            if (lane == 0) mbar_arrive(bars.s_empty(g));
 #pragma unroll
-            for (int h = 0; h < NH; ++h) x[h] = valid ? x[h] * P.scale : -kInf;
-            // tile max per head over the 128 keys
-            float *rb = red + (tile & 1) * 4 * 32;
-            const float wm = warp_reduce_heads<NH, true>(x, lane);
-            if (NH == 32 || (lane & 1) == 0) rb[w * 32 + my_head] = wm;
-            mbar_arrive(bars.red_full(tile & 1));
-            if (!wait_warp(bars.red_full(tile & 1), (tile >> 1) & 1u, abort_flag)) { ok = false; break; }
+            for (int i = 0; i < HH; ++i) y[i] = valid ? y[i] * P.scale : -kInf;
+            // tile max per head over the group's 64 keys
+            float *rb = red + (kg & 1) * kMaxHeads * 4;
+            const float wm = half_reduce<HH, true>(y, lane);
+            if (writer) rb[my_head * 4 + q] = wm;
+            mbar_arrive(bars.red_full(g, kg & 1));
+            if (!wait_warp(bars.red_full(g, kg & 1), (kg >> 1) & 1u, abort_flag)) { ok = false; break; }
             bool rescale = false;
             float alpha[NH];
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
-                const float tm = fmaxf(fmaxf(rb[h], rb[32 + h]), fmaxf(rb[64 + h], rb[96 + h]));
+                const float4 r4 = *reinterpret_cast<const float4 *>(rb + h * 4);
+                const float tm = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
                 m_true[h] = fmaxf(m_true[h], tm);
                 const float ref = tm - m_ref[h] > kSlack ? tm : m_ref[h];
                 alpha[h] = ref != m_ref[h] ? exp2f((m_ref[h] - ref) * kLog2e) : 1.f;
                 rescale |= ref != m_ref[h];
                 m_ref[h] = ref;
-                l_part[h] *= alpha[h];
             }
-            float p[NH];
+            float p[HH];
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                p[h] = valid ? exp2f((x[h] - m_ref[h]) * kLog2e) : 0.f;
-                l_part[h] += p[h];
+            for (int i = 0; i < HH; ++i) {
+                const float a = half ? alpha[HH + i] : alpha[i];
+                const float r = half ? m_ref[HH + i] : m_ref[i];
+                p[i] = valid ? exp2f((y[i] - r) * kLog2e) : 0.f;
+                l_part[i] = l_part[i] * a + p[i];
             }
-            // O (accumulated up to the previous tile) follows a moved reference
-            if (rescale && j > 0) {
-                if (!wait_warp(bars.o_done(), (tile - 1) & 1u, abort_flag)) { ok = false; break; }
+            // this group's O (accumulated up to its previous tile) follows a moved reference
+            if (rescale && mine > 0) {
+                if (!wait_warp(bars.o_done(g), (kg - 1) & 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int b = 0; b < P.npairs; ++b) {
 #pragma unroll
                     for (int c = 0; c < NH; c += 16) {
-                        const uint32_t ta = tmem + lane_addr + 2u * N + b * N + c;
+                        const uint32_t ta = tmem + lane_addr + o_col(P, g, b) + c;
                         float o[16];
                         tmem_ld16(ta, o);
 #pragma unroll
@@ -475,55 +525,98 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
                 }
                 tc_fence_before();
             }
-            // p as bf16 into this tile's P buffer once the MMA has finished with it
-            if (!wait_warp(bars.p_empty(sr.idx), sr.phase ^ 1u, abort_flag)) { ok = false; break; }
-            uint8_t *pb = smem + P.p_off + sr.idx * 2u * cb + p_key;
+            // p as bf16 into the group's P buffer once the MMA has finished with it
+            if (!wait_warp(bars.p_empty(g), (kg & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            {
+                uint8_t *pb = smem + P.p_off + g * cb + p_key;
 #pragma unroll
-            for (int h = 0; h < NH; ++h)
-                *reinterpret_cast<uint16_t *>(pb + (h >> 3) * 1024 + (h & 7) * 128 +
-                                              ((p_chunk ^ (uint32_t)(h & 7)) << 4)) = bf16_bits(p[h]);
+                for (int i = 0; i < HH; ++i) {
+                    const int h = hb + i;
+                    *reinterpret_cast<uint16_t *>(pb + (h >> 3) * 1024 + (h & 7) * 128 +
+                                                  ((p_chunk ^ (uint32_t)(h & 7)) << 4)) =
+                        bf16_bits(p[i]);
+                }
+            }
             fence_async_smem();
-            mbar_arrive(bars.p_full(sr.idx));
+            mbar_arrive(bars.p_full(g));
         }
         if (!ok) break;
-        // row totals of the fp32 sums (exchange buffers alternate by row)
-        float *sb = sumx + (nrow & 1) * 4 * 32;
+        // row totals of this group's fp32 sums (exchange buffers alternate by row)
+        float *sb = sumx + (nrow & 1) * kMaxHeads * 4;
         {
-            const float ws = warp_reduce_heads<NH, false>(l_part, lane);
-            if (NH == 32 || (lane & 1) == 0) sb[w * 32 + my_head] = ws;
-            mbar_arrive(bars.sum_full(nrow & 1));
-            if (!wait_warp(bars.sum_full(nrow & 1), (nrow >> 1) & 1u, abort_flag)) { ok = false; break; }
+            const float ws = half_reduce<HH, false>(l_part, lane);
+            if (writer) sb[my_head * 4 + q] = ws;
+            mbar_arrive(bars.sum_full(g, nrow & 1));
+            if (!wait_warp(bars.sum_full(g, nrow & 1), (nrow >> 1) & 1u, abort_flag)) { ok = false; break; }
         }
         float l_tot[NH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) l_tot[h] = (sb[h] + sb[32 + h]) + (sb[64 + h] + sb[96 + h]);
+        for (int h = 0; h < NH; ++h) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(sb + h * 4);
+            l_tot[h] = (s4.x + s4.y) + (s4.z + s4.w);
+        }
+        float *st = stat + (nrow & 1) * 3 * kMaxHeads;
+        if (g == 1) {
+            // hand the statistics to group 0
+            if (!wait_warp(bars.stat_empty(nrow & 1), ((nrow >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            if (warp == 4 && lane == 0) {
+                for (int h = 0; h < NH; ++h) {
+                    st[h] = m_ref[h];
+                    st[kMaxHeads + h] = m_true[h];
+                    st[2 * kMaxHeads + h] = l_tot[h];
+                }
+                mbar_arrive(bars.stat_full(nrow & 1));
+            }
+            __syncwarp();
+            ++nrow;
+            continue;
+        }
+        if (!wait_warp(bars.stat_full(nrow & 1), (nrow >> 1) & 1u, abort_flag)) { ok = false; break; }
+        // combine: c = the larger reference; weights of the two partial sums
+        const bool two = tiles >= 2;
+        float wa[NH], wb[NH], inv[NH];
+        float smx[NH], ssm[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            const float rb_ = st[h], tb = st[kMaxHeads + h], lb = st[2 * kMaxHeads + h];
+            const float c = two ? fmaxf(m_ref[h], rb_) : m_ref[h];
+            wa[h] = m_ref[h] > -kInf ? exp2f((m_ref[h] - c) * kLog2e) : 0.f;
+            wb[h] = two && rb_ > -kInf ? exp2f((rb_ - c) * kLog2e) : 0.f;
+            const float L = l_tot[h] * wa[h] + (two ? lb * wb[h] : 0.f);
+            inv[h] = L > 0.f ? 1.f / L : 0.f;
+            const float mt = two ? fmaxf(m_true[h], tb) : m_true[h];
+            smx[h] = mt;
+            ssm[h] = mt > -kInf ? L * exp2f((c - mt) * kLog2e) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.stat_empty(nrow & 1));
         if (!wait_warp(bars.o_full(), nrow & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int G = P.G;
         float *orow = P.out + (int64_t)row * G * P.Dm;
-        if (tiles > 0) {
-            for (int b = 0; b < P.npairs; ++b) {
+        for (int b = 0; b < P.npairs; ++b) {
 #pragma unroll
-                for (int c = 0; c < NH; c += 16) {
-                    float o[16];
-                    tmem_ld16(tmem + lane_addr + 2u * N + b * N + c, o);
+            for (int c = 0; c < NH; c += 16) {
+                float oa[16], ob[16];
+                if (tiles > 0) tmem_ld16(tmem + lane_addr + o_col(P, 0, b) + c, oa);
+                if (two) tmem_ld16(tmem + lane_addr + o_col(P, 1, b) + c, ob);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c + i < G)
-                            orow[(int64_t)(c + i) * P.Dm + 128 * b + key] =
-                                l_tot[c + i] > 0.f ? o[i] / l_tot[c + i] : 0.f;
+                for (int i = 0; i < 16; ++i) {
+                    const int h = c + i;
+                    if (h < G) {
+                        float o = 0.f;
+                        if (tiles > 0) o = oa[i] * wa[h];
+                        if (two) o += ob[i] * wb[h];
+                        orow[(int64_t)h * P.Dm + 128 * b + dlane] = o * inv[h];
+                    }
                 }
             }
-        } else {
-            for (int b = 0; b < P.npairs; ++b)
-                for (int h = 0; h < G; ++h) orow[(int64_t)h * P.Dm + 128 * b + key] = 0.f;
         }
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-            if (h == key && h < G) {
-                const bool any = m_true[h] > -kInf;
-                P.smax[(int64_t)row * G + h] = m_true[h];
-                P.ssum[(int64_t)row * G + h] = any ? l_tot[h] * exp2f((m_ref[h] - m_true[h]) * kLog2e) : 0.f;
+            if (h == dlane && h < G) {
+                P.smax[(int64_t)row * G + h] = smx[h];
+                P.ssum[(int64_t)row * G + h] = ssm[h];
             }
         }
         tc_fence_before();
@@ -551,29 +644,26 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.rs_full(i), 1);
-            mbar_init(bars.rs_empty(i), 1 + kSoftWarps + kGatherWarps);
+            mbar_init(bars.rs_empty(i), 2 + kSoftWarps + kGatherWarps);
             mbar_init(bars.q_full(i), 1);
             mbar_init(bars.q_empty(i), 1);
             mbar_init(bars.s_full(i), 1);
-            mbar_init(bars.s_empty(i), kSoftWarps);
-            mbar_init(bars.p_full(i), 32 * kSoftWarps);
+            mbar_init(bars.s_empty(i), 4);
+            mbar_init(bars.p_full(i), kGroupThreads);
             mbar_init(bars.p_empty(i), 1);
+            mbar_init(bars.o_done(i), 1);
+            mbar_init(bars.stat_full(i), 1);
+            mbar_init(bars.stat_empty(i), 4);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(bars.red_full(i, b), kGroupThreads);
+                mbar_init(bars.sum_full(i, b), kGroupThreads);
+            }
         }
-        mbar_init(bars.o_done(), 1);
         mbar_init(bars.o_full(), 1);
-        mbar_init(bars.o_empty(), kSoftWarps);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bars.red_full(i), 32 * kSoftWarps);
-            mbar_init(bars.sum_full(i), 32 * kSoftWarps);
-        }
-        for (int i = 0; i < kMaxPairSlots; ++i) {
-            mbar_init(bars.pair_full(i), kGatherThreads);
-            mbar_init(bars.pair_empty(i), 1);
-        }
-        for (int i = 0; i < kMaxRopeSlots; ++i) {
-            mbar_init(bars.rope_full(i), kGatherThreads);
-            mbar_init(bars.rope_empty(i), 1);
-        }
+        mbar_init(bars.o_empty(), 4);
+        for (int i = 0; i < kTileRing; ++i) mbar_init(bars.tile_full(i), kGatherThreads);
+        for (int i = 0; i < kMaxRopeSlots; ++i) mbar_init(bars.rope_empty(i), 1);
+        for (int i = 0; i < kMaxPairSlots; ++i) mbar_init(bars.pair_empty(i), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -595,7 +685,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (P.Dr > 0)
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_qr)) : "memory");
     }
-    if (warp == kMmaWarp) {
+    if (warp == kQkWarp) {
         tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
         tmem_relinquish();
     }
@@ -608,8 +698,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         softmax_role<NH>(P, smem, bars, abort_flag, tmem);
     } else if (warp == kSchedWarp) {
         scheduler_role(P, &tmap_q, &tmap_qr, smem, bars, abort_flag);
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role(P, smem, bars, abort_flag, tmem);
+    } else if (warp == kQkWarp) {
+        if (lane == 0) qk_role(P, smem, bars, abort_flag, tmem);
+        __syncwarp();
+    } else if (warp == kPvWarp) {
+        if (lane == 0) pv_role(P, smem, bars, abort_flag, tmem);
         __syncwarp();
     } else {
         gather_role(P, smem, bars, abort_flag);
@@ -618,7 +711,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) atomicOr(P.status, LI_DEVERR_TIMEOUT);
-    if (warp == kMmaWarp) {
+    if (warp == kQkWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, P.tmem_cols);
     }
@@ -646,23 +739,21 @@ bool attn_layout(const li_attn_args &a, AttnLayout *L) {
     L->N = N;
     L->npairs = npairs;
     L->q_bytes = (uint32_t)nqc * N * 128u;
-    const uint32_t p_bytes = 2u * 2u * N * 128u;           // two buffers of N x 128 keys bf16
+    const uint32_t p_bytes = 2u * N * 128u;                 // one N x 64-key bf16 tile per group
+    const int rope = a.Dr > 0 ? kMaxRopeSlots : 0;
+    // the MMA order keeps two tiles resident: at least 2 npairs pair slots; two Q buffers when
+    // they leave room for one more pair
     for (int q_bufs = 2; q_bufs >= 1; --q_bufs) {
         const uint32_t q_end = q_bufs * L->q_bytes;
         const uint32_t pair_off = (q_end + p_bytes + 1023u) / 1024u * 1024u;
-        const uint32_t avail = kTailOff > pair_off ? kTailOff - pair_off : 0;
-        int rope = a.Dr > 0 ? kMaxRopeSlots : 0;
-        int pairs = 0;
-        for (; rope >= (a.Dr > 0 ? 1 : 0); --rope) {
-            const uint32_t left = avail > rope * kChunk ? avail - rope * kChunk : 0;
-            pairs = (int)(left / kPair);
-            if (pairs > kMaxPairSlots) pairs = kMaxPairSlots;
-            if (pairs >= npairs + 1) break;                 // one pair of prefetch
-            if (rope == (a.Dr > 0 ? 1 : 0)) break;
-        }
-        // two Q buffers only when a pair of prefetch remains
-        if (q_bufs == 2 && pairs < npairs + 1) continue;
-        if (pairs < npairs) return false;
+        const uint32_t need = (uint32_t)rope * kChunk;
+        if (pair_off + need >= kTailOff) continue;
+        int pairs = (int)((kTailOff - pair_off - need) / kPair);
+        if (pairs > kMaxPairSlots) pairs = kMaxPairSlots;
+        // the gather may run at most this many tiles ahead of the scores (tile barrier ring)
+        if (pairs > (kTileRing - 2) * npairs) pairs = (kTileRing - 2) * npairs;
+        if (q_bufs == 2 && pairs < 2 * npairs + 1) continue;
+        if (pairs < 2 * npairs) return false;
         L->q_bufs = q_bufs;
         L->q_off = 0;
         L->p_off = q_end;
@@ -671,7 +762,7 @@ bool attn_layout(const li_attn_args &a, AttnLayout *L) {
         L->rope_off = pair_off + pairs * kPair;
         L->rope_slots = rope;
         uint32_t cols = 32;
-        while (cols < (uint32_t)(2 * N + npairs * N)) cols <<= 1;
+        while (cols < (uint32_t)(2 * N + 2 * npairs * N)) cols <<= 1;
         L->tmem_cols = cols;
         return true;
     }
@@ -711,11 +802,11 @@ cudaError_t launch_sparse_attention(const li_attn_args &a, uint32_t *status, int
     P.p_off = L.p_off;
     P.pair_off = L.pair_off;
     P.rope_off = L.rope_off;
-    // D fp32, A and B bf16, K-major A and B (S = K Q^T) / MN-major A (O^T = V^T P^T); N, M = 128
-    const uint32_t base = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(L.N >> 3) << 17) |
-                          ((uint32_t)(128 >> 4) << 24);
-    P.idesc_qk = base;
-    P.idesc_pv = base | (1u << 15);
+    // D fp32, A and B bf16, N; S = K Q^T: K-major A and B, M = 64; O^T = V^T P^T: MN-major A,
+    // M = 128
+    const uint32_t base = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(L.N >> 3) << 17);
+    P.idesc_qk = base | ((uint32_t)(kKeys >> 4) << 24);
+    P.idesc_pv = base | (1u << 15) | ((uint32_t)(128 >> 4) << 24);
     P.tmem_cols = L.tmem_cols;
     CUtensorMap mq, mr;
     if (!make_map_bf16(&mq, a.q, (uint64_t)rows * a.G, (uint64_t)a.Dm, (uint32_t)a.G))
