@@ -71,9 +71,6 @@ WORKLOAD_TEXT["sparse_attention"] = (
     "sparse attention over the selected keys: B=1, S1=S2=4096 causal, each row min(2048, i+1) "
     "selected keys (random, indexer-shaped), G=16 heads of Dm=512 + Dr=64, values = keys, bf16 "
     "inputs, fp32 outputs and statistics")
-# fp32 CUDA-core peak of the first backward version: 148 SMs x 128 fp32 lanes x 2 flops per FMA
-# x 1965 MHz (the maximum SM clock)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 # workloads whose keys (not rows) are split across GPUs: strong scaling, all-gather + merge
 KEY_SHARDED = ("long_row_decode",)
@@ -611,6 +608,7 @@ def run_kl(a, dev, world, rank):
     rows = kp_cpu.w.shape[0] * kp_cpu.w.shape[1]
     flops = kl_flops(kp_cpu)
     achieved = flops / (ms / 1e3) / 1e12
+    peaks = load_peaks()
     line = {"metric": "indexer backward query-rows/s", "value": rows * world / (ms / 1e3),
             "unit": "query-rows/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -619,10 +617,12 @@ def run_kl(a, dev, world, rank):
                        "l2": "flushed before every step by a 256 MB write outside the step's "
                              "CUDA events",
                        "parallelism": f"{world} independent replicas (one problem per GPU)"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS,
-                         "unit": "TFLOP/s", "frac": achieved / FP32_ALU_TFLOPS, "traffic": None,
-                         "kernel": "kl_row_kernel (CUDA cores, fp32; first version)",
-                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": None,
+                         "kernel": "kl_tc_kernel (tcgen05: main and indexer scores, d_qi and "
+                                   "d_ki products; fp32 softmax, loss and dS)",
+                         "peak_source": f"{peaks['source']} bf16 burst"},
             "clocks": clk, "gpu_launches": 3 * K}
     if rank == 0 and world == 1 and a.cpu_seconds > 0:
         from oracle import oracle as orc

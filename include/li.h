@@ -334,10 +334,16 @@ li_status li_merge_topk(const li_merge_args *args, void *stream);
  * (B,S1,1,topk) int32; softmax_max / softmax_sum (B,1,S1,G) fp32. Outputs, fp32: *loss (one
  * value), d_qi like qi, d_ki like ki (zeroed by the call, then accumulated), d_w like w.
  * G in [1, 128], Dm in [1, 576] and Dr in [0, 64] multiples of 8, H in [1, 64], topk in
- * [1, 2048]. Selected positions must lie in [0, S2); others set LI_DEVERR_LENGTHS and are
- * skipped. The workspace holds one fp32 per row plus the status word: li_kl_grad_workspace_size.
- * Stream-ordered, no allocation. d_ki is accumulated with atomic adds, so its rounding (not its
- * value beyond that) may differ from run to run; the loss is summed in a fixed order.
+ * [1, 2048]. Selected positions must lie in [0, S2) and be distinct within a row; others set
+ * LI_DEVERR_LENGTHS and are skipped. Stream-ordered, no allocation, loss summed in a fixed order.
+ * Two kernels: shapes with Dm a multiple of 64 up to 512, Dr 0 or 64, G <= 32 and H <= 64 run on
+ * the tensor cores (tcgen05: the scores and both gradient products; dS enters the products as a
+ * bf16 hi + lo pair, 16 significant bits), every output bit-reproducible: each CTA owns a fixed
+ * set of rows and adds its d_ki rows into its own slice of a partial buffer in the workspace,
+ * and the slices are summed per key in a fixed order. Other shapes run on CUDA cores with d_ki
+ * accumulated by atomic adds (rounding may differ from run to run). li_kl_grad_workspace_size
+ * gives the bytes: the status word, one fp32 per row, and on the tensor-core path
+ * SMs x B x S2 x 128 fp32 of partial d_ki (the SM count of the current device).
  */
 typedef struct li_kl_args {
     const void *q, *k, *q_rope, *k_rope;     /* bf16 main attention                          */

@@ -489,8 +489,22 @@ li_status validate_kl(const li_kl_args *a) {
         if (!aligned(p, 4)) return fail(LI_ERR_INVALID_ARG, "inputs must be 4-byte aligned");
     return LI_OK;
 }
+// Which backward kernel runs: the tensor-core kernel when the shapes fit it, unless
+// LI_KL_KERNEL=simple selects the CUDA-core one (a debugging switch).
+bool kl_use_tc(const li_kl_args *a, li::KlTcPlan *plan) {
+    const char *e = std::getenv("LI_KL_KERNEL");
+    if (e && std::strcmp(e, "simple") == 0) return false;
+    return li::kl_tc_plan(*a, plan);
+}
+size_t kl_row_loss_bytes(const li_kl_args *a) {
+    return ((size_t)a->batch * a->s1 * sizeof(float) + 255) / 256 * 256;
+}
+// status word | row losses | tensor-core path: the partial d_ki slices
 size_t kl_ws_bytes(const li_kl_args *a) {
-    return 256 + ((size_t)a->batch * a->s1 * sizeof(float) + 255) / 256 * 256;
+    li::KlTcPlan plan;
+    size_t n = 256 + kl_row_loss_bytes(a);
+    if (kl_use_tc(a, &plan)) n += li::kl_tc_partial_floats(*a, li::kl_tc_chunks(*a)) * sizeof(float);
+    return n;
 }
 }  // namespace
 
@@ -520,7 +534,16 @@ li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_b
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "workspace clear: %s", cudaGetErrorString(e));
     auto *status = static_cast<uint32_t *>(workspace);
     auto *row_loss = reinterpret_cast<float *>(static_cast<char *>(workspace) + 256);
-    e = li::launch_kl_grad(*args, row_loss, status, loss, d_qi, d_ki, d_w, cs);
+    li::KlTcPlan plan;
+    if (kl_use_tc(args, &plan)) {
+        auto *d_part = reinterpret_cast<float *>(static_cast<char *>(workspace) + 256 +
+                                                 kl_row_loss_bytes(args));
+        e = li::launch_kl_tc(*args, plan, row_loss, status, d_part, li::kl_tc_chunks(*args), d_qi,
+                             d_ki, d_w, cs);
+        if (e == cudaSuccess) e = li::launch_kl_loss(row_loss, (int64_t)args->batch * args->s1, loss, cs);
+    } else {
+        e = li::launch_kl_grad(*args, row_loss, status, loss, d_qi, d_ki, d_w, cs);
+    }
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
     return ok();
 }

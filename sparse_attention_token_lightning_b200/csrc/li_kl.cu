@@ -288,6 +288,10 @@ cudaError_t launch_kl_grad(const li_kl_args &a, float *row_loss, uint32_t *statu
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    return launch_kl_loss(row_loss, rows, loss, st);
+}
+
+cudaError_t launch_kl_loss(const float *row_loss, int64_t rows, float *loss, cudaStream_t st) {
     kl_loss_kernel<<<1, 1024, 0, st>>>(row_loss, rows, loss);
     return cudaGetLastError();
 }
