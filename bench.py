@@ -340,9 +340,45 @@ def run_reference_kl(a):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config},
+            "extrapolated_full_workload_ms": rows / (16 / t) * 1e3,
             "cpu_baseline": {"value": 16 / t, "unit": "query-rows/s", "cores": 1,
                              "kind": "oracle", "sample": "the 16 longest rows per step, one pinned host core"},
             "e2e": {"value": 16 / t, "unit": "query-rows/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_attn(a):
+    """The reference arm of the attention workload: the oracle on 8 seeded-random rows per step."""
+    import numpy as np
+    from oracle import oracle as orc
+    ap = synthetic.attn_config(a.config)
+    B, S1 = ap.q.shape[:2]
+    o = orc.default()
+    rng = np.random.default_rng(5)
+    R = 8
+    times = []
+    with one_core():
+        for s in range(a.warmup + a.steps):
+            part = ap.rows(rng.choice(B * S1, R, replace=False))
+            t0 = time.perf_counter()
+            o.sparse_attention(part)
+            if s >= a.warmup:
+                times.append(time.perf_counter() - t0)
+    t = statistics.mean(times)
+    line = {"metric": "sparse attention query-tokens/s", "value": R / t, "unit": "query-tokens/s",
+            "n_gpus": 1, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[a.config], "name": a.config,
+                       "step": f"the oracle on {R} seeded-random rows"},
+            "extrapolated_full_workload_ms": B * S1 / (R / t) * 1e3,
+            "cpu_baseline": {"value": R / t, "unit": "query-tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{R} seeded-random rows per step, one pinned host core",
+                             "host": host_cpu()},
+            "e2e": {"value": R / t, "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -355,6 +391,8 @@ def run_reference(a):
         return 0
     if a.config == "kl_backward":
         return run_reference_kl(a)
+    if a.config == "sparse_attention":
+        return run_reference_attn(a)
     pb = synthetic.config(a.config)
     step_seconds = a.ref_step_seconds
     for s in range(a.warmup):
