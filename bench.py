@@ -133,27 +133,31 @@ def score_kernel_bytes(pb, pairs) -> int:
     return key_bytes(pb) + q + w + table + pairs * 4
 
 
-# DRAM traffic of one score-kernel launch (dram__bytes_read.sum + dram__bytes_write.sum from one
-# ncu capture of `python bench.py [--config NAME] --steps 3 --warmup 3 --cpu-seconds 0 --no-e2e`),
-# with the sha256 of the score-kernel sources the counters were taken on; reported only while the
-# sources still match. Writes that stay in L2 when the kernel ends are not in the counter.
-SCORE_TRAFFIC = {
-    "causal_prefill": {"bytes": 68752128 + 9507840,
-                       "src_sha256": "b623c5865b8927a7cbd1c63a806547438de94eb902870e84c685e067617a720f"},
-    "paged_decode": {"bytes": 286280704 + 6545152,
-                     "src_sha256": "b623c5865b8927a7cbd1c63a806547438de94eb902870e84c685e067617a720f"},
+# DRAM traffic of one launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture of `python bench.py [--config NAME] --steps 3 --warmup 3 --cpu-seconds 0`
+# (plus --no-e2e for the indexer workloads)), with the sha256 of the kernel's sources the
+# counters were taken on; reported only while the sources still match. Writes that stay in L2
+# when the kernel ends are not in the counter.
+SCORE_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_score_tc.cu', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
+ATTN_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_attn.cu', 'sparse_attention_token_lightning_b200/csrc/li_attn.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
+KL_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_kl_tc.cu', 'sparse_attention_token_lightning_b200/csrc/li_kl.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
+KERNEL_TRAFFIC = {
+    "causal_prefill": {"bytes": 68748544 + 9403392, "sources": SCORE_SOURCES,
+                       "src_sha256": "10fff75115b23a2cfef41bfacd512bf2b2d8421bd9c8d94e3929755982b94dad"},
+    "sparse_attention": {"bytes": 114396416 + 92227072, "sources": ATTN_SOURCES,
+                         "src_sha256": "5006949e3c5ce6bbf0a84a1f7b760832de5548945894a00b16fbf9078ecf9157"},
+    "kl_backward": {"bytes": 446973440 + 607046912, "sources": KL_SOURCES,
+                    "src_sha256": "391cf2631960e7dab5bc74bf37bc7d758bc5ab39c63f483d0638ca83fea96e05"},
 }
-SCORE_SOURCES = ("sparse_attention_token_lightning_b200/csrc/li_score_tc.cu",
-                 "sparse_attention_token_lightning_b200/csrc/li_internal.cuh")
 
 
-def score_traffic(config: str):
+def kernel_traffic(config: str):
     import hashlib
-    rec = SCORE_TRAFFIC.get(config)
+    rec = KERNEL_TRAFFIC.get(config)
     if rec is None:
         return None
     h = hashlib.sha256()
-    for f in SCORE_SOURCES:
+    for f in rec["sources"]:
         h.update((ROOT / f).read_bytes())
     return rec["bytes"] if h.hexdigest() == rec["src_sha256"] else None
 
@@ -570,7 +574,7 @@ def run_attn(a, dev, world, rank):
                        "parallelism": f"{world} independent replicas (one problem per GPU)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "traffic": None,
+                         "traffic": kernel_traffic(a.config),
                          "kernel": "sparse_attn_kernel (gather + tcgen05 scores, softmax, "
                                    "value product)",
                          "peak_source": f"{peaks['source']} bf16 burst"},
@@ -657,7 +661,7 @@ def run_kl(a, dev, world, rank):
                        "parallelism": f"{world} independent replicas (one problem per GPU)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "traffic": None,
+                         "traffic": kernel_traffic(a.config),
                          "kernel": "kl_tc_kernel (tcgen05: main and indexer scores, d_qi and "
                                    "d_ki products; fp32 softmax, loss and dS)",
                          "peak_source": f"{peaks['source']} bf16 burst"},
@@ -884,7 +888,7 @@ def main():
         achieved = nbytes / (sc / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": score_traffic(a.config),
+                    "frac": achieved / peak, "traffic": kernel_traffic(a.config),
                     "algorithmic_bytes": nbytes,
                     "kernel": "score kernel (paged key gather + contraction + epilogue)",
                     "peak_source": f"{peaks['source']} HBM copy"}
@@ -893,7 +897,7 @@ def main():
         # fp8 contractions run at twice the bf16 rate (nominal dense 4.5 vs 2.25 PFLOP/s)
         peak = peaks["bf16_tflops"] * (2.0 if dtype == "fp8_e4m3" else 1.0)
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": score_traffic(a.config),
+                    "frac": achieved / peak, "traffic": kernel_traffic(a.config),
                     "algorithmic_bytes": score_kernel_bytes(pb_cpu, pairs),
                     "kernel": "score kernel (q.k contraction + ReLU/weight/head-sum epilogue)",
                     "peak_source": f"{peaks['source']} bf16 burst"
