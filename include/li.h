@@ -80,6 +80,10 @@ typedef enum li_dtype {
                                        after padding                                          */
 #define LI_DEVERR_DESCALE   0x80u   /* fp8 q/k: a q_descale or k_descale in use is not a positive
                                        finite number                                          */
+#define LI_DEVERR_BOUNDS    0x100u  /* bounds-checked build only (compiled with LI_DEBUG): a
+                                       computed shared- or global-memory index fell outside its
+                                       buffer; the access was skipped. Never set by the release
+                                       library, whose indices are bounded by construction.     */
 
 /*
  * Arguments of one indexer call. Mirrors the pages' prototypes (lightning_indexer, "Prototype":

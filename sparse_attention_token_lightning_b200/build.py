@@ -41,6 +41,14 @@ WAIT_TEST_LIB = PKG / "libli_waittest.so"
 WAIT_TEST_FLAGS = ("-DLI_WAIT_LIMIT_NS=1000000ull", "-DLI_TEST_NO_LOADS=1")
 
 
+# Bounds-checked build: every computed shared- or global-memory index the kernels form passes a
+# check first; a failing check sets LI_DEVERR_BOUNDS in the status word and the access is
+# skipped (see in_bounds() in csrc/li_internal.cuh). Same C ABI; loaded by the tests beside
+# libli.so, whose release kernels it must match bit for bit.
+DEBUG_LIB = PKG / "libli_debug.so"
+DEBUG_FLAGS = ("-DLI_DEBUG=1",)
+
+
 def up_to_date(lib: Path = LIB) -> bool:
     if not lib.exists():
         return False
@@ -51,6 +59,11 @@ def up_to_date(lib: Path = LIB) -> bool:
 def build_wait_test(force: bool = False, verbose: bool = False) -> Path:
     """libli_waittest.so (see WAIT_TEST_FLAGS)."""
     return build(force, verbose, WAIT_TEST_FLAGS, lib=WAIT_TEST_LIB, obj_sub="waittest")
+
+
+def build_debug(force: bool = False, verbose: bool = False) -> Path:
+    """libli_debug.so (see DEBUG_FLAGS)."""
+    return build(force, verbose, DEBUG_FLAGS, lib=DEBUG_LIB, obj_sub="debug")
 
 
 def build(force: bool = False, verbose: bool = False, extra=(), lib: Path = LIB,
@@ -89,4 +102,5 @@ def build(force: bool = False, verbose: bool = False, extra=(), lib: Path = LIB,
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     build_wait_test(force="--force" in sys.argv, verbose="-v" in sys.argv)
+    build_debug(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)

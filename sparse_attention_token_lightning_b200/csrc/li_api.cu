@@ -10,6 +10,8 @@
 #include <cstring>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "li_attn.cuh"
 #include "li_internal.cuh"
 #include "li_kl.cuh"
@@ -41,6 +43,16 @@ bool g_stage_events_on = false;
 void stage_mark(int i, cudaStream_t st) {
     if (g_stage_events_on && g_stage_events[i]) cudaEventRecord(g_stage_events[i], st);
 }
+
+// NVTX range around each entry point and each stage it enqueues, for timeline tools (Nsight
+// Systems); without a tool attached a push/pop pair costs a few nanoseconds. Building with
+// -DNVTX_DISABLE compiles them out.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -278,6 +290,7 @@ li_status li_metadata_workspace_size(const li_args *args, size_t *bytes) {
 }
 
 li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *stream) {
+    NvtxRange range("li_metadata");
     li::Problem p;
     li::Schedule s;
     li_status st = validate(args, &p, &s);
@@ -322,6 +335,7 @@ li_status li_indexer_workspace_size(const li_args *args, size_t *bytes) {
 li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
                      size_t workspace_bytes, int32_t *sparse_indices, float *sparse_values,
                      void *stream) {
+    NvtxRange range("li_indexer");
     li::Problem p;
     li::Schedule s;
     li_status st = validate(args, &p, &s);
@@ -355,6 +369,7 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
         stage_mark(1, cs);
     }
     if (!meta && !s.dense) {
+        NvtxRange r("li_indexer: schedule");
         stage_mark(0, cs);
         e = li::launch_metadata(p, s, inline_meta, cs);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "metadata launch: %s", cudaGetErrorString(e));
@@ -366,6 +381,8 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
     quant.q_descale = args->q_descale;
     quant.k_descale = args->k_descale;
     stage_mark(2, cs);
+    {
+    NvtxRange r("li_indexer: score");
     if (!use_simple_kernel()) {
         e = li::launch_score_tc(p, quant, s, meta, ws, scores, ld, cs, &launched);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
@@ -374,7 +391,9 @@ li_status li_indexer(const li_args *args, const void *metadata, void *workspace,
         e = li::launch_score_simple(p, quant, s, meta, ws, scores, ld, cs);
         if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
     }
+    }
     stage_mark(3, cs);
+    NvtxRange rsel("li_indexer: select");
     stage_mark(4, cs);
     const int pieces = li::select_pieces(p);
     if (pieces > 1) {
@@ -435,6 +454,7 @@ li_status li_set_stage_events(void *const *events, int32_t n_events) {
 }
 
 li_status li_merge_topk(const li_merge_args *a, void *stream) {
+    NvtxRange range("li_merge_topk");
     if (!a) return fail(LI_ERR_INVALID_ARG, "args is NULL");
     if (a->n_lists < 1 || a->n_lists > LI_MERGE_MAX_LISTS)
         return fail(LI_ERR_INVALID_ARG, "n_lists=%d outside [1, %d]", a->n_lists, LI_MERGE_MAX_LISTS);
@@ -518,6 +538,7 @@ li_status li_kl_grad_workspace_size(const li_kl_args *args, size_t *bytes) {
 
 li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_bytes, float *loss,
                      float *d_qi, float *d_ki, float *d_w, void *stream) {
+    NvtxRange range("li_kl_grad");
     li_status st = validate_kl(args);
     if (st != LI_OK) return st;
     if (!workspace || !aligned(workspace, 256))
@@ -591,6 +612,7 @@ li_status li_sparse_attention_workspace_size(const li_attn_args *args, size_t *b
 
 li_status li_sparse_attention(const li_attn_args *args, void *workspace, size_t workspace_bytes,
                               float *out, float *softmax_max, float *softmax_sum, void *stream) {
+    NvtxRange range("li_sparse_attention");
     li::AttnLayout L;
     li_status st = validate_attn(args, &L);
     if (st != LI_OK) return st;

@@ -230,7 +230,8 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
                 const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
                 if (v >= P.s2) err |= LI_DEVERR_LENGTHS;
                 // an unselected slot copies the batch's first key row (in bounds); its p is 0
-                const int64_t kr = key_base + (v >= 0 && v < P.s2 ? v : 0);
+                int64_t kr = key_base + (v >= 0 && v < P.s2 ? v : 0);
+                if (!idx_ok(kr, (int64_t)(P.rows / P.s1) * P.s2, P.status)) kr = 0;
                 krow[i] = P.k + kr * P.Dm + 8 * piece;
                 rrow[i] = P.Dr > 0 ? P.k_rope + kr * P.Dr + 8 * piece : nullptr;
             }
@@ -593,6 +594,7 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
         if (!wait_warp(bars.o_full(), nrow & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int G = P.G;
+        const bool row_ok = idx_ok(row, P.rows, P.status);
         float *orow = P.out + (int64_t)row * G * P.Dm;
         for (int b = 0; b < P.npairs; ++b) {
 #pragma unroll
@@ -603,7 +605,7 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int h = c + i;
-                    if (h < G) {
+                    if (h < G && row_ok) {
                         float o = 0.f;
                         if (tiles > 0) o = oa[i] * wa[h];
                         if (two) o += ob[i] * wb[h];
@@ -614,7 +616,7 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
         }
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-            if (h == dlane && h < G) {
+            if (h == dlane && h < G && row_ok) {
                 P.smax[(int64_t)row * G + h] = smx[h];
                 P.ssum[(int64_t)row * G + h] = ssm[h];
             }

@@ -340,6 +340,29 @@ __device__ inline void set_status(uint32_t *status, uint32_t bits) {
     if (bits) atomicOr(status, bits);
 }
 
+// Bounds-checked build (-DLI_DEBUG): the kernels pass each computed shared- or global-memory
+// index through in_bounds() before the access. A failing check sets LI_DEVERR_BOUNDS and the
+// caller skips the access (no trap: the context stays usable). The release build compiles every
+// check to `true`, so its code is unchanged.
+#ifdef LI_DEBUG
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t *status) {
+    if constexpr (kDebugBounds) {
+        if (!ok) {
+            if (status) atomicOr(status, LI_DEVERR_BOUNDS);
+            return false;
+        }
+    }
+    return true;
+}
+// Index i of a buffer of n elements.
+__device__ __forceinline__ bool idx_ok(int64_t i, int64_t n, uint32_t *status) {
+    return in_bounds(i >= 0 && i < n, status);
+}
+
 // Sets the message li_last_error_string() returns on this host thread.
 void set_last_error(const char *msg);
 

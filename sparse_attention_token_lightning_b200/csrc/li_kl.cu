@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(kT) kl_row_kernel(const KlParams P) {
             const int s = e / kDi, d = e % kDi;
             float acc = 0.0f;
             for (int h = 0; h < H; ++h) acc = fmaf(dS[h * kChunk + s], qi[h * kDi + d], acc);
-            if (acc != 0.0f) atomicAdd(&P.d_ki[(int64_t)kr[c0 + s] * kDi + d], acc);
+            if (acc != 0.0f && idx_ok(kr[c0 + s], (int64_t)(gridDim.x / P.s1) * P.s2, P.status))
+                atomicAdd(&P.d_ki[(int64_t)kr[c0 + s] * kDi + d], acc);
         }
         __syncthreads();
     }

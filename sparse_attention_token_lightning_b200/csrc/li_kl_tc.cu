@@ -201,6 +201,7 @@ __device__ void gather_role(const KlTcParams &P, uint8_t *smem, const Bars &bars
                     const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
                     if (pass == 0 && v >= P.s2) err |= LI_DEVERR_LENGTHS;
                     kr_[i] = key_base + (v >= 0 && v < P.s2 ? v : 0);
+                    if (!idx_ok(kr_[i], P.key_rows, P.status)) kr_[i] = 0;
                 }
                 if (pass == 0) {
                     for (int c = 0; c < P.nmc; ++c, mr.next(P.main_slots)) {
@@ -592,11 +593,13 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.dk_full(), dkph, abort_flag)) { ok = false; break; }
             dkph ^= 1u;
             tc_fence_after();
-            float *drow = slice + (key_base + (valid ? v : 0)) * kDi;
+            const int64_t dkr = key_base + (valid ? v : 0);
+            const bool dk_ok = idx_ok(dkr, P.key_rows, P.status);
+            float *drow = slice + dkr * kDi;
             for (int c = 0; c < kDi; c += 16) {
                 float a[16];
                 tmem_ld16(tmem + lane_addr + kColDk + c, a);
-                if (kl && valid) {
+                if (kl && valid && dk_ok) {
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
                         float4 o = *reinterpret_cast<float4 *>(drow + c + i);
@@ -616,7 +619,7 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         for (int c = 0; c < kDi; c += 16) {
             float a[16];
             tmem_ld16(tmem + lane_addr + kColDq + c, a);
-            if (kl && key < P.H) {
+            if (kl && key < P.H && idx_ok(row, P.rows, P.status)) {
                 float *dq = P.d_qi + ((int64_t)row * P.H + key) * kDi + c;
 #pragma unroll
                 for (int i = 0; i < 16; i += 4)

@@ -21,6 +21,7 @@
 // slot is written once (8 B, 4 B without values).
 #include <cstdint>
 
+#include "li_internal.cuh"
 #include "li_merge.cuh"
 
 namespace li {
@@ -202,7 +203,8 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
         }
 #pragma unroll
         for (int u = 0; u < kStageUnroll; ++u)
-            if (fe[u] >= 0) s_mem[fe[u]] = iv[u] >= 0 ? order_key(iv[u], vv[u]) : 0ull;
+            if (fe[u] >= 0 && idx_ok(fe[u], total_in, P.status))
+                s_mem[fe[u]] = iv[u] >= 0 ? order_key(iv[u], vv[u]) : 0ull;
     }
     __syncthreads();
     // input contract: within a list, keys strictly decrease until the padding (key 0) starts
@@ -284,6 +286,7 @@ __global__ void __launch_bounds__(kTreeThreads) merge_tree_kernel(const __grid_c
                         b = j < nb ? B[j] : 0ull;
                     }
                     if (last) {
+                        if (!idx_ok(pos, P.topk_out, P.status)) break;
                         oi[pos] = (int32_t)~(uint32_t)x;
                         if (ov) ov[pos] = key_value(x);
                     } else {

@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(kThreads) score_simple_kernel(Params sp) {
                         I = fmaf(ws_[h], fmaxf(s, 0.0f), I);
                     }
                 }
-                sp.scores[row * sp.ld + j] = I;
+                if (in_bounds(row < sp.p.rows && j < sp.ld, &sp.ws->status))
+                    sp.scores[row * sp.ld + j] = I;
             }
         }
     }

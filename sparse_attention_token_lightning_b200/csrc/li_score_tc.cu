@@ -245,7 +245,10 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
         // Q tile of the item (all heads of tq rows): two TMA loads, one per 64-wide K half.
         const int qb = it & 1;
         if (!mbar_wait(bars.q_empty(qb), ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (kIssueLoads && lane == 0) {
+        if (kIssueLoads && lane == 0 &&
+            !in_bounds((qb + 1) * 2u * P.q_half <= P.k_off, &P.ws->status)) {
+            mbar_arrive(bars.q_full(qb));            // bounds-checked build: skip the load
+        } else if (kIssueLoads && lane == 0) {
             const uint32_t qdst = sbase + qb * 2u * P.q_half;
             const int32_t y = row0 * N1;
             if constexpr (kQ8) {
@@ -270,6 +273,8 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             const uint32_t kdst = sbase + P.k_off + st * kStage;
             if (!kIssueLoads) {
                 // test build: no load and no arrive; the MMA warp's wait on k_full runs out
+            } else if (!in_bounds(P.k_off + (st + 1) * kStage <= kTailOff, &P.ws->status)) {
+                if (lane == 0) mbar_arrive(bars.k_full(st));   // bounds-checked build: skip
             } else if (pr == 0) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), kStage);
@@ -284,7 +289,9 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
                     pv = piece_row(P, b, j0, j1, pbase + lane);
                 }
                 const int32_t row = __shfl_sync(0xffffffffu, pv, (p0 - pbase + lane) & 31);
-                const bool mine = lane < pieces && row >= 0;
+                const bool mine = lane < pieces && row >= 0 &&
+                                  in_bounds((int64_t)row + pr <= (int64_t)P.p.num_blocks * P.p.block_size,
+                                            &P.ws->status);
                 const uint32_t loads = __ballot_sync(0xffffffffu, mine);
                 if (__ballot_sync(0xffffffffu, lane < pieces && row == -2)) err |= LI_DEVERR_TABLE;
                 if (lane == 0)
@@ -488,11 +495,13 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                     tmem_ld64(acc + group * 64, v);
                     float I = head_sum64(v, S.w + group * 64);
                     if constexpr (kQ8) I *= kd;
-                    if (j < hi1) out1[j] = I;
+                    if (j < hi1 && in_bounds(row0 + group < P.p.rows && j < P.ld, &P.ws->status))
+                        out1[j] = I;
                 } else if (jt < hi1) {
                     float I = head_sum(acc, S.w, group, N1);
                     if constexpr (kQ8) I *= kd;
-                    if (j < hi1) out1[j] = I;
+                    if (j < hi1 && in_bounds(row0 + group < P.p.rows && j < P.ld, &P.ws->status))
+                        out1[j] = I;
                 }
             } else {
                 for (int t = group; t < nq; t += kEpiGroups) {
@@ -507,7 +516,8 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                         I = head_sum(acc, S.w, t, N1);
                     }
                     if constexpr (kQ8) I *= kd;
-                    if (j < hi) P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
+                    if (j < hi && in_bounds(row0 + t < P.p.rows && j < P.ld, &P.ws->status))
+                        P.scores[(int64_t)(row0 + t) * P.ld + j] = I;
                 }
             }
             tc_fence_before();

@@ -34,6 +34,7 @@ struct Smem {
     float s_vmin, s_vmax;
     int32_t s_cut, s_maxbin, s_total;
     int32_t s_append;       // candidate append counter of the long-row path (only used there)
+    uint32_t *dbg;          // bounds-checked build: the status word (set at kernel start)
 };
 
 // Block-wide exclusive scan of cnt[0..kWarps*kDigits) in place (8 entries per thread).
@@ -169,11 +170,13 @@ __device__ void gather(const uint32_t *rowc, const float *src, int32_t n, int32_
         const uint32_t lt = lanemask_lt();
         if (is_gt) {
             const int32_t pos = run_gt + pre_g + __popc(bg & lt);
-            keyA[pos] = u;
-            idxA[pos] = e;
+            if (idx_ok(pos, m, sm.dbg)) {
+                keyA[pos] = u;
+                idxA[pos] = e;
+            }
         } else if (is_eq) {
             const int32_t r = run_eq + pre_e + __popc(be & lt);
-            if (r < need) {
+            if (r < need && idx_ok(gt + r, m, sm.dbg)) {
                 keyA[gt + r] = u;
                 idxA[gt + r] = e;
             }
@@ -228,8 +231,10 @@ __device__ bool sort_desc(int32_t m, uint32_t *keyA, int32_t *idxA, uint32_t *ke
             if (valid) {
                 const int32_t base = cnt[d * kWarps + warp];
                 const int32_t dst = base + __popc(peers & lanemask_lt());
-                kd[dst] = key;
-                id[dst] = is[e];
+                if (idx_ok(dst, m, sm.dbg)) {
+                    kd[dst] = key;
+                    id[dst] = is[e];
+                }
             }
             __syncwarp();
             if (valid && lane == __ffs(peers) - 1) cnt[d * kWarps + warp] += __popc(peers);
@@ -392,7 +397,7 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
         rb[i] = nb;
         if (e < n) {
             rb[i] = bucket_of(v[i], vmin, scale, nb);
-            atomicAdd(&hist[rb[i]], 1);
+            if (idx_ok(rb[i], nb, sm.dbg)) atomicAdd(&hist[rb[i]], 1);
         }
     }
     __syncthreads();
@@ -409,21 +414,26 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
 #pragma unroll
     for (int i = 0; i < kRegKeys; ++i) {
         const int32_t e = i * kThreads + tid;
-        if (rb[i] <= cutb) {                     // rb == nb for keys past n
+        if (rb[i] <= cutb && idx_ok(rb[i], nb, sm.dbg)) {   // rb == nb for keys past n
             const int32_t dst = atomicAdd(&hist[rb[i]], 1);
-            buf[dst] = ((uint64_t)score_key(v[i]) << 32) | (uint32_t)~(uint32_t)e;
-            bufb[dst] = (uint16_t)rb[i];
+            if (idx_ok(dst, m + kBinCap, sm.dbg)) {
+                buf[dst] = ((uint64_t)score_key(v[i]) << 32) | (uint32_t)~(uint32_t)e;
+                bufb[dst] = (uint16_t)rb[i];
+            }
         }
     }
     __syncthreads();
     // rank within the bucket; the top m land in the stage at their output slots, and the row is
     // then written out in slot order (contiguous stores instead of one scattered store per key)
-    const int32_t filled = hist[cutb];
+    int32_t filled = hist[cutb];
+    if (!in_bounds(filled >= 0 && filled <= m + kBinCap, sm.dbg)) filled = 0;
     for (int32_t p = tid; p < filled; p += kThreads) {
         const uint64_t x = buf[p];
         const int32_t b = bufb[p];
+        if (!idx_ok(b, nb, sm.dbg)) continue;
         const int32_t beg = b == 0 ? 0 : hist[b - 1];
         const int32_t end = hist[b];
+        if (!in_bounds(beg >= 0 && beg <= end && end <= filled, sm.dbg)) continue;
         int32_t rank = 0;
         for (int32_t a = beg; a < end; ++a) rank += buf[a] > x ? 1 : 0;
         const int32_t slot = beg + rank;
@@ -478,8 +488,10 @@ __device__ int cand_bucket_topk(const uint64_t *cand, int32_t n_c, int32_t m, in
     const float vmin = sm.s_vmin, vmax = sm.s_vmax;
     if (!(vmax - vmin > 0.0f) || !(vmax - vmin < kInf)) return 2;
     const float scale = (float)nb / (vmax - vmin);
-    for (int32_t p = tid; p < n_c; p += kThreads)
-        atomicAdd(&hist[bucket_of(key_score((uint32_t)(cand[p] >> 32)), vmin, scale, nb)], 1);
+    for (int32_t p = tid; p < n_c; p += kThreads) {
+        const int32_t rb = bucket_of(key_score((uint32_t)(cand[p] >> 32)), vmin, scale, nb);
+        if (idx_ok(rb, nb, sm.dbg)) atomicAdd(&hist[rb], 1);
+    }
     __syncthreads();
     switch (nb / kThreads) {
         case 1: scan_buckets<1>(hist, m, sm); break;
@@ -494,19 +506,24 @@ __device__ int cand_bucket_topk(const uint64_t *cand, int32_t n_c, int32_t m, in
     for (int32_t p = tid; p < n_c; p += kThreads) {
         const uint64_t x = cand[p];
         const int32_t rb = bucket_of(key_score((uint32_t)(x >> 32)), vmin, scale, nb);
-        if (rb <= cutb) {
+        if (rb <= cutb && idx_ok(rb, nb, sm.dbg)) {
             const int32_t dst = atomicAdd(&hist[rb], 1);
-            gbuf[dst] = x;
-            gbufb[dst] = (uint16_t)rb;
+            if (idx_ok(dst, m + kBinCap, sm.dbg)) {
+                gbuf[dst] = x;
+                gbufb[dst] = (uint16_t)rb;
+            }
         }
     }
     __syncthreads();
-    const int32_t filled = hist[cutb];
+    int32_t filled = hist[cutb];
+    if (!in_bounds(filled >= 0 && filled <= m + kBinCap, sm.dbg)) filled = 0;
     for (int32_t p = tid; p < filled; p += kThreads) {
         const uint64_t x = gbuf[p];
         const int32_t b = gbufb[p];
+        if (!idx_ok(b, nb, sm.dbg)) continue;
         const int32_t beg = b == 0 ? 0 : hist[b - 1];
         const int32_t end = hist[b];
+        if (!in_bounds(beg >= 0 && beg <= end && end <= filled, sm.dbg)) continue;
         int32_t rank = 0;
         for (int32_t a = beg; a < end; ++a) rank += gbuf[a] > x ? 1 : 0;
         const int32_t slot = beg + rank;
@@ -568,6 +585,7 @@ __device__ int long_row_topk(const float *src, int32_t n, int32_t m, int32_t *hi
     } else {
         __syncthreads();
     }
+    if (!in_bounds(n_c <= cand_cap, sm.dbg)) return 2;
     // pass 2: keys of bins 0..cut, 16 per thread per iteration: each thread packs its take flags
     // into a mask, a warp scan of the counts gives every thread its write position, and one
     // atomic per warp claims the warp's space
@@ -748,6 +766,10 @@ __global__ void __launch_bounds__(kThreads, kLong ? (kThreads >= 1024 ? 1 : 2) :
     // blocks start in index order; later rows of a causal window are the longer ones, so the
     // rows are taken last to first (longest first)
     const int32_t r = (int32_t)(gridDim.x - 1 - blockIdx.x);
+    if constexpr (kDebugBounds) {
+        if (threadIdx.x == 0) sm.dbg = &sp.ws->status;
+        __syncthreads();
+    }
     int32_t n, off;
     row_window(sp, r, &n, &off);
     const int32_t topk = sp.p.topk;
@@ -768,6 +790,10 @@ select_piece_kernel(Params sp, PieceParams pp) {
     const int32_t rows = (int32_t)(gridDim.x / pp.pieces);
     const int32_t r = rows - 1 - (int32_t)(blockIdx.x / pp.pieces);
     const int32_t c = (int32_t)(blockIdx.x % pp.pieces);
+    if constexpr (kDebugBounds) {
+        if (threadIdx.x == 0) sm.dbg = &sp.ws->status;
+        __syncthreads();
+    }
     int32_t n, off;
     row_window(sp, r, &n, &off);
     const int64_t start = (int64_t)c * pp.piece_len;

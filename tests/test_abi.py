@@ -42,6 +42,18 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, n)
 
 
+@pytest.mark.parametrize("which", ["debug", "waittest"])
+def test_test_builds_export_every_declared_symbol(which):
+    """The bounds-checked build and the wait-limit test build keep the same C ABI."""
+    path = libbuild.build_debug() if which == "debug" else libbuild.build_wait_test()
+    out = subprocess.run(["nm", "-D", "--defined-only", str(path)], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (li_[a-z_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert li.load(path).li_abi_version() == 5
+
+
 def test_abi_version(L):
     assert li.li_abi_version() == 5
 
