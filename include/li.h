@@ -183,8 +183,9 @@ li_status li_metadata(const li_args *args, void *metadata, size_t bytes, void *s
  *                 1 or 2 no schedule kernel runs
  *   kernels       kernels one li_indexer call launches with metadata == NULL (0 when there are no
  *                 query rows); one fewer schedule kernel when a metadata buffer is passed
- *   score_tc      1 when the score step runs on the tcgen05 kernel, 0 on the CUDA-core kernel
- *                 (paged caches whose block_size the TMA pieces cannot tile)
+ *   score_tc      1 when the score step runs on the tcgen05 kernel (every block_size of a
+ *                 paged cache included), 0 on the CUDA-core kernel (LI_SCORE_KERNEL=simple, or
+ *                 a shape outside the kernel's limits)
  *   select_pieces key pieces each row's selection is cut into (1: one CTA per row). Few very long
  *                 rows (decode over a long context) are split so that more SMs work on them;
  *                 the pieces' lists are merged as li_merge_topk merges key ranges, one more

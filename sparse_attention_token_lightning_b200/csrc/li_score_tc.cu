@@ -27,6 +27,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "li_internal.cuh"
 #include "li_sm100.cuh"
 
@@ -90,7 +92,9 @@ struct TcParams {
     int32_t N;            // MMA N
     int32_t tq;           // query rows per item
     uint32_t idesc;       // tcgen05 instruction descriptor
-    int32_t piece_rows;   // paged: keys per TMA load (min(block_size, 128)); 0 for dense keys
+    int32_t piece_rows;   // paged keys: > 0, keys per TMA load (the largest power of two dividing
+                          // block_size, at most 128); < 0, -(that power) below 8, the key rows
+                          // copied one by one (cp.async); 0 for dense keys
     int32_t stages;       // K ring depth
     int32_t n_acc;        // TMEM accumulators in use
     uint32_t acc_stride;  // TMEM columns per accumulator (power of two >= N)
@@ -129,9 +133,12 @@ __device__ __forceinline__ int32_t n_tiles_of(int32_t j0, int32_t j1) {
 // Paged keys: row in the key cache of piece pi of an item whose keys start at j0 (pieces of
 // piece_rows keys; j0 is a multiple of them). -1 past j1, -2 when the block-table entry is out
 // of range.
+__device__ __forceinline__ int32_t piece_len(const TcParams &P) {
+    return P.piece_rows < 0 ? -P.piece_rows : P.piece_rows;
+}
 __device__ __forceinline__ int32_t piece_row(const TcParams &P, int32_t b, int32_t j0, int32_t j1,
                                              int32_t pi) {
-    const int32_t jp = j0 + pi * P.piece_rows;
+    const int32_t jp = j0 + pi * piece_len(P);
     if (jp >= j1) return -1;
     const int32_t bs = P.p.block_size;
     const int32_t blk = P.p.block_table[(int64_t)b * P.p.bt_stride + jp / bs];
@@ -216,7 +223,7 @@ __device__ void scheduler(const TcParams &P, uint8_t *smem, const Bars &bars,
 // range through the ring; paged keys block by block through the block table.
 // kQ8: fp8 q/k, whose 128-element rows are one 128-byte box (two 64-element halves for 16-bit
 // types), so a Q tile and a K stage are half as many bytes and loads.
-template <bool kQ8>
+template <bool kQ8, bool kRows>
 __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtensorMap *tmk,
                          uint8_t *smem, const Bars &bars, volatile int *abort_flag) {
     constexpr uint32_t kStage = kQ8 ? kKHalfBytes : kKStageBytes;
@@ -265,7 +272,8 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
         // lanes 0..pieces-1 each load one piece of the tile.
         const int32_t nt = n_tiles_of(j0, j1);
         const int pr = P.piece_rows;
-        const int pieces = pr ? kKeyTile / pr : 0;
+        const int pieces = pr > 0 ? kKeyTile / pr : 0;
+        int prev_st = -1;                   // row-copy mode: the stage whose arrival is pending
         for (int32_t tile = 0; tile < nt; ++tile, kr.next(P.stages)) {
             const int st = kr.idx;
             if (!mbar_wait(bars.k_empty(st), kr.phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -275,6 +283,42 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
                 // test build: no load and no arrive; the MMA warp's wait on k_full runs out
             } else if (!in_bounds(P.k_off + (st + 1) * kStage <= kTailOff, &P.ws->status)) {
                 if (lane == 0) mbar_arrive(bars.k_full(st));   // bounds-checked build: skip
+            } else if constexpr (kRows) {
+                // block sizes that are not a multiple of 8: the key rows are copied one by one
+                // (cp.async, eight lanes per 128-byte half row) into the same 128-byte swizzled
+                // layout the TMA writes; lane l copies chunk l % 8 of keys l / 8 + 4 i. Each
+                // lane arrives on a stage's full barrier (32 arrivals) once its copies of that
+                // stage have landed and are fenced for the tensor cores, one tile later, so two
+                // tiles' copies are in flight.
+                const int32_t g = -pr;
+                const int kq = lane >> 3, ch = lane & 7;
+                const char *kbase = reinterpret_cast<const char *>(P.p.k);
+                const int64_t cache_rows = (int64_t)P.p.num_blocks * P.p.block_size;
+#pragma unroll 4
+                for (int i = 0; i < kKeyTile / 4; ++i) {
+                    const int key = kq + 4 * i;
+                    const int32_t j = jt + key;
+                    int32_t row = -1;
+                    if (j < j1) {
+                        const int32_t q = j - j0;
+                        row = piece_row(P, b, j0, j1, q / g);
+                        if (row >= 0) row += q % g;
+                    }
+                    if (row == -2) err |= LI_DEVERR_TABLE;
+                    if (row >= 0 && idx_ok(row, cache_rows, &P.ws->status)) {
+                        const char *src = kbase + (int64_t)row * kRowBytes + ch * 16;
+                        const uint32_t dst = kdst + (uint32_t)key * 128u + (uint32_t)((ch ^ (key & 7)) << 4);
+                        cp_async16(dst, src);
+                        if constexpr (!kQ8) cp_async16(dst + kKHalfBytes, src + 128);
+                    }
+                }
+                cp_async_commit();
+                if (prev_st >= 0) {
+                    cp_async_wait<1>();
+                    fence_async_smem();
+                    mbar_arrive(bars.k_full(prev_st));
+                }
+                prev_st = st;
             } else if (pr == 0) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bars.k_full(st), kStage);
@@ -306,9 +350,16 @@ __device__ void producer(const TcParams &P, const CUtensorMap *tmq, const CUtens
             }
             __syncwarp();
         }
+        if (kRows && prev_st >= 0) {        // row-copy mode: the item's last stage
+            cp_async_wait<0>();
+            fence_async_smem();
+            mbar_arrive(bars.k_full(prev_st));
+        }
         if (!ok) break;
         if (lane == 0) mbar_arrive(bars.sl_empty(sl));
     }
+    // no copy may still be writing shared memory when the CTA leaves
+    if constexpr (kRows) asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok) *abort_flag = 1;
     if (lane == 0 && err) set_status(&P.ws->status, err);
 }
@@ -389,6 +440,30 @@ __device__ __forceinline__ float head_sum64(const float (&v)[64], const float *w
     return (a01.x + a01.y) + (a23.x + a23.y);
 }
 
+// The same sum with the 64 columns read from TMEM in two halves of 32: fewer live registers,
+// the same additions in the same order. The fp8 instantiations take it (with one 64-column
+// load their key-scale registers spill at the kernel's 96-register budget); the 16-bit ones
+// keep the single load, which measures faster there.
+__device__ __forceinline__ float head_sum64_tmem(uint32_t taddr, const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(taddr + 32u * half, v);
+#pragma unroll
+        for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 ww = w4[8 * half + h4];
+            const float x0 = v[4 * h4 + 0], x2 = v[4 * h4 + 2];
+            a01 = __ffma2_rn(make_float2(ww.x, ww.y),
+                             make_float2(x0 + fabsf(x0), fmaxf(v[4 * h4 + 1], 0.f)), a01);
+            a23 = __ffma2_rn(make_float2(ww.z, ww.w),
+                             make_float2(x2 + fabsf(x2), fmaxf(v[4 * h4 + 3], 0.f)), a23);
+        }
+    }
+    return (a01.x + a01.y) + (a23.x + a23.y);
+}
+
 // The same sum for any N1: row t's columns [t*N1, (t+1)*N1) of the accumulator at acc, read 16
 // columns at a time; even columns carry halved weights.
 __device__ __forceinline__ float head_sum(uint32_t acc, const float *w, int t, int N1) {
@@ -450,16 +525,17 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
             if (t >= nt || jj >= j1) return 0.0f;
             int64_t kr = (int64_t)S.k_row0 + jj;
             if (P.piece_rows) {
-                const int32_t pc = (jj - j0) / P.piece_rows;
+                const int32_t pl = piece_len(P);
+                const int32_t pc = (jj - j0) / pl;
                 int32_t prow = pc < 32 ? S.prow[pc] : -1;
                 if (pc >= 32) {
                     const int32_t bs = P.p.block_size;
                     const int32_t blk = P.p.block_table[(int64_t)S.b * P.p.bt_stride + jj / bs];
-                    prow = blk >= 0 && blk < P.p.num_blocks ? blk * bs + (jj - jj % P.piece_rows) % bs
+                    prow = blk >= 0 && blk < P.p.num_blocks ? blk * bs + (jj - jj % pl) % bs
                                                             : -2;
                 }
                 if (prow < 0) return 0.0f;
-                kr = (int64_t)prow + (jj - j0) % P.piece_rows;
+                kr = (int64_t)prow + (jj - j0) % pl;
             }
             has = true;
             return __ldg(P.qd.k_descale + kr);
@@ -491,9 +567,14 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
             const uint32_t acc = tmem_base + lane_addr + ab * P.acc_stride;
             if (one_row) {
                 if (N1 == 64 && jt < hi1) {
-                    float v[64];
-                    tmem_ld64(acc + group * 64, v);
-                    float I = head_sum64(v, S.w + group * 64);
+                    float I;
+                    if constexpr (kQ8) {
+                        I = head_sum64_tmem(acc + group * 64, S.w + group * 64);
+                    } else {
+                        float v[64];
+                        tmem_ld64(acc + group * 64, v);
+                        I = head_sum64(v, S.w + group * 64);
+                    }
                     if constexpr (kQ8) I *= kd;
                     if (j < hi1 && in_bounds(row0 + group < P.p.rows && j < P.ld, &P.ws->status))
                         out1[j] = I;
@@ -509,9 +590,13 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
                     if (jt >= hi) continue;                       // tile past this row's window
                     float I;
                     if (N1 == 64) {
-                        float v[64];
-                        tmem_ld64(acc + t * 64, v);
-                        I = head_sum64(v, S.w + t * 64);
+                        if constexpr (kQ8) {
+                            I = head_sum64_tmem(acc + t * 64, S.w + t * 64);
+                        } else {
+                            float v[64];
+                            tmem_ld64(acc + t * 64, v);
+                            I = head_sum64(v, S.w + t * 64);
+                        }
                     } else {
                         I = head_sum(acc, S.w, t, N1);
                     }
@@ -535,7 +620,7 @@ __device__ void epilogue(const TcParams &P, uint8_t *smem, const Bars &bars,
 
 // kW: li_dtype of w (the weights are staged as fp32; q and k go to the MMA as they are);
 // kQ8: fp8 q/k with scales.
-template <int kW, bool kQ8>
+template <int kW, bool kQ8, bool kRows>
 __global__ void __launch_bounds__(kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const TcParams P) {
@@ -561,7 +646,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff + 4);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(bars.k_full(s), 1);
+            mbar_init(bars.k_full(s), kRows ? 32 : 1);   // row copies: one arrival per lane
             mbar_init(bars.k_empty(s), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -593,7 +678,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        producer<kQ8>(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
+        producer<kQ8, kRows>(P, &tmap_q, &tmap_k, smem, bars, abort_flag);
     } else if (warp == kSchedWarp) {
         if (blockIdx.x == 0) check_batch_keys(P.p, P.view, &P.ws->status, lane, 32);
         scheduler<kW, kQ8>(P, smem, bars, abort_flag, n_items);
@@ -635,17 +720,14 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows,
 }  // namespace
 
 // Shape checks of the tensor-core kernel: MMA width 16..256, at least two key stages in shared
-// memory, paged blocks the TMA pieces tile (a multiple of 8 dividing 128, or a multiple of 128),
-// and 16-byte aligned q and k for the tensor maps.
+// memory and 16-byte aligned q and k for the tensor maps. Every paged block size is taken: TMA
+// pieces of the largest power of two dividing it (capped at 128) when that is 8 or more, row
+// copies otherwise.
 bool score_tc_eligible(const Problem &p, const Schedule &s) {
     if (s.max_items <= 0 || p.rows <= 0) return false;
     const int N = (s.tq * p.n_heads + 15) / 16 * 16;
     if (N > kNmax || N < 16) return false;
     if ((kTailOff - 4u * (uint32_t)N * 128u) / kKStageBytes < 2) return false;
-    if (p.layout_k == LI_LAYOUT_PA_BSND) {
-        const int bs = p.block_size;
-        if (bs <= kKeyTile ? (bs % 8 != 0 || kKeyTile % bs != 0) : bs % kKeyTile != 0) return false;
-    }
     return (reinterpret_cast<uintptr_t>(p.q) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.k) & 15) == 0;
 }
 
@@ -684,14 +766,13 @@ cudaError_t launch_score_tc(const Problem &p, const Quant &qd, const Schedule &s
     if (P.stages < 2) return cudaSuccess;
     uint64_t k_rows = 0;
     if (p.layout_k == LI_LAYOUT_PA_BSND) {
+        // pieces: the largest power of two dividing the block size, at most a tile; each piece
+        // lies inside one block and one tile. TMA loads pieces of 8 rows or more (whole
+        // 1024-byte swizzle atoms); smaller ones are copied row by row.
         const int bs = p.block_size;
-        if (bs <= kKeyTile) {
-            if (bs % 8 != 0 || kKeyTile % bs != 0) return cudaSuccess;
-            P.piece_rows = bs;
-        } else {
-            if (bs % kKeyTile != 0) return cudaSuccess;
-            P.piece_rows = kKeyTile;
-        }
+        const int low = bs & -bs;
+        const int piece = low < kKeyTile ? low : kKeyTile;
+        P.piece_rows = piece >= 8 ? piece : -piece;
         k_rows = (uint64_t)p.num_blocks * bs;
     } else {
         P.piece_rows = 0;
@@ -701,15 +782,22 @@ cudaError_t launch_score_tc(const Problem &p, const Quant &qd, const Schedule &s
                             p.n_heads;
     CUtensorMap mq, mk;
     if (!make_map(&mq, p.q, q_rows, (uint32_t)P.N, p.dtype_qk)) return cudaSuccess;
-    if (!make_map(&mk, p.k, k_rows, P.piece_rows ? (uint32_t)P.piece_rows : (uint32_t)kKeyTile,
+    if (!make_map(&mk, p.k, k_rows,
+                  P.piece_rows > 0 ? (uint32_t)P.piece_rows : P.piece_rows < 0 ? 1u : (uint32_t)kKeyTile,
                   p.dtype_qk))
         return cudaSuccess;
-    auto kern = q8 ? (p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32, true>
-                      : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16, true>
-                                                   : score_tc_kernel<LI_DTYPE_BF16, true>)
-                   : (p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32, false>
-                      : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16, false>
-                                                   : score_tc_kernel<LI_DTYPE_BF16, false>);
+    // row-copy mode (block sizes that are not a multiple of 8) has instantiations of its own,
+    // so the TMA kernels' code is unchanged by it
+    const bool rows = P.piece_rows < 0;
+    auto pick = [&](auto q8c, auto rowsc) {
+        constexpr bool Q8 = decltype(q8c)::value, R = decltype(rowsc)::value;
+        return p.dtype_w == LI_DTYPE_FP32   ? score_tc_kernel<LI_DTYPE_FP32, Q8, R>
+             : p.dtype_w == LI_DTYPE_FP16 ? score_tc_kernel<LI_DTYPE_FP16, Q8, R>
+                                          : score_tc_kernel<LI_DTYPE_BF16, Q8, R>;
+    };
+    using T = std::true_type;
+    using F = std::false_type;
+    auto kern = q8 ? (rows ? pick(T{}, T{}) : pick(T{}, F{})) : (rows ? pick(F{}, T{}) : pick(F{}, F{}));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;

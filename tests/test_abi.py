@@ -274,11 +274,13 @@ def test_plan_reports_schedule_and_kernel_count(L):
     st_a, n_split = _ws_status(_args(max_seqlen_k=1 << 20, **long_row))
     st_b, n_whole = _ws_status(_args(max_seqlen_k=(1 << 20) - 128, **long_row))
     assert st_a == st_b == 0
-    # block sizes the TMA pieces cannot tile go to the CUDA-core score kernel
-    pl = li.li_plan(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
-                          block_table_stride=64, num_blocks=64, block_size=12,
-                          max_seqlen_k=512))
-    assert pl["score_tc"] == 0 and pl["kernels"] == 3 and pl["dense"] == 0
+    # every block size runs on the tensor-core score kernel (12: pieces of 4 rows, copied row
+    # by row; 1 and 1024 too)
+    for bs in (1, 12, 48, 1000, 1024):
+        pl = li.li_plan(_args(layout_k=2, k_len=0, seqused_k=0x40000, block_table=0x50000,
+                              block_table_stride=64, num_blocks=64, block_size=bs,
+                              max_seqlen_k=512))
+        assert pl["score_tc"] == 1 and pl["kernels"] == 3 and pl["dense"] == 0, bs
     # no query rows: nothing launches
     assert li.li_plan(_args(batch=0))["kernels"] == 0
     # argument errors come back as status codes

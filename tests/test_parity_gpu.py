@@ -87,6 +87,17 @@ SMALL = {
     # few query blocks and long windows: key ranges split across work items
     "paged_decode_split": lambda: synthetic.paged([5000, 3000, 100], 1, 64, 256, block_size=64,
                                                   seed=51),
+    # block sizes the TMA pieces do not tile at 8 rows: pieces of the largest power of two
+    # dividing the block size (24: 8, 1000: 8) or row copies below 8 (3, 100: 4, 6: 2)
+    "paged_bs3": lambda: synthetic.paged([200, 31, 2], 2, 16, 32, block_size=3, seed=64),
+    "paged_bs6_tnd_q": lambda: synthetic.paged([150, 40], 0, 8, 24, block_size=6, seed=65,
+                                               layout_q="TND", lens_q=[20, 7]),
+    "paged_bs24": lambda: synthetic.paged([500, 130], 2, 64, 100, block_size=24, seed=66),
+    "paged_bs100_decode": lambda: synthetic.paged([1300, 700, 90], 1, 64, 128, block_size=100,
+                                                  seed=67),
+    "paged_bs1000": lambda: synthetic.paged([2500, 999], 1, 32, 200, block_size=1000, seed=68),
+    "paged_bs1024": lambda: synthetic.paged([3000, 1025, 1], 2, 64, 256, block_size=1024,
+                                            seed=69),
 }
 
 
@@ -97,12 +108,25 @@ def test_small_parity(orc, name):
     parity.check(orc, pb, gi, gv, label=name)
 
 
+@pytest.mark.parametrize("name", [n for n in SMALL if n.startswith("paged")])
+def test_every_block_size_takes_the_tensor_core_kernel(name):
+    """Paged keys of any block size in [1, 1024] run on the tcgen05 score kernel: TMA pieces of
+    the largest power of two dividing the block size when that is 8 or more, row copies
+    otherwise (lightning_indexer, "Constraints": block size 1 to 1024)."""
+    pb = SMALL[name]()
+    assert li.li_plan(li.make_args(pb))["score_tc"] == 1
+
+
 EXACT = {
     "bsnd_causal": lambda: synthetic.bsnd(2, 333, 333, 64, 100, 3, seed=20, integer=True),
     "bsnd_n4_nomask": lambda: synthetic.bsnd(1, 100, 260, 4, 300, 0, seed=21, integer=True),
     "tnd": lambda: synthetic.tnd([5, 200, 1], [129, 200, 700], 16, 64, 3, seed=22, integer=True),
     "paged": lambda: synthetic.paged([500, 64, 65], 2, 64, 96, block_size=64, seed=23,
                                      integer=True, spare_blocks=2),
+    "paged_bs1_rows": lambda: synthetic.paged([300, 64, 5], 2, 16, 96, block_size=1, seed=24,
+                                              integer=True, spare_blocks=3),
+    "paged_bs48_pieces": lambda: synthetic.paged([500, 47], 1, 64, 128, block_size=48, seed=25,
+                                                 integer=True),
 }
 
 
@@ -169,6 +193,8 @@ FP8_CASES = {
     "paged_bs16_long_fp8": lambda: Q8(SMALL["paged_bs16_long"]()),
     "paged_decode_split_fp8": lambda: Q8(SMALL["paged_decode_split"]()),
     "paged_bs256_nomask_fp8": lambda: Q8(SMALL["paged_bs256_nomask"]()),
+    "paged_bs3_fp8": lambda: Q8(SMALL["paged_bs3"]()),
+    "paged_bs100_decode_fp8": lambda: Q8(SMALL["paged_bs100_decode"]()),
 }
 
 
