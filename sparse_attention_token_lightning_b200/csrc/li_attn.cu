@@ -286,6 +286,7 @@ __device__ void qk_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
             const int g = j & 1;
             if (!wait_(bars.s_empty(g), (kg[g] & 1u) ^ 1u, abort_flag)) { ok = false; break; }
             if (!wait_(bars.tile_full(tr.idx), tr.phase, abort_flag)) { ok = false; break; }
+            fence_async_smem();                  // the gathered rows, for the async proxy
             tc_fence_after();
             const uint32_t d_s = tmem + g * N;
             for (int b = 0; b < P.npairs; ++b, pq.next(P.pair_slots)) {
@@ -343,6 +344,7 @@ __device__ void pv_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
                 break;
             }
             if (!wait_(bars.p_full(g), kg[g] & 1u, abort_flag)) { ok = false; break; }
+            fence_async_smem();
             tc_fence_after();
             const uint32_t pa = sbase + P.p_off + g * cb;
             for (int b = 0; b < P.npairs; ++b, pv.next(P.pair_slots)) {

@@ -269,6 +269,7 @@ __device__ void mma_role(const KlTcParams &P, uint8_t *smem, const Bars &bars,
         for (int j = 0; j < tiles && ok; ++j, tr.next(kTileRing)) {
             if (!wait_(bars.s_empty(), sph ^ 1u, abort_flag)) { ok = false; break; }
             if (!wait_(bars.tile_full(tr.idx), tr.phase, abort_flag)) { ok = false; break; }
+            fence_async_smem();                  // the gathered rows, for the async proxy
             tc_fence_after();
             for (int c = 0; c < P.nmc; ++c, mr.next(P.main_slots)) {
                 const uint64_t a = sw128_desc(sbase + P.main_off + mr.idx * kChunk);
@@ -290,6 +291,7 @@ __device__ void mma_role(const KlTcParams &P, uint8_t *smem, const Bars &bars,
         for (int j = 0; j < tiles && ok; ++j, tr.next(kTileRing)) {
             if (!wait_(bars.s_empty(), sph ^ 1u, abort_flag)) { ok = false; break; }
             if (!wait_(bars.tile_full(tr.idx), tr.phase, abort_flag)) { ok = false; break; }
+            fence_async_smem();                  // the gathered rows, for the async proxy
             tc_fence_after();
             const uint32_t ki_addr = sbase + P.ki_off + kr.idx * 2u * kChunk;
             indexer_scores(ki_addr);
