@@ -79,7 +79,7 @@ constexpr uint32_t kTailOff = kSmemBytes - kTailBytes;
 constexpr uint32_t kRowSlotOff = kTailOff + 8 * kNumBars;
 constexpr uint32_t kXchOff = (kRowSlotOff + 2 * sizeof(RowSlot) + 15) / 16 * 16;
 constexpr uint32_t kDwOff = kXchOff + 2 * 4 * 4;
-constexpr uint32_t kRowDataOff = kDwOff + 2 * 64 * 4 * 4;
+constexpr uint32_t kRowDataOff = kDwOff + 64 * 4 * 4;
 constexpr uint32_t kFlagOff = kRowDataOff + (64 + 32 + 32) * 4;
 static_assert(kFlagOff + 16 <= kSmemBytes, "shared memory tail");
 static_assert(kTailOff % 1024 == 0, "tail alignment");
@@ -402,7 +402,7 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
     float *iarr = reinterpret_cast<float *>(smem + P.iarr_off);
     float *rw = reinterpret_cast<float *>(smem + kRowDataOff);        // w[64]
     float *rmax = rw + 64, *rsum = rw + 96;                           // softmax max / sum [32]
-    float *dwx = reinterpret_cast<float *>(smem + kDwOff);            // [2][64 heads][4 warps]
+    float *dwx = reinterpret_cast<float *>(smem + kDwOff);            // [64 heads][4 warps]
     const float kInf = __int_as_float(0x7f800000);
     uint32_t sph = 0, dsph = 0, dkph = 0, nrow_dq = 0, use = 0;
     bool ok = true;
@@ -508,7 +508,14 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         if (!epi_reduce(loss, false, use, smem, bars, abort_flag)) { ok = false; break; }
         if (tid == 0) P.row_loss[row] = loss;
         // ---- pass 2: dS, d_w, d_qi and the dK rows ------------------------------------------------
-        float dw_acc = 0.f;                                           // head tid < 64
+        // d_w: each warp adds its tiles' per-head sums into its own column of dwx (one owner per
+        // entry, tile order); the four columns are added in warp order at the row's end. The
+        // previous row's final read of dwx came before the exchanges above.
+        if (lane < 16) {
+            const int qb = quad_base(lane);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dwx[(qb + i) * 4 + warp] = 0.f;
+        }
         float *slice = P.d_part + (int64_t)blockIdx.x * P.key_rows * kDi;
         for (int j = 0; j < tiles; ++j) {
             const int pos = kKeys * j + key;
@@ -576,38 +583,50 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             }
             fence_async_smem();
             mbar_arrive(bars.ds_full());
-            // d_w: per-head sums over the tile's keys (lanes 0-15 of the four warps), fixed order
+            // this key's previous partial dK row (the first half) is loaded now, so the load is in
+            // flight during the d_w sums and the wait for the product
+            const int64_t dkr = key_base + (valid ? v : 0);
+            const bool dk_on = kl && valid && idx_ok(dkr, P.key_rows, P.status);
+            float4 *drow = reinterpret_cast<float4 *>(slice + dkr * kDi);
+            float4 old[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) old[i] = dk_on ? drow[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            // d_w: per-head sums over this warp's 16 keys, added to the warp's own column
             {
-                float *db = dwx + (j & 1) * 64 * 4;
 #pragma unroll
                 for (int h = 0; h < 64; ++h) dwp[h] = kl ? dwp[h] : 0.f;
                 quad_reduce64(dwp, lane);
                 if (lane < 16) {
                     const int qb = quad_base(lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) db[(qb + i) * 4 + warp] = dwp[i];
+                    for (int i = 0; i < 4; ++i) dwx[(qb + i) * 4 + warp] += dwp[i];
                 }
-                float d0 = 0.f;
-                if (!epi_reduce(d0, false, use, smem, bars, abort_flag)) { ok = false; break; }
-                if (tid < 64) dw_acc += (db[tid * 4] + db[tid * 4 + 1]) + (db[tid * 4 + 2] + db[tid * 4 + 3]);
             }
-            // this tile's dK rows into the CTA's slice of the partial buffer
+            // this tile's dK rows into the CTA's slice of the partial buffer, in two halves
             if (!wait_warp(bars.dk_full(), dkph, abort_flag)) { ok = false; break; }
             dkph ^= 1u;
             tc_fence_after();
-            const int64_t dkr = key_base + (valid ? v : 0);
-            const bool dk_ok = idx_ok(dkr, P.key_rows, P.status);
-            float *drow = slice + dkr * kDi;
-            for (int c = 0; c < kDi; c += 16) {
-                float a[16];
-                tmem_ld16(tmem + lane_addr + kColDk + c, a);
-                if (kl && valid && dk_ok) {
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4) {
-                        float4 o = *reinterpret_cast<float4 *>(drow + c + i);
-                        o.x += a[i]; o.y += a[i + 1]; o.z += a[i + 2]; o.w += a[i + 3];
-                        *reinterpret_cast<float4 *>(drow + c + i) = o;
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        old[i] = dk_on ? drow[16 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c += 16) {
+                    float a[16];
+                    tmem_ld16(tmem + lane_addr + kColDk + 64 * half + c, a);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float4 o = old[c / 4 + i];
+                        o.x += a[4 * i]; o.y += a[4 * i + 1]; o.z += a[4 * i + 2]; o.w += a[4 * i + 3];
+                        old[c / 4 + i] = o;
                     }
+                }
+                if (dk_on) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) drow[16 * half + i] = old[i];
                 }
             }
             tc_fence_before();
@@ -632,7 +651,13 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.dq_empty());
         ++nrow_dq;
-        if (tid < P.H) P.d_w[(int64_t)row * P.H + tid] = dw_acc;
+        {
+            float d0 = 0.f;                  // orders the four warps' dwx columns before the sums
+            if (!epi_reduce(d0, false, use, smem, bars, abort_flag)) { ok = false; break; }
+        }
+        if (tid < P.H)
+            P.d_w[(int64_t)row * P.H + tid] =
+                (dwx[tid * 4] + dwx[tid * 4 + 1]) + (dwx[tid * 4 + 2] + dwx[tid * 4 + 3]);
         // the d_part rows written above are read by later rows of this CTA through the same
         // threads or others: order them before the next row's updates
         __threadfence_block();
