@@ -384,9 +384,6 @@ __device__ __forceinline__ void quad_reduce64(float (&a)[64], int lane) {
     }
 }
 
-__device__ __forceinline__ uint16_t bf16_bits(float x) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
-}
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 template <int NG>
@@ -405,6 +402,7 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
     float *dwx = reinterpret_cast<float *>(smem + kDwOff);            // [64 heads][4 warps]
     const float kInf = __int_as_float(0x7f800000);
     uint32_t sph = 0, dsph = 0, dkph = 0, nrow_dq = 0, use = 0;
+    const float scale2 = P.scale * kLog2e;                // scale in log2 units
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it & 1;
@@ -429,9 +427,10 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             float dummy = 0.f;
             if (!epi_reduce(dummy, false, use, smem, bars, abort_flag)) { ok = false; break; }
             if (tid < 64) rw[tid] = tid < P.H ? bf16_val(P.w[(int64_t)row * P.H + tid]) : 0.f;
+            // staged for the exponent's FMA: max in log2 units and the reciprocal of the sum
             if (tid < 32) {
-                rmax[tid] = tid < P.G ? P.smax[(int64_t)row * P.G + tid] : 0.f;
-                rsum[tid] = tid < P.G ? P.ssum[(int64_t)row * P.G + tid] : 1.f;
+                rmax[tid] = tid < P.G ? P.smax[(int64_t)row * P.G + tid] * kLog2e : 0.f;
+                rsum[tid] = tid < P.G ? 1.f / P.ssum[(int64_t)row * P.G + tid] : 1.f;
             }
             if (!epi_reduce(dummy, false, use, smem, bars, abort_flag)) { ok = false; break; }
         }
@@ -443,33 +442,46 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.s_full(), sph, abort_flag)) { ok = false; break; }
             sph ^= 1u;
             tc_fence_after();
-            float sm[NG];
-            {
-                float a[16];
-                tmem_ld16(tmem + lane_addr + kColSm, a);
+            // both score sets loaded with one wait, then the buffer is released at once
+            uint32_t smr[NG / 16][16], sir[4][16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) sm[i] = a[i];
-                if constexpr (NG == 32) {
-                    tmem_ld16(tmem + lane_addr + kColSm + 16, a);
+            for (int c = 0; c < NG / 16; ++c) tmem_ld16_nowait(tmem + lane_addr + kColSm + 16 * c, smr[c]);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) sm[16 + i] = a[i];
+            for (int c = 0; c < 4; ++c) {
+                if (16 * c < P.Nh) {
+                    tmem_ld16_nowait(tmem + lane_addr + kColSi + 16 * c, sir[c]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) sir[c][i] = 0u;
                 }
             }
-            float I = 0.f;
-            for (int c = 0; c < P.Nh; c += 16) {
-                float a[16];
-                tmem_ld16(tmem + lane_addr + kColSi + c, a);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) I = fmaf(rw[c + i], fmaxf(a[i], 0.f), I);
-            }
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_empty());
+            // I = sum_h w_h ReLU(S~_h), two heads per packed FMA
+            float2 ia = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    const float2 w2 = *reinterpret_cast<const float2 *>(rw + 16 * c + i);
+                    ia = __ffma2_rn(w2, make_float2(fmaxf(__uint_as_float(sir[c][i]), 0.f),
+                                                    fmaxf(__uint_as_float(sir[c][i + 1]), 0.f)), ia);
+                }
+            }
+            const float I = ia.x + ia.y;
+            // p^ = sum_g exp(scale S_g - max_g) / sum_g: exp2 of one FMA, times the staged 1 / sum
             float ph = 0.f;
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
-                if (g < P.G)
-                    ph += exp2f((P.scale * sm[g] - rmax[g]) * kLog2e) / rsum[g];
+            for (int c = 0; c < NG / 16; ++c) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int g = 16 * c + i;
+                    if (g < P.G)
+                        ph = fmaf(exp2f(fmaf(__uint_as_float(smr[c][i]), scale2, -rmax[g])), rsum[g], ph);
+                }
+            }
             if (kl && pos < tiles * kKeys) {
                 parr[pos] = valid ? ph : 0.f;
                 iarr[pos] = valid ? I : -kInf;
@@ -527,18 +539,17 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             tc_fence_after();
             // this tile's S~ (the MMA recomputes it into the same columns for the next tile once
             // released)
-            float sv[64];
+            uint32_t svr[4][16];
 #pragma unroll
-            for (int c = 0; c < 64; c += 16) {
-                float a[16];
-                if (c < P.Nh) tmem_ld16(tmem + lane_addr + kColSi + c, a);
-                else {
+            for (int c = 0; c < 4; ++c) {
+                if (16 * c < P.Nh) {
+                    tmem_ld16_nowait(tmem + lane_addr + kColSi + 16 * c, svr[c]);
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) a[i] = 0.f;
+                    for (int i = 0; i < 16; ++i) svr[c][i] = 0u;
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) sv[c + i] = a[i];
             }
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_empty());
@@ -549,7 +560,7 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             float dwp[64];
 #pragma unroll
             for (int c = 0; c < 64; c += 16) {
-                const float *a = sv + c;
+                const uint32_t *a = svr[c / 16];
                 uint32_t hi[8], lo[8];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
@@ -557,15 +568,18 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int h = c + i + u;
-                        const float s = a[i + u];
+                        const float s = __uint_as_float(a[i + u]);
                         ds2[u] = valid && h < P.H && s > 0.f ? dI * rw[h] : 0.f;
                         dwp[h] = valid && h < P.H ? dI * fmaxf(s, 0.f) : 0.f;
                     }
-                    const uint16_t h0 = bf16_bits(ds2[0]), h1 = bf16_bits(ds2[1]);
-                    const uint16_t l0 = bf16_bits(ds2[0] - bf16_val(h0));
-                    const uint16_t l1 = bf16_bits(ds2[1] - bf16_val(h1));
-                    hi[i / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                    lo[i / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                    // hi = bf16(dS) and lo = bf16(dS - hi), two heads per conversion
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(ds2[0], ds2[1]);
+                    const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h2);
+                    const __nv_bfloat162 l2 =
+                        __floats2bfloat162_rn(ds2[0] - __uint_as_float(hb << 16),
+                                              ds2[1] - __uint_as_float(hb & 0xffff0000u));
+                    hi[i / 2] = hb;
+                    lo[i / 2] = *reinterpret_cast<const uint32_t *>(&l2);
                 }
                 if (kl) {
                     // this key's row, 16-byte chunks (c / 8, c / 8 + 1), swizzled by key % 8
