@@ -17,10 +17,13 @@
 // in its row order, into its own slice c of a partial buffer [C][key rows][128]; a second kernel
 // sums the C slices of every key in slice order, so d_key_index is bit-reproducible (no atomics).
 //
-// Warp roles: 0-3 epilogue (thread = key or head of the M = 64 TMEM layouts: lanes 0-15 of each
-// quarter), 4 MMA (and TMEM), 5 scheduler (row slots, Q tiles by TMA), 6-9 gather (cp.async of
-// the selected key rows into 128-byte swizzled 64-dim chunks). Every wait is bounded in time.
+// Warp roles: 0-7 epilogue (thread = key or head of the M = 64 TMEM layouts: lanes 0-15 of each
+// quarter; warps q and q + 4 share quarter q and split each key's heads and dK dims in halves),
+// 8 MMA (and TMEM), 9 scheduler (row slots, Q tiles by TMA), 10-13 gather (cp.async of the
+// selected key rows into 128-byte swizzled 64-dim chunks). Every wait is bounded in time.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "li_internal.cuh"
 #include "li_kl.cuh"
@@ -34,8 +37,8 @@ using namespace sm100;
 constexpr int kKeys = 64;
 constexpr uint32_t kChunk = kKeys * 128;            // 64 keys x 64 dims bf16: 8 KB
 constexpr int kDi = 128;
-constexpr int kEpiWarps = 4, kMmaWarp = 4, kSchedWarp = 5, kGatherWarp0 = 6, kGatherWarps = 4;
-constexpr int kThreads = 32 * 10;
+constexpr int kEpiWarps = 8, kMmaWarp = 8, kSchedWarp = 9, kGatherWarp0 = 10, kGatherWarps = 4;
+constexpr int kThreads = 32 * 14;
 constexpr int kGatherThreads = 32 * kGatherWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr uint32_t kSmemBytes = 232448;
@@ -72,13 +75,13 @@ struct Bars {
     __device__ uint32_t main_empty(int i) const { return at(16 + kTileRing + kMaxKiSlots + i); }
 };
 constexpr int kNumBars = 16 + kTileRing + kMaxKiSlots + kMaxMainSlots;
-// tail: barriers | row slots | scalar exchange [2][4] | d_w exchange [2][64][4] | w, max, sum of
+// tail: barriers | row slots | scalar exchange [2][8 warps] | d_w sums [64][4] | w, max, sum of
 // the row [64 + 32 + 32] | TMEM slot, abort flag
 constexpr uint32_t kTailBytes = 4096;
 constexpr uint32_t kTailOff = kSmemBytes - kTailBytes;
 constexpr uint32_t kRowSlotOff = kTailOff + 8 * kNumBars;
 constexpr uint32_t kXchOff = (kRowSlotOff + 2 * sizeof(RowSlot) + 15) / 16 * 16;
-constexpr uint32_t kDwOff = kXchOff + 2 * 4 * 4;
+constexpr uint32_t kDwOff = kXchOff + 2 * kEpiWarps * 4;
 constexpr uint32_t kRowDataOff = kDwOff + 64 * 4 * 4;
 constexpr uint32_t kFlagOff = kRowDataOff + (64 + 32 + 32) * 4;
 static_assert(kFlagOff + 16 <= kSmemBytes, "shared memory tail");
@@ -352,29 +355,32 @@ __device__ __forceinline__ bool epi_reduce(float &v, bool is_max, uint32_t &use,
         const float x = __shfl_xor_sync(0xffffffffu, v, o);
         v = is_max ? fmaxf(v, x) : v + x;
     }
-    float *xb = reinterpret_cast<float *>(smem + kXchOff) + (use & 1) * 4;
+    float *xb = reinterpret_cast<float *>(smem + kXchOff) + (use & 1) * kEpiWarps;
     if (lane == 0) xb[warp] = v;
     mbar_arrive(bars.xch(use & 1));
     const bool ok = wait_warp(bars.xch(use & 1), (use >> 1) & 1u, abort_flag);
-    v = is_max ? fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3])) : (xb[0] + xb[1]) + (xb[2] + xb[3]);
+    static_assert(kEpiWarps == 8, "eight partials");
+    v = is_max ? fmaxf(fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3])),
+                       fmaxf(fmaxf(xb[4], xb[5]), fmaxf(xb[6], xb[7])))
+               : ((xb[0] + xb[1]) + (xb[2] + xb[3])) + ((xb[4] + xb[5]) + (xb[6] + xb[7]));
     ++use;
     return ok;
 }
 
-// Sums of 64 per-head values over the 16 lanes of a half-warp, transposed: afterwards lane l
-// (of either half) holds the sums of heads quad_base(l) .. + 3 in a[0..3], where lanes with bit
-// (8 >> s) set kept the upper half at step s.
-__device__ __forceinline__ int quad_base(int lane) {
-    return ((lane >> 3) & 1) * 32 + ((lane >> 2) & 1) * 16 + ((lane >> 1) & 1) * 8 + (lane & 1) * 4;
+// Sums of 32 per-head values over the 16 lanes of a half-warp, transposed: afterwards lane l
+// (of either half) holds the sums of heads pair_base(l) and pair_base(l) + 1 in a[0..1], where
+// lanes with bit (8 >> s) set kept the upper half at step s.
+__device__ __forceinline__ int pair_base(int lane) {
+    return ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 + ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
 }
-__device__ __forceinline__ void quad_reduce64(float (&a)[64], int lane) {
+__device__ __forceinline__ void pair_reduce32(float (&a)[32], int lane) {
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         const int bit = 8 >> s;
-        const int half = 32 >> s;
+        const int half = 16 >> s;
         const bool up = (lane & bit) != 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 16; ++i) {
             if (i < half) {
                 const float keep = up ? a[i + half] : a[i];
                 const float send = up ? a[i] : a[i + half];
@@ -390,19 +396,24 @@ template <int NG>
 __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &bars,
                               volatile int *abort_flag, uint32_t tmem) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tid = threadIdx.x;                          // 0..127
+    const int tid = threadIdx.x;                          // 0..kEpiThreads-1
+    const int q = warp & 3;                               // TMEM lane quarter
+    const int hf = warp >> 2;                             // half: heads (and dK dims) of the key
     const bool kl = lane < 16;                            // lanes holding a key (or head) row
-    const int key = 16 * warp + (lane & 15);              // key of the tile / head of d_qi
-    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    const int key = 16 * q + (lane & 15);                 // key of the tile / head of d_qi
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
-    float *parr = reinterpret_cast<float *>(smem + P.parr_off);
-    float *iarr = reinterpret_cast<float *>(smem + P.iarr_off);
+    const int arr_n = (P.topk + kKeys - 1) / kKeys * kKeys;
+    float *parr = reinterpret_cast<float *>(smem + P.parr_off);       // [2 halves][arr_n]
+    float *iarr = reinterpret_cast<float *>(smem + P.iarr_off);       // [2 halves][arr_n]
     float *rw = reinterpret_cast<float *>(smem + kRowDataOff);        // w[64]
     float *rmax = rw + 64, *rsum = rw + 96;                           // softmax max / sum [32]
-    float *dwx = reinterpret_cast<float *>(smem + kDwOff);            // [64 heads][4 warps]
+    float *dwx = reinterpret_cast<float *>(smem + kDwOff);            // [64 heads][4 quarters]
     const float kInf = __int_as_float(0x7f800000);
     uint32_t sph = 0, dsph = 0, dkph = 0, nrow_dq = 0, use = 0;
     const float scale2 = P.scale * kLog2e;                // scale in log2 units
+    constexpr int kMainHalf = NG / 2;                     // main heads of this half
+    const int h0 = 32 * hf;                               // first indexer head of this half
     bool ok = true;
     for (int it = 0; ok; ++it) {
         const int sl = it & 1;
@@ -434,7 +445,7 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             }
             if (!epi_reduce(dummy, false, use, smem, bars, abort_flag)) { ok = false; break; }
         }
-        // ---- pass 1: p^ and I of every selected key -------------------------------------------
+        // ---- pass 1: each half's share of p^ and I of every selected key ----------------------
         for (int j = 0; j < tiles; ++j) {
             const int pos = kKeys * j + key;
             const int32_t v = kl && pos < P.topk ? __ldg(ir + pos) : -1;
@@ -442,14 +453,14 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.s_full(), sph, abort_flag)) { ok = false; break; }
             sph ^= 1u;
             tc_fence_after();
-            // both score sets loaded with one wait, then the buffer is released at once
-            uint32_t smr[NG / 16][16], sir[4][16];
+            // this half's main heads and indexer heads, loaded with one wait, then released
+            uint32_t smr[NG / 16][16], sir[2][16];
 #pragma unroll
             for (int c = 0; c < NG / 16; ++c) tmem_ld16_nowait(tmem + lane_addr + kColSm + 16 * c, smr[c]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (16 * c < P.Nh) {
-                    tmem_ld16_nowait(tmem + lane_addr + kColSi + 16 * c, sir[c]);
+            for (int c = 0; c < 2; ++c) {
+                if (h0 + 16 * c < P.Nh) {
+                    tmem_ld16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, sir[c]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) sir[c][i] = 0u;
@@ -459,47 +470,54 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_empty());
-            // I = sum_h w_h ReLU(S~_h), two heads per packed FMA
+            // I share = sum over this half's heads of w_h ReLU(S~_h), two heads per packed FMA
             float2 ia = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
-                    const float2 w2 = *reinterpret_cast<const float2 *>(rw + 16 * c + i);
+                    const float2 w2 = *reinterpret_cast<const float2 *>(rw + h0 + 16 * c + i);
                     ia = __ffma2_rn(w2, make_float2(fmaxf(__uint_as_float(sir[c][i]), 0.f),
                                                     fmaxf(__uint_as_float(sir[c][i + 1]), 0.f)), ia);
                 }
             }
-            const float I = ia.x + ia.y;
-            // p^ = sum_g exp(scale S_g - max_g) / sum_g: exp2 of one FMA, times the staged 1 / sum
-            float ph = 0.f;
+            // p^ share = sum over this half's main heads of exp(scale S_g - max_g) / sum_g
+            // (register indices fixed at compile time for each half)
+            auto main_share = [&](auto half_c) -> float {
+                constexpr int G0 = decltype(half_c)::value * kMainHalf;
+                float acc = 0.f;
 #pragma unroll
-            for (int c = 0; c < NG / 16; ++c) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int g = 16 * c + i;
-                    if (g < P.G)
-                        ph = fmaf(exp2f(fmaf(__uint_as_float(smr[c][i]), scale2, -rmax[g])), rsum[g], ph);
+                for (int i = 0; i < kMainHalf; ++i) {
+                    const int g = G0 + i;
+                    const float sg = __uint_as_float(smr[g / 16][g % 16]);
+                    if (g < P.G) acc = fmaf(exp2f(fmaf(sg, scale2, -rmax[g])), rsum[g], acc);
                 }
-            }
+                return acc;
+            };
+            const float ph = hf == 0 ? main_share(std::integral_constant<int, 0>{})
+                                     : main_share(std::integral_constant<int, 1>{});
             if (kl && pos < tiles * kKeys) {
-                parr[pos] = valid ? ph : 0.f;
-                iarr[pos] = valid ? I : -kInf;
+                parr[hf * arr_n + pos] = valid ? ph : 0.f;
+                iarr[hf * arr_n + pos] = valid ? ia.x + ia.y : (hf == 0 ? -kInf : 0.f);
             }
         }
         if (!ok) break;
         // ---- row statistics, loss and dI ----------------------------------------------------------
         const int n = tiles * kKeys;
-        float zp = 0.f, im = -kInf;
         {
-            // every thread's own positions are written by lanes 0-15 of all four warps: the
-            // exchange orders those writes before these reads
+            // the two halves' shares, written by lanes 0-15 of every epilogue warp: the exchange
+            // orders those writes before these reads; p^ and I are their sums (half 0 + half 1)
             float d0 = 0.f;
             if (!epi_reduce(d0, false, use, smem, bars, abort_flag)) { ok = false; break; }
         }
+        float zp = 0.f, im = -kInf;
         for (int e = tid; e < n; e += kEpiThreads) {
-            zp += parr[e];
-            im = fmaxf(im, iarr[e]);
+            const float pe = parr[e] + parr[arr_n + e];
+            const float ie = iarr[e] + iarr[arr_n + e];
+            parr[e] = pe;
+            iarr[e] = ie;
+            zp += pe;
+            im = fmaxf(im, ie);
         }
         if (!epi_reduce(zp, false, use, smem, bars, abort_flag)) { ok = false; break; }
         if (!epi_reduce(im, true, use, smem, bars, abort_flag)) { ok = false; break; }
@@ -519,14 +537,13 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         }
         if (!epi_reduce(loss, false, use, smem, bars, abort_flag)) { ok = false; break; }
         if (tid == 0) P.row_loss[row] = loss;
-        // ---- pass 2: dS, d_w, d_qi and the dK rows ------------------------------------------------
-        // d_w: each warp adds its tiles' per-head sums into its own column of dwx (one owner per
-        // entry, tile order); the four columns are added in warp order at the row's end. The
-        // previous row's final read of dwx came before the exchanges above.
+        // ---- pass 2: dS, d_w, d_qi and the dK rows, each half its heads and dims ---------------
+        // d_w: each (head, quarter) entry of dwx has one owner (the half holding the head), which
+        // adds its tiles' sums in tile order; the four quarters are added in order at the row's
+        // end. The previous row's final read of dwx came before the exchanges above.
         if (lane < 16) {
-            const int qb = quad_base(lane);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dwx[(qb + i) * 4 + warp] = 0.f;
+            for (int i = 0; i < 2; ++i) dwx[(h0 + pair_base(lane) + i) * 4 + q] = 0.f;
         }
         float *slice = P.d_part + (int64_t)blockIdx.x * P.key_rows * kDi;
         for (int j = 0; j < tiles; ++j) {
@@ -537,13 +554,13 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.s_full(), sph, abort_flag)) { ok = false; break; }
             sph ^= 1u;
             tc_fence_after();
-            // this tile's S~ (the MMA recomputes it into the same columns for the next tile once
-            // released)
-            uint32_t svr[4][16];
+            // this tile's S~, this half's heads (the MMA recomputes the columns for the next tile
+            // once released)
+            uint32_t svr[2][16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (16 * c < P.Nh) {
-                    tmem_ld16_nowait(tmem + lane_addr + kColSi + 16 * c, svr[c]);
+            for (int c = 0; c < 2; ++c) {
+                if (h0 + 16 * c < P.Nh) {
+                    tmem_ld16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, svr[c]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) svr[c][i] = 0u;
@@ -557,20 +574,20 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.ds_empty(), dsph ^ 1u, abort_flag)) { ok = false; break; }
             dsph ^= 1u;
             uint8_t *dsb = smem + P.ds_off;
-            float dwp[64];
+            float dwp[32];
 #pragma unroll
-            for (int c = 0; c < 64; c += 16) {
-                const uint32_t *a = svr[c / 16];
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t *a = svr[c];
                 uint32_t hi[8], lo[8];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     float ds2[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int h = c + i + u;
+                        const int h = h0 + 16 * c + i + u;
                         const float s = __uint_as_float(a[i + u]);
                         ds2[u] = valid && h < P.H && s > 0.f ? dI * rw[h] : 0.f;
-                        dwp[h] = valid && h < P.H ? dI * fmaxf(s, 0.f) : 0.f;
+                        dwp[16 * c + i + u] = valid && h < P.H ? dI * fmaxf(s, 0.f) : 0.f;
                     }
                     // hi = bf16(dS) and lo = bf16(dS - hi), two heads per conversion
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(ds2[0], ds2[1]);
@@ -582,10 +599,11 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
                     lo[i / 2] = *reinterpret_cast<const uint32_t *>(&l2);
                 }
                 if (kl) {
-                    // this key's row, 16-byte chunks (c / 8, c / 8 + 1), swizzled by key % 8
+                    // this key's row, 16-byte chunks (hc / 8, hc / 8 + 1) of head column
+                    // hc = h0 + 16 c, swizzled by key % 8
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const uint32_t chunk = (uint32_t)(c / 8 + u);
+                        const uint32_t chunk = (uint32_t)((h0 + 16 * c) / 8 + u);
                         const uint32_t off = (uint32_t)(key >> 3) * 1024u + (uint32_t)(key & 7) * 128u +
                                              ((chunk ^ (uint32_t)(key & 7)) << 4);
                         *reinterpret_cast<uint4 *>(dsb + off) =
@@ -597,76 +615,80 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             }
             fence_async_smem();
             mbar_arrive(bars.ds_full());
-            // this key's previous partial dK row (the first half) is loaded now, so the load is in
-            // flight during the d_w sums and the wait for the product
+            // this key's previous partial dK row (this half's 64 dims) is loaded now, so the load
+            // is in flight during the d_w sums and the wait for the product
             const int64_t dkr = key_base + (valid ? v : 0);
             const bool dk_on = kl && valid && idx_ok(dkr, P.key_rows, P.status);
-            float4 *drow = reinterpret_cast<float4 *>(slice + dkr * kDi);
+            float4 *drow = reinterpret_cast<float4 *>(slice + dkr * kDi) + 16 * hf;
             float4 old[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) old[i] = dk_on ? drow[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-            // d_w: per-head sums over this warp's 16 keys, added to the warp's own column
+            // d_w: this half's per-head sums over the warp's 16 keys, added to its dwx entries
             {
 #pragma unroll
-                for (int h = 0; h < 64; ++h) dwp[h] = kl ? dwp[h] : 0.f;
-                quad_reduce64(dwp, lane);
+                for (int h = 0; h < 32; ++h) dwp[h] = kl ? dwp[h] : 0.f;
+                pair_reduce32(dwp, lane);
                 if (lane < 16) {
-                    const int qb = quad_base(lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dwx[(qb + i) * 4 + warp] += dwp[i];
+                    for (int i = 0; i < 2; ++i) dwx[(h0 + pair_base(lane) + i) * 4 + q] += dwp[i];
                 }
             }
-            // this tile's dK rows into the CTA's slice of the partial buffer, in two halves
+            // this tile's dK rows (this half's dims) into the CTA's slice of the partial buffer
             if (!wait_warp(bars.dk_full(), dkph, abort_flag)) { ok = false; break; }
             dkph ^= 1u;
             tc_fence_after();
+            {
+                uint32_t dkv[4][16];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (half == 1) {
+                for (int c = 0; c < 4; ++c)
+                    tmem_ld16_nowait(tmem + lane_addr + kColDk + 64 * hf + 16 * c, dkv[c]);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        old[i] = dk_on ? drow[16 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) {
-                    float a[16];
-                    tmem_ld16(tmem + lane_addr + kColDk + 64 * half + c, a);
+                for (int c = 0; c < 4; ++c) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        float4 o = old[c / 4 + i];
-                        o.x += a[4 * i]; o.y += a[4 * i + 1]; o.z += a[4 * i + 2]; o.w += a[4 * i + 3];
-                        old[c / 4 + i] = o;
+                        float4 o = old[4 * c + i];
+                        o.x += __uint_as_float(dkv[c][4 * i]);
+                        o.y += __uint_as_float(dkv[c][4 * i + 1]);
+                        o.z += __uint_as_float(dkv[c][4 * i + 2]);
+                        o.w += __uint_as_float(dkv[c][4 * i + 3]);
+                        old[4 * c + i] = o;
                     }
-                }
-                if (dk_on) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) drow[16 * half + i] = old[i];
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.dk_empty());
-        }
-        if (!ok) break;
-        // ---- the row's d_qi and d_w -----------------------------------------------------------
-        if (!wait_warp(bars.dq_full(), nrow_dq & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        for (int c = 0; c < kDi; c += 16) {
-            float a[16];
-            tmem_ld16(tmem + lane_addr + kColDq + c, a);
-            if (kl && key < P.H && idx_ok(row, P.rows, P.status)) {
-                float *dq = P.d_qi + ((int64_t)row * P.H + key) * kDi + c;
+            if (dk_on) {
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    *reinterpret_cast<float4 *>(dq + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+                for (int i = 0; i < 16; ++i) drow[i] = old[i];
             }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.dq_empty());
+        if (!ok) break;
+        // ---- the row's d_qi (this half's dims) and d_w --------------------------------------------
+        if (!wait_warp(bars.dq_full(), nrow_dq & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        {
+            uint32_t dqv[4][16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld16_nowait(tmem + lane_addr + kColDq + 64 * hf + 16 * c, dqv[c]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.dq_empty());
+            if (kl && key < P.H && idx_ok(row, P.rows, P.status)) {
+                float4 *dq = reinterpret_cast<float4 *>(P.d_qi + ((int64_t)row * P.H + key) * kDi + 64 * hf);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dq[4 * c + i] = make_float4(__uint_as_float(dqv[c][4 * i]), __uint_as_float(dqv[c][4 * i + 1]),
+                                                    __uint_as_float(dqv[c][4 * i + 2]), __uint_as_float(dqv[c][4 * i + 3]));
+            }
+        }
         ++nrow_dq;
         {
-            float d0 = 0.f;                  // orders the four warps' dwx columns before the sums
+            float d0 = 0.f;                  // orders every half's dwx entries before the sums
             if (!epi_reduce(d0, false, use, smem, bars, abort_flag)) { ok = false; break; }
         }
         if (tid < P.H)
@@ -807,10 +829,10 @@ bool kl_tc_plan(const li_kl_args &a, KlTcPlan *L) {
     L->ds_off = off;
     off += 2u * kChunk;
     const uint32_t arr = (uint32_t)((a.topk + kKeys - 1) / kKeys * kKeys) * 4u;
-    L->parr_off = off;
-    off += arr;
+    L->parr_off = off;                                   // two halves' shares, then p^ / dI
+    off += 2 * arr;
     L->iarr_off = off;
-    off += arr;
+    off += 2 * arr;
     off = (off + 1023u) / 1024u * 1024u;
     L->ki_off = off;
     L->ki_slots = 2;
