@@ -142,12 +142,12 @@ SCORE_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_score_tc.cu', 's
 ATTN_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_attn.cu', 'sparse_attention_token_lightning_b200/csrc/li_attn.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
 KL_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_kl_tc.cu', 'sparse_attention_token_lightning_b200/csrc/li_kl.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
 KERNEL_TRAFFIC = {
-    "causal_prefill": {"bytes": 68748544 + 9403392, "sources": SCORE_SOURCES,
-                       "src_sha256": "10fff75115b23a2cfef41bfacd512bf2b2d8421bd9c8d94e3929755982b94dad"},
-    "sparse_attention": {"bytes": 114396416 + 92227072, "sources": ATTN_SOURCES,
-                         "src_sha256": "5006949e3c5ce6bbf0a84a1f7b760832de5548945894a00b16fbf9078ecf9157"},
-    "kl_backward": {"bytes": 446973440 + 607046912, "sources": KL_SOURCES,
-                    "src_sha256": "391cf2631960e7dab5bc74bf37bc7d758bc5ab39c63f483d0638ca83fea96e05"},
+    "causal_prefill": {"bytes": 68750592 + 9553152, "sources": SCORE_SOURCES,
+                       "src_sha256": "4e4dabfaabcda2bf99f669f38e2fce627f3f181d28fe5231f9dfe916655b35f3"},
+    "sparse_attention": {"bytes": 113965568 + 91356160, "sources": ATTN_SOURCES,
+                         "src_sha256": "d0e4959646efe3081b8634981ea7ec2d13860a18dd64cd9532942416654fddf6"},
+    "kl_backward": {"bytes": 334605824 + 611836416, "sources": KL_SOURCES,
+                    "src_sha256": "0f6e31b98b67a32d92f5c2e7ea82d445bb71fff776bb30e1da0d708a70704d41"},
 }
 
 
