@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LI_ABI_VERSION 5
+#define LI_ABI_VERSION 6
 
 typedef enum li_layout {
     LI_LAYOUT_BSND = 0,     /* dense batch: q (B,S1,N1,D), k (B,S2,1,D), w (B,S1,N1)            */
@@ -375,14 +375,23 @@ li_status li_kl_grad(const li_kl_args *args, void *workspace, size_t workspace_b
  * [reading] the value rows are the key rows (all Dm dims; the rope dims only enter the scores).
  * The statistics m and l are the inputs li_kl_grad takes as softmax_max / softmax_sum.
  *
- * Layout BSND, all bf16 and dense: q (B,S1,G,Dm), k (B,S2,1,Dm), q_rope (B,S1,G,Dr) and k_rope
- * (B,S2,1,Dr) or both NULL (Dr = 0); sparse_indices (B,S1,1,topk) int32, positions in the row's
- * batch (as li_indexer writes them without output_idx_offset); a negative entry selects nothing,
- * an entry >= S2 selects nothing and sets LI_DEVERR_LENGTHS. Entries may repeat (each counts).
+ * Layouts, all bf16: q (B,S1,G,Dm) and q_rope (B,S1,G,Dr); keys either dense, layout_k =
+ * LI_LAYOUT_BSND: k (B,S2,1,Dm) and k_rope (B,S2,1,Dr), or paged, layout_k = LI_LAYOUT_PA_BSND
+ * (lightning_indexer, "Prototype": block_table and the paged key cache): k (num_blocks,
+ * block_size,1,Dm) and k_rope (num_blocks,block_size,1,Dr), key position v of batch b in cache
+ * row block_table[b * block_table_stride + v / block_size] * block_size + v % block_size.
+ * q_rope and k_rope are both NULL when Dr = 0. sparse_indices (B,S1,1,topk) int32, positions in
+ * the row's batch (as li_indexer writes them without output_idx_offset; S2 bounds them for both
+ * layouts); a negative entry selects nothing, an entry >= S2 selects nothing and sets
+ * LI_DEVERR_LENGTHS, a block-table entry outside [0, num_blocks) selects nothing and sets
+ * LI_DEVERR_TABLE. Entries may repeat (each counts).
  * Outputs, fp32: out (B,S1,G,Dm); softmax_max and softmax_sum (B,1,S1,G). A row that selects no
  * key gets out = 0, softmax_max = -inf, softmax_sum = 0.
  * Limits: G in [1, 32], Dm in {128, 256, 384, 512}, Dr in {0, 64}, topk in [1, 8192], S2 >= 1
- * when there are rows, scale > 0; q, k, q_rope, k_rope 16-byte aligned, the rest 4-byte aligned.
+ * when there are rows, scale > 0; q, k, q_rope, k_rope 16-byte aligned, the rest 4-byte aligned;
+ * PA_BSND: block_size in [1, 1024], num_blocks >= 1, block_table_stride >= ceil(S2/block_size);
+ * BSND: the block-table fields 0 / NULL. Argument errors return LI_ERR_INVALID_ARG before any
+ * launch.
  * Numerics: products and sums in fp32 on the tensor cores; the softmax weights enter the value
  * product rounded to bf16 (the normaliser l is the fp32 sum of the unrounded weights).
  * The workspace (li_sparse_attention_workspace_size: 256 bytes) holds the device status word
@@ -395,6 +404,10 @@ typedef struct li_attn_args {
     float scale;
     int32_t batch, s1, s2;                  /* B, S1 (query rows per batch), S2 (keys per batch) */
     int32_t G, Dm, Dr, topk;
+    int32_t layout_k;                       /* LI_LAYOUT_BSND or LI_LAYOUT_PA_BSND               */
+    const int32_t *block_table;             /* PA_BSND: (B, block_table_stride); else NULL       */
+    int32_t block_table_stride;             /* PA_BSND: >= ceil(S2 / block_size); else 0         */
+    int32_t num_blocks, block_size;         /* PA_BSND: >= 1 and 1..1024; else 0                 */
     int32_t reserved;                       /* must be 0                                         */
 } li_attn_args;
 li_status li_sparse_attention_workspace_size(const li_attn_args *args, size_t *bytes);

@@ -502,6 +502,7 @@ li_status validate_kl(const li_kl_args *a) {
         return fail(LI_ERR_INVALID_ARG, "a required input is NULL");
     if ((a->Dr > 0) != (a->q_rope != nullptr) || (a->Dr > 0) != (a->k_rope != nullptr))
         return fail(LI_ERR_INVALID_ARG, "q_rope and k_rope go with Dr > 0, and only with it");
+
     if (!(a->scale > 0.0f)) return fail(LI_ERR_INVALID_ARG, "scale must be positive");
     const void *ptrs[] = {a->q, a->k, a->q_rope, a->k_rope, a->qi, a->ki, a->w, a->sparse_indices,
                           a->softmax_max, a->softmax_sum};
@@ -591,6 +592,24 @@ li_status validate_attn(const li_attn_args *a, li::AttnLayout *L) {
         return fail(LI_ERR_INVALID_ARG, "q, k and sparse_indices are required");
     if ((a->Dr > 0) != (a->q_rope != nullptr) || (a->Dr > 0) != (a->k_rope != nullptr))
         return fail(LI_ERR_INVALID_ARG, "q_rope and k_rope go with Dr > 0, and only with it");
+    if (a->layout_k == LI_LAYOUT_PA_BSND) {
+        if (a->block_size < 1 || a->block_size > 1024)
+            return fail(LI_ERR_INVALID_ARG, "block_size=%d outside [1, 1024]", a->block_size);
+        if (a->num_blocks < 1) return fail(LI_ERR_INVALID_ARG, "num_blocks must be >= 1");
+        if ((int64_t)a->num_blocks * a->block_size > INT32_MAX)
+            return fail(LI_ERR_UNSUPPORTED, "more than 2^31-1 cache rows");
+        const int64_t need = ((int64_t)a->s2 + a->block_size - 1) / a->block_size;
+        if (a->block_table_stride < need)
+            return fail(LI_ERR_INVALID_ARG, "block_table_stride=%d below ceil(S2 / block_size)=%lld",
+                        a->block_table_stride, (long long)need);
+        if (rows > 0 && (!a->block_table || !aligned(a->block_table, 4)))
+            return fail(LI_ERR_INVALID_ARG, "PA_BSND needs a 4-byte aligned block_table");
+    } else if (a->layout_k == LI_LAYOUT_BSND) {
+        if (a->block_table || a->block_table_stride || a->num_blocks || a->block_size)
+            return fail(LI_ERR_INVALID_ARG, "block_table fields are for PA_BSND only");
+    } else {
+        return fail(LI_ERR_INVALID_ARG, "layout_k=%d must be BSND or PA_BSND", a->layout_k);
+    }
     if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->q_rope, 16) ||
         !aligned(a->k_rope, 16) || !aligned(a->sparse_indices, 4))
         return fail(LI_ERR_INVALID_ARG, "q, k and the rope parts must be 16-byte aligned");

@@ -111,6 +111,9 @@ static_assert(kTailOff % 1024 == 0, "tail alignment");
 struct AttnParams {
     const uint16_t *k, *k_rope;          // key rows (Dm) and their rope dims (Dr), bf16
     const int32_t *indices;              // [rows][topk]
+    const int32_t *block_table;          // paged keys: [B][bt_stride]; null for dense keys
+    int64_t key_rows;                    // rows of k: B * S2, or num_blocks * block_size
+    int32_t bt_stride, block_size, num_blocks, pad0;
     float *out, *smax, *ssum;            // [rows][G][Dm], [rows][G], [rows][G]
     uint32_t *status;
     int32_t *ticket;
@@ -178,7 +181,8 @@ __device__ void scheduler_role(const AttnParams &P, const CUtensorMap *tmq, cons
             S.row = row;
             S.tiles = tiles;
             S.n_eff = n_eff;
-            S.key_base = row >= 0 ? (int64_t)(row / P.s1) * P.s2 : 0;
+            // dense keys: the batch's first key row; paged keys: the batch (its block-table row)
+            S.key_base = row < 0 ? 0 : P.block_table ? (int64_t)(row / P.s1) : (int64_t)(row / P.s1) * P.s2;
             mbar_arrive(bars.rs_full(sl));
         }
         __syncwarp();
@@ -201,6 +205,7 @@ __device__ void scheduler_role(const AttnParams &P, const CUtensorMap *tmq, cons
 }
 
 // ---- gather: the selected key rows of each tile into the pair and rope slots -------------------
+template <bool kPaged>
 __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
                             volatile int *abort_flag) {
     const int t = threadIdx.x - 32 * kGatherWarp0;      // 0..127
@@ -229,9 +234,21 @@ __device__ void gather_role(const AttnParams &P, uint8_t *smem, const Bars &bars
                 const int pos = kKeys * j + key0 + 16 * i;
                 const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
                 if (v >= P.s2) err |= LI_DEVERR_LENGTHS;
-                // an unselected slot copies the batch's first key row (in bounds); its p is 0
-                int64_t kr = key_base + (v >= 0 && v < P.s2 ? v : 0);
-                if (!idx_ok(kr, (int64_t)(P.rows / P.s1) * P.s2, P.status)) kr = 0;
+                // an unselected slot copies an in-bounds row (the batch's first key, or cache row
+                // 0); its p is 0
+                int64_t kr;
+                if constexpr (kPaged) {
+                    // paged keys: the row of position v through the batch's block table
+                    kr = 0;
+                    if (v >= 0 && v < P.s2) {
+                        const int32_t blk = __ldg(P.block_table + key_base * P.bt_stride + v / P.block_size);
+                        if (blk >= 0 && blk < P.num_blocks) kr = (int64_t)blk * P.block_size + v % P.block_size;
+                        else err |= LI_DEVERR_TABLE;
+                    }
+                } else {
+                    kr = key_base + (v >= 0 && v < P.s2 ? v : 0);
+                }
+                if (!idx_ok(kr, P.key_rows, P.status)) kr = 0;
                 krow[i] = P.k + kr * P.Dm + 8 * piece;
                 rrow[i] = P.Dr > 0 ? P.k_rope + kr * P.Dr + 8 * piece : nullptr;
             }
@@ -416,7 +433,7 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 // key 16 q + (lane % 16) of the tile (q = warp % 4, the TMEM lanes of M = 64 scores) and heads
 // (lane / 16) HH .. + HH - 1 of it. Group 1 hands its statistics to group 0, which combines the
 // two partial outputs and writes the row.
-template <int NH>
+template <int NH, bool kPaged>
 __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bars,
                              volatile int *abort_flag, uint32_t tmem) {
     constexpr int HH = NH / 2;
@@ -459,7 +476,13 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
         for (int j = g; j < tiles; j += 2, ++kg, ++mine) {
             const int pos = kKeys * j + key;
             const int32_t v = pos < P.topk ? __ldg(ir + pos) : -1;
-            const bool valid = v >= 0 && v < P.s2;
+            bool valid = v >= 0 && v < P.s2;
+            if (kPaged && valid) {
+                // paged keys: a block-table entry out of range selects nothing (the gather
+                // reported it)
+                const int32_t blk = __ldg(P.block_table + (int64_t)(row / P.s1) * P.bt_stride + v / P.block_size);
+                valid = blk >= 0 && blk < P.num_blocks;
+            }
             if (!wait_warp(bars.s_full(g), kg & 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             float x[16];
@@ -631,7 +654,7 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
     if (!ok) *abort_flag = 1;
 }
 
-template <int NH>
+template <int NH, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_qr,
                    const AttnParams P) {
@@ -699,7 +722,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
 
     if (warp < kSoftWarps) {
-        softmax_role<NH>(P, smem, bars, abort_flag, tmem);
+        softmax_role<NH, kPaged>(P, smem, bars, abort_flag, tmem);
     } else if (warp == kSchedWarp) {
         scheduler_role(P, &tmap_q, &tmap_qr, smem, bars, abort_flag);
     } else if (warp == kQkWarp) {
@@ -709,7 +732,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (lane == 0) pv_role(P, smem, bars, abort_flag, tmem);
         __syncwarp();
     } else {
-        gather_role(P, smem, bars, abort_flag);
+        gather_role<kPaged>(P, smem, bars, abort_flag);
     }
 
     tc_fence_before();
@@ -783,6 +806,15 @@ cudaError_t launch_sparse_attention(const li_attn_args &a, uint32_t *status, int
     P.k = static_cast<const uint16_t *>(a.k);
     P.k_rope = static_cast<const uint16_t *>(a.k_rope);
     P.indices = a.sparse_indices;
+    if (a.layout_k == LI_LAYOUT_PA_BSND) {
+        P.block_table = a.block_table;
+        P.bt_stride = a.block_table_stride;
+        P.block_size = a.block_size;
+        P.num_blocks = a.num_blocks;
+        P.key_rows = (int64_t)a.num_blocks * a.block_size;
+    } else {
+        P.key_rows = (int64_t)a.batch * a.s2;
+    }
     P.out = out;
     P.smax = smax;
     P.ssum = ssum;
@@ -821,7 +853,10 @@ cudaError_t launch_sparse_attention(const li_attn_args &a, uint32_t *status, int
     } else {
         mr = mq;
     }
-    auto kern = L.N <= 16 ? sparse_attn_kernel<16> : sparse_attn_kernel<32>;
+    // paged keys have instantiations of their own, so the dense kernels carry no paged code
+    const bool paged = a.layout_k == LI_LAYOUT_PA_BSND;
+    auto kern = L.N <= 16 ? (paged ? sparse_attn_kernel<16, true> : sparse_attn_kernel<16, false>)
+                          : (paged ? sparse_attn_kernel<32, true> : sparse_attn_kernel<32, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;

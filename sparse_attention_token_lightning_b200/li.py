@@ -95,7 +95,10 @@ class LiAttnArgs(ctypes.Structure):
         ("k_rope", ctypes.c_void_p), ("sparse_indices", ctypes.c_void_p),
         ("scale", ctypes.c_float), ("batch", ctypes.c_int32), ("s1", ctypes.c_int32),
         ("s2", ctypes.c_int32), ("G", ctypes.c_int32), ("Dm", ctypes.c_int32),
-        ("Dr", ctypes.c_int32), ("topk", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("Dr", ctypes.c_int32), ("topk", ctypes.c_int32), ("layout_k", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p), ("block_table_stride", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -376,6 +379,16 @@ def make_attn_args(ap) -> LiAttnArgs:
     a.batch, a.s1, a.s2 = B, S1, ap.k.shape[1]
     a.G, a.Dm, a.Dr = G, Dm, 0 if ap.q_rope is None else ap.q_rope.shape[-1]
     a.topk = ap.sparse_indices.shape[-1]
+    bt = getattr(ap, "block_table", None)
+    if bt is not None:
+        # paged keys: k is the cache (num_blocks, block_size, 1, Dm), S2 the logical length
+        a.layout_k = LAYOUTS["PA_BSND"]
+        a.block_table = bt.data_ptr()
+        a.block_table_stride = bt.shape[1]
+        a.num_blocks, a.block_size = ap.k.shape[0], ap.k.shape[1]
+        a.s2 = int(ap.s2)
+    else:
+        a.layout_k = LAYOUTS["BSND"]
     return a
 
 

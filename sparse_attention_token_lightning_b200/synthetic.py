@@ -416,8 +416,12 @@ class AttnProblem:
     sparse_indices: torch.Tensor    # (B, S1, 1, topk) int32
     key_base: torch.Tensor          # (B * S1,) int64: key row of position 0 of the row's batch
     scale: float
+    # paged keys: k / k_rope are caches (num_blocks, block_size, 1, D) read through block_table
+    # (B, width); s2 is the logical key count per batch. None / 0 for dense keys.
+    block_table: Optional[torch.Tensor] = None
+    s2: int = 0
 
-    TENSORS = ("q", "k", "q_rope", "k_rope", "sparse_indices", "key_base")
+    TENSORS = ("q", "k", "q_rope", "k_rope", "sparse_indices", "key_base", "block_table")
 
     def to(self, device) -> "AttnProblem":
         kw = {f: (None if getattr(self, f) is None else getattr(self, f).to(device))
@@ -464,6 +468,31 @@ def attn_bsnd(B, S1, S2, G, Dm, Dr, topk, seed=0, causal=True, scale=None, name=
     return AttnProblem(name=name, q=q, k=k, q_rope=q_rope, k_rope=k_rope, sparse_indices=sel,
                        key_base=key_base,
                        scale=float(scale) if scale is not None else 1.0 / math.sqrt(Dm + Dr))
+
+
+def attn_paged(ap: AttnProblem, block_size: int, seed: int = 0, spare_blocks: int = 0) -> AttnProblem:
+    """The same problem with its keys in a paged cache: batch b's ceil(S2 / block_size) blocks are
+    taken from a seeded random permutation of all physical blocks (plus `spare_blocks` unused
+    ones); key position v of batch b sits in block block_table[b, v // block_size] at row
+    v % block_size. Positions past S2 in a batch's last block are zero."""
+    g = _gen(seed)
+    B, S2 = ap.k.shape[0], ap.k.shape[1]
+    nb = -(-S2 // block_size)
+    NB = B * nb + int(spare_blocks)
+    perm = torch.randperm(NB, generator=g)[: B * nb].reshape(B, nb).to(torch.int32)
+
+    def page(t):
+        if t is None:
+            return None
+        D = t.shape[-1]
+        cache = torch.zeros((NB, block_size, 1, D), dtype=t.dtype)
+        flat = torch.zeros((B, nb * block_size, 1, D), dtype=t.dtype)
+        flat[:, :S2] = t
+        cache[perm.reshape(-1).long()] = flat.reshape(B * nb, block_size, 1, D)
+        return cache
+
+    return ap.replace(k=page(ap.k), k_rope=page(ap.k_rope), block_table=perm, s2=S2,
+                      name=ap.name + f"_paged{block_size}")
 
 
 def attn_config(name: str, seed: int = 0) -> AttnProblem:

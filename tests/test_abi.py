@@ -51,11 +51,11 @@ def test_test_builds_export_every_declared_symbol(which):
     exported = set(re.findall(r" T (li_[a-z_]+)$", out, flags=re.M))
     missing = [n for n in declared_functions() if n not in exported]
     assert not missing, missing
-    assert li.load(path).li_abi_version() == 5
+    assert li.load(path).li_abi_version() == 6
 
 
 def test_abi_version(L):
-    assert li.li_abi_version() == 5
+    assert li.li_abi_version() == 6
 
 
 @pytest.mark.parametrize("cls,cname", [(li.LiArgs, "li_args"), (li.LiPlanInfo, "li_plan_info")])
@@ -289,6 +289,13 @@ def test_plan_reports_schedule_and_kernel_count(L):
     assert L.li_plan(ctypes.byref(_args()), None) == 1
 
 
+def _paged(**over):
+    """Paged-key fields of li_attn_args (S2 = 64 keys in blocks of 32), with overrides."""
+    kw = dict(layout_k=2, block_table=0x60000, block_table_stride=2, num_blocks=8, block_size=32)
+    kw.update(over)
+    return kw
+
+
 def _attn_args(**kw):
     a = li.LiAttnArgs()
     a.q, a.k, a.sparse_indices = 0x10000, 0x20000, 0x30000
@@ -303,7 +310,12 @@ def _attn_args(**kw):
     dict(G=0), dict(G=33), dict(Dm=64), dict(Dm=576), dict(Dm=200), dict(Dr=32),
     dict(Dr=64), dict(q_rope=0x40000, k_rope=0x50000), dict(topk=0), dict(topk=8193),
     dict(scale=0.0), dict(scale=float("inf")), dict(reserved=1), dict(batch=-1), dict(s2=0),
-    dict(q=None), dict(sparse_indices=None), dict(q=0x10008), dict(sparse_indices=0x30002)])
+    dict(q=None), dict(sparse_indices=None), dict(q=0x10008), dict(sparse_indices=0x30002),
+    # key layouts: TND is not one; PA_BSND needs a block table, a block size in [1, 1024], at
+    # least one block and a table wide enough for S2; BSND takes none of the paged fields
+    dict(layout_k=1), _paged(block_table=None), _paged(block_size=0), _paged(block_size=1025),
+    _paged(num_blocks=0), _paged(block_table_stride=1), _paged(block_table=0x60002),
+    dict(block_table=0x60000), dict(block_size=32)])
 def test_invalid_attention_args_rejected_on_host(L, kw):
     n = ctypes.c_size_t(0)
     assert L.li_sparse_attention_workspace_size(ctypes.byref(_attn_args(**kw)), ctypes.byref(n)) == 1
@@ -312,7 +324,9 @@ def test_invalid_attention_args_rejected_on_host(L, kw):
 
 @pytest.mark.parametrize("kw", [dict(), dict(Dr=64, q_rope=0x40000, k_rope=0x50000),
                                 dict(G=32, Dm=512, Dr=64, q_rope=0x40000, k_rope=0x50000),
-                                dict(G=1, Dm=128), dict(batch=0, s2=0)])
+                                dict(G=1, Dm=128), dict(batch=0, s2=0), _paged(),
+                                _paged(block_size=1, block_table_stride=64),
+                                _paged(block_size=1024, block_table_stride=1)])
 def test_attention_args_accepted(L, kw):
     n = ctypes.c_size_t(0)
     assert L.li_sparse_attention_workspace_size(ctypes.byref(_attn_args(**kw)), ctypes.byref(n)) == 0

@@ -166,6 +166,51 @@ def test_deterministic_reruns():
         assert torch.equal(x.view(torch.int32), y.view(torch.int32))
 
 
+PAGED = {
+    # (dense problem, block size, spare blocks)
+    "g16_dm512_rope_bs64": (lambda: SMALL["g16_dm512_rope"](), 64, 3),
+    "g5_dm128_bs1": (lambda: SMALL["g5_dm128"](), 1, 7),
+    "g20_dm384_nomask_bs48": (lambda: SMALL["g20_dm384_nomask"](), 48, 0),
+    "interleaved_padding_bs16": (lambda: _interleaved(11), 16, 2),
+}
+
+
+@pytest.mark.parametrize("name", list(PAGED))
+def test_paged_keys_match_dense_keys(orc, name):
+    """Keys in a paged cache (PA_BSND, blocks in a seeded random order) give the same outputs as
+    the dense keys, bit for bit (the same rows are gathered in the same order), and the oracle's
+    values on the dense problem."""
+    make, bs, spare = PAGED[name]
+    ap = make()
+    pp = synthetic.attn_paged(ap, bs, seed=5, spare_blocks=spare)
+    a = run(ap)
+    b = run(pp)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    check_attention(orc, ap, *b, label=name)
+
+
+def test_paged_bad_block_table_entry_reported(orc):
+    ap = synthetic.attn_bsnd(1, 30, 70, 4, 128, 0, 20, seed=12)
+    pp = synthetic.attn_paged(ap, 16, seed=2)
+    bt = pp.block_table.clone()
+    bt[0, 1] = bt.max() + 5                          # positions 16..31 point past the cache
+    pp = pp.replace(block_table=bt)
+    g = pp.to("cuda")
+    a = li.make_attn_args(g)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    out = torch.empty((1, 30, 4, 128), dtype=torch.float32, device="cuda")
+    sm = torch.empty((1, 1, 30, 4), dtype=torch.float32, device="cuda")
+    ss = torch.empty((1, 1, 30, 4), dtype=torch.float32, device="cuda")
+    li.li_sparse_attention(a, ws, out, sm, ss)
+    st, bits = li.li_check_status(ws)
+    assert st == 6 and bits & li.DEVERR_TABLE
+    # the affected keys select nothing: the rows equal the oracle on the selection without them
+    sel = ap.sparse_indices.clone()
+    sel[(sel >= 16) & (sel < 32)] = -1
+    check_attention(orc, ap.replace(sparse_indices=sel), out, sm, ss, label="bad table")
+
+
 def test_out_of_range_index_reported():
     ap = synthetic.attn_bsnd(1, 20, 30, 4, 128, 0, 16, seed=10)
     ap.sparse_indices[0, 3, 0, 2] = 30                 # == S2: selects nothing, reported

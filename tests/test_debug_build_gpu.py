@@ -99,6 +99,8 @@ ATTN = {
     "g16_dm512_rope": lambda: synthetic.attn_bsnd(1, 300, 300, 16, 512, 64, 200, seed=1),
     "g20_dm384_nomask": lambda: synthetic.attn_bsnd(1, 64, 500, 20, 384, 64, 500, seed=4,
                                                     causal=False),
+    "g16_paged_bs48": lambda: synthetic.attn_paged(
+        synthetic.attn_bsnd(2, 100, 300, 16, 512, 64, 150, seed=6), 48, seed=1, spare_blocks=2),
 }
 
 
