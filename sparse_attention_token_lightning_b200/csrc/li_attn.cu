@@ -16,8 +16,10 @@
 //   warp 8      scheduler: takes a ticket, finds the row's last selected position (the tile
 //               count), publishes the row, and loads the row's Q tile (all heads, Dm + Dr dims)
 //               with TMA into a 128-byte swizzled buffer
-//   warps 11-14 gather: each tile's 64 key rows are copied with cp.async (16 bytes per thread and
-//               copy, eight threads per 128-byte segment) into 128-byte swizzled chunks of 64 dims;
+//   warps 11-14 gather: each tile's 64 key rows (dense keys at the batch's row plus the index, or
+//               paged keys through the batch's block-table row; the paged instantiations carry
+//               that lookup) are copied with cp.async (16 bytes per thread and copy, eight
+//               threads per 128-byte segment) into 128-byte swizzled chunks of 64 dims;
 //               two chunks form a 16 KB pair slot, the rope dims an 8 KB rope slot; one barrier
 //               per tile signals its arrival
 //   warp 9      allocates TMEM; one thread issues the scores S = sum over chunks K_chunk Q_chunk^T
