@@ -144,8 +144,8 @@ KL_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_kl_tc.cu', 'sparse_
 KERNEL_TRAFFIC = {
     "causal_prefill": {"bytes": 68750592 + 9553152, "sources": SCORE_SOURCES,
                        "src_sha256": "4e4dabfaabcda2bf99f669f38e2fce627f3f181d28fe5231f9dfe916655b35f3"},
-    "sparse_attention": {"bytes": 114084352 + 91415296, "sources": ATTN_SOURCES,
-                         "src_sha256": "d6bef0d881ed0c50cd328964ffcdaf2968f155ef6283200922da98fc7a404e8b"},
+    "sparse_attention": {"bytes": 113986816 + 90557952, "sources": ATTN_SOURCES,
+                         "src_sha256": "b645dcc38def059a2d33028e0c098f925b9346a7daef84161156994a2e9d97bc"},
     "kl_backward": {"bytes": 334605824 + 611836416, "sources": KL_SOURCES,
                     "src_sha256": "0f6e31b98b67a32d92f5c2e7ea82d445bb71fff776bb30e1da0d708a70704d41"},
 }

@@ -469,9 +469,10 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
         if (lane == 0) mbar_arrive(bars.rs_empty(sl));
         if (row < 0) break;
         const int32_t *ir = P.indices + (int64_t)row * P.topk;
-        float m_ref[NH], m_true[NH], l_part[HH];
+        // references and true maxima of this thread's heads hb .. hb + HH - 1
+        float mr[HH], mt[HH], l_part[HH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) { m_ref[h] = -kInf; m_true[h] = -kInf; }
+        for (int i = 0; i < HH; ++i) { mr[i] = -kInf; mt[i] = -kInf; }
 #pragma unroll
         for (int i = 0; i < HH; ++i) l_part[i] = 0.f;
         int mine = 0;                                    // tiles of this group in the row
@@ -516,30 +517,39 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
             if (writer) rb[my_head * 4 + q] = wm;
             mbar_arrive(bars.red_full(g, kg & 1));
             if (!wait_warp(bars.red_full(g, kg & 1), (kg >> 1) & 1u, abort_flag)) { ok = false; break; }
-            bool rescale = false;
-            float alpha[NH];
+            // this thread's heads only; the other half of the warp holds the rest
+            bool moved = false;
+            float alpha[HH];
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                const float4 r4 = *reinterpret_cast<const float4 *>(rb + h * 4);
+            for (int i = 0; i < HH; ++i) {
+                const float4 r4 = *reinterpret_cast<const float4 *>(rb + (hb + i) * 4);
                 const float tm = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                m_true[h] = fmaxf(m_true[h], tm);
-                const float ref = tm - m_ref[h] > kSlack ? tm : m_ref[h];
-                alpha[h] = ref != m_ref[h] ? exp2f((m_ref[h] - ref) * kLog2e) : 1.f;
-                rescale |= ref != m_ref[h];
-                m_ref[h] = ref;
+                mt[i] = fmaxf(mt[i], tm);
+                const float ref = tm - mr[i] > kSlack ? tm : mr[i];
+                alpha[i] = ref != mr[i] ? exp2f((mr[i] - ref) * kLog2e) : 1.f;
+                moved |= ref != mr[i];
+                mr[i] = ref;
             }
+            // every warp of the group sees the same tile maxima, so the vote is group-wide
+            const bool rescale = __any_sync(0xffffffffu, moved);
             float p[HH];
 #pragma unroll
             for (int i = 0; i < HH; ++i) {
-                const float a = half ? alpha[HH + i] : alpha[i];
-                const float r = half ? m_ref[HH + i] : m_ref[i];
-                p[i] = valid ? exp2f((y[i] - r) * kLog2e) : 0.f;
-                l_part[i] = l_part[i] * a + p[i];
+                p[i] = valid ? exp2f((y[i] - mr[i]) * kLog2e) : 0.f;
+                l_part[i] = l_part[i] * alpha[i] + p[i];
             }
             // this group's O (accumulated up to its previous tile) follows a moved reference
             if (rescale && mine > 0) {
                 if (!wait_warp(bars.o_done(g), (kg - 1) & 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
+                // every head's factor: own half and the other half's, from lane ^ 16
+                float af[NH];
+#pragma unroll
+                for (int i = 0; i < HH; ++i) {
+                    const float other = __shfl_xor_sync(0xffffffffu, alpha[i], 16);
+                    af[i] = half ? other : alpha[i];
+                    af[HH + i] = half ? alpha[i] : other;
+                }
                 for (int b = 0; b < P.npairs; ++b) {
 #pragma unroll
                     for (int c = 0; c < NH; c += 16) {
@@ -547,7 +557,7 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
                         float o[16];
                         tmem_ld16(ta, o);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] *= alpha[c + i];
+                        for (int i = 0; i < 16; ++i) o[i] *= af[c + i];
                         tmem_st16(ta, o);
                     }
                 }
@@ -576,6 +586,17 @@ __device__ void softmax_role(const AttnParams &P, uint8_t *smem, const Bars &bar
             if (writer) sb[my_head * 4 + q] = ws;
             mbar_arrive(bars.sum_full(g, nrow & 1));
             if (!wait_warp(bars.sum_full(g, nrow & 1), (nrow >> 1) & 1u, abort_flag)) { ok = false; break; }
+        }
+        // every head's reference and true maximum (own half and the other half's)
+        float m_ref[NH], m_true[NH];
+#pragma unroll
+        for (int i = 0; i < HH; ++i) {
+            const float orr = __shfl_xor_sync(0xffffffffu, mr[i], 16);
+            const float ort = __shfl_xor_sync(0xffffffffu, mt[i], 16);
+            m_ref[i] = half ? orr : mr[i];
+            m_ref[HH + i] = half ? mr[i] : orr;
+            m_true[i] = half ? ort : mt[i];
+            m_true[HH + i] = half ? mt[i] : ort;
         }
         float l_tot[NH];
 #pragma unroll
