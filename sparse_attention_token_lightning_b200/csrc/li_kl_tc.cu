@@ -367,29 +367,6 @@ __device__ __forceinline__ bool epi_reduce(float &v, bool is_max, uint32_t &use,
     return ok;
 }
 
-// Sums of 32 per-head values over the 16 lanes of a half-warp, transposed: afterwards lane l
-// (of either half) holds the sums of heads pair_base(l) and pair_base(l) + 1 in a[0..1], where
-// lanes with bit (8 >> s) set kept the upper half at step s.
-__device__ __forceinline__ int pair_base(int lane) {
-    return ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 + ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
-}
-__device__ __forceinline__ void pair_reduce32(float (&a)[32], int lane) {
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int bit = 8 >> s;
-        const int half = 16 >> s;
-        const bool up = (lane & bit) != 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (i < half) {
-                const float keep = up ? a[i + half] : a[i];
-                const float send = up ? a[i] : a[i + half];
-                a[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-            }
-        }
-    }
-}
-
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 template <int NG>
@@ -401,6 +378,10 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
     const int hf = warp >> 2;                             // half: heads (and dK dims) of the key
     const bool kl = lane < 16;                            // lanes holding a key (or head) row
     const int key = 16 * q + (lane & 15);                 // key of the tile / head of d_qi
+    // the 16-lane TMEM loads spread a quarter's 16 keys over the whole warp: lane pair
+    // (t, t ^ 2) shares key key2, each lane the heads of parity par
+    const int key2 = 16 * q + (lane >> 2) + 8 * (lane & 1);
+    const int par = (lane >> 1) & 1;
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     const RowSlot *slots = reinterpret_cast<const RowSlot *>(smem + kRowSlotOff);
     const int arr_n = (P.topk + kKeys - 1) / kKeys * kKeys;
@@ -412,7 +393,6 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
     const float kInf = __int_as_float(0x7f800000);
     uint32_t sph = 0, dsph = 0, dkph = 0, nrow_dq = 0, use = 0;
     const float scale2 = P.scale * kLog2e;                // scale in log2 units
-    constexpr int kMainHalf = NG / 2;                     // main heads of this half
     const int h0 = 32 * hf;                               // first indexer head of this half
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -447,58 +427,61 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         }
         // ---- pass 1: each half's share of p^ and I of every selected key ----------------------
         for (int j = 0; j < tiles; ++j) {
-            const int pos = kKeys * j + key;
-            const int32_t v = kl && pos < P.topk ? __ldg(ir + pos) : -1;
-            const bool valid = v >= 0 && v < P.s2;
+            const int pos2 = kKeys * j + key2;
+            const int32_t v2 = pos2 < P.topk ? __ldg(ir + pos2) : -1;
+            const bool valid2 = v2 >= 0 && v2 < P.s2;
             if (!wait_warp(bars.s_full(), sph, abort_flag)) { ok = false; break; }
             sph ^= 1u;
             tc_fence_after();
-            // this half's main heads and indexer heads, loaded with one wait, then released
-            uint32_t smr[NG / 16][16], sir[2][16];
+            // this half's main and indexer heads of key key2, the parity-par ones in this lane,
+            // loaded with one wait, then released
+            uint32_t smr[NG / 16][8], sir[2][8];
 #pragma unroll
-            for (int c = 0; c < NG / 16; ++c) tmem_ld16_nowait(tmem + lane_addr + kColSm + 16 * c, smr[c]);
+            for (int c = 0; c < NG / 16; ++c) tmem_ld16x16_nowait(tmem + lane_addr + kColSm + 16 * c, smr[c]);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 if (h0 + 16 * c < P.Nh) {
-                    tmem_ld16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, sir[c]);
+                    tmem_ld16x16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, sir[c]);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) sir[c][i] = 0u;
+                    for (int i = 0; i < 8; ++i) sir[c][i] = 0u;
                 }
             }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_empty());
-            // I share = sum over this half's heads of w_h ReLU(S~_h), two heads per packed FMA
-            float2 ia = make_float2(0.f, 0.f);
+            // I share over this lane's indexer heads h0 + 16 c + par + 2 i
+            float ia = 0.f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    const float2 w2 = *reinterpret_cast<const float2 *>(rw + h0 + 16 * c + i);
-                    ia = __ffma2_rn(w2, make_float2(fmaxf(__uint_as_float(sir[c][i]), 0.f),
-                                                    fmaxf(__uint_as_float(sir[c][i + 1]), 0.f)), ia);
-                }
-            }
-            // p^ share = sum over this half's main heads of exp(scale S_g - max_g) / sum_g
+                for (int i = 0; i < 8; ++i)
+                    ia = fmaf(rw[h0 + 16 * c + par + 2 * i], fmaxf(__uint_as_float(sir[c][i]), 0.f), ia);
+            // p^ share over this lane's main heads of the half: g = par + 2 i of 16 columns
             // (register indices fixed at compile time for each half)
             auto main_share = [&](auto half_c) -> float {
-                constexpr int G0 = decltype(half_c)::value * kMainHalf;
+                constexpr int HF = decltype(half_c)::value;
+                constexpr int C = NG == 16 ? 0 : HF;              // the 16 columns of this half
+                constexpr int I0 = NG == 16 ? 4 * HF : 0;         // registers of this half
+                constexpr int NI = NG == 16 ? 4 : 8;
                 float acc = 0.f;
 #pragma unroll
-                for (int i = 0; i < kMainHalf; ++i) {
-                    const int g = G0 + i;
-                    const float sg = __uint_as_float(smr[g / 16][g % 16]);
+                for (int i = I0; i < I0 + NI; ++i) {
+                    const int g = 16 * C + par + 2 * i;
+                    const float sg = __uint_as_float(smr[C][i]);
                     if (g < P.G) acc = fmaf(exp2f(fmaf(sg, scale2, -rmax[g])), rsum[g], acc);
                 }
                 return acc;
             };
-            const float ph = hf == 0 ? main_share(std::integral_constant<int, 0>{})
-                                     : main_share(std::integral_constant<int, 1>{});
-            if (kl && pos < tiles * kKeys) {
-                parr[hf * arr_n + pos] = valid ? ph : 0.f;
-                iarr[hf * arr_n + pos] = valid ? ia.x + ia.y : (hf == 0 ? -kInf : 0.f);
+            float ph = hf == 0 ? main_share(std::integral_constant<int, 0>{})
+                               : main_share(std::integral_constant<int, 1>{});
+            // the key's half-shares: this lane's heads plus the partner lane's
+            ph += __shfl_xor_sync(0xffffffffu, ph, 2);
+            ia += __shfl_xor_sync(0xffffffffu, ia, 2);
+            if (par == 0 && pos2 < tiles * kKeys) {
+                parr[hf * arr_n + pos2] = valid2 ? ph : 0.f;
+                iarr[hf * arr_n + pos2] = valid2 ? ia : (hf == 0 ? -kInf : 0.f);
             }
         }
         if (!ok) break;
@@ -541,29 +524,32 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
         // d_w: each (head, quarter) entry of dwx has one owner (the half holding the head), which
         // adds its tiles' sums in tile order; the four quarters are added in order at the row's
         // end. The previous row's final read of dwx came before the exchanges above.
-        if (lane < 16) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) dwx[(h0 + pair_base(lane) + i) * 4 + q] = 0.f;
-        }
+        // the head whose d_w sum over a quarter's keys this lane holds after the reduction below
+        const int dw_idx = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + (lane & 1);
+        const int dw_head = h0 + 16 * (dw_idx >> 3) + par + 2 * (dw_idx & 7);
+        dwx[dw_head * 4 + q] = 0.f;
         float *slice = P.d_part + (int64_t)blockIdx.x * P.key_rows * kDi;
         for (int j = 0; j < tiles; ++j) {
-            const int pos = kKeys * j + key;
+            const int pos = kKeys * j + key;                  // dK rows: lanes 0-15, key `key`
             const int32_t v = kl && pos < P.topk ? __ldg(ir + pos) : -1;
             const bool valid = v >= 0 && v < P.s2;
-            const float dI = kl && pos < n ? parr[pos] : 0.f;
+            const int pos2 = kKeys * j + key2;                // dS and d_w: every lane, key `key2`
+            const int32_t v2 = pos2 < P.topk ? __ldg(ir + pos2) : -1;
+            const bool valid2 = v2 >= 0 && v2 < P.s2;
+            const float dI2 = pos2 < n ? parr[pos2] : 0.f;
             if (!wait_warp(bars.s_full(), sph, abort_flag)) { ok = false; break; }
             sph ^= 1u;
             tc_fence_after();
-            // this tile's S~, this half's heads (the MMA recomputes the columns for the next tile
-            // once released)
-            uint32_t svr[2][16];
+            // this tile's S~, this half's heads of key key2, the parity-par ones in this lane (the
+            // MMA recomputes the columns for the next tile once released)
+            uint32_t svr[2][8];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 if (h0 + 16 * c < P.Nh) {
-                    tmem_ld16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, svr[c]);
+                    tmem_ld16x16_nowait(tmem + lane_addr + kColSi + h0 + 16 * c, svr[c]);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) svr[c][i] = 0u;
+                    for (int i = 0; i < 8; ++i) svr[c][i] = 0u;
                 }
             }
             tmem_wait_ld();
@@ -574,43 +560,47 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             if (!wait_warp(bars.ds_empty(), dsph ^ 1u, abort_flag)) { ok = false; break; }
             dsph ^= 1u;
             uint8_t *dsb = smem + P.ds_off;
-            float dwp[32];
+            // dS and the d_w terms of this lane's 16 heads h0 + 16 c + par + 2 i (index 8 c + i)
+            float dsv[16], dwp[16];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const uint32_t *a = svr[c];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int h = h0 + 16 * c + par + 2 * i;
+                    const float sv = __uint_as_float(svr[c][i]);
+                    dsv[8 * c + i] = valid2 && h < P.H && sv > 0.f ? dI2 * rw[h] : 0.f;
+                    dwp[8 * c + i] = valid2 && h < P.H ? dI2 * fmaxf(sv, 0.f) : 0.f;
+                }
+            }
+            {
+                // consecutive head pairs: lane par = 0 assembles heads h0 .. h0 + 15 of key2
+                // (its even heads, the partner's odd ones), lane par = 1 heads h0 + 16 .. h0 + 31
                 uint32_t hi[8], lo[8];
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    float ds2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int h = h0 + 16 * c + i + u;
-                        const float s = __uint_as_float(a[i + u]);
-                        ds2[u] = valid && h < P.H && s > 0.f ? dI * rw[h] : 0.f;
-                        dwp[16 * c + i + u] = valid && h < P.H ? dI * fmaxf(s, 0.f) : 0.f;
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float send = par ? dsv[i] : dsv[8 + i];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+                    const float ev = par ? recv : dsv[i];
+                    const float od = par ? dsv[8 + i] : recv;
                     // hi = bf16(dS) and lo = bf16(dS - hi), two heads per conversion
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(ds2[0], ds2[1]);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(ev, od);
                     const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h2);
-                    const __nv_bfloat162 l2 =
-                        __floats2bfloat162_rn(ds2[0] - __uint_as_float(hb << 16),
-                                              ds2[1] - __uint_as_float(hb & 0xffff0000u));
-                    hi[i / 2] = hb;
-                    lo[i / 2] = *reinterpret_cast<const uint32_t *>(&l2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(ev - __uint_as_float(hb << 16),
+                                                                    od - __uint_as_float(hb & 0xffff0000u));
+                    hi[i] = hb;
+                    lo[i] = *reinterpret_cast<const uint32_t *>(&l2);
                 }
-                if (kl) {
-                    // this key's row, 16-byte chunks (hc / 8, hc / 8 + 1) of head column
-                    // hc = h0 + 16 c, swizzled by key % 8
+                // key2's row, 16-byte chunks of heads hb2 .. hb2 + 15, swizzled by key2 % 8
+                const int hb2 = h0 + 16 * par;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t chunk = (uint32_t)((h0 + 16 * c) / 8 + u);
-                        const uint32_t off = (uint32_t)(key >> 3) * 1024u + (uint32_t)(key & 7) * 128u +
-                                             ((chunk ^ (uint32_t)(key & 7)) << 4);
-                        *reinterpret_cast<uint4 *>(dsb + off) =
-                            make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
-                        *reinterpret_cast<uint4 *>(dsb + kChunk + off) =
-                            make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
-                    }
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t chunk = (uint32_t)(hb2 / 8 + u);
+                    const uint32_t off = (uint32_t)(key2 >> 3) * 1024u + (uint32_t)(key2 & 7) * 128u +
+                                         ((chunk ^ (uint32_t)(key2 & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(dsb + off) =
+                        make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+                    *reinterpret_cast<uint4 *>(dsb + kChunk + off) =
+                        make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
                 }
             }
             fence_async_smem();
@@ -623,15 +613,25 @@ __device__ void epilogue_role(const KlTcParams &P, uint8_t *smem, const Bars &ba
             float4 old[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) old[i] = dk_on ? drow[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-            // d_w: this half's per-head sums over the warp's 16 keys, added to its dwx entries
+            // d_w: per-head sums over the quarter's 16 keys (lanes differing in bits 0, 2, 3, 4);
+            // each step halves the values a lane holds, the lanes with the step's bit set keeping
+            // the upper half, so lane l ends with head dw_head
             {
 #pragma unroll
-                for (int h = 0; h < 32; ++h) dwp[h] = kl ? dwp[h] : 0.f;
-                pair_reduce32(dwp, lane);
-                if (lane < 16) {
+                for (int st = 0; st < 4; ++st) {
+                    const int m = st == 0 ? 16 : st == 1 ? 8 : st == 2 ? 4 : 1;
+                    const int half_n = 8 >> st;
+                    const bool up = (lane & m) != 0;
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) dwx[(h0 + pair_base(lane) + i) * 4 + q] += dwp[i];
+                    for (int k = 0; k < 8; ++k) {
+                        if (k < half_n) {
+                            const float keep = up ? dwp[k + half_n] : dwp[k];
+                            const float send = up ? dwp[k] : dwp[k + half_n];
+                            dwp[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                        }
+                    }
                 }
+                dwx[dw_head * 4 + q] += dwp[0];
             }
             // this tile's dK rows (this half's dims) into the CTA's slice of the partial buffer
             if (!wait_warp(bars.dk_full(), dkph, abort_flag)) { ok = false; break; }

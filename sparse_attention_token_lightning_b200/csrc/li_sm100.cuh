@@ -185,6 +185,17 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[1
         : "r"(taddr)
         : "memory");
 }
+// 16 TMEM lanes x 16 fp32 columns spread over the whole warp (shape 16x64b, 8 registers):
+// thread t holds lane (t >> 2) + 8 (t & 1) of the 16, columns ((t >> 1) & 1) + 2 i, i < 8.
+// No wait: several loads in flight, then one tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld16x16_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
