@@ -142,12 +142,12 @@ SCORE_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_score_tc.cu', 's
 ATTN_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_attn.cu', 'sparse_attention_token_lightning_b200/csrc/li_attn.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
 KL_SOURCES = ('sparse_attention_token_lightning_b200/csrc/li_kl_tc.cu', 'sparse_attention_token_lightning_b200/csrc/li_kl.cuh', 'sparse_attention_token_lightning_b200/csrc/li_internal.cuh', 'sparse_attention_token_lightning_b200/csrc/li_sm100.cuh')
 KERNEL_TRAFFIC = {
-    "causal_prefill": {"bytes": 68750592 + 9553152, "sources": SCORE_SOURCES,
-                       "src_sha256": "4e4dabfaabcda2bf99f669f38e2fce627f3f181d28fe5231f9dfe916655b35f3"},
-    "sparse_attention": {"bytes": 113986816 + 90557952, "sources": ATTN_SOURCES,
-                         "src_sha256": "b645dcc38def059a2d33028e0c098f925b9346a7daef84161156994a2e9d97bc"},
-    "kl_backward": {"bytes": 334605824 + 611836416, "sources": KL_SOURCES,
-                    "src_sha256": "0f6e31b98b67a32d92f5c2e7ea82d445bb71fff776bb30e1da0d708a70704d41"},
+    "causal_prefill": {"bytes": 68751360 + 9356800, "sources": SCORE_SOURCES,
+                       "src_sha256": "0095f6af9f2a659de9051d799cffc612e39053c51bce781b29188ccd99b6dbb1"},
+    "sparse_attention": {"bytes": 114988544 + 90959360, "sources": ATTN_SOURCES,
+                         "src_sha256": "85c665056494cd6af8891ba21c3073d1d5b42028e4eb8c30becb916f8f960201"},
+    "kl_backward": {"bytes": 340291840 + 611383296, "sources": KL_SOURCES,
+                    "src_sha256": "b6e122e3ad169be982fbbcac26ef1a02db549224c351af4bc4412770a057ef56"},
 }
 
 
