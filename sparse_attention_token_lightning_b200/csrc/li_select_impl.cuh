@@ -32,7 +32,7 @@ struct Smem {
     int32_t s_skip[4];      // one flag per sort pass, so no pass resets a flag still being read
     float red_min[kWarps], red_max[kWarps];
     float s_vmin, s_vmax;
-    int32_t s_cut, s_maxbin, s_total;
+    int32_t s_cut, s_maxbin;
     int32_t s_append;       // candidate append counter of the long-row path (only used there)
     uint32_t *dbg;          // bounds-checked build: the status word (set at kernel start)
 };
@@ -256,9 +256,10 @@ __device__ __forceinline__ int32_t bucket_of(float v, float vmin, float scale, i
     return nb - 1 - b;
 }
 
-// Block-wide exclusive scan of one value per thread; returns the thread's exclusive prefix and
-// leaves the total in *total.
-__device__ __forceinline__ int32_t block_exclusive_scan(int32_t x, int32_t *total, Smem &sm) {
+// Block-wide exclusive scan of one value per thread; returns the thread's exclusive prefix. One
+// barrier: every warp adds up the totals of the warps before it itself. The caller must pass a
+// barrier before sm.wsum is written again.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t x, Smem &sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t incl = x;
 #pragma unroll
@@ -268,70 +269,89 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t x, int32_t *tota
     }
     if (lane == 31) sm.wsum[0][warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        const int32_t v = lane < kWarps ? sm.wsum[0][lane] : 0;
-        int32_t vi = v;
+    int32_t before = lane < warp ? sm.wsum[0][lane] : 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t t = __shfl_up_sync(0xffffffffu, vi, o);
-            if (lane >= o) vi += t;
-        }
-        if (lane < kWarps) sm.wsum[1][lane] = vi - v;
-        if (lane == 31) sm.s_total = vi;
-    }
-    __syncthreads();
-    *total = sm.s_total;
-    return sm.wsum[1][warp] + incl - x;
+    for (int o = kWarps / 2; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+    return __shfl_sync(0xffffffffu, before, 0) + incl - x;
 }
 
 // Turns the bucket counts into output start positions (exclusive scan in bucket order),
 // records the bucket holding output position m-1 in sm.s_cut and the largest count among the
-// buckets that start before m in sm.s_maxbin. Thread t owns buckets [PER*t, PER*(t+1)), read and
-// written with vector accesses (no bank conflicts).
+// buckets that start before m in sm.s_maxbin. PER = nb / kThreads buckets per thread. From
+// PER = 4 on, warp w owns the 32 PER buckets from 32 PER w on and reads them in steps of 32 int4
+// (lane l of step q holds buckets 4 (32 q + l) .. + 3 of the warp's range: consecutive lanes
+// read consecutive 16 bytes, no bank conflicts); a warp scan per step and a carry give each
+// lane its prefix within the warp, one barrier the warps' prefixes. Below 4, thread t owns
+// buckets [PER t, PER (t + 1)).
 template <int PER>
 __device__ __forceinline__ void scan_buckets(int32_t *hist, int32_t m, Smem &sm) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    int32_t c[PER];
-    if constexpr (PER >= 8) {
-#pragma unroll
-        for (int q = 0; q < PER / 4; ++q) {
-            const int4 a = reinterpret_cast<const int4 *>(hist)[(PER / 4) * tid + q];
-            c[4 * q + 0] = a.x; c[4 * q + 1] = a.y; c[4 * q + 2] = a.z; c[4 * q + 3] = a.w;
-        }
-    } else if constexpr (PER == 4) {
-        const int4 a = reinterpret_cast<const int4 *>(hist)[tid];
-        c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
-    } else if constexpr (PER == 2) {
-        const int2 a = reinterpret_cast<const int2 *>(hist)[tid];
-        c[0] = a.x; c[1] = a.y;
-    } else {
-        c[0] = hist[tid];
-    }
-    int32_t local = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) local += c[i];
-    int32_t total;
-    int32_t run = block_exclusive_scan(local, &total, sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t lmax = 0, cut = -1;
+    if constexpr (PER >= 4) {
+        constexpr int kSteps = PER / 4;
+        int4 *h4 = reinterpret_cast<int4 *>(hist) + warp * 32 * kSteps + lane;
+        int32_t pre[kSteps];
+        int32_t carry = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int32_t x = c[i];
-        c[i] = run;
-        if (run <= m - 1 && m - 1 < run + x) cut = PER * tid + i;
-        if (run < m && x > lmax) lmax = x;
-        run += x;
-    }
-    if constexpr (PER >= 8) {
+        for (int q = 0; q < kSteps; ++q) {
+            const int4 c = h4[32 * q];
+            const int32_t x = c.x + c.y + c.z + c.w;
+            int32_t incl = x;
 #pragma unroll
-        for (int q = 0; q < PER / 4; ++q)
-            reinterpret_cast<int4 *>(hist)[(PER / 4) * tid + q] =
-                make_int4(c[4 * q + 0], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
-    } else if constexpr (PER == 4) {
-        reinterpret_cast<int4 *>(hist)[tid] = make_int4(c[0], c[1], c[2], c[3]);
-    } else if constexpr (PER == 2) {
-        reinterpret_cast<int2 *>(hist)[tid] = make_int2(c[0], c[1]);
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            pre[q] = carry + incl - x;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) sm.wsum[0][warp] = carry;
+        __syncthreads();
+        int32_t before = lane < warp ? sm.wsum[0][lane] : 0;
+#pragma unroll
+        for (int o = kWarps / 2; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+        before = __shfl_sync(0xffffffffu, before, 0);
+#pragma unroll
+        for (int q = 0; q < kSteps; ++q) {
+            const int4 c = h4[32 * q];
+            int32_t x[4] = {c.x, c.y, c.z, c.w};
+            int32_t run = before + pre[q];
+            const int32_t b0 = 4 * ((warp * kSteps + q) * 32 + lane);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int32_t cnt = x[i];
+                x[i] = run;
+                if (run <= m - 1 && m - 1 < run + cnt) cut = b0 + i;
+                if (run < m && cnt > lmax) lmax = cnt;
+                run += cnt;
+            }
+            h4[32 * q] = make_int4(x[0], x[1], x[2], x[3]);
+        }
     } else {
-        hist[tid] = c[0];
+        int32_t c[PER];
+        if constexpr (PER == 2) {
+            const int2 a = reinterpret_cast<const int2 *>(hist)[tid];
+            c[0] = a.x; c[1] = a.y;
+        } else {
+            c[0] = hist[tid];
+        }
+        int32_t local = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) local += c[i];
+        int32_t run = block_exclusive_scan(local, sm);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int32_t x = c[i];
+            c[i] = run;
+            if (run <= m - 1 && m - 1 < run + x) cut = PER * tid + i;
+            if (run < m && x > lmax) lmax = x;
+            run += x;
+        }
+        if constexpr (PER == 2) {
+            reinterpret_cast<int2 *>(hist)[tid] = make_int2(c[0], c[1]);
+        } else {
+            hist[tid] = c[0];
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
@@ -340,64 +360,83 @@ __device__ __forceinline__ void scan_buckets(int32_t *hist, int32_t m, Smem &sm)
 }
 
 constexpr int kRegKeys = 4096 / kThreads;   // keys per thread held in registers (rows <= 4096)
+constexpr int kRegQuads = kRegKeys / 4;     // of them, float4 slots
+static_assert(kRegKeys % 4 == 0, "register keys come in float4 slots");
 
-// Short-row path (n <= kRegKeys * kThreads): each thread keeps its keys (e = i*kThreads + tid)
-// and their buckets in registers across the passes; one read of the row.
-// Returns 1 when the outputs [0, m) are written, 3 when all scores tie (*vtie set), 2 when the
-// caller must take the exact radix path.
+// Short-row path (n <= kRegKeys * kThreads): the row is read once with float4 loads (slot i of
+// thread tid holds keys 4 (i kThreads + tid) .. + 3) and each key and its bucket stay in
+// registers across the passes. Only the first ceil(n / (4 kThreads)) slots are live (a
+// block-uniform bound), and only the last of them can reach past the row's end. The row must
+// start 16-byte aligned and be readable up to n rounded up to 4 keys: score rows are padded to a
+// multiple of 4 floats, and row pieces start at multiples of 128 keys.
+// Returns 1 when the stage holds the m output composites in slot order, 3 when all scores tie
+// (*vtie set), 2 when the caller must take the exact radix path.
 __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *hist,
-                               uint64_t *buf, uint16_t *bufb, uint64_t *stage, int32_t off,
-                               int32_t *oi, float *ov, Smem &sm, float *vtie) {
+                               uint64_t *buf, uint16_t *bufb, uint64_t *stage, Smem &sm,
+                               float *vtie) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float kInf = __int_as_float(0x7f800000);
+    const int32_t live = (n + 4 * kThreads - 1) / (4 * kThreads);
     int32_t nb = kThreads;
     while (nb < n && nb < kNbMax) nb <<= 1;
     for (int i = tid; i < nb / 4; i += kThreads) reinterpret_cast<int4 *>(hist)[i] = make_int4(0, 0, 0, 0);
     if (tid == 0) { sm.s_cut = nb - 1; sm.s_maxbin = 0; }
+    const float4 *src4 = reinterpret_cast<const float4 *>(src);
     float v[kRegKeys];
     float lo = kInf, hi = -kInf;
 #pragma unroll
-    for (int i = 0; i < kRegKeys; ++i) {
-        const int32_t e = i * kThreads + tid;
-        float x = 0.0f;
-        if (e < n) {
-            x = __ldg(src + e);
-            x = x == 0.0f ? 0.0f : x;
-            lo = fminf(lo, x);
-            hi = fmaxf(hi, x);
+    for (int i = 0; i < kRegQuads; ++i) {
+        const int32_t e0 = 4 * (i * kThreads + tid);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < live) {
+            if (e0 < n && idx_ok(e0, (n + 3) & ~3, sm.dbg)) x = __ldg(src4 + (e0 >> 2));
+            // keys past the row's end leave the minimum and maximum alone (-0 and +0 need no
+            // care: they land in the same bucket and have the same composite key)
+            lo = fminf(lo, e0 + 0 < n ? x.x : kInf);
+            lo = fminf(lo, e0 + 1 < n ? x.y : kInf);
+            lo = fminf(lo, e0 + 2 < n ? x.z : kInf);
+            lo = fminf(lo, e0 + 3 < n ? x.w : kInf);
+            hi = fmaxf(hi, e0 + 0 < n ? x.x : -kInf);
+            hi = fmaxf(hi, e0 + 1 < n ? x.y : -kInf);
+            hi = fmaxf(hi, e0 + 2 < n ? x.z : -kInf);
+            hi = fmaxf(hi, e0 + 3 < n ? x.w : -kInf);
         }
-        v[i] = x;
+        v[4 * i + 0] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
+    // one barrier: every warp combines the warps' partial results itself (in the same order, so
+    // all warps agree)
     if (lane == 0) { sm.red_min[warp] = lo; sm.red_max[warp] = hi; }
     __syncthreads();
-    if (warp == 0) {
-        lo = lane < kWarps ? sm.red_min[lane] : kInf;
-        hi = lane < kWarps ? sm.red_max[lane] : -kInf;
+    lo = lane < kWarps ? sm.red_min[lane] : kInf;
+    hi = lane < kWarps ? sm.red_max[lane] : -kInf;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        if (lane == 0) { sm.s_vmin = lo; sm.s_vmax = hi; }
+    for (int o = kWarps / 2; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    __syncthreads();
-    const float vmin = sm.s_vmin, vmax = sm.s_vmax;
-    if (vmin == vmax) { *vtie = vmin; return 3; }
+    const float vmin = __shfl_sync(0xffffffffu, lo, 0), vmax = __shfl_sync(0xffffffffu, hi, 0);
+    if (vmin == vmax) { *vtie = vmin == 0.0f ? 0.0f : vmin; return 3; }
     if (!(vmax - vmin < kInf)) return 2;
     const float scale = (float)nb / (vmax - vmin);
     int32_t rb[kRegKeys];
 #pragma unroll
-    for (int i = 0; i < kRegKeys; ++i) {
-        const int32_t e = i * kThreads + tid;
-        rb[i] = nb;
-        if (e < n) {
-            rb[i] = bucket_of(v[i], vmin, scale, nb);
-            if (idx_ok(rb[i], nb, sm.dbg)) atomicAdd(&hist[rb[i]], 1);
+    for (int i = 0; i < kRegQuads; ++i) {
+        const int32_t e0 = 4 * (i * kThreads + tid);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rb[4 * i + j] = nb;     // nb: no key (past the row's end)
+        if (i < live) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (e0 + j < n) {
+                    rb[4 * i + j] = bucket_of(v[4 * i + j], vmin, scale, nb);
+                    if (idx_ok(rb[4 * i + j], nb, sm.dbg)) atomicAdd(&hist[rb[4 * i + j]], 1);
+                }
+            }
         }
     }
     __syncthreads();
@@ -412,19 +451,25 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
     if (sm.s_maxbin > kBinCap) return 2;
     const int32_t cutb = sm.s_cut;
 #pragma unroll
-    for (int i = 0; i < kRegKeys; ++i) {
-        const int32_t e = i * kThreads + tid;
-        if (rb[i] <= cutb && idx_ok(rb[i], nb, sm.dbg)) {   // rb == nb for keys past n
-            const int32_t dst = atomicAdd(&hist[rb[i]], 1);
-            if (idx_ok(dst, m + kBinCap, sm.dbg)) {
-                buf[dst] = ((uint64_t)score_key(v[i]) << 32) | (uint32_t)~(uint32_t)e;
-                bufb[dst] = (uint16_t)rb[i];
+    for (int i = 0; i < kRegQuads; ++i) {
+        if (i < live) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int32_t k = 4 * i + j;
+                const int32_t e = 4 * (i * kThreads + tid) + j;
+                if (rb[k] <= cutb && idx_ok(rb[k], nb, sm.dbg)) {   // rb == nb past the end
+                    const int32_t dst = atomicAdd(&hist[rb[k]], 1);
+                    if (idx_ok(dst, m + kBinCap, sm.dbg)) {
+                        buf[dst] = ((uint64_t)score_key(v[k]) << 32) | (uint32_t)~(uint32_t)e;
+                        bufb[dst] = (uint16_t)rb[k];
+                    }
+                }
             }
         }
     }
     __syncthreads();
-    // rank within the bucket; the top m land in the stage at their output slots, and the row is
-    // then written out in slot order (contiguous stores instead of one scattered store per key)
+    // rank within the bucket (two composites per step); the top m land in the stage at their
+    // output slots, which the caller writes out in slot order
     int32_t filled = hist[cutb];
     if (!in_bounds(filled >= 0 && filled <= m + kBinCap, sm.dbg)) filled = 0;
     for (int32_t p = tid; p < filled; p += kThreads) {
@@ -435,17 +480,32 @@ __device__ int reg_bucket_topk(const float *src, int32_t n, int32_t m, int32_t *
         const int32_t end = hist[b];
         if (!in_bounds(beg >= 0 && beg <= end && end <= filled, sm.dbg)) continue;
         int32_t rank = 0;
-        for (int32_t a = beg; a < end; ++a) rank += buf[a] > x ? 1 : 0;
+        int32_t a = beg;
+        for (; a + 1 < end; a += 2) rank += (buf[a] > x ? 1 : 0) + (buf[a + 1] > x ? 1 : 0);
+        if (a < end) rank += buf[a] > x ? 1 : 0;
         const int32_t slot = beg + rank;
         if (slot < m) stage[slot] = x;
     }
-    __syncthreads();
-    for (int32_t s = tid; s < m; s += kThreads) {
-        const uint64_t x = stage[s];
-        oi[s] = (int32_t)~(uint32_t)x + off;
-        if (ov) ov[s] = key_score((uint32_t)(x >> 32));
-    }
     return 1;
+}
+
+// Writes a row's output slots [0, topk): slots below m from the staged composites, the rest
+// padding (-1 / -inf), one slot per thread and step (four slots per thread with 16-byte stores
+// measured slower).
+__device__ __forceinline__ void emit_stage(const uint64_t *stage, int32_t m, int32_t topk,
+                                           int32_t off, int32_t *oi, float *ov) {
+    const float kNegInf = -__int_as_float(0x7f800000);
+    for (int32_t s = threadIdx.x; s < topk; s += kThreads) {
+        int32_t id = -1;
+        float val = kNegInf;
+        if (s < m) {
+            const uint64_t x = stage[s];
+            id = (int32_t)~(uint32_t)x + off;
+            val = key_score((uint32_t)(x >> 32));
+        }
+        oi[s] = id;
+        if (ov) ov[s] = val;
+    }
 }
 
 // Linear-bucket sort of candidates held in shared memory as (score key << 32 | ~index)
@@ -683,8 +743,14 @@ __device__ __forceinline__ void select_body(const Params &sp, int32_t n, int32_t
     int mode = 0;
     bool inB = false;
     float vtie = 0.0f;
+    int32_t written = 0;
     if (m > 0 && n <= kRegKeys * kThreads) {
-        mode = reg_bucket_topk(src, n, m, hist, buf, bufb, stage, off, oi, ov, sm, &vtie);
+        mode = reg_bucket_topk(src, n, m, hist, buf, bufb, stage, sm, &vtie);
+        if (mode == 1) {
+            __syncthreads();
+            emit_stage(stage, m, topk, off, oi, ov);
+            written = topk;
+        }
         if (mode == 2) {
             uint32_t prefix = 0u, mask = 0u;
             int32_t need = m;
@@ -697,6 +763,7 @@ __device__ __forceinline__ void select_body(const Params &sp, int32_t n, int32_t
         uint64_t *sbuf = cand + sp.cand_cap;
         uint16_t *sbufb = reinterpret_cast<uint16_t *>(sbuf + topk + kBinCap);
         mode = long_row_topk(src, n, m, hist, cand, sp.cand_cap, sbuf, sbufb, off, oi, ov, sm);
+        if (mode == 1) written = m;
         if (mode == 2) {
             uint32_t prefix = 0u, mask = 0u;
             int32_t need = m;
@@ -709,8 +776,8 @@ __device__ __forceinline__ void select_body(const Params &sp, int32_t n, int32_t
     if (mode == 2 && tid == 0) atomicAdd(&sp.ws->exact_rows, 1);
     const uint32_t *kf = inB ? keyB : keyA;
     const int32_t *jf = inB ? idxB : idxA;
-    // the bucket path has written slots [0, m) already
-    for (int32_t s = (mode == 1 ? m : 0) + tid; s < topk; s += kThreads) {
+    // the bucket paths have written slots [0, written) already
+    for (int32_t s = written + tid; s < topk; s += kThreads) {
         int32_t id = -1;
         float v = kNegInf;
         if (s < m) {
